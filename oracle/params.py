@@ -121,9 +121,13 @@ def lloyd_max_beta(d: int, levels: int):
         raise ValueError("the coordinate density needs d >= 3")
     probs = np.arange(1, levels) / levels
     init = np.array([_beta_quantile(p, d) for p in probs])
-    return lloyd_max(lambda a, b: _beta_mass(a, b, d),
+    c, _ = lloyd_max(lambda a, b: _beta_mass(a, b, d),
                      lambda a, b: _beta_first_moment(a, b, d),
                      levels, -1.0, 1.0, init)
+    # f_d is even, so the exact quantizer is odd-symmetric; make the computed one exactly
+    # so (the middle boundary is then exactly 0 and y = 0 sits on it, going to the lower cell)
+    c = 0.5 * (c - c[::-1])
+    return c, 0.5 * (c[:-1] + c[1:])
 
 
 def _beta_quantile(p: float, d: int) -> float:

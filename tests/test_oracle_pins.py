@@ -170,8 +170,8 @@ def test_codebook_fixed_point_under_gauss_legendre(d, levels):
 def test_codebook_symmetric_and_sorted(d, levels):
     c, t = lloyd_max_beta(d, levels)
     assert np.all(np.diff(c) > 0)
-    assert np.abs(c + c[::-1]).max() < 1e-15
-    assert abs(t[levels // 2 - 1]) < 1e-15
+    assert np.abs(c + c[::-1]).max() == 0.0
+    assert t[levels // 2 - 1] == 0.0
 
 
 def _max1960():
