@@ -1,0 +1,215 @@
+/*
+ * tq.h -- TurboQuant hot path for NVIDIA B200 (sm_100a): C ABI of libtq.so
+ *
+ * TurboQuant quantizes each key / value vector online and without calibration data:
+ * it stores the vector's norm, rotates its direction by a fixed random orthogonal
+ * matrix Pi, rounds each rotated coordinate to a Lloyd-Max codebook fitted to the
+ * Beta-type coordinate density, and (for keys) adds a 1-bit QJL sign sketch of the
+ * residual so that inner products are estimated without bias.  Attention and
+ * vector search then read the packed codes directly.
+ *
+ * Sources cited below:
+ *   [ZX]  zingnex.cn thread "TurboQuant：接近理论极限的KV缓存量化方案" -- sections
+ *         "随机旋转与Beta分布", "两阶段内积量化".
+ *   [TQN] turboquant.net landing page -- sections "PolarQuant：极坐标变换 / 坐标分布公式",
+ *         "伪代码实现步骤" (预计算 Lloyd-Max 质心, 生成随机旋转矩阵, Quant / DeQuant 函数,
+ *         集成到 Attention), "潜在挑战与解决方案" (随机旋转开销, 残差 norm 存储).
+ *   [ADM] admirer.cn news article on Google Research's TurboQuant -- paragraphs on
+ *         PolarQuant, QJL, the b-1 + 1 bit two-stage pipeline, vector search.
+ *
+ * Conventions shared by every call
+ *   - All data buffers are owned by the caller; pointers marked "device" must be CUDA
+ *     device (or managed) memory on the context's device, "host" pointers host memory.
+ *   - Calls never allocate device memory except tq_init (which owns the context's
+ *     parameter buffers).  Scratch space is passed in as a caller-owned workspace
+ *     whose size is given by the matching *_workspace_size query.
+ *   - Every call returns a status (TQ_OK or a TQ_ERR_* code) and never aborts.  On
+ *     error, tq_last_error() returns a message for the calling thread.  Kernels are
+ *     launched asynchronously on the given stream (NULL = legacy default stream);
+ *     execution errors surface at the caller's next synchronisation.
+ *   - A context is immutable after tq_init and may be used from several threads and
+ *     streams at once.
+ *
+ * Packed code layout (produced by tq_quantize_kv, read by every other call)
+ *   A context with dimension d, MSE bits k (k = bits-1 in prod mode, k = bits in MSE
+ *   mode) stores each vector as
+ *     - P bit planes over d_pad = 32*ceil(d/32) coordinate positions, P = k+1 in prod
+ *       mode (k index planes, then 1 sign plane), P = k in MSE mode;
+ *     - fp16 norm ||x|| (and, prod mode, fp16 residual norm ||r||) in separate arrays.
+ *   The code record of one vector is code_bytes = P*d_pad/8 bytes, divided into 4
+ *   quarters of P*d_pad/32 bytes.  Quarter q holds coordinate positions
+ *   [q*d_pad/4, (q+1)*d_pad/4); inside a quarter, plane p occupies the d_pad/32 bytes at
+ *   offset p*d_pad/32, and bit b of that chunk (bit b%8 of byte b/8, LSB first) belongs
+ *   to position q*d_pad/4 + b.  So for plane p and position i:
+ *       byte = (i / (d_pad/4)) * (P*d_pad/32) + p*(d_pad/32) + (i % (d_pad/4)) / 8
+ *       bit  = (i % (d_pad/4)) % 8
+ *   Index plane p (p < k) holds bit p of idx_i, the codebook index of rotated
+ *   coordinate y_i (binary, LSB = plane 0; centroids are sorted ascending).  The sign
+ *   plane (p = k, prod mode) holds s_j = [(S r)_j >= 0] for projection row j.
+ *   Positions i >= d are zero.  Slot t of a tq_packed buffer starts at
+ *   codes + t*code_bytes.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct tq_ctx tq_ctx;
+/* Same type as cudaStream_t; NULL selects the legacy default stream. */
+typedef struct CUstream_st* tq_stream_t;
+
+enum tq_mode {
+  TQ_MODE_PROD = 0, /* keys: (bits-1)-bit MSE codebook + 1-bit QJL sign of the residual, m = d */
+  TQ_MODE_MSE = 1   /* values: bits-bit MSE codebook only */
+};
+
+enum tq_dtype { TQ_DTYPE_F32 = 0, TQ_DTYPE_BF16 = 1, TQ_DTYPE_F16 = 2 };
+
+enum tq_status {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1, /* null pointer, negative size, mismatched contexts, bad dtype */
+  TQ_ERR_UNSUPPORTED = 2, /* d or bits outside the supported range, misaligned pointer */
+  TQ_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  TQ_ERR_ALLOC = 4,       /* tq_init could not allocate host or device memory */
+  TQ_ERR_WORKSPACE = 5,   /* workspace pointer null or smaller than the size query */
+  TQ_ERR_INTERNAL = 6     /* a kernel's own consistency check failed */
+};
+
+/* Caller-owned device storage for packed vectors (one context's codes). */
+typedef struct tq_packed {
+  uint8_t* codes;  /* device [cap][code_bytes]; must be 16-byte aligned */
+  uint16_t* norm;  /* device [cap] fp16 bit patterns of ||x|| */
+  uint16_t* rnorm; /* device [cap] fp16 bit patterns of ||r||; prod mode only (NULL in MSE mode) */
+  int64_t cap;     /* number of slots */
+} tq_packed;
+
+/* Static description of a context. */
+typedef struct tq_info {
+  int d;          /* vector (or channel-group) dimension */
+  int bits;       /* total bits per coordinate */
+  int k;          /* MSE index bits: bits-1 (prod) or bits (MSE) */
+  int m;          /* QJL projection rows (= d in prod mode, 0 in MSE mode) */
+  int mode;       /* TQ_MODE_* */
+  int planes;     /* P: bit planes per vector */
+  int d_pad;      /* 32*ceil(d/32) */
+  int code_bytes; /* P*d_pad/8 */
+  uint64_t seed;
+} tq_info;
+
+/* tq_init -- build a context: Pi, S, M = S Pi^T and the Lloyd-Max codebook, on the
+ * current CUDA device.  [TQN] "生成随机旋转矩阵" (Pi from the QR of a seeded Gaussian
+ * d x d matrix, column signs fixed so that R_ii > 0), "预计算 Lloyd-Max 质心" (codebook of
+ * 2^k levels on f_d(x) = Gamma(d/2)/(sqrt(pi) Gamma((d-1)/2)) (1-x^2)^((d-3)/2), computed
+ * once), [TQN] "随机旋转开销" (generate once, reuse); [ADM] two-stage pipeline (b-1 MSE
+ * bits + 1 QJL bit; Gaussian S with m = d rows).
+ * Random draws: SplitMix64 seeded with `seed` (output i = mix(seed + (i+1)*0x9E3779B97F4A7C15)),
+ * uniforms ((w>>11)+1)*2^-53, Box-Muller pairs (cos, sin); G (d x d, row-major) first,
+ * then S (d x d, row-major).
+ * Arguments: d in [3, 4096]; bits in [2, 5] (prod) or [1, 4] (MSE); mode TQ_MODE_*.
+ * On success *out owns host and device memory released by tq_free.
+ * Errors: TQ_ERR_INVALID_ARG (out NULL, bad mode), TQ_ERR_UNSUPPORTED (d or bits out of
+ * range), TQ_ERR_ALLOC, TQ_ERR_CUDA. */
+int tq_init(tq_ctx** out, int d, int bits, uint64_t seed, int mode);
+
+/* tq_host_params -- the same parameters as tq_init, computed on the host only (no CUDA
+ * device needed), for verification.  Output pointers as in tq_get_params (any may be NULL).
+ * Errors: as tq_init's argument checks. */
+int tq_host_params(int d, int bits, uint64_t seed, int mode, double* Pi, double* S, double* centroids,
+                   double* boundaries);
+
+/* Release a context (NULL is ignored).  The caller must ensure no work using it is
+ * still queued on any stream. */
+void tq_free(tq_ctx* ctx);
+
+/* Fill *info (host pointer). */
+int tq_get_info(const tq_ctx* ctx, tq_info* info);
+
+/* Host float64 copies of the parameters, for verification.  Any pointer may be NULL.
+ * Pi [d*d] row-major (y = Pi x), S [m*d] row-major (prod mode; zero rows in MSE
+ * mode are not written), centroids [2^k] ascending, boundaries [2^k - 1]. */
+int tq_get_params(const tq_ctx* ctx, double* Pi, double* S, double* centroids, double* boundaries);
+
+/* tq_quantize_kv -- quantize n vectors.  [TQN] "Quant / DeQuant 函数" (y = Pi x, nearest
+ * centroid per coordinate), "PolarQuant：极坐标变换" (norm stored, direction quantized),
+ * "残差 norm 存储" (||r|| as one fp16), [ADM] QJL paragraph (sign of S r).
+ * Per vector x (row v of the input):
+ *   norm = fp16_rn(||x||); y = Pi x / ||x||; idx_i = #{j : y_i > t_j};
+ *   prod mode: r = y - c[idx] (rotated residual; ||r|| equals ||x/||x|| - Pi^T c[idx]||),
+ *              rnorm = fp16_rn(||r||), s = [ M r >= 0 ] with M = S Pi^T (= S (x/||x|| - Pi^T c[idx])).
+ *   A zero vector stores norm = rnorm = 0, the index of y = 0 and all signs 1.
+ * x: device, n rows of d elements of x_dtype (TQ_DTYPE_F32 / BF16 / F16), row v at
+ *    x + v*ld elements; ld >= d.  Any channel slice of a wider row is passed by offsetting x.
+ * dst: packed storage; vector v goes to slot dst_slot[v] (device int64 array) or, when
+ *    dst_slot is NULL, to slot v.  Every slot must be < dst->cap.
+ * Errors: TQ_ERR_INVALID_ARG (NULL pointers, n < 0, ld < d, rnorm NULL in prod mode),
+ * TQ_ERR_UNSUPPORTED (misaligned codes), TQ_ERR_CUDA. */
+int tq_quantize_kv(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld,
+                   const tq_packed* dst, const int64_t* dst_slot, tq_stream_t stream);
+
+/* tq_dequantize -- MSE reconstruction x_hat = norm * Pi^T c[idx] of n stored vectors
+ * ([TQN] "Quant / DeQuant 函数").  Vector v is read from slot src_slot[v] (device int64) or
+ * slot v when src_slot is NULL, and written to out + v*ld (device float32, ld >= d). */
+int tq_dequantize(const tq_ctx* ctx, const tq_packed* src, const int64_t* src_slot, int64_t n,
+                  float* out, int64_t ld, tq_stream_t stream);
+
+/* tq_prepare_queries -- rotate queries once: out[a] = (Pi q_a [d floats], S q_a [m floats])
+ * ([TQN] "集成到 Attention": the query side of the QJL estimate).  q: device float32
+ * [nq][ld]; out: device float32 [nq][d + m]. */
+int tq_prepare_queries(const tq_ctx* ctx, const float* q, int64_t nq, int64_t ld, float* out,
+                       tq_stream_t stream);
+
+/* tq_attn_logits -- estimated inner products of nq queries with the keys in slots
+ * 0..n-1 ([ADM] "computing attention logits" on 4-bit keys; [ZX] "两阶段内积量化"):
+ *   logits[a*n + b] = norm_b * ( <Pi q_a, c[idx_b]> + sqrt(pi/2)/m * rnorm_b * <S q_a, 2 s_b - 1> )
+ * (prod mode; MSE-mode contexts give the first term only).  q: device float32 [nq][d];
+ * logits: device float32 [nq][n].  workspace: device, >= tq_attn_logits_workspace_size. */
+size_t tq_attn_logits_workspace_size(const tq_ctx* ctx, int64_t nq);
+int tq_attn_logits(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* keys, int64_t n,
+                   float* logits, void* workspace, size_t ws_bytes, tq_stream_t stream);
+
+/* tq_decode_attention -- one decode step of attention over a quantized KV cache
+ * ([TQN] "集成到 Attention": k_quant / v_quant replace the cache, QJL estimates <q,k>;
+ *  values are MSE-dequantized):
+ *   for batch b, query head h (kv head h / (Hq/Hkv)), tokens t < seq_lens[b]:
+ *     l_t = scale * sum_g est_g(q[b,h, group g], key g of token t)
+ *     out[b,h,:] = sum_t softmax(l)_t * v_hat_t,  v_hat_t[group g] = vnorm * Pi_vg^T c_vg[idx]
+ * Channel group g covers channels [group_off[g], group_off[g+1]) of the head dimension D;
+ * kctx[g] (prod) and vctx[g] (MSE) must have d = group width.  kcache[g] / vcache[g]
+ * hold slot ((b*Hkv + hk)*max_len + t) for token t of sequence b, kv head hk.
+ * q: device [B][Hq][D] of q_dtype (F32 or BF16); seq_lens: device int32 [B], each in
+ * [0, max_len] (a sequence of length 0 gives zeros); out: device float32 [B][Hq][D].
+ * group_off is a host array of ngroups+1 ints with group_off[0] = 0, group_off[ngroups] = D.
+ * Hq must be a multiple of Hkv.  workspace: device, >= tq_decode_workspace_size. */
+size_t tq_decode_workspace_size(int B, int Hq, int Hkv, int D, int ngroups, int64_t max_len);
+int tq_decode_attention(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off,
+                        int ngroups, const void* q, int q_dtype, const tq_packed* kcache,
+                        const tq_packed* vcache, const int32_t* seq_lens, int B, int Hq, int Hkv,
+                        int D, int64_t max_len, float scale, float* out, void* workspace,
+                        size_t ws_bytes, tq_stream_t stream);
+
+/* tq_search_topk -- top-k stored vectors (slots 0..N-1) of each query by the estimated
+ * inner product ([TQN] "向量搜索中的应用"; [ADM] vector-search paragraph).  Ties keep the
+ * lower id first.  q: device float32 [nq][d]; scores: device float32 [nq][k] (descending);
+ * ids: device int64 [nq][k].  1 <= k <= 64, k <= N.
+ * workspace: device, >= tq_search_workspace_size(ctx, nq, N, k). */
+size_t tq_search_workspace_size(const tq_ctx* ctx, int64_t nq, int64_t N, int k);
+int tq_search_topk(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* db, int64_t N,
+                   int k, float* scores, int64_t* ids, void* workspace, size_t ws_bytes,
+                   tq_stream_t stream);
+
+/* Message describing the calling thread's most recent error ("" if none). */
+const char* tq_last_error(void);
+
+/* Number of kernels this library has launched in this process (all streams). */
+uint64_t tq_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

@@ -1,0 +1,24 @@
+// Kernel-family selection for each hot-path call.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace tq {
+
+int launch_quantize(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld, const tq_packed* dst,
+                    const int64_t* slots, cudaStream_t st) {
+  return launch_quantize_simt(ctx, x, x_dtype, n, ld, dst, slots, st);
+}
+
+int launch_logits(const tq_ctx* ctx, const float* qprep, int64_t nq, const tq_packed* keys, int64_t n,
+                  float* logits, cudaStream_t st) {
+  return launch_logits_simt(ctx, qprep, nq, keys, n, logits, st);
+}
+
+int launch_decode(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G, const void* q,
+                  int q_dtype, const tq_packed* kc, const tq_packed* vc, const int32_t* seq_lens, int B, int Hq,
+                  int Hkv, int D, int64_t max_len, float scale, float* out, void* ws, cudaStream_t st) {
+  return launch_decode_simt(kctx, vctx, off, G, q, q_dtype, kc, vc, seq_lens, B, Hq, Hkv, D, max_len, scale, out, ws,
+                            st);
+}
+
+}  // namespace tq

@@ -1,0 +1,36 @@
+// Launchers of the libtq kernels (host side).
+#pragma once
+
+#include "common.cuh"
+
+namespace tq {
+
+int launch_quantize_simt(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld,
+                         const tq_packed* dst, const int64_t* slots, cudaStream_t st);
+int launch_dequantize_simt(const tq_ctx* ctx, const tq_packed* src, const int64_t* slots, int64_t n,
+                           float* out, int64_t ld, cudaStream_t st);
+int launch_prepare_queries(const tq_ctx* ctx, const void* q, int q_dtype, int64_t nq, int64_t ld, float* out,
+                           int64_t out_ld, cudaStream_t st);
+int launch_logits_simt(const tq_ctx* ctx, const float* qprep, int64_t nq, const tq_packed* keys, int64_t n,
+                       float* logits, cudaStream_t st);
+void decode_geometry(int B, int Hkv, int64_t max_len, int* nsplit, int* chunk);
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int ngroups, int64_t max_len, int qp_ld);
+int launch_decode_simt(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G, const void* q,
+                       int q_dtype, const tq_packed* kc, const tq_packed* vc, const int32_t* seq_lens, int B, int Hq,
+                       int Hkv, int D, int64_t max_len, float scale, float* out, void* ws, cudaStream_t st);
+size_t search_workspace_bytes(const tq_ctx* ctx, int64_t nq, int64_t N, int k);
+int launch_search_simt(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* db, int64_t N, int k,
+                       float* scores, int64_t* ids, void* ws, cudaStream_t st);
+
+}  // namespace tq
+
+namespace tq {
+// Dispatchers: pick the fastest kernel family that supports the shape.
+int launch_quantize(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld, const tq_packed* dst,
+                    const int64_t* slots, cudaStream_t st);
+int launch_logits(const tq_ctx* ctx, const float* qprep, int64_t nq, const tq_packed* keys, int64_t n,
+                  float* logits, cudaStream_t st);
+int launch_decode(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G, const void* q,
+                  int q_dtype, const tq_packed* kc, const tq_packed* vc, const int32_t* seq_lens, int B, int Hq,
+                  int Hkv, int D, int64_t max_len, float scale, float* out, void* ws, cudaStream_t st);
+}  // namespace tq

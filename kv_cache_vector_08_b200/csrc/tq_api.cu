@@ -1,0 +1,321 @@
+// C ABI of libtq: argument checking, context construction and kernel dispatch.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace tq {
+
+namespace {
+thread_local std::string g_error;
+std::atomic<uint64_t> g_launches{0};
+}  // namespace
+
+void set_error(const std::string& msg) { g_error = msg; }
+
+int fail(int code, const std::string& msg) {
+  g_error = msg;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  g_error = std::string(what) + ": " + cudaGetErrorString(e);
+  return TQ_ERR_CUDA;
+}
+
+void count_launch(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+int check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return TQ_OK;
+}
+
+namespace {
+
+int check_device(const tq_ctx* ctx) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev != ctx->device) return fail(TQ_ERR_INVALID_ARG, "context belongs to another CUDA device than the current one");
+  return TQ_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_packed(const tq_ctx* ctx, const tq_packed* pk, const char* name) {
+  if (!pk) return fail(TQ_ERR_INVALID_ARG, std::string(name) + " is NULL");
+  if (!pk->codes || !pk->norm) return fail(TQ_ERR_INVALID_ARG, std::string(name) + ": codes/norm pointer is NULL");
+  if (ctx->mode == TQ_MODE_PROD && !pk->rnorm)
+    return fail(TQ_ERR_INVALID_ARG, std::string(name) + ": rnorm is required for a prod-mode context");
+  if (pk->cap < 0) return fail(TQ_ERR_INVALID_ARG, std::string(name) + ": negative capacity");
+  if (!aligned(pk->codes, 16)) return fail(TQ_ERR_UNSUPPORTED, std::string(name) + ": codes must be 16-byte aligned");
+  return TQ_OK;
+}
+
+int alloc_copy(float** dst, const std::vector<double>& src) {
+  std::vector<float> f(src.size());
+  for (size_t i = 0; i < src.size(); ++i) f[i] = (float)src[i];
+  cudaError_t e = cudaMalloc(dst, f.size() * sizeof(float));
+  if (e != cudaSuccess) {
+    *dst = nullptr;
+    return fail(TQ_ERR_ALLOC, std::string("cudaMalloc: ") + cudaGetErrorString(e));
+  }
+  e = cudaMemcpy(*dst, f.data(), f.size() * sizeof(float), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(params)");
+  return TQ_OK;
+}
+
+std::vector<double> transpose(const std::vector<double>& a, int rows, int cols) {
+  std::vector<double> t((size_t)rows * cols);
+  for (int i = 0; i < rows; ++i)
+    for (int j = 0; j < cols; ++j) t[(size_t)j * rows + i] = a[(size_t)i * cols + j];
+  return t;
+}
+
+void release(tq_ctx* c) {
+  if (!c) return;
+  cudaFree(c->Pi);
+  cudaFree(c->PiT);
+  cudaFree(c->S);
+  cudaFree(c->ST);
+  cudaFree(c->MT);
+  delete c;
+}
+
+int check_args_common(int d, int bits, int mode) {
+  if (mode != TQ_MODE_PROD && mode != TQ_MODE_MSE) return fail(TQ_ERR_INVALID_ARG, "mode must be TQ_MODE_PROD or TQ_MODE_MSE");
+  if (d < 3 || d > 4096) return fail(TQ_ERR_UNSUPPORTED, "d must be in [3, 4096]");
+  if (mode == TQ_MODE_PROD && (bits < 2 || bits > 5)) return fail(TQ_ERR_UNSUPPORTED, "prod mode needs bits in [2, 5]");
+  if (mode == TQ_MODE_MSE && (bits < 1 || bits > 4)) return fail(TQ_ERR_UNSUPPORTED, "MSE mode needs bits in [1, 4]");
+  return TQ_OK;
+}
+
+}  // namespace
+}  // namespace tq
+
+using namespace tq;
+
+extern "C" {
+
+const char* tq_last_error(void) { return g_error.c_str(); }
+
+uint64_t tq_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int tq_host_params(int d, int bits, uint64_t seed, int mode, double* Pi, double* S, double* centroids,
+                   double* boundaries) {
+  int r = check_args_common(d, bits, mode);
+  if (r != TQ_OK) return r;
+  HostParams p;
+  if (!build_params(d, bits, seed, mode, &p)) return fail(TQ_ERR_INVALID_ARG, "bad parameters");
+  if (Pi) std::memcpy(Pi, p.Pi.data(), p.Pi.size() * sizeof(double));
+  if (S && mode == TQ_MODE_PROD) std::memcpy(S, p.S.data(), p.S.size() * sizeof(double));
+  if (centroids) std::memcpy(centroids, p.centroids.data(), p.centroids.size() * sizeof(double));
+  if (boundaries) std::memcpy(boundaries, p.boundaries.data(), p.boundaries.size() * sizeof(double));
+  return TQ_OK;
+}
+
+int tq_init(tq_ctx** out, int d, int bits, uint64_t seed, int mode) {
+  if (!out) return fail(TQ_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  int r = check_args_common(d, bits, mode);
+  if (r != TQ_OK) return r;
+  tq_ctx* c = new (std::nothrow) tq_ctx();
+  if (!c) return fail(TQ_ERR_ALLOC, "host allocation failed");
+  cudaError_t e = cudaGetDevice(&c->device);
+  if (e != cudaSuccess) {
+    delete c;
+    return cuda_fail(e, "cudaGetDevice");
+  }
+  if (!build_params(d, bits, seed, mode, &c->host)) {
+    delete c;
+    return fail(TQ_ERR_INVALID_ARG, "bad parameters");
+  }
+  const HostParams& h = c->host;
+  c->mode = mode;
+  c->bits = bits;
+  c->m = h.m;
+  Layout& L = c->lay;
+  L.d = d;
+  L.k = h.k;
+  L.d_pad = ((d + 31) / 32) * 32;
+  L.planes = h.k + (mode == TQ_MODE_PROD ? 1 : 0);
+  L.code_bytes = L.planes * L.d_pad / 8;
+  L.quarter = L.d_pad / 4;
+  L.chunk = L.d_pad / 32;
+  L.qbytes = L.planes * L.chunk;
+  Codebook& cb = c->cb;
+  cb.K = 1 << h.k;
+  for (int j = 0; j < kMaxLevels; ++j) {
+    cb.c[j] = j < cb.K ? (float)h.centroids[j] : 0.f;
+    cb.t[j] = j < cb.K - 1 ? (float)h.boundaries[j] : INFINITY;
+  }
+  c->sqrt_pi_over_2_over_m = mode == TQ_MODE_PROD ? (float)(std::sqrt(M_PI / 2.0) / h.m) : 0.f;
+  if ((r = alloc_copy(&c->Pi, h.Pi)) != TQ_OK || (r = alloc_copy(&c->PiT, transpose(h.Pi, d, d))) != TQ_OK) {
+    release(c);
+    return r;
+  }
+  if (mode == TQ_MODE_PROD) {
+    if ((r = alloc_copy(&c->S, h.S)) != TQ_OK || (r = alloc_copy(&c->ST, transpose(h.S, h.m, d))) != TQ_OK ||
+        (r = alloc_copy(&c->MT, transpose(h.M, h.m, d))) != TQ_OK) {
+      release(c);
+      return r;
+    }
+  }
+  *out = c;
+  return TQ_OK;
+}
+
+void tq_free(tq_ctx* ctx) { release(ctx); }
+
+int tq_get_info(const tq_ctx* ctx, tq_info* info) {
+  if (!ctx || !info) return fail(TQ_ERR_INVALID_ARG, "NULL argument");
+  info->d = ctx->lay.d;
+  info->bits = ctx->bits;
+  info->k = ctx->lay.k;
+  info->m = ctx->m;
+  info->mode = ctx->mode;
+  info->planes = ctx->lay.planes;
+  info->d_pad = ctx->lay.d_pad;
+  info->code_bytes = ctx->lay.code_bytes;
+  info->seed = ctx->host.seed;
+  return TQ_OK;
+}
+
+int tq_get_params(const tq_ctx* ctx, double* Pi, double* S, double* centroids, double* boundaries) {
+  if (!ctx) return fail(TQ_ERR_INVALID_ARG, "ctx is NULL");
+  const HostParams& h = ctx->host;
+  if (Pi) std::memcpy(Pi, h.Pi.data(), h.Pi.size() * sizeof(double));
+  if (S && ctx->mode == TQ_MODE_PROD) std::memcpy(S, h.S.data(), h.S.size() * sizeof(double));
+  if (centroids) std::memcpy(centroids, h.centroids.data(), h.centroids.size() * sizeof(double));
+  if (boundaries) std::memcpy(boundaries, h.boundaries.data(), h.boundaries.size() * sizeof(double));
+  return TQ_OK;
+}
+
+int tq_quantize_kv(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld, const tq_packed* dst,
+                   const int64_t* dst_slot, tq_stream_t stream) {
+  if (!ctx) return fail(TQ_ERR_INVALID_ARG, "ctx is NULL");
+  if (n < 0) return fail(TQ_ERR_INVALID_ARG, "n < 0");
+  if (n > 0 && !x) return fail(TQ_ERR_INVALID_ARG, "x is NULL");
+  if (ld < ctx->lay.d) return fail(TQ_ERR_INVALID_ARG, "ld < d");
+  if (x_dtype != TQ_DTYPE_F32 && x_dtype != TQ_DTYPE_BF16 && x_dtype != TQ_DTYPE_F16)
+    return fail(TQ_ERR_INVALID_ARG, "x_dtype must be TQ_DTYPE_F32, BF16 or F16");
+  int r = check_packed(ctx, dst, "dst");
+  if (r != TQ_OK) return r;
+  if (!dst_slot && n > dst->cap) return fail(TQ_ERR_INVALID_ARG, "n exceeds dst->cap");
+  if ((r = check_device(ctx)) != TQ_OK) return r;
+  return launch_quantize(ctx, x, x_dtype, n, ld, dst, dst_slot, (cudaStream_t)stream);
+}
+
+int tq_dequantize(const tq_ctx* ctx, const tq_packed* src, const int64_t* src_slot, int64_t n, float* out,
+                  int64_t ld, tq_stream_t stream) {
+  if (!ctx) return fail(TQ_ERR_INVALID_ARG, "ctx is NULL");
+  if (n < 0) return fail(TQ_ERR_INVALID_ARG, "n < 0");
+  if (n > 0 && !out) return fail(TQ_ERR_INVALID_ARG, "out is NULL");
+  if (ld < ctx->lay.d) return fail(TQ_ERR_INVALID_ARG, "ld < d");
+  int r = check_packed(ctx, src, "src");
+  if (r != TQ_OK) return r;
+  if (!src_slot && n > src->cap) return fail(TQ_ERR_INVALID_ARG, "n exceeds src->cap");
+  if ((r = check_device(ctx)) != TQ_OK) return r;
+  return launch_dequantize_simt(ctx, src, src_slot, n, out, ld, (cudaStream_t)stream);
+}
+
+int tq_prepare_queries(const tq_ctx* ctx, const float* q, int64_t nq, int64_t ld, float* out, tq_stream_t stream) {
+  if (!ctx) return fail(TQ_ERR_INVALID_ARG, "ctx is NULL");
+  if (nq < 0) return fail(TQ_ERR_INVALID_ARG, "nq < 0");
+  if (nq > 0 && (!q || !out)) return fail(TQ_ERR_INVALID_ARG, "NULL q or out");
+  if (ld < ctx->lay.d) return fail(TQ_ERR_INVALID_ARG, "ld < d");
+  int r = check_device(ctx);
+  if (r != TQ_OK) return r;
+  return launch_prepare_queries(ctx, q, TQ_DTYPE_F32, nq, ld, out, ctx->lay.d + ctx->m, (cudaStream_t)stream);
+}
+
+size_t tq_attn_logits_workspace_size(const tq_ctx* ctx, int64_t nq) {
+  if (!ctx || nq < 0) return 0;
+  return (size_t)nq * (ctx->lay.d + ctx->m) * sizeof(float);
+}
+
+int tq_attn_logits(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* keys, int64_t n, float* logits,
+                   void* workspace, size_t ws_bytes, tq_stream_t stream) {
+  if (!ctx) return fail(TQ_ERR_INVALID_ARG, "ctx is NULL");
+  if (nq < 0 || n < 0) return fail(TQ_ERR_INVALID_ARG, "negative size");
+  if (nq > 0 && (!q || !logits) && n > 0) return fail(TQ_ERR_INVALID_ARG, "NULL q or logits");
+  int r = check_packed(ctx, keys, "keys");
+  if (r != TQ_OK) return r;
+  if (n > keys->cap) return fail(TQ_ERR_INVALID_ARG, "n exceeds keys->cap");
+  size_t need = tq_attn_logits_workspace_size(ctx, nq);
+  if (need > 0 && (!workspace || ws_bytes < need)) return fail(TQ_ERR_WORKSPACE, "workspace too small");
+  if ((r = check_device(ctx)) != TQ_OK) return r;
+  if (nq == 0 || n == 0) return TQ_OK;
+  float* qprep = static_cast<float*>(workspace);
+  r = launch_prepare_queries(ctx, q, TQ_DTYPE_F32, nq, ctx->lay.d, qprep, ctx->lay.d + ctx->m, (cudaStream_t)stream);
+  if (r != TQ_OK) return r;
+  return launch_logits(ctx, qprep, nq, keys, n, logits, (cudaStream_t)stream);
+}
+
+size_t tq_decode_workspace_size(int B, int Hq, int Hkv, int D, int ngroups, int64_t max_len) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || ngroups <= 0 || max_len < 0) return 0;
+  return decode_workspace_bytes(B, Hq, Hkv, D, ngroups, max_len, D);
+}
+
+int tq_decode_attention(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off, int ngroups,
+                        const void* q, int q_dtype, const tq_packed* kcache, const tq_packed* vcache,
+                        const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len, float scale,
+                        float* out, void* workspace, size_t ws_bytes, tq_stream_t stream) {
+  if (!kctx || !vctx || !group_off || !kcache || !vcache) return fail(TQ_ERR_INVALID_ARG, "NULL argument");
+  if (ngroups < 1 || ngroups > 4) return fail(TQ_ERR_UNSUPPORTED, "ngroups must be in [1, 4]");
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_len < 0) return fail(TQ_ERR_INVALID_ARG, "bad sizes");
+  if (Hq % Hkv != 0) return fail(TQ_ERR_INVALID_ARG, "Hq must be a multiple of Hkv");
+  if (q_dtype != TQ_DTYPE_F32 && q_dtype != TQ_DTYPE_BF16) return fail(TQ_ERR_INVALID_ARG, "q_dtype must be F32 or BF16");
+  if (group_off[0] != 0 || group_off[ngroups] != D) return fail(TQ_ERR_INVALID_ARG, "group_off must span [0, D]");
+  if (B == 0) return TQ_OK;
+  if (!q || !seq_lens || !out) return fail(TQ_ERR_INVALID_ARG, "NULL q, seq_lens or out");
+  for (int g = 0; g < ngroups; ++g) {
+    const tq_ctx* kc = kctx[g];
+    const tq_ctx* vc = vctx[g];
+    if (!kc || !vc) return fail(TQ_ERR_INVALID_ARG, "NULL context");
+    int w = group_off[g + 1] - group_off[g];
+    if (w <= 0) return fail(TQ_ERR_INVALID_ARG, "group_off must be increasing");
+    if (kc->mode != TQ_MODE_PROD || vc->mode != TQ_MODE_MSE)
+      return fail(TQ_ERR_INVALID_ARG, "key contexts must be prod mode, value contexts MSE mode");
+    if (kc->lay.d != w || vc->lay.d != w) return fail(TQ_ERR_INVALID_ARG, "context dimension differs from its group width");
+    int r = check_packed(kc, &kcache[g], "kcache");
+    if (r != TQ_OK) return r;
+    if ((r = check_packed(vc, &vcache[g], "vcache")) != TQ_OK) return r;
+    int64_t need = (int64_t)B * Hkv * max_len;
+    if (kcache[g].cap < need || vcache[g].cap < need) return fail(TQ_ERR_INVALID_ARG, "cache capacity below B*Hkv*max_len");
+    if ((r = check_device(kc)) != TQ_OK) return r;
+  }
+  size_t need = tq_decode_workspace_size(B, Hq, Hkv, D, ngroups, max_len);
+  if (!workspace || ws_bytes < need) return fail(TQ_ERR_WORKSPACE, "workspace too small");
+  return launch_decode(kctx, vctx, group_off, ngroups, q, q_dtype, kcache, vcache, seq_lens, B, Hq, Hkv, D, max_len,
+                       scale, out, workspace, (cudaStream_t)stream);
+}
+
+size_t tq_search_workspace_size(const tq_ctx* ctx, int64_t nq, int64_t N, int k) {
+  if (!ctx || nq < 0 || N < 0 || k < 1) return 0;
+  return search_workspace_bytes(ctx, nq, N, k);
+}
+
+int tq_search_topk(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* db, int64_t N, int k,
+                   float* scores, int64_t* ids, void* workspace, size_t ws_bytes, tq_stream_t stream) {
+  if (!ctx) return fail(TQ_ERR_INVALID_ARG, "ctx is NULL");
+  if (ctx->mode != TQ_MODE_PROD) return fail(TQ_ERR_INVALID_ARG, "search needs a prod-mode context");
+  if (nq < 0 || N < 1) return fail(TQ_ERR_INVALID_ARG, "bad sizes");
+  if (k < 1 || k > 64 || k > N) return fail(TQ_ERR_UNSUPPORTED, "k must be in [1, min(64, N)]");
+  int r = check_packed(ctx, db, "db");
+  if (r != TQ_OK) return r;
+  if (N > db->cap) return fail(TQ_ERR_INVALID_ARG, "N exceeds db->cap");
+  if (nq > 0 && (!q || !scores || !ids)) return fail(TQ_ERR_INVALID_ARG, "NULL q, scores or ids");
+  size_t need = tq_search_workspace_size(ctx, nq, N, k);
+  if (!workspace || ws_bytes < need) return fail(TQ_ERR_WORKSPACE, "workspace too small");
+  if ((r = check_device(ctx)) != TQ_OK) return r;
+  return launch_search_simt(ctx, q, nq, db, N, k, scores, ids, workspace, (cudaStream_t)stream);
+}
+
+}  // extern "C"

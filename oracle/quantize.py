@@ -44,7 +44,8 @@ def quantize(params: dict, x: np.ndarray, idx_override: np.ndarray | None = None
     and sign stages can be re-run with another implementation's indices for the
     coordinates that sit on a decision boundary.
     Returns dict(idx [n,d] int64, signs [n,m] uint8 or None, norm [n], rnorm [n] or None,
-    y [n,d] float64, proj [n,m] float64 or None) -- norms already rounded to fp16.
+    y [n,d] float64, proj [n,m] float64 or None) -- norms rounded to fp16 -- plus the
+    unrounded norm_exact / rnorm_exact.
     """
     x = np.asarray(x, dtype=np.float64)
     Pi, c, t = params["Pi"], params["centroids"], params["boundaries"]
@@ -54,7 +55,8 @@ def quantize(params: dict, x: np.ndarray, idx_override: np.ndarray | None = None
     u[n == 0.0] = 0.0
     y = u @ Pi.T                       # y = Pi u for every row
     idx = nearest_index(y, t) if idx_override is None else np.asarray(idx_override, dtype=np.int64)
-    out = dict(idx=idx, norm=fp16_round(n), y=y, signs=None, rnorm=None, proj=None)
+    out = dict(idx=idx, norm=fp16_round(n), norm_exact=n, y=y, signs=None, rnorm=None,
+               rnorm_exact=None, proj=None)
     if params["mode"] == MODE_PROD:
         r = u - c[idx] @ Pi            # r = u - Pi^T c[idx]
         rn = np.sqrt(np.sum(r * r, axis=1))
@@ -63,7 +65,7 @@ def quantize(params: dict, x: np.ndarray, idx_override: np.ndarray | None = None
         zero = n == 0.0
         rn[zero] = 0.0
         signs[zero] = 1
-        out.update(rnorm=fp16_round(rn), signs=signs, proj=z)
+        out.update(rnorm=fp16_round(rn), rnorm_exact=rn, signs=signs, proj=z)
     return out
 
 

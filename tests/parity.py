@@ -1,0 +1,87 @@
+"""Comparison rules between the CUDA path and the float64 oracle.
+
+* Indices and sign bits: bit-exact, except coordinates whose oracle value lies within
+  1e-6 of a decision boundary (|y_i - t_j| < 1e-6, or |(S r)_j| < 1e-6).  The number of
+  such mismatches must not exceed 1e-4 of the coordinates.  When an exempt index differs,
+  the oracle's residual and sign stages are re-run with the CUDA path's indices for
+  that vector before the signs are compared.
+* Norms: equal as fp16, except where the float64 value lies within 1e-6 (relative) of an
+  fp16 rounding midpoint.
+* Logits and attention outputs: |gpu - oracle| <= 1e-3 + 2e-3 |oracle| elementwise.
+"""
+import numpy as np
+
+import oracle
+import layout
+
+IDX_EPS = 1e-6
+ATOL, RTOL = 1e-3, 2e-3
+
+
+def fp16_midpoint_exempt(v: np.ndarray) -> np.ndarray:
+    v = np.asarray(v, dtype=np.float64)
+    lo = (v * (1 - 1e-6)).astype(np.float16)
+    hi = (v * (1 + 1e-6)).astype(np.float16)
+    return lo != hi
+
+
+def check_codes(oparams: dict, x64: np.ndarray, codes: np.ndarray, norm16: np.ndarray, rnorm16=None,
+                label: str = "") -> dict:
+    """Compare packed GPU codes of rows x64 with the oracle; returns mismatch counts."""
+    d, k, prod = oparams["d"], oparams["k"], oparams["mode"] == 0
+    o = oracle.quantize(oparams, x64)
+    idx, signs, pad = layout.unpack(codes, d, k, prod)
+    assert (pad == 0).all(), label + ": padding bits must be zero"
+    t = oparams["boundaries"]
+    near = np.min(np.abs(o["y"][..., None] - t), axis=-1) < IDX_EPS
+    diff_idx = idx != o["idx"]
+    bad = diff_idx & ~near
+    assert not bad.any(), "%s: %d index mismatches away from a boundary (first at %s)" % (
+        label, bad.sum(), np.argwhere(bad)[:3].tolist())
+    n_coords = idx.size
+    assert diff_idx.sum() <= 1e-4 * n_coords, "%s: %d exempt index mismatches" % (label, diff_idx.sum())
+    res = dict(idx_mismatch=int(diff_idx.sum()), idx_exempt=int(near.sum()), sign_mismatch=0)
+    norm = np.asarray(norm16, dtype=np.float64)
+    nbad = (norm != o["norm"]) & ~fp16_midpoint_exempt(o["norm_exact"])
+    assert not nbad.any(), "%s: %d norm mismatches (first row %d: gpu %r oracle %r exact %r)" % (
+        label, nbad.sum(), np.argmax(nbad), norm[np.argmax(nbad)], o["norm"][np.argmax(nbad)],
+        o["norm_exact"][np.argmax(nbad)])
+    if prod:
+        rows = np.any(diff_idx, axis=1)
+        ref = o
+        if rows.any():
+            ref = oracle.quantize(oparams, x64, idx_override=idx)   # the GPU's indices
+        snear = np.abs(ref["proj"]) < IDX_EPS
+        dsig = signs != ref["signs"]
+        sbad = dsig & ~snear
+        assert not sbad.any(), "%s: %d sign mismatches away from 0 (first at %s, proj %r)" % (
+            label, sbad.sum(), np.argwhere(sbad)[:3].tolist(), ref["proj"][tuple(np.argwhere(sbad)[0])])
+        assert dsig.sum() <= 1e-4 * signs.size
+        res["sign_mismatch"] = int(dsig.sum())
+        rn = np.asarray(rnorm16, dtype=np.float64)
+        rbad = (rn != ref["rnorm"]) & ~fp16_midpoint_exempt(ref["rnorm_exact"])
+        assert not rbad.any(), "%s: %d residual-norm mismatches (first row %d: gpu %r oracle %r exact %r)" % (
+            label, rbad.sum(), np.argmax(rbad), rn[np.argmax(rbad)], ref["rnorm"][np.argmax(rbad)],
+            ref["rnorm_exact"][np.argmax(rbad)])
+    return res
+
+
+def assert_close(gpu, ref, label=""):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    err = np.abs(gpu - ref)
+    tol = ATOL + RTOL * np.abs(ref)
+    bad = err > tol
+    assert not bad.any(), "%s: %d of %d elements outside 1e-3 + 2e-3|ref| (worst err %.3g at %s, ref %.5g)" % (
+        label, bad.sum(), bad.size, err.max(), np.unravel_index(np.argmax(err - tol), err.shape),
+        ref.ravel()[np.argmax(err - tol)])
+    return float(err.max())
+
+
+def codes_dict(codes, norm16, rnorm16, d, k, prod):
+    """Unpacked GPU codes in the oracle's format (stored norms upcast)."""
+    idx, signs, _ = layout.unpack(codes, d, k, prod)
+    out = dict(idx=idx, norm=np.asarray(norm16, dtype=np.float64), signs=signs,
+               rnorm=None if rnorm16 is None else np.asarray(rnorm16, dtype=np.float64))
+    return out

@@ -1,0 +1,281 @@
+"""CUDA path vs float64 oracle, element by element, through the C ABI (needs a B200)."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+import layout
+import parity
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+import kv_cache_vector_08_b200 as tq  # noqa: E402
+
+DEV = torch.device("cuda", 0)
+
+
+def _bf16_rows(n, d, seed, outliers=False):
+    x = W.gaussian((n, d), seed, W.STREAM_KEYS)
+    if outliers:
+        x[:, [3, 17, 60, 101][: max(1, d // 32)]] *= 8.0
+    return W.round_bf16(x)
+
+
+def _quantize(ctx, x_np, dtype, slots=None, cap=None):
+    n = x_np.shape[0]
+    x = torch.tensor(x_np, dtype=dtype, device=DEV)
+    pk = tq.alloc_packed(ctx, cap or n)
+    s = None if slots is None else torch.tensor(slots, dtype=torch.int64, device=DEV)
+    tq.quantize_kv(ctx, x, pk, slots=s)
+    torch.cuda.synchronize()
+    return pk
+
+
+def _host(pk, rows=None):
+    sel = slice(None) if rows is None else torch.tensor(rows, device=DEV)
+    codes = pk.codes[sel].cpu().numpy()
+    norm = pk.norm[sel].float().cpu().numpy()
+    rn = None if pk.rnorm is None else pk.rnorm[sel].float().cpu().numpy()
+    return codes, norm, rn
+
+
+# ------------------------------------------------------------------------------ params
+@pytest.mark.parametrize("d,bits,mode", [(128, 4, 0), (64, 3, 1), (1536, 4, 0)])
+def test_device_context_params_match_oracle(d, bits, mode):
+    ctx = tq.Context(d, bits, 1000 + bits, mode)
+    p = ctx.params()
+    o = oracle.make_params(d, bits, 1000 + bits, mode)
+    assert np.abs(p["Pi"] - o["Pi"]).max() < 1e-10
+    assert np.abs(p["centroids"] - o["centroids"]).max() < 1e-10
+    assert (ctx.d_pad, ctx.planes, ctx.code_bytes) == layout.geometry(d, o["k"], mode == 0)
+
+
+# ---------------------------------------------------------------------------- quantize
+def test_quantize_toy_config_fp32():
+    """Keys N=4096 x 128 fp32 N(0,1) from seed 0, b = 3 (2-bit MSE + 1-bit QJL, m = 128)."""
+    keys, _ = W.toy_inputs(0)
+    ctx = tq.Context(128, 3, 1000, tq.MODE_PROD)
+    pk = _quantize(ctx, keys, torch.float32)
+    codes, norm, rn = _host(pk)
+    res = parity.check_codes(oracle.make_params(128, 3, 1000, 0), keys.astype(np.float64), codes, norm, rn, "toy")
+    print("toy quantize", res)
+
+
+@pytest.mark.parametrize("d,bits,mode,n,dtype", [
+    (128, 4, 0, 3000, "bf16"), (128, 4, 1, 3000, "bf16"),      # Llama-shaped keys / values
+    (64, 4, 0, 1031, "bf16"), (64, 3, 0, 1031, "bf16"), (64, 2, 0, 517, "bf16"),
+    (64, 4, 1, 1031, "bf16"), (64, 3, 1, 1031, "bf16"), (64, 2, 1, 517, "bf16"),
+    (128, 5, 0, 300, "f16"), (128, 1, 1, 300, "fp32"),
+    (200, 4, 0, 257, "fp32"), (1536, 4, 0, 65, "fp32"), (16, 3, 0, 129, "fp32"),
+    (128, 4, 0, 1, "bf16"), (128, 4, 0, 127, "bf16"), (128, 4, 0, 129, "bf16"),
+])
+def test_quantize_matches_oracle(d, bits, mode, n, dtype):
+    seed = 1000 + 2 * bits + mode
+    if dtype == "fp32":
+        x = W.unit_gaussian(n, d, 3, 11) * 3.0
+    else:
+        x = _bf16_rows(n, d, 5, outliers=True)
+    tdt = {"bf16": torch.bfloat16, "f16": torch.float16, "fp32": torch.float32}[dtype]
+    if dtype == "f16":
+        x = x.astype(np.float16).astype(np.float32)
+    ctx = tq.Context(d, bits, seed, mode)
+    pk = _quantize(ctx, x, tdt)
+    codes, norm, rn = _host(pk)
+    res = parity.check_codes(oracle.make_params(d, bits, seed, mode), x.astype(np.float64), codes, norm, rn,
+                             "d=%d b=%d mode=%d" % (d, bits, mode))
+    print(d, bits, mode, n, res)
+
+
+def test_quantize_zero_rows_and_scattered_slots():
+    d, n = 128, 300
+    x = _bf16_rows(n, d, 9)
+    x[[0, 17, 299]] = 0.0
+    rng = np.random.default_rng(4)
+    slots = rng.permutation(1000)[:n]
+    ctx = tq.Context(d, 4, 77, tq.MODE_PROD)
+    pk = _quantize(ctx, x, torch.bfloat16, slots=slots, cap=1000)
+    codes, norm, rn = _host(pk, rows=slots)
+    parity.check_codes(oracle.make_params(d, 4, 77, 0), x.astype(np.float64), codes, norm, rn, "zero+slots")
+    assert norm[0] == 0 and rn[0] == 0
+    # slots that were not written stay zero
+    untouched = np.setdiff1d(np.arange(1000), slots)
+    assert pk.codes[torch.tensor(untouched, device=DEV)].abs().sum().item() == 0
+
+
+def test_quantize_strided_channel_group():
+    """A group's channels are a slice of wider rows: x + offset, ld = row width."""
+    full = _bf16_rows(500, 128, 13)
+    xt = torch.tensor(full, dtype=torch.bfloat16, device=DEV)
+    ctx = tq.Context(64, 3, 1003, tq.MODE_PROD)
+    pk = tq.alloc_packed(ctx, 500)
+    tq.quantize_kv(ctx, xt[:, 64:], pk)
+    torch.cuda.synchronize()
+    codes, norm, rn = _host(pk)
+    parity.check_codes(oracle.make_params(64, 3, 1003, 0), full[:, 64:].astype(np.float64), codes, norm, rn, "slice")
+
+
+# -------------------------------------------------------------------------- dequantize
+@pytest.mark.parametrize("d,bits,mode", [(128, 4, 1), (64, 3, 0), (200, 2, 1)])
+def test_dequantize_matches_oracle(d, bits, mode):
+    x = _bf16_rows(333, d, 21)
+    ctx = tq.Context(d, bits, 5, mode)
+    pk = _quantize(ctx, x, torch.bfloat16)
+    out = tq.dequantize(ctx, pk, 333).cpu().numpy()
+    codes, norm, rn = _host(pk)
+    cd = parity.codes_dict(codes, norm, rn, d, ctx.k, mode == 0)
+    ref = oracle.dequantize(oracle.make_params(d, bits, 5, mode), cd["idx"], cd["norm"])
+    parity.assert_close(out, ref, "dequant")
+
+
+# ------------------------------------------------------------------------------ logits
+def test_logits_toy_config():
+    """16 queries x 4096 keys: logits from the GPU codes vs the oracle estimator on the
+    same codes, and vs the oracle's end-to-end quantize + estimate."""
+    keys, queries = W.toy_inputs(0)
+    op = oracle.make_params(128, 3, 1000, 0)
+    ctx = tq.Context(128, 3, 1000, tq.MODE_PROD)
+    pk = _quantize(ctx, keys, torch.float32)
+    q = torch.tensor(queries, device=DEV)
+    lg = tq.attn_logits(ctx, q, pk, 4096).cpu().numpy()
+    codes, norm, rn = _host(pk)
+    ref = oracle.estimate_inner_products(op, queries.astype(np.float64), parity.codes_dict(codes, norm, rn, 128, 2, True))
+    parity.assert_close(lg, ref, "logits(gpu codes)")
+    e2e = oracle.estimate_inner_products(op, queries.astype(np.float64), oracle.quantize(op, keys.astype(np.float64)))
+    parity.assert_close(lg, e2e, "logits(end to end)")
+
+
+@pytest.mark.parametrize("d,bits,n,nq", [(128, 4, 1000, 3), (64, 2, 777, 9), (200, 4, 300, 5), (128, 3, 1, 1)])
+def test_logits_on_oracle_codes(d, bits, n, nq):
+    """Codes produced by the oracle, packed on the host and uploaded: isolates the logits
+    kernel from the quantizer."""
+    op = oracle.make_params(d, bits, 31, 0)
+    x = _bf16_rows(n, d, 2).astype(np.float64)
+    o = oracle.quantize(op, x)
+    codes = layout.pack(o["idx"], o["signs"], d, op["k"])
+    ctx = tq.Context(d, bits, 31, tq.MODE_PROD)
+    pk = tq.alloc_packed(ctx, n)
+    pk.codes.copy_(torch.tensor(codes, device=DEV))
+    pk.norm.copy_(torch.tensor(o["norm"], dtype=torch.float16, device=DEV))
+    pk.rnorm.copy_(torch.tensor(o["rnorm"], dtype=torch.float16, device=DEV))
+    qn = W.gaussian((nq, d), 8, W.STREAM_QUERIES).astype(np.float32)
+    lg = tq.attn_logits(ctx, torch.tensor(qn, device=DEV), pk, n).cpu().numpy()
+    parity.assert_close(lg, oracle.estimate_inner_products(op, qn.astype(np.float64), o), "logits")
+
+
+def test_prepare_queries():
+    ctx = tq.Context(128, 4, 3, tq.MODE_PROD)
+    q = W.gaussian((7, 128), 1, 2).astype(np.float32)
+    out = tq.prepare_queries(ctx, torch.tensor(q, device=DEV)).cpu().numpy()
+    qt, qs = oracle.prepare_query(oracle.make_params(128, 4, 3, 0), q.astype(np.float64))
+    assert np.abs(out[:, :128] - qt).max() < 1e-4
+    assert np.abs(out[:, 128:] - qs).max() < 1e-3
+
+
+# ------------------------------------------------------------------------------ decode
+def _decode_case(B, Hkv, Hq, D, groups, seq_lens, max_len, seed, q_dtype=torch.bfloat16):
+    rng = np.random.default_rng(seed)
+    K = W.round_bf16(rng.standard_normal((B, Hkv, max_len, D)))
+    V = W.round_bf16(rng.standard_normal((B, Hkv, max_len, D)) * rng.lognormal(0, 0.5, (B, 1, max_len, 1)))
+    qn = W.round_bf16(rng.standard_normal((B, Hq, D)))
+    kctx, vctx, kc, vc, kp, vp, offs = [], [], [], [], [], [], []
+    for gi, (off, w, kb, vb) in enumerate(groups):
+        kx = tq.Context(w, kb, 1000 + 2 * gi, tq.MODE_PROD)
+        vx = tq.Context(w, vb, 1001 + 2 * gi, tq.MODE_MSE)
+        kpk = tq.alloc_packed(kx, B * Hkv * max_len)
+        vpk = tq.alloc_packed(vx, B * Hkv * max_len)
+        # prefill: token t of (b, h) -> slot (b*Hkv + h)*max_len + t, only t < seq_len
+        rows, slots = [], []
+        for b in range(B):
+            for h in range(Hkv):
+                for t in range(seq_lens[b]):
+                    rows.append((b, h, t))
+                    slots.append((b * Hkv + h) * max_len + t)
+        if rows:
+            ridx = np.array(rows)
+            st = torch.tensor(slots, dtype=torch.int64, device=DEV)
+            kr = torch.tensor(K[ridx[:, 0], ridx[:, 1], ridx[:, 2]][:, off:off + w].copy(), dtype=torch.bfloat16, device=DEV)
+            vr = torch.tensor(V[ridx[:, 0], ridx[:, 1], ridx[:, 2]][:, off:off + w].copy(), dtype=torch.bfloat16, device=DEV)
+            tq.quantize_kv(kx, kr, kpk, slots=st)
+            tq.quantize_kv(vx, vr, vpk, slots=st)
+        kctx.append(kx); vctx.append(vx); kc.append(kpk); vc.append(vpk)
+        kp.append(oracle.make_params(w, kb, 1000 + 2 * gi, 0))
+        vp.append(oracle.make_params(w, vb, 1001 + 2 * gi, 1))
+        offs.append(off)
+    offs.append(D)
+    sl = torch.tensor(seq_lens, dtype=torch.int32, device=DEV)
+    q = torch.tensor(qn, dtype=q_dtype, device=DEV)
+    scale = 1.0 / math.sqrt(D)
+    out = tq.decode_attention(kctx, vctx, offs, q, kc, vc, sl, Hkv, max_len, scale).cpu().numpy()
+    # oracle on the GPU's stored codes
+    kcodes, vcodes = [], []
+    for gi, (off, w, kb, vb) in enumerate(groups):
+        c, n_, r_ = _host(kc[gi])
+        d1 = parity.codes_dict(c, n_, r_, w, kb - 1, True)
+        kcodes.append({k: (None if v is None else v.reshape(B, Hkv, max_len, *v.shape[1:])) for k, v in d1.items()})
+        c, n_, _ = _host(vc[gi])
+        d2 = parity.codes_dict(c, n_, None, w, vb, False)
+        vcodes.append({k: v.reshape(B, Hkv, max_len, *v.shape[1:]) for k, v in d2.items() if v is not None})
+    ref = oracle.decode_attention(kp, vp, offs, qn.astype(np.float64), kcodes, vcodes, seq_lens, scale)
+    return out, ref, (K, V, qn, kp, vp, offs)
+
+
+@pytest.mark.parametrize("groups", [((0, 128, 4, 4),), ((0, 64, 4, 4), (64, 64, 3, 3)), ((0, 64, 3, 3), (64, 64, 2, 2))])
+def test_decode_matches_oracle(groups):
+    out, ref, _ = _decode_case(2, 2, 8, 128, groups, [300, 37], 320, 1)
+    parity.assert_close(out, ref, "decode %s" % (groups,))
+
+
+def test_decode_edge_lengths():
+    """Empty sequence -> zeros; single token -> that token's dequantized value; ragged tails."""
+    out, ref, (K, V, qn, kp, vp, offs) = _decode_case(4, 1, 4, 128, ((0, 128, 4, 4),), [0, 1, 129, 255], 256, 2)
+    assert np.all(out[0] == 0.0)
+    parity.assert_close(out, ref, "edge")
+
+
+def test_decode_end_to_end_matches_oracle_pipeline():
+    """GPU quantize + decode vs oracle quantize + decode on the same bf16 inputs."""
+    groups = ((0, 128, 4, 4),)
+    B, Hkv, Hq, D, T = 1, 2, 8, 128, 200
+    out, _, (K, V, qn, kp, vp, offs) = _decode_case(B, Hkv, Hq, D, groups, [T], T, 3)
+    ko = oracle.quantize(kp[0], K.reshape(-1, D).astype(np.float64))
+    vo = oracle.quantize(vp[0], V.reshape(-1, D).astype(np.float64))
+    kcodes = [{k: (None if v is None else v.reshape(B, Hkv, T, *v.shape[1:])) for k, v in
+               dict(idx=ko["idx"], norm=ko["norm"], signs=ko["signs"], rnorm=ko["rnorm"]).items()}]
+    vcodes = [dict(idx=vo["idx"].reshape(B, Hkv, T, D), norm=vo["norm"].reshape(B, Hkv, T))]
+    ref = oracle.decode_attention(kp, vp, offs, qn.astype(np.float64), kcodes, vcodes, [T], 1 / math.sqrt(D))
+    parity.assert_close(out, ref, "e2e decode")
+
+
+# ------------------------------------------------------------------------------ search
+@pytest.mark.parametrize("d,N,k", [(128, 5000, 10), (200, 3000, 10), (64, 100, 64)])
+def test_search_topk_matches_oracle(d, N, k):
+    db = W.unit_gaussian(N, d, 1, 10)
+    db[N // 2] = db[7]                        # an exact tie: lower id must come first
+    qs = W.unit_gaussian(6, d, 1, 3)
+    qs[0] = db[7]
+    ctx = tq.Context(d, 4, 12, tq.MODE_PROD)
+    pk = _quantize(ctx, db, torch.float32)
+    scores, ids = tq.search_topk(ctx, torch.tensor(qs, device=DEV), pk, N, k)
+    scores, ids = scores.cpu().numpy(), ids.cpu().numpy()
+    codes, norm, rn = _host(pk)
+    op = oracle.make_params(d, 4, 12, 0)
+    cd = parity.codes_dict(codes, norm, rn, d, 3, True)
+    est = oracle.estimate_inner_products(op, qs.astype(np.float64), cd)
+    ref_s, ref_i = oracle.search_topk(op, qs.astype(np.float64), cd, k)
+    parity.assert_close(scores, ref_s, "top-k scores")
+    for a in range(len(qs)):
+        assert len(set(ids[a])) == k
+        parity.assert_close(scores[a], est[a, ids[a]], "score of returned id")
+        # ids agree wherever the oracle's scores are separated by more than the tolerance
+        gap = np.abs(np.diff(np.sort(est[a])[::-1][: k + 1]))
+        if gap.min() > 2 * (parity.ATOL + parity.RTOL * np.abs(ref_s[a]).max()):
+            assert list(ids[a]) == list(ref_i[a])
+    row = list(ids[0])
+    if 7 in row and N // 2 in row and scores[0][row.index(7)] == scores[0][row.index(N // 2)]:
+        assert row.index(7) < row.index(N // 2)        # equal scores: lower id first
