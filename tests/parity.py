@@ -85,3 +85,20 @@ def codes_dict(codes, norm16, rnorm16, d, k, prod):
     out = dict(idx=idx, norm=np.asarray(norm16, dtype=np.float64), signs=signs,
                rnorm=None if rnorm16 is None else np.asarray(rnorm16, dtype=np.float64))
     return out
+
+
+def reconciled_oracle_codes(oparams: dict, x64: np.ndarray, codes: np.ndarray) -> dict:
+    """The oracle's own codes for rows x64, except that rows where the GPU chose another
+    index for a coordinate within 1e-6 of a boundary (the exempt case) are re-run through
+    the oracle with the GPU's indices.  End-to-end comparisons use these codes."""
+    d, k, prod = oparams["d"], oparams["k"], oparams["mode"] == 0
+    o = oracle.quantize(oparams, x64)
+    idx, _, _ = layout.unpack(codes, d, k, prod)
+    rows = np.any(idx != o["idx"], axis=1)
+    if rows.any():
+        fixed = oracle.quantize(oparams, x64[rows], idx_override=idx[rows])
+        for key in ("idx", "signs", "norm", "rnorm"):
+            if o[key] is not None:
+                o[key] = o[key].copy()
+                o[key][rows] = fixed[key]
+    return dict(idx=o["idx"], signs=o["signs"], norm=o["norm"], rnorm=o["rnorm"], rows_reconciled=int(rows.sum()))

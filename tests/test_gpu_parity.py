@@ -146,7 +146,9 @@ def test_logits_toy_config():
     codes, norm, rn = _host(pk)
     ref = oracle.estimate_inner_products(op, queries.astype(np.float64), parity.codes_dict(codes, norm, rn, 128, 2, True))
     parity.assert_close(lg, ref, "logits(gpu codes)")
-    e2e = oracle.estimate_inner_products(op, queries.astype(np.float64), oracle.quantize(op, keys.astype(np.float64)))
+    rec = parity.reconciled_oracle_codes(op, keys.astype(np.float64), codes)
+    assert rec["rows_reconciled"] <= 4
+    e2e = oracle.estimate_inner_products(op, queries.astype(np.float64), rec)
     parity.assert_close(lg, e2e, "logits(end to end)")
 
 
@@ -222,6 +224,7 @@ def _decode_case(B, Hkv, Hq, D, groups, seq_lens, max_len, seed, q_dtype=torch.b
         d2 = parity.codes_dict(c, n_, None, w, vb, False)
         vcodes.append({k: v.reshape(B, Hkv, max_len, *v.shape[1:]) for k, v in d2.items() if v is not None})
     ref = oracle.decode_attention(kp, vp, offs, qn.astype(np.float64), kcodes, vcodes, seq_lens, scale)
+    _decode_case.last_caches = (kc, vc)
     return out, ref, (K, V, qn, kp, vp, offs)
 
 
@@ -243,8 +246,9 @@ def test_decode_end_to_end_matches_oracle_pipeline():
     groups = ((0, 128, 4, 4),)
     B, Hkv, Hq, D, T = 1, 2, 8, 128, 200
     out, _, (K, V, qn, kp, vp, offs) = _decode_case(B, Hkv, Hq, D, groups, [T], T, 3)
-    ko = oracle.quantize(kp[0], K.reshape(-1, D).astype(np.float64))
-    vo = oracle.quantize(vp[0], V.reshape(-1, D).astype(np.float64))
+    kg, vg = _decode_case.last_caches
+    ko = parity.reconciled_oracle_codes(kp[0], K.reshape(-1, D).astype(np.float64), _host(kg[0])[0])
+    vo = parity.reconciled_oracle_codes(vp[0], V.reshape(-1, D).astype(np.float64), _host(vg[0])[0])
     kcodes = [{k: (None if v is None else v.reshape(B, Hkv, T, *v.shape[1:])) for k, v in
                dict(idx=ko["idx"], norm=ko["norm"], signs=ko["signs"], rnorm=ko["rnorm"]).items()}]
     vcodes = [dict(idx=vo["idx"].reshape(B, Hkv, T, D), norm=vo["norm"].reshape(B, Hkv, T))]
