@@ -192,6 +192,31 @@ int tq_decode_attention(const tq_ctx* const* kctx, const tq_ctx* const* vctx, co
                         int D, int64_t max_len, float scale, float* out, void* workspace,
                         size_t ws_bytes, tq_stream_t stream);
 
+/* Size in bytes of the library-owned scratch array used by tq_decode_attention_static. */
+#define TQ_DECODE_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+
+/* tq_decode_attention_static -- tq_decode_attention for callers that cannot allocate
+ * device memory.  The pages have no counterpart to this call; it exists for callers such
+ * as plug-ins hosted by an engine that owns all device memory through its own pool, or
+ * latency-critical serving loops that may not call cudaMalloc (which can synchronise
+ * the device) on the decode path.  Such a caller passes only inputs and outputs; the
+ * split-K scratch (prepared queries, per-split softmax partials) lives in a fixed array of
+ * TQ_DECODE_STATIC_SCRATCH_BYTES bytes in this library's device memory, which every GPU
+ * that loads the library holds until the process exits.  The call allocates nothing.
+ * Arguments, layout and results are those of tq_decode_attention.
+ * Set-up: the first call on each device (with that device current) looks up the array's
+ * device address once; make that first call before any stream capture.
+ * Shared state: every call uses the same array and leaves its contents behind; nothing in
+ * it needs to start at zero.  Calls whose GPU work overlaps (on different streams, or
+ * from different host threads) race on the array, so serialise them.
+ * Errors: TQ_ERR_WORKSPACE when the shape needs more scratch than the array holds
+ * (tq_decode_workspace_size > TQ_DECODE_STATIC_SCRATCH_BYTES; use tq_decode_attention
+ * with a caller workspace instead), otherwise those of tq_decode_attention. */
+int tq_decode_attention_static(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off,
+                               int ngroups, const void* q, int q_dtype, const tq_packed* kcache,
+                               const tq_packed* vcache, const int32_t* seq_lens, int B, int Hq, int Hkv, int D,
+                               int64_t max_len, float scale, float* out, tq_stream_t stream);
+
 /* tq_search_topk -- top-k stored vectors (slots 0..N-1) of each query by the estimated
  * inner product ([TQN] "向量搜索中的应用"; [ADM] vector-search paragraph).  Ties keep the
  * lower id first.  q: device float32 [nq][d]; scores: device float32 [nq][k] (descending);
