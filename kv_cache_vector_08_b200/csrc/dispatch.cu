@@ -17,6 +17,9 @@ int launch_logits(const tq_ctx* ctx, const float* qprep, int64_t nq, const tq_pa
 int launch_decode(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G, const void* q,
                   int q_dtype, const tq_packed* kc, const tq_packed* vc, const int32_t* seq_lens, int B, int Hq,
                   int Hkv, int D, int64_t max_len, float scale, float* out, void* ws, cudaStream_t st) {
+  int r = launch_decode_mma(kctx, vctx, off, G, q, q_dtype, kc, vc, seq_lens, B, Hq, Hkv, D, max_len, scale, out, ws,
+                            st);
+  if (r != kNotHandled) return r;
   return launch_decode_simt(kctx, vctx, off, G, q, q_dtype, kc, vc, seq_lens, B, Hq, Hkv, D, max_len, scale, out, ws,
                             st);
 }

@@ -492,7 +492,7 @@ __global__ void __launch_bounds__(kDecTile) decode_split_simt_kernel(DecodeArgs 
 
 struct MergeArgs {
   const float* part;
-  int nsplit, D, G, Hq;
+  int nsplit, D, G;
   int off[kMaxGroups + 1];
   const float* PiV[kMaxGroups];  // value rotations [d_g][d_g]
   float* out;
@@ -798,11 +798,16 @@ int launch_decode_simt(const tq_ctx* const* kctx, const tq_ctx* const* vctx, con
   count_launch();
   int r = check_launch("decode_split_simt_kernel");
   if (r != TQ_OK) return r;
+  return launch_decode_merge(vctx, off, G, part, nsplit, B * Hq, D, out, st);
+}
+
+int launch_decode_merge(const tq_ctx* const* vctx, const int* off, int G, const float* part, int nsplit, int BHq,
+                        int D, float* out, cudaStream_t st) {
   MergeArgs M{};
-  M.part = part; M.nsplit = nsplit; M.D = D; M.G = G; M.Hq = Hq; M.out = out;
+  M.part = part; M.nsplit = nsplit; M.D = D; M.G = G; M.out = out;
   for (int g = 0; g < G; ++g) { M.off[g] = off[g]; M.PiV[g] = vctx[g]->Pi; }
   M.off[G] = D;
-  decode_merge_kernel<<<B * Hq, 128, (D + nsplit) * sizeof(float), st>>>(M);
+  decode_merge_kernel<<<BHq, 128, (D + nsplit) * sizeof(float), st>>>(M);
   count_launch();
   return check_launch("decode_merge_kernel");
 }

@@ -283,3 +283,15 @@ def test_search_topk_matches_oracle(d, N, k):
     row = list(ids[0])
     if 7 in row and N // 2 in row and scores[0][row.index(7)] == scores[0][row.index(N // 2)]:
         assert row.index(7) < row.index(N // 2)        # equal scores: lower id first
+
+
+@pytest.mark.parametrize("Hkv,Hq", [(2, 4), (1, 8), (3, 12)])
+def test_decode_other_gqa_ratios(Hkv, Hq):
+    """GQA ratios 2, 8 (SIMT kernel) and 4 with three kv heads (tensor-core kernel)."""
+    out, ref, _ = _decode_case(2, Hkv, Hq, 128, ((0, 128, 4, 4),), [100, 33], 128, 7)
+    parity.assert_close(out, ref, "gqa %d/%d" % (Hq, Hkv))
+
+
+def test_decode_fp32_queries_and_128_2bit_keys():
+    out, ref, _ = _decode_case(1, 2, 8, 128, ((0, 128, 3, 3),), [513], 600, 8, q_dtype=torch.float32)
+    parity.assert_close(out, ref, "fp32 q, 3-bit keys / values")
