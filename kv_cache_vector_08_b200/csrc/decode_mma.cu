@@ -103,23 +103,11 @@ __device__ __forceinline__ uint32_t selector(const uint32_t* w, int qq) {
   return s;
 }
 
-// fp16 centroid table split into low/high bytes, 8 entries per register pair.
+// fp16 centroid table split into low/high bytes, 8 entries per register pair (built on
+// the host from the context's codebook).
 struct Lut {
   uint32_t lo[4], hi[4];  // lo[0..1]: low bytes of c[0..7], lo[2..3]: of c[8..15]
 };
-
-__device__ __forceinline__ Lut make_lut(const float* c, int K) {
-  Lut t;
-  uint32_t lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};
-  for (int j = 0; j < 16; ++j) {
-    uint16_t b = j < K ? __half_as_ushort(__float2half_rn(c[j])) : 0;
-    lo[j / 4] |= (uint32_t)(b & 0xFF) << (8 * (j % 4));
-    hi[j / 4] |= (uint32_t)(b >> 8) << (8 * (j % 4));
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) { t.lo[i] = lo[i]; t.hi[i] = hi[i]; }
-  return t;
-}
 
 // Two half2 registers: fp16 centroids of the coordinates selected by the 4 nibbles of
 // `sel` (pairs nibble 0,1 and nibble 2,3).  NB index bits; the 4th bit (NB == 4) chooses
@@ -147,7 +135,8 @@ struct MmaGroup {
   const uint16_t* krnorm;
   const uint8_t* vcodes;
   const uint16_t* vnorm;
-  float kc[16], vc[16];
+  const float* PiV;    // value rotation [d_g][d_g] row-major (float32)
+  Lut klut, vlut;      // fp16 key / value centroid tables
   float coef;          // sqrt(pi/2)/m
   int off;             // first channel of the group
   int kbytes, vbytes;  // record sizes
@@ -159,9 +148,14 @@ struct MmaArgs {
   int64_t max_len;
   float scale_log2;    // softmax scale * log2(e)
   const int32_t* seq_lens;
-  const float* qprep;  // [B*Hq][G][2*qp_ld]
-  float* part;         // [B*Hq][nsplit][D+2]
+  const float* qprep;  // [B*Hq][G][2*qp_ld]: (Pi q, S q) of each group
+  float* part;         // [B*Hq][nsplit][D+2]: (m, l, acc) per split
+  int* done;           // [B*Hkv] finished-split counters (zeroed by the prep kernel)
+  float* out;          // [B*Hq][D]
 };
+
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void allow_dependent_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
 // Query fragments of one group for this thread, built once per CTA.
 template <class GC>
@@ -173,8 +167,8 @@ struct QFrag {
 template <class GC>
 __device__ __forceinline__ void load_qfrag(QFrag<GC>& f, const MmaArgs& A, int gi, int b, int hk, int lane) {
   const int g = lane >> 2, l = lane & 3;
-  const int head = hk * kRep + (g & 3);
-  const bool lo_part = g >= 4;
+  const int head = hk * kRep + (g >> 1);   // column n = g: head n/2, hi (n even) or lo (n odd) half
+  const bool lo_part = (g & 1) != 0;
   const float* src = A.qprep + ((size_t)(b * A.Hq + head) * A.G + gi) * 2 * A.qp_ld;
   const float* qt = src;
   const float* qs = src + GC::DG;
@@ -247,10 +241,44 @@ __device__ __forceinline__ void group_values(const Lut& vl, const uint32_t (&w0)
       uint32_t x0f, x0s, x1f, x1s;  // token g / g+8, coordinate blocks f = 0 (first) and 1 (second)
       lookup<GC::KV>(vl, s0 >> (16 * hh), ((b40 >> (16 * hh)) & 0xFFFFu) | 0x3210u, x0f, x0s);
       lookup<GC::KV>(vl, s1 >> (16 * hh), ((b41 >> (16 * hh)) & 0xFFFFu) | 0x3210u, x1f, x1s);
-      // rows (coordinates) g: block f = 0, g+8: block f = 1; k (tokens) 2l.. from token g block, 2l+8.. from g+8
+      // rows (coordinates) g: block f = 0, g+8: block f = 1; k (tokens) 2l.. from token g, 2l+8.. from g+8
       mma16816(acc[mb], movT(x0f), movT(x0s), movT(x1f), movT(x1s), pb0, pb1);
     }
   }
+}
+
+// Everything a thread loads for one 16-token tile of one group.
+template <class GC>
+struct TileData {
+  uint32_t ka[GC::PK], kb[GC::PK], va[GC::PV], vb[GC::PV];
+  unsigned short nka, nkb, rka, rkb, nva, nvb;
+};
+
+template <class GC>
+__device__ __forceinline__ void load_tile(TileData<GC>& t, const MmaGroup& gr, int64_t sa, int64_t sb, int l) {
+  load_quarter<GC::Q, GC::PK>(gr.kcodes + sa * gr.kbytes, l, t.ka);
+  load_quarter<GC::Q, GC::PK>(gr.kcodes + sb * gr.kbytes, l, t.kb);
+  load_quarter<GC::Q, GC::PV>(gr.vcodes + sa * gr.vbytes, l, t.va);
+  load_quarter<GC::Q, GC::PV>(gr.vcodes + sb * gr.vbytes, l, t.vb);
+  t.nka = __ldg(gr.knorm + sa);
+  t.nkb = __ldg(gr.knorm + sb);
+  t.rka = __ldg(gr.krnorm + sa);
+  t.rkb = __ldg(gr.krnorm + sb);
+  t.nva = __ldg(gr.vnorm + sa);
+  t.nvb = __ldg(gr.vnorm + sb);
+}
+
+__device__ __forceinline__ float h2f(unsigned short h) { return __half2float(__ushort_as_half(h)); }
+
+template <class GC>
+__device__ __forceinline__ void tile_logits(const TileData<GC>& t, const QFrag<GC>& qf, const Lut& kl,
+                                            const MmaGroup& gr, float& la, float& lb) {
+  float mse[4], sgn[4];
+  group_logits<GC>(qf, kl, t.ka, t.kb, mse, sgn);
+  // columns 2l, 2l+1 are the hi and lo halves of head l
+  const float ca = gr.coef * h2f(t.rka), cb = gr.coef * h2f(t.rkb);
+  la += h2f(t.nka) * fmaf(ca, sgn[0] + sgn[1], mse[0] + mse[1]);
+  lb += h2f(t.nkb) * fmaf(cb, sgn[2] + sgn[3], mse[2] + mse[3]);
 }
 
 template <class G0, class G1>
@@ -259,6 +287,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_mma_kernel(MmaArgs A) {
   using G1c = typename std::conditional<TWO, G1, G0>::type;
   __shared__ float s_m[kWarps][kRep], s_l[kWarps][kRep];
   __shared__ float s_acc[kWarps][kRep][256];
+  __shared__ int s_last;
   const int split = blockIdx.x, bh = blockIdx.y;
   const int b = bh / A.Hkv, hk = bh % A.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -267,189 +296,112 @@ __global__ void __launch_bounds__(kWarps * 32) decode_mma_kernel(MmaArgs A) {
   const int t_begin = split * A.chunk;
   const int t_end = min(T, t_begin + A.chunk);
   const int64_t slot0 = (int64_t)bh * A.max_len;
+  constexpr int kStride = kWarps * 16;
 
+  // The first tile's codes are inputs of this call: fetch them before waiting for the
+  // query-preparation kernel that precedes this one on the stream.
+  TileData<G0> c0;
+  TileData<G1c> c1;
+  int ts = t_begin + warp * 16;
+  if (ts < t_end) {
+    const int64_t sa = slot0 + min(ts + g, T - 1), sb = slot0 + min(ts + g + 8, T - 1);
+    load_tile<G0>(c0, A.g[0], sa, sb, l);
+    if constexpr (TWO) load_tile<G1c>(c1, A.g[1], sa, sb, l);
+  }
+  const Lut kl0 = A.g[0].klut, vl0 = A.g[0].vlut;
+  const Lut kl1 = A.g[TWO ? 1 : 0].klut, vl1 = A.g[TWO ? 1 : 0].vlut;
+  grid_dependency_wait();
   QFrag<G0> qf0;
   load_qfrag<G0>(qf0, A, 0, b, hk, lane);
   QFrag<G1c> qf1;
   if constexpr (TWO) load_qfrag<G1c>(qf1, A, 1, b, hk, lane);
-  const Lut kl0 = make_lut(A.g[0].kc, 1 << G0::KK), vl0 = make_lut(A.g[0].vc, 1 << G0::KV);
-  Lut kl1, vl1;
-  if constexpr (TWO) {
-    kl1 = make_lut(A.g[1].kc, 1 << G1c::KK);
-    vl1 = make_lut(A.g[1].vc, 1 << G1c::KV);
-  }
+
   float acc0[G0::NKB][4];
   float acc1[G1c::NKB][4];
 #pragma unroll
   for (int i = 0; i < G0::NKB; ++i) acc0[i][0] = acc0[i][1] = acc0[i][2] = acc0[i][3] = 0.f;
 #pragma unroll
   for (int i = 0; i < G1c::NKB; ++i) acc1[i][0] = acc1[i][1] = acc1[i][2] = acc1[i][3] = 0.f;
-  // softmax state for heads h0 = 2(l&1), h0+1 (log2 domain); l_run is this thread's partial sum
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-  const bool hi_cols = l < 2;
+  // softmax state of head l (log2 domain); l_run is this lane's partial sum over its tokens
+  float m_run = -INFINITY, l_run = 0.f;
 
-  for (int ts = t_begin + warp * 16; ts < t_end; ts += kWarps * 16) {
-    const int ta = ts + g, tb = ts + g + 8;
-    const bool va = ta < t_end, vb = tb < t_end;
-    const int64_t sa = slot0 + min(ta, T - 1), sb = slot0 + min(tb, T - 1);
-    float logit_a[2] = {0.f, 0.f}, logit_b[2] = {0.f, 0.f};
-    uint32_t vw0a[G0::PV], vw0b[G0::PV];
-    uint32_t vw1a[G1c::PV], vw1b[G1c::PV];
-    float nva0, nvb0, nva1 = 0.f, nvb1 = 0.f;
-    {
-      const MmaGroup& gr = A.g[0];
-      uint32_t ka[G0::PK], kb_[G0::PK];
-      load_quarter<G0::Q, G0::PK>(gr.kcodes + sa * gr.kbytes, l, ka);
-      load_quarter<G0::Q, G0::PK>(gr.kcodes + sb * gr.kbytes, l, kb_);
-      load_quarter<G0::Q, G0::PV>(gr.vcodes + sa * gr.vbytes, l, vw0a);
-      load_quarter<G0::Q, G0::PV>(gr.vcodes + sb * gr.vbytes, l, vw0b);
-      const float nka = __half2float(__ushort_as_half(__ldg(gr.knorm + sa)));
-      const float nkb = __half2float(__ushort_as_half(__ldg(gr.knorm + sb)));
-      const float rka = __half2float(__ushort_as_half(__ldg(gr.krnorm + sa)));
-      const float rkb = __half2float(__ushort_as_half(__ldg(gr.krnorm + sb)));
-      nva0 = __half2float(__ushort_as_half(__ldg(gr.vnorm + sa)));
-      nvb0 = __half2float(__ushort_as_half(__ldg(gr.vnorm + sb)));
-      float mse[4], sgn[4];
-      group_logits<G0>(qf0, kl0, ka, kb_, mse, sgn);
-      // columns 2l, 2l+1: add the hi/lo halves held by lanes l and l^2
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        mse[i] += __shfl_xor_sync(0xffffffffu, mse[i], 2);
-        sgn[i] += __shfl_xor_sync(0xffffffffu, sgn[i], 2);
-      }
-      logit_a[0] = nka * (mse[0] + gr.coef * rka * sgn[0]);
-      logit_a[1] = nka * (mse[1] + gr.coef * rka * sgn[1]);
-      logit_b[0] = nkb * (mse[2] + gr.coef * rkb * sgn[2]);
-      logit_b[1] = nkb * (mse[3] + gr.coef * rkb * sgn[3]);
+  for (; ts < t_end; ts += kStride) {
+    // prefetch the next tile while this one is computed
+    TileData<G0> n0;
+    TileData<G1c> n1;
+    const int tn = ts + kStride;
+    if (tn < t_end) {
+      const int64_t sa = slot0 + min(tn + g, T - 1), sb = slot0 + min(tn + g + 8, T - 1);
+      load_tile<G0>(n0, A.g[0], sa, sb, l);
+      if constexpr (TWO) load_tile<G1c>(n1, A.g[1], sa, sb, l);
     }
-    if constexpr (TWO) {
-      const MmaGroup& gr = A.g[1];
-      uint32_t ka[G1c::PK], kb_[G1c::PK];
-      load_quarter<G1c::Q, G1c::PK>(gr.kcodes + sa * gr.kbytes, l, ka);
-      load_quarter<G1c::Q, G1c::PK>(gr.kcodes + sb * gr.kbytes, l, kb_);
-      load_quarter<G1c::Q, G1c::PV>(gr.vcodes + sa * gr.vbytes, l, vw1a);
-      load_quarter<G1c::Q, G1c::PV>(gr.vcodes + sb * gr.vbytes, l, vw1b);
-      const float nka = __half2float(__ushort_as_half(__ldg(gr.knorm + sa)));
-      const float nkb = __half2float(__ushort_as_half(__ldg(gr.knorm + sb)));
-      const float rka = __half2float(__ushort_as_half(__ldg(gr.krnorm + sa)));
-      const float rkb = __half2float(__ushort_as_half(__ldg(gr.krnorm + sb)));
-      nva1 = __half2float(__ushort_as_half(__ldg(gr.vnorm + sa)));
-      nvb1 = __half2float(__ushort_as_half(__ldg(gr.vnorm + sb)));
-      float mse[4], sgn[4];
-      group_logits<G1c>(qf1, kl1, ka, kb_, mse, sgn);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        mse[i] += __shfl_xor_sync(0xffffffffu, mse[i], 2);
-        sgn[i] += __shfl_xor_sync(0xffffffffu, sgn[i], 2);
-      }
-      logit_a[0] += nka * (mse[0] + gr.coef * rka * sgn[0]);
-      logit_a[1] += nka * (mse[1] + gr.coef * rka * sgn[1]);
-      logit_b[0] += nkb * (mse[2] + gr.coef * rkb * sgn[2]);
-      logit_b[1] += nkb * (mse[3] + gr.coef * rkb * sgn[3]);
-    }
-    // online softmax, log2 domain, heads h0 and h0+1 of this lane
-    float la[2], lb[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      la[h] = va ? logit_a[h] * A.scale_log2 : -INFINITY;
-      lb[h] = vb ? logit_b[h] * A.scale_log2 : -INFINITY;
-    }
-    float mt[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float v = fmaxf(la[h], lb[h]);
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-      mt[h] = v;
-    }
-    if (mt[0] > m_run[0] || mt[1] > m_run[1]) {
-      float alpha[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float mn = fmaxf(m_run[h], mt[h]);
-        alpha[h] = exp2f(m_run[h] - mn);
-        m_run[h] = mn;
-        l_run[h] *= alpha[h];
-      }
+    float la = 0.f, lb = 0.f;
+    tile_logits<G0>(c0, qf0, kl0, A.g[0], la, lb);
+    if constexpr (TWO) tile_logits<G1c>(c1, qf1, kl1, A.g[1], la, lb);
+    // online softmax (log2 domain) of head l over tokens g, g+8 of the tile
+    la = (ts + g < t_end) ? la * A.scale_log2 : -INFINITY;
+    lb = (ts + g + 8 < t_end) ? lb * A.scale_log2 : -INFINITY;
+    float mt = fmaxf(la, lb);
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+    if (mt > m_run) {
+      const float alpha = exp2f(m_run - mt);
+      m_run = mt;
+      l_run *= alpha;
 #pragma unroll
       for (int i = 0; i < G0::NKB; ++i) {
-        acc0[i][0] *= alpha[0]; acc0[i][1] *= alpha[1]; acc0[i][2] *= alpha[0]; acc0[i][3] *= alpha[1];
+        acc0[i][0] *= alpha; acc0[i][1] *= alpha; acc0[i][2] *= alpha; acc0[i][3] *= alpha;
       }
       if constexpr (TWO) {
 #pragma unroll
         for (int i = 0; i < G1c::NKB; ++i) {
-          acc1[i][0] *= alpha[0]; acc1[i][1] *= alpha[1]; acc1[i][2] *= alpha[0]; acc1[i][3] *= alpha[1];
+          acc1[i][0] *= alpha; acc1[i][1] *= alpha; acc1[i][2] *= alpha; acc1[i][3] *= alpha;
         }
       }
     }
-    float pa[2], pb[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      pa[h] = exp2f(la[h] - m_run[h]);
-      pb[h] = exp2f(lb[h] - m_run[h]);
-      l_run[h] += pa[h] + pb[h];
-    }
-    // probability operand [P_hi | P_lo], weighted by each group's value norm
+    const float pa = exp2f(la - m_run), pb = exp2f(lb - m_run);
+    l_run += pa + pb;
+    // probability operand: columns 2l, 2l+1 = hi and lo halves of p * ||v|| for head l
     auto pfrag = [&](float na, float nb, uint32_t& b0, uint32_t& b1) {
-      float wa0 = pa[0] * na, wa1 = pa[1] * na, wb0 = pb[0] * nb, wb1 = pb[1] * nb;
-      if (!hi_cols) {
-        wa0 -= __half2float(__float2half_rn(wa0));
-        wa1 -= __half2float(__float2half_rn(wa1));
-        wb0 -= __half2float(__float2half_rn(wb0));
-        wb1 -= __half2float(__float2half_rn(wb1));
-      }
-      b0 = movT(pack_h2(wa0, wa1));
-      b1 = movT(pack_h2(wb0, wb1));
+      const float wa = pa * na, wb = pb * nb;
+      const float ha = __half2float(__float2half_rn(wa)), hb = __half2float(__float2half_rn(wb));
+      b0 = movT(pack_h2(ha, wa - ha));
+      b1 = movT(pack_h2(hb, wb - hb));
     };
     uint32_t pb0, pb1;
-    pfrag(nva0, nvb0, pb0, pb1);
-    group_values<G0>(vl0, vw0a, vw0b, pb0, pb1, acc0);
+    pfrag(h2f(c0.nva), h2f(c0.nvb), pb0, pb1);
+    group_values<G0>(vl0, c0.va, c0.vb, pb0, pb1, acc0);
     if constexpr (TWO) {
-      pfrag(nva1, nvb1, pb0, pb1);
-      group_values<G1c>(vl1, vw1a, vw1b, pb0, pb1, acc1);
+      pfrag(h2f(c1.nva), h2f(c1.nvb), pb0, pb1);
+      group_values<G1c>(vl1, c1.va, c1.vb, pb0, pb1, acc1);
     }
+    c0 = n0;
+    if constexpr (TWO) c1 = n1;
   }
 
-  // ---- warp state -> shared memory
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    float v = l_run[h];
-    v += __shfl_xor_sync(0xffffffffu, v, 4);
-    v += __shfl_xor_sync(0xffffffffu, v, 8);
-    v += __shfl_xor_sync(0xffffffffu, v, 16);
-    l_run[h] = v;
-  }
-  const int h0 = 2 * (l & 1);
-  if (g == 0 && l < 2) {
-    s_m[warp][h0] = m_run[0];
-    s_m[warp][h0 + 1] = m_run[1];
-    s_l[warp][h0] = l_run[0];
-    s_l[warp][h0 + 1] = l_run[1];
+  // ---- warp state -> shared memory (lane (g, l) holds head l)
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 4);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 8);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
+  if (g == 0) {
+    s_m[warp][l] = m_run;
+    s_l[warp][l] = l_run;
   }
   auto store_acc = [&](auto& acc, auto gc_tag, int off) {
     using GC = decltype(gc_tag);
 #pragma unroll
     for (int mb = 0; mb < GC::NKB; ++mb) {
-      float v0 = acc[mb][0] + __shfl_xor_sync(0xffffffffu, acc[mb][0], 2);
-      float v1 = acc[mb][1] + __shfl_xor_sync(0xffffffffu, acc[mb][1], 2);
-      float v2 = acc[mb][2] + __shfl_xor_sync(0xffffffffu, acc[mb][2], 2);
-      float v3 = acc[mb][3] + __shfl_xor_sync(0xffffffffu, acc[mb][3], 2);
-      if (l < 2) {
-        const int qq = mb & 3, hh = mb >> 2;
-        const int c0 = GC::Q * (g >> 1) + qq + 16 * hh + 4 * (g & 1);   // row g: block f = 0
-        const int c1 = c0 + 8;                                           // row g+8: block f = 1
-        s_acc[warp][h0][off + c0] = v0;
-        s_acc[warp][h0 + 1][off + c0] = v1;
-        s_acc[warp][h0][off + c1] = v2;
-        s_acc[warp][h0 + 1][off + c1] = v3;
-      }
+      const int qq = mb & 3, hh = mb >> 2;
+      const int c0_ = GC::Q * (g >> 1) + qq + 16 * hh + 4 * (g & 1);   // row g: block f = 0
+      s_acc[warp][l][off + c0_] = acc[mb][0] + acc[mb][1];
+      s_acc[warp][l][off + c0_ + 8] = acc[mb][2] + acc[mb][3];          // row g+8: block f = 1
     }
   };
   store_acc(acc0, G0{}, A.g[0].off);
   if constexpr (TWO) store_acc(acc1, G1c{}, A.g[1].off);
   __syncthreads();
-  // ---- merge the warps; one partial per (query head, split), m in natural-log units
+  // ---- merge the warps: one partial per (query head, split); m in natural-log units
   const float ln2 = 0.69314718055994531f;
   for (int e = threadIdx.x; e < kRep * A.D; e += blockDim.x) {
     const int h = e / A.D, c = e % A.D;
@@ -470,17 +422,142 @@ __global__ void __launch_bounds__(kWarps * 32) decode_mma_kernel(MmaArgs A) {
     }
     dst[2 + c] = acc;
   }
+  // ---- the last split of this (sequence, kv head) to finish merges all splits
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(A.done + bh, 1) == A.nsplit - 1) ? 1 : 0;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  float* wts = &s_acc[0][0][0];                  // reuse: [kRep][nsplit] weights (nsplit <= 512)
+  float* rot = &s_acc[2][0][0];                  // [kRep][D] merged rotated-basis accumulators
+  for (int h = warp; h < kRep; h += kWarps) {
+    const float* P = A.part + (size_t)(b * A.Hq + hk * kRep + h) * A.nsplit * (A.D + 2);
+    float M = -INFINITY;
+    for (int s = lane; s < A.nsplit; s += 32) M = fmaxf(M, __ldcg(P + (size_t)s * (A.D + 2)));
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    for (int s = lane; s < A.nsplit; s += 32) {
+      const float ms = __ldcg(P + (size_t)s * (A.D + 2));
+      const float w = (ms == -INFINITY) ? 0.f : __expf(ms - M);
+      wts[h * 512 + s] = w;
+      L += w * __ldcg(P + (size_t)s * (A.D + 2) + 1);
+    }
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    __syncwarp();
+    for (int s = lane; s < A.nsplit; s += 32) wts[h * 512 + s] *= inv;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < kRep * A.D; e += blockDim.x) {
+    const int h = e / A.D, c = e % A.D;
+    const float* P = A.part + (size_t)(b * A.Hq + hk * kRep + h) * A.nsplit * (A.D + 2) + 2 + c;
+    float a0 = 0.f, a1 = 0.f;
+    int s = 0;
+    for (; s + 1 < A.nsplit; s += 2) {
+      a0 = fmaf(wts[h * 512 + s], __ldcg(P + (size_t)s * (A.D + 2)), a0);
+      a1 = fmaf(wts[h * 512 + s + 1], __ldcg(P + (size_t)(s + 1) * (A.D + 2)), a1);
+    }
+    if (s < A.nsplit) a0 = fmaf(wts[h * 512 + s], __ldcg(P + (size_t)s * (A.D + 2)), a0);
+    rot[h * 256 + c] = a0 + a1;
+  }
+  __syncthreads();
+  // o = Pi_v^T acc per group: o[off+j] = sum_i Pi_v[i][j] acc[off+i]
+  for (int c = threadIdx.x; c < A.D; c += blockDim.x) {
+    const int gi = (A.G > 1 && c >= A.g[1].off) ? 1 : 0;
+    const MmaGroup& gr = A.g[gi];
+    const int dg = (gi == 0) ? (A.G > 1 ? A.g[1].off : A.D) : A.D - gr.off;
+    const int j = c - gr.off;
+    float o[kRep] = {0.f, 0.f, 0.f, 0.f};
+    const float* Pi = gr.PiV + j;
+#pragma unroll 8
+    for (int i = 0; i < dg; ++i) {
+      const float p = __ldg(Pi + (size_t)i * dg);
+#pragma unroll
+      for (int h = 0; h < kRep; ++h) o[h] = fmaf(p, rot[h * 256 + gr.off + i], o[h]);
+    }
+#pragma unroll
+    for (int h = 0; h < kRep; ++h) A.out[(size_t)(b * A.Hq + hk * kRep + h) * A.D + c] = o[h];
+  }
+}
+
+// (Pi q, S q) for a 32-row x 32-output tile of the prepared-query matrix per CTA (the
+// rows are the B*Hq query rows, the outputs the 2*d_g coordinates of Pi q and S q);
+// CTA (0, 0) of group 0 also clears the completion counters.
+template <typename T>
+__global__ void __launch_bounds__(256) decode_prep_kernel(const T* __restrict__ q, int rows, int D, int off, int dg,
+                                                          const float* __restrict__ PiT, const float* __restrict__ ST,
+                                                          float* __restrict__ qprep, int G, int gi, int qp_ld,
+                                                          int* __restrict__ done, int ndone) {
+  __shared__ float qs[32][129];
+  __shared__ float ms[128][33];
+  allow_dependent_launch();
+  const int o0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && gi == 0)
+    for (int i = threadIdx.x; i < ndone; i += blockDim.x) done[i] = 0;
+  for (int e = threadIdx.x; e < 32 * dg; e += blockDim.x) {
+    const int r = e / dg, j = e % dg;
+    float v = 0.f;
+    if (r0 + r < rows) {
+      if constexpr (std::is_same<T, float>::value) v = q[(size_t)(r0 + r) * D + off + j];
+      else v = __bfloat162float(q[(size_t)(r0 + r) * D + off + j]);
+    }
+    qs[r][j] = v;
+  }
+  for (int e = threadIdx.x; e < 32 * dg; e += blockDim.x) {
+    const int j = e / 32, c = e % 32, o = o0 + c;
+    float v = 0.f;
+    if (o < dg) v = __ldg(PiT + (size_t)j * dg + o);
+    else if (o < 2 * dg) v = __ldg(ST + (size_t)j * dg + (o - dg));
+    ms[j][c] = v;
+  }
+  __syncthreads();
+  const int r = threadIdx.x >> 3, c0 = (threadIdx.x & 7) * 4;
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int j = 0; j < dg; ++j) {
+    const float x = qs[r][j];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = fmaf(ms[j][c0 + i], x, a[i]);
+  }
+  if (r0 + r < rows)
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (o0 + c0 + i < 2 * dg) qprep[((size_t)(r0 + r) * G + gi) * 2 * qp_ld + o0 + c0 + i] = a[i];
 }
 
 template <class G0, class G1>
 int launch_mma_t(const MmaArgs& A, int nsplit, int BHkv, cudaStream_t st) {
-  dim3 grid(nsplit, BHkv);
-  decode_mma_kernel<G0, G1><<<grid, kWarps * 32, 0, st>>>(A);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nsplit, BHkv);
+  cfg.blockDim = dim3(kWarps * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_mma_kernel<G0, G1>, A);
   count_launch();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(decode_mma_kernel)");
   return check_launch("decode_mma_kernel");
 }
 
 }  // namespace
+
+Lut host_lut(const Codebook& cb) {
+  Lut t{};
+  for (int j = 0; j < 16; ++j) {
+    uint16_t b = 0;
+    if (j < cb.K) {
+      __half h = __float2half_rn(cb.c[j]);
+      b = *reinterpret_cast<uint16_t*>(&h);
+    }
+    t.lo[j / 4] |= (uint32_t)(b & 0xFF) << (8 * (j % 4));
+    t.hi[j / 4] |= (uint32_t)(b >> 8) << (8 * (j % 4));
+  }
+  return t;
+}
 
 // Returns kNotHandled when the shape is outside this kernel's instantiations.
 int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G, const void* q,
@@ -503,41 +580,46 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
   const bool ok = (G == 1 && (sig[0] == 12834 || sig[0] == 12823)) || is(6434, 6423) || is(6423, 6412);
   if (!ok) return kNotHandled;
 
-  int qp_ld = 0;
-  for (int g = 0; g < G; ++g) qp_ld = std::max(qp_ld, kctx[g]->lay.d);
-  int nsplit, chunk;
-  decode_geometry(B, Hkv, max_len, &nsplit, &chunk);
-  float* qprep = static_cast<float*>(ws);
-  size_t qp_bytes = (size_t)B * Hq * G * 2 * qp_ld * sizeof(float);
-  float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + ((qp_bytes + 255) / 256) * 256);
+  const DecodeWs W = decode_ws(B, Hq, Hkv, D, G, max_len);
+  if (W.nsplit > 512) return kNotHandled;
+  char* base = static_cast<char*>(ws);
+  float* qprep = reinterpret_cast<float*>(base + W.qp);
+  float* part = reinterpret_cast<float*>(base + W.part);
+  int* done = reinterpret_cast<int*>(base + W.cnt);
   for (int g = 0; g < G; ++g) {
-    int esz = q_dtype == TQ_DTYPE_F32 ? 4 : 2;
-    const char* qg = static_cast<const char*>(q) + (size_t)off[g] * esz;
-    int r = launch_prepare_queries(kctx[g], qg, q_dtype, (int64_t)B * Hq, D, qprep + (size_t)g * 2 * qp_ld,
-                                   (int64_t)G * 2 * qp_ld, st);
+    const int dg = kctx[g]->lay.d;
+    const dim3 pgrid(div_up(2 * dg, 32), div_up(B * Hq, 32));
+    if (q_dtype == TQ_DTYPE_F32)
+      decode_prep_kernel<float><<<pgrid, 256, 0, st>>>(static_cast<const float*>(q), B * Hq, D, off[g], dg,
+                                                       kctx[g]->PiT, kctx[g]->ST, qprep, G, g, D, done, B * Hkv);
+    else
+      decode_prep_kernel<__nv_bfloat16><<<pgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), B * Hq, D, off[g],
+                                                               dg, kctx[g]->PiT, kctx[g]->ST, qprep, G, g, D, done,
+                                                               B * Hkv);
+    count_launch();
+    int r = check_launch("decode_prep_kernel");
     if (r != TQ_OK) return r;
   }
   MmaArgs A{};
-  A.B = B; A.Hq = Hq; A.Hkv = Hkv; A.D = D; A.nsplit = nsplit; A.chunk = chunk; A.qp_ld = qp_ld; A.G = G;
+  A.B = B; A.Hq = Hq; A.Hkv = Hkv; A.D = D; A.nsplit = W.nsplit; A.chunk = W.chunk; A.qp_ld = D; A.G = G;
   A.max_len = max_len; A.scale_log2 = scale * 1.4426950408889634f; A.seq_lens = seq_lens; A.qprep = qprep;
-  A.part = part;
+  A.part = part; A.done = done; A.out = out;
   for (int g = 0; g < G; ++g) {
     MmaGroup& gr = A.g[g];
     gr.kcodes = kc[g].codes; gr.knorm = kc[g].norm; gr.krnorm = kc[g].rnorm;
     gr.vcodes = vc[g].codes; gr.vnorm = vc[g].norm;
-    for (int j = 0; j < 16; ++j) { gr.kc[j] = kctx[g]->cb.c[j]; gr.vc[j] = vctx[g]->cb.c[j]; }
+    gr.PiV = vctx[g]->Pi;
+    gr.klut = host_lut(kctx[g]->cb);
+    gr.vlut = host_lut(vctx[g]->cb);
     gr.coef = kctx[g]->sqrt_pi_over_2_over_m;
     gr.off = off[g];
     gr.kbytes = kctx[g]->lay.code_bytes;
     gr.vbytes = vctx[g]->lay.code_bytes;
   }
-  int r;
-  if (G == 1 && sig[0] == 12834) r = launch_mma_t<C128_34, void>(A, nsplit, B * Hkv, st);
-  else if (G == 1) r = launch_mma_t<C128_23, void>(A, nsplit, B * Hkv, st);
-  else if (is(6434, 6423)) r = launch_mma_t<C64_34, C64_23>(A, nsplit, B * Hkv, st);
-  else r = launch_mma_t<C64_23, C64_12>(A, nsplit, B * Hkv, st);
-  if (r != TQ_OK) return r;
-  return launch_decode_merge(vctx, off, G, part, nsplit, B * Hq, D, out, st);
+  if (G == 1 && sig[0] == 12834) return launch_mma_t<C128_34, void>(A, W.nsplit, B * Hkv, st);
+  if (G == 1) return launch_mma_t<C128_23, void>(A, W.nsplit, B * Hkv, st);
+  if (is(6434, 6423)) return launch_mma_t<C64_34, C64_23>(A, W.nsplit, B * Hkv, st);
+  return launch_mma_t<C64_23, C64_12>(A, W.nsplit, B * Hkv, st);
 }
 
 }  // namespace tq

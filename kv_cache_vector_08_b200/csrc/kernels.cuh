@@ -17,6 +17,11 @@ int launch_prepare_queries(const tq_ctx* ctx, const void* q, int q_dtype, int64_
 int launch_logits_simt(const tq_ctx* ctx, const float* qprep, int64_t nq, const tq_packed* keys, int64_t n,
                        float* logits, cudaStream_t st);
 void decode_geometry(int B, int Hkv, int64_t max_len, int* nsplit, int* chunk);
+struct DecodeWs {
+  size_t qp, part, cnt, total;  // byte offsets of the regions and total size
+  int nsplit, chunk;
+};
+DecodeWs decode_ws(int B, int Hq, int Hkv, int D, int G, int64_t max_len);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int ngroups, int64_t max_len, int qp_ld);
 int launch_decode_simt(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G, const void* q,
                        int q_dtype, const tq_packed* kc, const tq_packed* vc, const int32_t* seq_lens, int B, int Hq,

@@ -731,24 +731,37 @@ int launch_logits_simt(const tq_ctx* ctx, const float* qprep, int64_t nq, const 
   return check_launch("logits_simt_kernel");
 }
 
-// split-K geometry shared by the size query and the launch
+// split-K geometry shared by the size query and every decode launch: the context is cut
+// into chunks of whole 64-token tiles so that about 3 CTAs per SM are in flight.
 void decode_geometry(int B, int Hkv, int64_t max_len, int* nsplit, int* chunk) {
-  int64_t tiles = (max_len + kDecTile - 1) / kDecTile;
+  constexpr int64_t kTile = 64;
+  int64_t tiles = (max_len + kTile - 1) / kTile;
   if (tiles < 1) tiles = 1;
-  int64_t want = (2 * 148 + (int64_t)B * Hkv - 1) / ((int64_t)B * Hkv);  // ~2 CTAs per SM
+  int64_t bh = (int64_t)B * Hkv;
+  int64_t want = (3 * 148 + bh - 1) / bh;   // one wave at 3 CTAs per SM
   if (want < 1) want = 1;
+  if (want > 512) want = 512;
   if (want > tiles) want = tiles;
   int64_t tiles_per = (tiles + want - 1) / want;
-  *chunk = (int)(tiles_per * kDecTile);
+  *chunk = (int)(tiles_per * kTile);
   *nsplit = (int)((tiles + tiles_per - 1) / tiles_per);
 }
 
-size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int ngroups, int64_t max_len, int qp_ld) {
-  int nsplit, chunk;
-  decode_geometry(B, Hkv, max_len, &nsplit, &chunk);
-  size_t qp = (size_t)B * Hq * ngroups * 2 * qp_ld * sizeof(float);
-  size_t part = (size_t)B * Hq * nsplit * (D + 2) * sizeof(float);
-  return ((qp + 255) / 256) * 256 + part;
+// Workspace: prepared queries [B*Hq][G][2*D], split partials [B*Hq][nsplit][D+2],
+// completion counters [B*Hkv] (each region 256-byte aligned).
+DecodeWs decode_ws(int B, int Hq, int Hkv, int D, int G, int64_t max_len) {
+  DecodeWs w{};
+  decode_geometry(B, Hkv, max_len, &w.nsplit, &w.chunk);
+  auto up = [](size_t x) { return ((x + 255) / 256) * 256; };
+  w.qp = 0;
+  w.part = up((size_t)B * Hq * G * 2 * D * sizeof(float));
+  w.cnt = w.part + up((size_t)B * Hq * w.nsplit * (D + 2) * sizeof(float));
+  w.total = w.cnt + up((size_t)B * Hkv * sizeof(int));
+  return w;
+}
+
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int ngroups, int64_t max_len, int) {
+  return decode_ws(B, Hq, Hkv, D, ngroups, max_len).total;
 }
 
 int launch_decode_simt(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G, const void* q,
@@ -758,13 +771,11 @@ int launch_decode_simt(const tq_ctx* const* kctx, const tq_ctx* const* vctx, con
   const int rep = Hq / Hkv;
   if (rep > kMaxRep) return fail(TQ_ERR_UNSUPPORTED, "at most 8 query heads per kv head");
   if (D > 2 * kDecTile) return fail(TQ_ERR_UNSUPPORTED, "head dimension above 256");
-  int qp_ld = 0;
-  for (int g = 0; g < G; ++g) qp_ld = std::max(qp_ld, kctx[g]->lay.d);
-  int nsplit, chunk;
-  decode_geometry(B, Hkv, max_len, &nsplit, &chunk);
-  float* qprep = static_cast<float*>(ws);
-  size_t qp_bytes = (size_t)B * Hq * G * 2 * qp_ld * sizeof(float);
-  float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + ((qp_bytes + 255) / 256) * 256);
+  const int qp_ld = D;
+  const DecodeWs W = decode_ws(B, Hq, Hkv, D, G, max_len);
+  const int nsplit = W.nsplit, chunk = W.chunk;
+  float* qprep = reinterpret_cast<float*>(static_cast<char*>(ws) + W.qp);
+  float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + W.part);
   // query preparation per group: rows (b, h) of q restricted to the group's channels
   for (int g = 0; g < G; ++g) {
     int esz = q_dtype == TQ_DTYPE_F32 ? 4 : 2;
