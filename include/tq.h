@@ -126,6 +126,12 @@ int tq_host_params(int d, int bits, uint64_t seed, int mode, double* Pi, double*
  * still queued on any stream. */
 void tq_free(tq_ctx* ctx);
 
+/* Kernel-side failure report: a tensor-core kernel whose pipeline wait exceeds its time
+ * limit (2 s) records a non-zero code in the context's device error word, stops its work
+ * and exits cleanly instead of hanging.  This call synchronises the device, copies the
+ * word to *code (0 = no failure) and clears it. */
+int tq_get_device_error(const tq_ctx* ctx, int* code);
+
 /* Fill *info (host pointer). */
 int tq_get_info(const tq_ctx* ctx, tq_info* info);
 

@@ -77,6 +77,7 @@ def lib():
         "tq_search_topk": (I, [P, P, I64, PK, I64, I, P, P, P, SZ, P]),
         "tq_last_error": (ctypes.c_char_p, []),
         "tq_kernel_launch_count": (U64, []),
+        "tq_get_device_error": (I, [P, ctypes.POINTER(I)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -163,6 +164,12 @@ class Context:
         p = lambda a: None if a is None else a.ctypes.data_as(ctypes.c_void_p)
         _check(lib().tq_get_params(self._h, p(Pi), p(S), p(c), p(t)))
         return dict(Pi=Pi, S=S, centroids=c, boundaries=t[:K - 1], mode=self.mode, k=self.k, m=self.m, d=d)
+
+    def device_error(self) -> int:
+        """Kernel-side failure code recorded for this context (0 = none); clears it."""
+        v = ctypes.c_int(0)
+        _check(lib().tq_get_device_error(self._h, ctypes.byref(v)))
+        return v.value
 
     def close(self):
         if getattr(self, "_h", None) is not None and self._h.value:

@@ -52,6 +52,11 @@ struct tq_ctx {
   float* S = nullptr;     // [m][d]
   float* ST = nullptr;    // [d][m]
   float* MT = nullptr;    // [d][m]    (S Pi^T)^T
+  // tensor-core operands (d in {64, 128}): Pi as three bf16 splits [3][d][d] and
+  // 16 * M as two fp16 splits [2][d][d], row-major
+  void* Pi_split = nullptr;
+  void* M_split = nullptr;
+  int* dev_err = nullptr;  // device error word written by kernels that detect a stuck pipeline
 };
 
 namespace tq {

@@ -2,10 +2,27 @@
 #include "common.cuh"
 #include "kernels.cuh"
 
+#include <cstdlib>
+
 namespace tq {
+
+// TQ_FORCE_SIMT=1 routes every call to the CUDA-core kernels (used to cross-check the
+// tensor-core kernels against the CUDA-core rung on the same inputs).
+bool force_simt() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("TQ_FORCE_SIMT");
+    v = (e && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
 
 int launch_quantize(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld, const tq_packed* dst,
                     const int64_t* slots, cudaStream_t st) {
+  if (!force_simt()) {
+    int r = launch_quantize_tc(ctx, x, x_dtype, n, ld, dst, slots, st);
+    if (r != kNotHandled) return r;
+  }
   return launch_quantize_simt(ctx, x, x_dtype, n, ld, dst, slots, st);
 }
 
@@ -17,9 +34,11 @@ int launch_logits(const tq_ctx* ctx, const float* qprep, int64_t nq, const tq_pa
 int launch_decode(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G, const void* q,
                   int q_dtype, const tq_packed* kc, const tq_packed* vc, const int32_t* seq_lens, int B, int Hq,
                   int Hkv, int D, int64_t max_len, float scale, float* out, void* ws, cudaStream_t st) {
-  int r = launch_decode_mma(kctx, vctx, off, G, q, q_dtype, kc, vc, seq_lens, B, Hq, Hkv, D, max_len, scale, out, ws,
-                            st);
-  if (r != kNotHandled) return r;
+  if (!force_simt()) {
+    int r = launch_decode_mma(kctx, vctx, off, G, q, q_dtype, kc, vc, seq_lens, B, Hq, Hkv, D, max_len, scale, out,
+                              ws, st);
+    if (r != kNotHandled) return r;
+  }
   return launch_decode_simt(kctx, vctx, off, G, q, q_dtype, kc, vc, seq_lens, B, Hq, Hkv, D, max_len, scale, out, ws,
                             st);
 }

@@ -26,6 +26,8 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int ngroups, int64_
 int launch_decode_simt(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G, const void* q,
                        int q_dtype, const tq_packed* kc, const tq_packed* vc, const int32_t* seq_lens, int B, int Hq,
                        int Hkv, int D, int64_t max_len, float scale, float* out, void* ws, cudaStream_t st);
+int launch_quantize_tc(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld, const tq_packed* dst,
+                       const int64_t* slots, cudaStream_t st);
 int launch_decode_merge(const tq_ctx* const* vctx, const int* off, int G, const float* part, int nsplit, int BHq,
                         int D, float* out, cudaStream_t st);
 int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G, const void* q,

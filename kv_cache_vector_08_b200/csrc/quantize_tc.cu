@@ -1,0 +1,420 @@
+// Quantize on the 5th-generation tensor cores (tcgen05 + TMEM, operands staged by TMA).
+//
+// turboquant.net "Quant / DeQuant 函数": y = Pi x, nearest Lloyd-Max centroid per rotated
+// coordinate; admirer.cn QJL paragraph: signs of the projected residual.  For a tile of
+// 128 vectors the two projections are dense contractions:
+//
+//   D_y [128 x d] = X [128 x d] * Pi^T            x bf16 (exact), Pi = Pi_hi + Pi_mid + Pi_lo (bf16)
+//   D_z [128 x d] = R [128 x d] * M^T             R = r * 2^8 (fp16 hi + lo), M * 2^4 (fp16 hi + lo)
+//
+// Pi x is fp32-accurate (three bf16 splits of Pi against the exact bf16 input), so the
+// norm comes for free as ||Pi x|| = ||x||.  The residual r = y - c[idx] lives in the
+// rotated basis, and S r = (S Pi^T) y-residual = M r, so the QJL projection is a second
+// GEMM with A taken straight from tensor memory (hi*hi + hi*lo + lo*hi products).
+//
+// Roles (192 threads): warp 0 issues TMA loads (constants once, then one x tile per
+// stage), warp 1 allocates TMEM and issues the MMAs, warps 2-5 are the epilogue
+// (thread = one vector = one TMEM lane).  Every mbarrier wait is bounded; a timeout sets
+// the context's error word and the CTA winds down (TMEM is always released).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace tq {
+namespace {
+
+using namespace sm100;
+
+constexpr int kTileM = 128;
+constexpr uint64_t kWaitNs = 2000000000ull;   // a pipeline wait longer than 2 s is declared stuck
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColY = 0, kColR = 128, kColZ = 256;
+constexpr float kRScale = 256.f;   // the residual enters the QJL GEMM as r * 2^8 (M as 16 * M)
+
+struct QtArgs {
+  int64_t n;
+  const int64_t* slots;
+  uint8_t* codes;
+  uint16_t* norm;
+  uint16_t* rnorm;
+  int* err;
+  float c[16], t[16];
+};
+
+// Shared-memory plan (all operand regions 1024-byte aligned).
+template <int D, bool PROD, int NST>
+struct Smem {
+  static constexpr int KA = D / 64;                       // 128-byte K atoms per row
+  static constexpr int PI_SPLIT = D * D * 2;              // bytes of one bf16 split of Pi
+  static constexpr int M_SPLIT = D * D * 2;
+  static constexpr int X_TILE = kTileM * D * 2;
+  static constexpr int OFF_PI = 0;
+  static constexpr int OFF_M = OFF_PI + 3 * PI_SPLIT;
+  static constexpr int OFF_X = OFF_M + (PROD ? 2 * M_SPLIT : 0);
+  static constexpr int OFF_BAR = OFF_X + NST * X_TILE;
+  static constexpr int BYTES = OFF_BAR + 256 + 1024;      // barriers + alignment slack
+};
+
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int D, bool PROD, int K>
+__global__ void __launch_bounds__(192, 1) quantize_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
+                                                             const __grid_constant__ CUtensorMap tm_pi,
+                                                             const __grid_constant__ CUtensorMap tm_m, QtArgs A) {
+  constexpr int NST = PROD ? 2 : 3;
+  using SM = Smem<D, PROD, NST>;
+  constexpr int KA = SM::KA;
+  constexpr int NK = D / 16;             // k-steps per product
+  constexpr int LEVELS = 1 << K;
+  constexpr int P = K + (PROD ? 1 : 0);  // bit planes
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::OFF_BAR);
+  uint64_t* full_x = bars;               // [NST] TMA -> MMA
+  uint64_t* empty_x = bars + NST;        // [NST] MMA -> TMA
+  uint64_t* const_full = bars + 2 * NST; // constants loaded
+  uint64_t* y_full = const_full + 1;     // MMA -> epilogue
+  uint64_t* y_empty = y_full + 1;        // epilogue -> MMA
+  uint64_t* r_full = y_empty + 1;        // epilogue -> MMA (residual written to TMEM)
+  uint64_t* z_full = r_full + 1;         // MMA -> epilogue
+  uint64_t* z_empty = z_full + 1;        // epilogue -> MMA
+  uint64_t* drain = z_empty + 1;          // MMA issuer: all issued MMAs complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ntiles = (A.n + kTileM - 1) / kTileM;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(full_x + s, 1);
+      mbar_init(empty_x + s, 1);
+    }
+    mbar_init(const_full, 1);
+    mbar_init(y_full, 1);
+    mbar_init(y_empty, 128);
+    mbar_init(r_full, 128);
+    mbar_init(z_full, 1);
+    mbar_init(z_empty, 128);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const volatile int* abort_v = abort_flag;
+  auto fail = [&](int code) {
+    atomicExch(abort_flag, 1);
+    if (A.err) atomicCAS(A.err, 0, code);
+  };
+  auto wait = [&](uint64_t* bar, uint32_t parity) { return mbar_wait(bar, parity, abort_v, kWaitNs); };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tm_x);
+      mbar_arrive_expect_tx(const_full, 3 * SM::PI_SPLIT + (PROD ? 2 * SM::M_SPLIT : 0));
+      for (int s = 0; s < 3; ++s)
+        for (int a = 0; a < KA; ++a)
+          tma_load_2d(smem + SM::OFF_PI + s * SM::PI_SPLIT + a * D * 128, &tm_pi, 64 * a, s * D, const_full);
+      if (PROD)
+        for (int s = 0; s < 2; ++s)
+          for (int a = 0; a < KA; ++a)
+            tma_load_2d(smem + SM::OFF_M + s * SM::M_SPLIT + a * D * 128, &tm_m, 64 * a, s * D, const_full);
+      int it = 0;
+      int pending[NST];                  // parity of the last load issued into each stage, -1: none
+      for (int s = 0; s < NST; ++s) pending[s] = -1;
+      for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+        const int s = it % NST;
+        const uint32_t ph = (it / NST) & 1;
+        if (!wait(empty_x + s, ph ^ 1)) { fail(101); break; }
+        mbar_arrive_expect_tx(full_x + s, SM::X_TILE);
+        for (int a = 0; a < KA; ++a)
+          tma_load_2d(smem + SM::OFF_X + s * SM::X_TILE + a * kTileM * 128, &tm_x, 64 * a, (int)(tile * kTileM),
+                      full_x + s);
+        pending[s] = (int)ph;
+      }
+      // copies still in flight land before the CTA releases its shared memory
+      mbar_wait(const_full, 0, nullptr, kWaitNs);
+      for (int s = 0; s < NST; ++s)
+        if (pending[s] >= 0) mbar_wait(full_x + s, (uint32_t)pending[s], nullptr, kWaitNs);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idy = idesc_f16(kTileM, D, 1), idz = idesc_f16(kTileM, D, 0);
+      const uint32_t pi_addr = smem_u32(smem + SM::OFF_PI), m_addr = smem_u32(smem + SM::OFF_M);
+      bool ok = wait(const_full, 0);
+      if (!ok) fail(102);
+      int it = 0;
+      for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
+        const int s = it % NST;
+        const uint32_t ph = (it / NST) & 1, pt = it & 1;
+        if (!wait(full_x + s, ph) || !wait(y_empty, pt ^ 1)) { fail(103); break; }
+        tc_fence_after();
+        const uint32_t x_addr = smem_u32(smem + SM::OFF_X + s * SM::X_TILE);
+        for (int sp = 0; sp < 3; ++sp)
+          for (int ks = 0; ks < NK; ++ks) {
+            const int a = ks >> 2, kk = ks & 3;
+            const uint64_t da = desc_sw128(x_addr + a * kTileM * 128 + kk * 32);
+            const uint64_t db = desc_sw128(pi_addr + sp * SM::PI_SPLIT + a * D * 128 + kk * 32);
+            mma_ss(tmem + kColY, da, db, idy, (sp | ks) ? 1u : 0u);
+          }
+        mma_commit(empty_x + s);
+        mma_commit(y_full);
+        if (PROD) {
+          if (!wait(r_full, pt) || !wait(z_empty, pt ^ 1)) { fail(104); break; }
+          tc_fence_after();
+          // z = R_hi M_hi + R_hi M_lo + R_lo M_hi   (A from TMEM: 2 fp16 per column)
+          for (int sp = 0; sp < 3; ++sp) {
+            const uint32_t a_col = kColR + (sp == 2 ? D / 2 : 0);
+            const int msp = (sp == 1) ? 1 : 0;
+            for (int ks = 0; ks < NK; ++ks) {
+              const int a = ks >> 2, kk = ks & 3;
+              const uint64_t db = desc_sw128(m_addr + msp * SM::M_SPLIT + a * D * 128 + kk * 32);
+              mma_ts(tmem + kColZ, tmem + a_col + ks * 8, db, idz, (sp | ks) ? 1u : 0u);
+            }
+          }
+          mma_commit(z_full);
+        }
+      }
+      // every MMA issued above completes before TMEM is released
+      mma_commit(drain);
+      mbar_wait(drain, 0, nullptr, kWaitNs);
+    }
+  } else {
+    // ------------------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;                       // TMEM lanes 32*quarter .. +31
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    int it = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+      const uint32_t pt = it & 1;
+      if (!wait(y_full, pt)) { fail(105); break; }
+      tc_fence_after();
+      // pass 1: ||x||^2 = ||Pi x||^2 from the accumulator row
+      float n2 = 0.f;
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + kColY + c, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) n2 = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), n2);
+      }
+      const float nrm = sqrtf(n2);
+      const float inv = nrm > 0.f ? 1.f / nrm : 0.f;
+      uint32_t planes[P][D / 32];
+#pragma unroll
+      for (int p = 0; p < P; ++p)
+#pragma unroll
+        for (int w = 0; w < D / 32; ++w) planes[p][w] = 0u;
+      float rn2 = 0.f;
+      // pass 2: y = Pi x / ||x||, nearest centroid, residual (scaled, split into fp16 hi / lo)
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + kColY + c, r);
+        tmem_ld_wait();
+        float rs[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float yy = __uint_as_float(r[i]) * inv;
+          int idx = 0;
+#pragma unroll
+          for (int j = 0; j < LEVELS - 1; ++j) idx += (yy > A.t[j]) ? 1 : 0;
+          float cv = A.c[0];
+#pragma unroll
+          for (int j = 1; j < LEVELS; ++j) cv = (idx == j) ? A.c[j] : cv;
+          const float rr = yy - cv;
+          rn2 = fmaf(rr, rr, rn2);
+          rs[i] = rr * kRScale;
+#pragma unroll
+          for (int p = 0; p < K; ++p) planes[p][c / 32] |= (uint32_t)((idx >> p) & 1) << i;
+        }
+        if (PROD) {
+          uint32_t hi[16], lo[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a0 = rs[2 * i], a1 = rs[2 * i + 1];
+            const float h0 = __half2float(__float2half_rn(a0)), h1 = __half2float(__float2half_rn(a1));
+            hi[i] = pack_h2(h0, h1);
+            lo[i] = pack_h2(a0 - h0, a1 - h1);
+          }
+          tmem_st16(lane_base + kColR + c / 2, hi);
+          tmem_st16(lane_base + kColR + D / 2 + c / 2, lo);
+        }
+      }
+      if (PROD) tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(y_empty);                            // D_y may be overwritten now
+      const int64_t v = tile * kTileM + row;
+      if (PROD) {
+        mbar_arrive(r_full);
+        if (!wait(z_full, pt)) { fail(106); break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(lane_base + kColZ + c, r);
+          tmem_ld_wait();
+          uint32_t w = 0;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w |= (__uint_as_float(r[i]) >= 0.f ? 1u : 0u) << i;
+          planes[K][c / 32] = (nrm > 0.f) ? w : 0xFFFFFFFFu;
+        }
+        tc_fence_before();
+        mbar_arrive(z_empty);
+      }
+      if (v < A.n) {
+        const int64_t slot = A.slots ? A.slots[v] : v;
+        A.norm[slot] = __half_as_ushort(__float2half_rn(nrm));
+        if (PROD) A.rnorm[slot] = nrm > 0.f ? __half_as_ushort(__float2half_rn(sqrtf(rn2))) : (uint16_t)0;
+        uint8_t* rec = A.codes + slot * (int64_t)(P * D / 8);
+        if constexpr (D == 128) {
+          // quarter q = 32 coordinates: one 32-bit word per plane
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t w[P];
+#pragma unroll
+            for (int p = 0; p < P; ++p) w[p] = planes[p][q];
+            if constexpr (P == 4) {
+              *reinterpret_cast<uint4*>(rec + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+            } else {
+#pragma unroll
+              for (int p = 0; p < P; ++p) *reinterpret_cast<uint32_t*>(rec + q * 4 * P + 4 * p) = w[p];
+            }
+          }
+        } else {
+          // D == 64: quarter q = 16 coordinates: one 16-bit half word per plane
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+#pragma unroll
+            for (int p = 0; p < P; ++p) {
+              const uint32_t w = planes[p][q >> 1] >> (16 * (q & 1));
+              *reinterpret_cast<uint16_t*>(rec + q * 2 * P + 2 * p) = (uint16_t)(w & 0xFFFFu);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------ host
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encoder() {
+  static EncodeTiled fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  }
+  return fn;
+}
+
+// 2-D row-major map [rows][cols] of 16-bit elements, box {64 columns, box_rows rows},
+// 128-byte swizzle (the canonical K-major operand layout of tcgen05.mma).
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t rows, uint64_t cols,
+              uint64_t row_stride_bytes, uint32_t box_rows) {
+  EncodeTiled enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, bool PROD, int K>
+int launch_tc_t(const tq_ctx* ctx, const void* x, int64_t n, int64_t ld, const tq_packed* dst, const int64_t* slots,
+                cudaStream_t st) {
+  constexpr int NST = PROD ? 2 : 3;
+  using SM = Smem<D, PROD, NST>;
+  CUtensorMap tx, tp, tm;
+  if (!make_map(&tx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)n, D, (uint64_t)ld * 2, kTileM))
+    return fail(TQ_ERR_UNSUPPORTED, "cuTensorMapEncodeTiled rejected the input (needs 16-byte aligned rows)");
+  if (!make_map(&tp, ctx->Pi_split, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3 * D, D, D * 2, D))
+    return fail(TQ_ERR_INTERNAL, "tensor map for Pi splits");
+  if (PROD) {
+    if (!make_map(&tm, ctx->M_split, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2 * D, D, D * 2, D))
+      return fail(TQ_ERR_INTERNAL, "tensor map for M splits");
+  } else {
+    tm = tp;
+  }
+  QtArgs a{};
+  a.n = n;
+  a.slots = slots;
+  a.codes = dst->codes;
+  a.norm = dst->norm;
+  a.rnorm = dst->rnorm;
+  a.err = ctx->dev_err;
+  for (int j = 0; j < 16; ++j) {
+    a.c[j] = ctx->cb.c[j];
+    a.t[j] = ctx->cb.t[j];
+  }
+  auto kern = quantize_tc_kernel<D, PROD, K>;
+  // one CTA per SM: it owns all 512 TMEM columns (more than half the shared memory forces it)
+  const int smem_bytes = SM::BYTES > 120 * 1024 ? SM::BYTES : 120 * 1024;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(quantize_tc)");
+  const int64_t ntiles = (n + kTileM - 1) / kTileM;
+  int sms = 148;
+  int dev = ctx->device;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = (int)std::min<int64_t>(ntiles, sms);
+  kern<<<grid, 192, smem_bytes, st>>>(tx, tp, tm, a);
+  count_launch();
+  return check_launch("quantize_tc_kernel");
+}
+
+}  // namespace
+
+// bf16 input, d in {64, 128}, k in [1, 4]; other shapes return kNotHandled.
+int launch_quantize_tc(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld, const tq_packed* dst,
+                       const int64_t* slots, cudaStream_t st) {
+  if (x_dtype != TQ_DTYPE_BF16 || !ctx->Pi_split) return kNotHandled;
+  const int d = ctx->lay.d, k = ctx->lay.k;
+  if ((d != 64 && d != 128) || (ld * 2) % 16 != 0 || (reinterpret_cast<uintptr_t>(x) % 16) != 0) return kNotHandled;
+  if (n < kTileM) return kNotHandled;   // small batches: the CUDA-core kernel
+  const bool prod = ctx->mode == TQ_MODE_PROD;
+#define TQ_TC_CASE(DD, PP, KK) \
+  if (d == DD && prod == PP && k == KK) return launch_tc_t<DD, PP, KK>(ctx, x, n, ld, dst, slots, st);
+  TQ_TC_CASE(128, true, 3) TQ_TC_CASE(128, true, 2) TQ_TC_CASE(128, true, 1)
+  TQ_TC_CASE(128, false, 4) TQ_TC_CASE(128, false, 3) TQ_TC_CASE(128, false, 2)
+  TQ_TC_CASE(64, true, 3) TQ_TC_CASE(64, true, 2) TQ_TC_CASE(64, true, 1)
+  TQ_TC_CASE(64, false, 4) TQ_TC_CASE(64, false, 3) TQ_TC_CASE(64, false, 2)
+#undef TQ_TC_CASE
+  return kNotHandled;
+}
+
+}  // namespace tq

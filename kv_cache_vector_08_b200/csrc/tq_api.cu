@@ -78,8 +78,48 @@ std::vector<double> transpose(const std::vector<double>& a, int rows, int cols) 
   return t;
 }
 
+// bf16 / fp16 splits of the tensor-core operands: Pi = hi + mid + lo (bf16, ~24 bits),
+// 16*M = hi + lo (fp16, ~22 bits); each split row-major [d][d].
+int alloc_splits(tq_ctx* c) {
+  const HostParams& h = c->host;
+  const int d = c->lay.d;
+  const size_t nn = (size_t)d * d;
+  std::vector<__nv_bfloat16> pis(3 * nn);
+  for (size_t i = 0; i < nn; ++i) {
+    double v = h.Pi[i];
+    __nv_bfloat16 a = __float2bfloat16_rn((float)v);
+    double r1 = v - (double)__bfloat162float(a);
+    __nv_bfloat16 b = __float2bfloat16_rn((float)r1);
+    double r2 = r1 - (double)__bfloat162float(b);
+    pis[i] = a;
+    pis[nn + i] = b;
+    pis[2 * nn + i] = __float2bfloat16_rn((float)r2);
+  }
+  cudaError_t e = cudaMalloc(&c->Pi_split, pis.size() * sizeof(__nv_bfloat16));
+  if (e != cudaSuccess) return fail(TQ_ERR_ALLOC, std::string("cudaMalloc: ") + cudaGetErrorString(e));
+  e = cudaMemcpy(c->Pi_split, pis.data(), pis.size() * sizeof(__nv_bfloat16), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(Pi splits)");
+  if (c->mode == TQ_MODE_PROD) {
+    std::vector<__half> ms(2 * nn);
+    for (size_t i = 0; i < nn; ++i) {
+      double v = 16.0 * h.M[i];
+      __half a = __float2half_rn((float)v);
+      ms[i] = a;
+      ms[nn + i] = __float2half_rn((float)(v - (double)__half2float(a)));
+    }
+    e = cudaMalloc(&c->M_split, ms.size() * sizeof(__half));
+    if (e != cudaSuccess) return fail(TQ_ERR_ALLOC, std::string("cudaMalloc: ") + cudaGetErrorString(e));
+    e = cudaMemcpy(c->M_split, ms.data(), ms.size() * sizeof(__half), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(M splits)");
+  }
+  return TQ_OK;
+}
+
 void release(tq_ctx* c) {
   if (!c) return;
+  cudaFree(c->Pi_split);
+  cudaFree(c->M_split);
+  cudaFree(c->dev_err);
   cudaFree(c->Pi);
   cudaFree(c->PiT);
   cudaFree(c->S);
@@ -167,7 +207,36 @@ int tq_init(tq_ctx** out, int d, int bits, uint64_t seed, int mode) {
       return r;
     }
   }
+  if (d == 64 || d == 128) {
+    if ((r = alloc_splits(c)) != TQ_OK) {
+      release(c);
+      return r;
+    }
+  }
+  e = cudaMalloc(&c->dev_err, sizeof(int));
+  if (e != cudaSuccess) {
+    release(c);
+    return fail(TQ_ERR_ALLOC, std::string("cudaMalloc: ") + cudaGetErrorString(e));
+  }
+  e = cudaMemset(c->dev_err, 0, sizeof(int));
+  if (e != cudaSuccess) {
+    release(c);
+    return cuda_fail(e, "cudaMemset(error word)");
+  }
   *out = c;
+  return TQ_OK;
+}
+
+int tq_get_device_error(const tq_ctx* ctx, int* code) {
+  if (!ctx || !code) return fail(TQ_ERR_INVALID_ARG, "NULL argument");
+  int v = 0;
+  cudaError_t e = cudaMemcpy(&v, ctx->dev_err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(error word)");
+  *code = v;
+  if (v != 0) {
+    e = cudaMemset(ctx->dev_err, 0, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(error word)");
+  }
   return TQ_OK;
 }
 

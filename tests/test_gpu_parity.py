@@ -74,6 +74,8 @@ def test_quantize_toy_config_fp32():
     (128, 5, 0, 300, "f16"), (128, 1, 1, 300, "fp32"),
     (200, 4, 0, 257, "fp32"), (1536, 4, 0, 65, "fp32"), (16, 3, 0, 129, "fp32"),
     (128, 4, 0, 1, "bf16"), (128, 4, 0, 127, "bf16"), (128, 4, 0, 129, "bf16"),
+    (128, 2, 0, 700, "bf16"), (128, 3, 1, 700, "bf16"), (128, 2, 1, 700, "bf16"),   # tensor-core variants
+    (64, 2, 1, 300, "bf16"), (128, 4, 0, 40000, "bf16"), (64, 4, 1, 40000, "bf16"),  # many tiles per CTA
 ])
 def test_quantize_matches_oracle(d, bits, mode, n, dtype):
     seed = 1000 + 2 * bits + mode
@@ -89,6 +91,7 @@ def test_quantize_matches_oracle(d, bits, mode, n, dtype):
     codes, norm, rn = _host(pk)
     res = parity.check_codes(oracle.make_params(d, bits, seed, mode), x.astype(np.float64), codes, norm, rn,
                              "d=%d b=%d mode=%d" % (d, bits, mode))
+    assert ctx.device_error() == 0
     print(d, bits, mode, n, res)
 
 
