@@ -12,10 +12,14 @@
 // rotated basis, and S r = (S Pi^T) y-residual = M r, so the QJL projection is a second
 // GEMM with A taken straight from tensor memory (hi*hi + hi*lo + lo*hi products).
 //
-// Roles (192 threads): warp 0 issues TMA loads (constants once, then one x tile per
-// stage), warp 1 allocates TMEM and issues the MMAs, warps 2-5 are the epilogue
-// (thread = one vector = one TMEM lane).  Every mbarrier wait is bounded; a timeout sets
-// the context's error word and the CTA winds down (TMEM is always released).
+// Roles (576 threads, one persistent CTA per SM): warp 0 issues TMA loads (constants
+// once, then the x tiles one 128-byte K atom at a time), warp 1 allocates TMEM and issues
+// the MMAs, warps 2-17 are the epilogue: thread (row, w) owns vector `row` of the tile and
+// coordinates [w d/4, (w+1) d/4), i.e. exactly one quarter of its packed record.  Two TMEM
+// accumulator buffers (each holding a tile's Pi x, then its QJL projection) and two
+// residual buffers let the MMAs of the next tile run under the epilogue of this one.
+// Every mbarrier wait is bounded; a timeout sets the context's error word and the CTA
+// winds down (in-flight copies and MMAs are drained and TMEM is always released).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -32,8 +36,11 @@ using namespace sm100;
 constexpr int kTileM = 128;
 constexpr uint64_t kWaitNs = 2000000000ull;   // a pipeline wait longer than 2 s is declared stuck
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColY = 0, kColR = 128, kColZ = 256;
-constexpr float kRScale = 256.f;   // the residual enters the QJL GEMM as r * 2^8 (M as 16 * M)
+constexpr uint32_t kColBuf0 = 0, kColR0 = 256;  // accumulators [2] x 128 cols, residuals [2] x 128 cols
+constexpr float kRScale = 256.f;              // the residual enters the QJL GEMM as r * 2^8 (M as 16 * M)
+constexpr int kEpiWarps = 16;                 // 4 warpgroups: thread = (vector row, quarter of its coords)
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kEpiThreads = 32 * kEpiWarps;
 
 struct QtArgs {
   int64_t n;
@@ -45,18 +52,21 @@ struct QtArgs {
   float c[16], t[16];
 };
 
-// Shared-memory plan (all operand regions 1024-byte aligned).
-template <int D, bool PROD, int NST>
+// Shared-memory plan (operand regions 1024-byte aligned); x is staged per 128-byte K atom
+// (128 rows x 64 columns bf16 = 16 KB) so loads of the next tile overlap the MMAs.
+template <int D, bool PROD>
 struct Smem {
-  static constexpr int KA = D / 64;                       // 128-byte K atoms per row
-  static constexpr int PI_SPLIT = D * D * 2;              // bytes of one bf16 split of Pi
+  static constexpr int KA = D / 64;
+  static constexpr int ATOM = kTileM * 128;
+  static constexpr int PI_SPLIT = D * D * 2;
   static constexpr int M_SPLIT = D * D * 2;
-  static constexpr int X_TILE = kTileM * D * 2;
+  static constexpr int NSLOT = (D == 128 && PROD) ? 3 : 4;
   static constexpr int OFF_PI = 0;
   static constexpr int OFF_M = OFF_PI + 3 * PI_SPLIT;
   static constexpr int OFF_X = OFF_M + (PROD ? 2 * M_SPLIT : 0);
-  static constexpr int OFF_BAR = OFF_X + NST * X_TILE;
-  static constexpr int BYTES = OFF_BAR + 256 + 1024;      // barriers + alignment slack
+  static constexpr int OFF_XCH = OFF_X + NSLOT * ATOM;          // float [2][4][128] x 2 (norm partials)
+  static constexpr int OFF_BAR = OFF_XCH + 2 * 2 * 4 * kTileM * 4;
+  static constexpr int BYTES = OFF_BAR + 256 + 1024;            // barriers + alignment slack
 };
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
@@ -65,27 +75,33 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 }
 
 template <int D, bool PROD, int K>
-__global__ void __launch_bounds__(192, 1) quantize_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
-                                                             const __grid_constant__ CUtensorMap tm_pi,
-                                                             const __grid_constant__ CUtensorMap tm_m, QtArgs A) {
-  constexpr int NST = PROD ? 2 : 3;
-  using SM = Smem<D, PROD, NST>;
-  constexpr int KA = SM::KA;
+__global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
+                                                                  const __grid_constant__ CUtensorMap tm_pi,
+                                                                  const __grid_constant__ CUtensorMap tm_m, QtArgs A) {
+  using SM = Smem<D, PROD>;
+  constexpr int KA = SM::KA, NSLOT = SM::NSLOT;
   constexpr int NK = D / 16;             // k-steps per product
+  constexpr int CQ = D / 4;              // coordinates per epilogue thread (one record quarter)
   constexpr int LEVELS = 1 << K;
   constexpr int P = K + (PROD ? 1 : 0);  // bit planes
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* s_n = reinterpret_cast<float*>(smem + SM::OFF_XCH);          // [2][4][128] partial ||y||^2
+  float* s_rn = s_n + 2 * 4 * kTileM;                                  // [2][4][128] partial ||r||^2
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::OFF_BAR);
-  uint64_t* full_x = bars;               // [NST] TMA -> MMA
-  uint64_t* empty_x = bars + NST;        // [NST] MMA -> TMA
-  uint64_t* const_full = bars + 2 * NST; // constants loaded
-  uint64_t* y_full = const_full + 1;     // MMA -> epilogue
-  uint64_t* y_empty = y_full + 1;        // epilogue -> MMA
-  uint64_t* r_full = y_empty + 1;        // epilogue -> MMA (residual written to TMEM)
-  uint64_t* z_full = r_full + 1;         // MMA -> epilogue
-  uint64_t* z_empty = z_full + 1;        // epilogue -> MMA
-  uint64_t* drain = z_empty + 1;          // MMA issuer: all issued MMAs complete
+  uint64_t* full_x = bars;                  // [NSLOT] TMA -> MMA
+  uint64_t* empty_x = bars + NSLOT;         // [NSLOT] MMA -> TMA
+  uint64_t* const_full = bars + 2 * NSLOT;  // constant operands landed
+  // Every barrier below exists once per accumulator buffer: a barrier completes its next
+  // phase only after each of its waiters has seen the previous one, so parity waits never
+  // skip a phase even when one role runs a whole tile ahead of another.
+  uint64_t* y_full = const_full + 1;        // [2] MMA -> epilogue (Pi x ready)
+  uint64_t* z_full = y_full + 2;            // [2] MMA -> epilogue (QJL projection ready)
+  uint64_t* r_full = z_full + 2;            // [2] epilogue -> MMA (residual in TMEM)
+  uint64_t* buf_empty = r_full + 2;         // [2] epilogue -> MMA (accumulator buffer free)
+  uint64_t* xn = buf_empty + 2;             // [2] norm partials written
+  uint64_t* xr = xn + 2;                    // [2] residual-norm partials written
+  uint64_t* drain = xr + 2;                 // MMA issuer: every issued MMA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
@@ -93,16 +109,19 @@ __global__ void __launch_bounds__(192, 1) quantize_tc_kernel(const __grid_consta
   const int64_t ntiles = (A.n + kTileM - 1) / kTileM;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < NSLOT; ++s) {
       mbar_init(full_x + s, 1);
       mbar_init(empty_x + s, 1);
     }
     mbar_init(const_full, 1);
-    mbar_init(y_full, 1);
-    mbar_init(y_empty, 128);
-    mbar_init(r_full, 128);
-    mbar_init(z_full, 1);
-    mbar_init(z_empty, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(y_full + b, 1);
+      mbar_init(z_full + b, 1);
+      mbar_init(r_full + b, kEpiThreads);
+      mbar_init(buf_empty + b, kEpiThreads);
+      mbar_init(xn + b, kEpiThreads);
+      mbar_init(xr + b, kEpiThreads);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -135,22 +154,23 @@ __global__ void __launch_bounds__(192, 1) quantize_tc_kernel(const __grid_consta
         for (int s = 0; s < 2; ++s)
           for (int a = 0; a < KA; ++a)
             tma_load_2d(smem + SM::OFF_M + s * SM::M_SPLIT + a * D * 128, &tm_m, 64 * a, s * D, const_full);
-      int it = 0;
-      int pending[NST];                  // parity of the last load issued into each stage, -1: none
-      for (int s = 0; s < NST; ++s) pending[s] = -1;
-      for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-        const int s = it % NST;
-        const uint32_t ph = (it / NST) & 1;
-        if (!wait(empty_x + s, ph ^ 1)) { fail(101); break; }
-        mbar_arrive_expect_tx(full_x + s, SM::X_TILE);
-        for (int a = 0; a < KA; ++a)
-          tma_load_2d(smem + SM::OFF_X + s * SM::X_TILE + a * kTileM * 128, &tm_x, 64 * a, (int)(tile * kTileM),
-                      full_x + s);
-        pending[s] = (int)ph;
+      int pending[NSLOT];                 // parity of the load in flight in each slot, -1: none
+      for (int s = 0; s < NSLOT; ++s) pending[s] = -1;
+      int64_t q = 0;                      // atom loads issued
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+        for (int a = 0; a < KA; ++a, ++q) {
+          const int s = (int)(q % NSLOT);
+          const uint32_t ph = (uint32_t)((q / NSLOT) & 1);
+          if (!wait(empty_x + s, ph ^ 1)) { fail(101); ok = false; break; }
+          mbar_arrive_expect_tx(full_x + s, SM::ATOM);
+          tma_load_2d(smem + SM::OFF_X + s * SM::ATOM, &tm_x, 64 * a, (int)(tile * kTileM), full_x + s);
+          pending[s] = (int)ph;
+        }
       }
       // copies still in flight land before the CTA releases its shared memory
       mbar_wait(const_full, 0, nullptr, kWaitNs);
-      for (int s = 0; s < NST; ++s)
+      for (int s = 0; s < NSLOT; ++s)
         if (pending[s] >= 0) mbar_wait(full_x + s, (uint32_t)pending[s], nullptr, kWaitNs);
     }
   } else if (warp == 1) {
@@ -160,158 +180,201 @@ __global__ void __launch_bounds__(192, 1) quantize_tc_kernel(const __grid_consta
       const uint32_t pi_addr = smem_u32(smem + SM::OFF_PI), m_addr = smem_u32(smem + SM::OFF_M);
       bool ok = wait(const_full, 0);
       if (!ok) fail(102);
-      int it = 0;
-      for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
-        const int s = it % NST;
-        const uint32_t ph = (it / NST) & 1, pt = it & 1;
-        if (!wait(full_x + s, ph) || !wait(y_empty, pt ^ 1)) { fail(103); break; }
+      // z = (R_hi + R_lo)(M_hi + M_lo) without the lo*lo term, into the tile's buffer
+      auto issue_z = [&](int t) -> bool {
+        const int par = t & 1;
+        if (!wait(r_full + par, (uint32_t)((t >> 1) & 1))) { fail(104); return false; }
         tc_fence_after();
-        const uint32_t x_addr = smem_u32(smem + SM::OFF_X + s * SM::X_TILE);
-        for (int sp = 0; sp < 3; ++sp)
+        const uint32_t dz = tmem + kColBuf0 + 128 * par, rz = tmem + kColR0 + 128 * par;
+        for (int sp = 0; sp < 3; ++sp) {
+          const uint32_t a_col = rz + (sp == 2 ? D / 2 : 0);
+          const int msp = (sp == 1) ? 1 : 0;
           for (int ks = 0; ks < NK; ++ks) {
-            const int a = ks >> 2, kk = ks & 3;
-            const uint64_t da = desc_sw128(x_addr + a * kTileM * 128 + kk * 32);
-            const uint64_t db = desc_sw128(pi_addr + sp * SM::PI_SPLIT + a * D * 128 + kk * 32);
-            mma_ss(tmem + kColY, da, db, idy, (sp | ks) ? 1u : 0u);
+            const uint64_t db = desc_sw128(m_addr + msp * SM::M_SPLIT + (ks >> 2) * D * 128 + (ks & 3) * 32);
+            mma_ts(dz, a_col + ks * 8, db, idz, (sp | ks) ? 1u : 0u);
           }
-        mma_commit(empty_x + s);
-        mma_commit(y_full);
-        if (PROD) {
-          if (!wait(r_full, pt) || !wait(z_empty, pt ^ 1)) { fail(104); break; }
-          tc_fence_after();
-          // z = R_hi M_hi + R_hi M_lo + R_lo M_hi   (A from TMEM: 2 fp16 per column)
-          for (int sp = 0; sp < 3; ++sp) {
-            const uint32_t a_col = kColR + (sp == 2 ? D / 2 : 0);
-            const int msp = (sp == 1) ? 1 : 0;
-            for (int ks = 0; ks < NK; ++ks) {
-              const int a = ks >> 2, kk = ks & 3;
-              const uint64_t db = desc_sw128(m_addr + msp * SM::M_SPLIT + a * D * 128 + kk * 32);
-              mma_ts(tmem + kColZ, tmem + a_col + ks * 8, db, idz, (sp | ks) ? 1u : 0u);
-            }
-          }
-          mma_commit(z_full);
         }
+        mma_commit(z_full + par);
+        return true;
+      };
+      int it = 0;
+      int64_t q = 0;
+      for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
+        const int par = it & 1;
+        if (!wait(buf_empty + par, (uint32_t)(((it >> 1) & 1) ^ 1))) { fail(103); ok = false; break; }
+        tc_fence_after();
+        const uint32_t dy = tmem + kColBuf0 + 128 * par;
+        for (int a = 0; a < KA; ++a, ++q) {
+          const int s = (int)(q % NSLOT);
+          if (!wait(full_x + s, (uint32_t)((q / NSLOT) & 1))) { fail(103); ok = false; break; }
+          tc_fence_after();
+          const uint32_t x_addr = smem_u32(smem + SM::OFF_X + s * SM::ATOM);
+          for (int sp = 0; sp < 3; ++sp)
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t da = desc_sw128(x_addr + kk * 32);
+              const uint64_t db = desc_sw128(pi_addr + sp * SM::PI_SPLIT + a * D * 128 + kk * 32);
+              mma_ss(dy, da, db, idy, (a | sp | kk) ? 1u : 0u);
+            }
+          mma_commit(empty_x + s);
+        }
+        if (!ok) break;
+        mma_commit(y_full + par);
+        if (PROD && it >= 1 && !issue_z(it - 1)) { ok = false; break; }
       }
+      if (PROD && ok && it >= 1) issue_z(it - 1);
       // every MMA issued above completes before TMEM is released
       mma_commit(drain);
       mbar_wait(drain, 0, nullptr, kWaitNs);
     }
   } else {
     // ------------------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;                       // TMEM lanes 32*quarter .. +31
-    const int row = quarter * 32 + lane;
-    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    int it = 0;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-      const uint32_t pt = it & 1;
-      if (!wait(y_full, pt)) { fail(105); break; }
-      tc_fence_after();
-      // pass 1: ||x||^2 = ||Pi x||^2 from the accumulator row
-      float n2 = 0.f;
-#pragma unroll
-      for (int c = 0; c < D; c += 32) {
+    const int ew = warp - 2, wg = ew >> 2;             // wg: which quarter of the coordinates
+    const int tq = warp & 3;                           // TMEM lanes 32*tq .. +31
+    const int row = tq * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(tq * 32) << 16);
+    const int c0 = wg * CQ;
+    // state of the tile whose QJL signs are still to come
+    uint32_t pend_planes[K];
+    float pend_n = 0.f;
+    int64_t pend_v = -1;
+    auto load_cols = [&](uint32_t col, float (&v)[CQ]) {
+      if constexpr (CQ == 32) {
         uint32_t r[32];
-        tmem_ld32(lane_base + kColY + c, r);
+        tmem_ld32(lane_base + col, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) n2 = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), n2);
-      }
-      const float nrm = sqrtf(n2);
-      const float inv = nrm > 0.f ? 1.f / nrm : 0.f;
-      uint32_t planes[P][D / 32];
-#pragma unroll
-      for (int p = 0; p < P; ++p)
-#pragma unroll
-        for (int w = 0; w < D / 32; ++w) planes[p][w] = 0u;
-      float rn2 = 0.f;
-      // pass 2: y = Pi x / ||x||, nearest centroid, residual (scaled, split into fp16 hi / lo)
-#pragma unroll
-      for (int c = 0; c < D; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(lane_base + kColY + c, r);
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      } else {
+        uint32_t r[16];
+        tmem_ld16(lane_base + col, r);
         tmem_ld_wait();
-        float rs[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float yy = __uint_as_float(r[i]) * inv;
-          int idx = 0;
-#pragma unroll
-          for (int j = 0; j < LEVELS - 1; ++j) idx += (yy > A.t[j]) ? 1 : 0;
-          float cv = A.c[0];
-#pragma unroll
-          for (int j = 1; j < LEVELS; ++j) cv = (idx == j) ? A.c[j] : cv;
-          const float rr = yy - cv;
-          rn2 = fmaf(rr, rr, rn2);
-          rs[i] = rr * kRScale;
-#pragma unroll
-          for (int p = 0; p < K; ++p) planes[p][c / 32] |= (uint32_t)((idx >> p) & 1) << i;
-        }
-        if (PROD) {
-          uint32_t hi[16], lo[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float a0 = rs[2 * i], a1 = rs[2 * i + 1];
-            const float h0 = __half2float(__float2half_rn(a0)), h1 = __half2float(__float2half_rn(a1));
-            hi[i] = pack_h2(h0, h1);
-            lo[i] = pack_h2(a0 - h0, a1 - h1);
-          }
-          tmem_st16(lane_base + kColR + c / 2, hi);
-          tmem_st16(lane_base + kColR + D / 2 + c / 2, lo);
-        }
+        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
       }
-      if (PROD) tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(y_empty);                            // D_y may be overwritten now
-      const int64_t v = tile * kTileM + row;
-      if (PROD) {
-        mbar_arrive(r_full);
-        if (!wait(z_full, pt)) { fail(106); break; }
-        tc_fence_after();
+    };
+    // one record quarter: planes[0..P-1] of this thread's CQ coordinates
+    auto store_quarter = [&](int64_t v, const uint32_t* pl, float nrm, float rn2) {
+      if (v >= A.n) return;
+      const int64_t slot = A.slots ? A.slots[v] : v;
+      uint8_t* rec = A.codes + slot * (int64_t)(P * D / 8) + wg * (P * D / 32);
+      if constexpr (CQ == 32) {
+        if constexpr (P == 4) *reinterpret_cast<uint4*>(rec) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+        else if constexpr (P == 2) *reinterpret_cast<uint2*>(rec) = make_uint2(pl[0], pl[1]);
+        else
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t r[32];
-          tmem_ld32(lane_base + kColZ + c, r);
-          tmem_ld_wait();
-          uint32_t w = 0;
+          for (int p = 0; p < P; ++p) reinterpret_cast<uint32_t*>(rec)[p] = pl[p];
+      } else {
+        if constexpr (P == 4) *reinterpret_cast<uint2*>(rec) = make_uint2(pl[0] | (pl[1] << 16), pl[2] | (pl[3] << 16));
+        else if constexpr (P == 2) *reinterpret_cast<uint32_t*>(rec) = pl[0] | (pl[1] << 16);
+        else
 #pragma unroll
-          for (int i = 0; i < 32; ++i) w |= (__uint_as_float(r[i]) >= 0.f ? 1u : 0u) << i;
-          planes[K][c / 32] = (nrm > 0.f) ? w : 0xFFFFFFFFu;
-        }
-        tc_fence_before();
-        mbar_arrive(z_empty);
+          for (int p = 0; p < P; ++p) reinterpret_cast<uint16_t*>(rec)[p] = (uint16_t)pl[p];
       }
-      if (v < A.n) {
-        const int64_t slot = A.slots ? A.slots[v] : v;
+      if (wg == 0) {
         A.norm[slot] = __half_as_ushort(__float2half_rn(nrm));
         if (PROD) A.rnorm[slot] = nrm > 0.f ? __half_as_ushort(__float2half_rn(sqrtf(rn2))) : (uint16_t)0;
-        uint8_t* rec = A.codes + slot * (int64_t)(P * D / 8);
-        if constexpr (D == 128) {
-          // quarter q = 32 coordinates: one 32-bit word per plane
+      }
+    };
+    // signs of tile t's QJL projection, then its record quarter
+    auto finish_z = [&](int t) -> bool {
+      const int par = t & 1;
+      if (!wait(z_full + par, (uint32_t)((t >> 1) & 1))) { fail(106); return false; }
+      tc_fence_after();
+      float z[CQ];
+      load_cols(kColBuf0 + 128 * par + c0, z);
+      uint32_t w = 0;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t w[P];
+      for (int i = 0; i < CQ; ++i) w |= (z[i] >= 0.f ? 1u : 0u) << i;
+      if (pend_n == 0.f) w = (CQ == 32) ? 0xFFFFFFFFu : 0xFFFFu;
+      float rn2 = 0.f;
+      if (wg == 0) {
+        if (!wait(xr + par, (uint32_t)((t >> 1) & 1))) { fail(107); return false; }
 #pragma unroll
-            for (int p = 0; p < P; ++p) w[p] = planes[p][q];
-            if constexpr (P == 4) {
-              *reinterpret_cast<uint4*>(rec + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-            } else {
+        for (int g = 0; g < 4; ++g) rn2 += s_rn[(par * 4 + g) * kTileM + row];
+      }
+      tc_fence_before();
+      mbar_arrive(buf_empty + par);
+      uint32_t pl[P];
 #pragma unroll
-              for (int p = 0; p < P; ++p) *reinterpret_cast<uint32_t*>(rec + q * 4 * P + 4 * p) = w[p];
-            }
-          }
-        } else {
-          // D == 64: quarter q = 16 coordinates: one 16-bit half word per plane
+      for (int p = 0; p < K; ++p) pl[p] = pend_planes[p];
+      pl[P - 1] = w;
+      store_quarter(pend_v, pl, pend_n, rn2);
+      return true;
+    };
+    int it = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+      const int par = it & 1;
+      if (!wait(y_full + par, (uint32_t)((it >> 1) & 1))) { fail(105); ok = false; break; }
+      tc_fence_after();
+      float y[CQ];
+      load_cols(kColBuf0 + 128 * par + c0, y);
+      float n2p = 0.f;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+      for (int i = 0; i < CQ; ++i) n2p = fmaf(y[i], y[i], n2p);
+      s_n[(par * 4 + wg) * kTileM + row] = n2p;
+      mbar_arrive(xn + par);
+      if (!wait(xn + par, (uint32_t)((it >> 1) & 1))) { fail(108); ok = false; break; }
+      float n2 = 0.f;
 #pragma unroll
-            for (int p = 0; p < P; ++p) {
-              const uint32_t w = planes[p][q >> 1] >> (16 * (q & 1));
-              *reinterpret_cast<uint16_t*>(rec + q * 2 * P + 2 * p) = (uint16_t)(w & 0xFFFFu);
-            }
-          }
+      for (int g = 0; g < 4; ++g) n2 += s_n[(par * 4 + g) * kTileM + row];
+      const float nrm = sqrtf(n2);
+      const float inv = nrm > 0.f ? 1.f / nrm : 0.f;
+      uint32_t planes[P];
+#pragma unroll
+      for (int p = 0; p < P; ++p) planes[p] = 0u;
+      float rn2p = 0.f;
+      float rs[CQ];
+#pragma unroll
+      for (int i = 0; i < CQ; ++i) {
+        const float yy = y[i] * inv;
+        int idx = 0;
+#pragma unroll
+        for (int j = 0; j < LEVELS - 1; ++j) idx += (yy > A.t[j]) ? 1 : 0;
+        float cv = A.c[0];
+#pragma unroll
+        for (int j = 1; j < LEVELS; ++j) cv = (idx == j) ? A.c[j] : cv;
+        const float rr = yy - cv;
+        rn2p = fmaf(rr, rr, rn2p);
+        rs[i] = rr * kRScale;
+#pragma unroll
+        for (int p = 0; p < K; ++p) planes[p] |= (uint32_t)((idx >> p) & 1) << i;
+      }
+      const int64_t v = tile * kTileM + row;
+      if (PROD) {
+        uint32_t hi[CQ / 2], lo[CQ / 2];
+#pragma unroll
+        for (int i = 0; i < CQ / 2; ++i) {
+          const float a0 = rs[2 * i], a1 = rs[2 * i + 1];
+          const float h0 = __half2float(__float2half_rn(a0)), h1 = __half2float(__float2half_rn(a1));
+          hi[i] = pack_h2(h0, h1);
+          lo[i] = pack_h2(a0 - h0, a1 - h1);
         }
+        const uint32_t rz = lane_base + kColR0 + 128 * par + c0 / 2;
+        if constexpr (CQ == 32) {
+          tmem_st16(rz, hi);
+          tmem_st16(rz + D / 2, lo);
+        } else {
+          tmem_st8(rz, hi);
+          tmem_st8(rz + D / 2, lo);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(r_full + par);
+        s_rn[(par * 4 + wg) * kTileM + row] = rn2p;
+        mbar_arrive(xr + par);
+        if (it >= 1 && !finish_z(it - 1)) { ok = false; break; }
+#pragma unroll
+        for (int p = 0; p < K; ++p) pend_planes[p] = planes[p];
+        pend_n = nrm;
+        pend_v = v;
+      } else {
+        tc_fence_before();
+        mbar_arrive(buf_empty + par);
+        store_quarter(v, planes, nrm, 0.f);
       }
     }
+    if (PROD && ok && it >= 1) finish_z(it - 1);
   }
   tc_fence_before();
   __syncthreads();
@@ -358,8 +421,7 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t
 template <int D, bool PROD, int K>
 int launch_tc_t(const tq_ctx* ctx, const void* x, int64_t n, int64_t ld, const tq_packed* dst, const int64_t* slots,
                 cudaStream_t st) {
-  constexpr int NST = PROD ? 2 : 3;
-  using SM = Smem<D, PROD, NST>;
+  using SM = Smem<D, PROD>;
   CUtensorMap tx, tp, tm;
   if (!make_map(&tx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)n, D, (uint64_t)ld * 2, kTileM))
     return fail(TQ_ERR_UNSUPPORTED, "cuTensorMapEncodeTiled rejected the input (needs 16-byte aligned rows)");
@@ -392,7 +454,7 @@ int launch_tc_t(const tq_ctx* ctx, const void* x, int64_t n, int64_t ld, const t
   int dev = ctx->device;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = (int)std::min<int64_t>(ntiles, sms);
-  kern<<<grid, 192, smem_bytes, st>>>(tx, tp, tm, a);
+  kern<<<grid, kThreads, smem_bytes, st>>>(tx, tp, tm, a);
   count_launch();
   return check_launch("quantize_tc_kernel");
 }
