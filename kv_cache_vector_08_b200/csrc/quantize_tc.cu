@@ -49,7 +49,10 @@ struct QtArgs {
   uint16_t* norm;
   uint16_t* rnorm;
   int* err;
-  float c[16], t[16];
+  // symmetric codebook: boundaries t[L/2-1+j] = pos_t[j-1] (j >= 1, the middle one is 0),
+  // centroids c[L/2+j] = mag[j] = -c[L/2-1-j]
+  float pos_t[8];
+  float mag[8];
 };
 
 // Shared-memory plan (operand regions 1024-byte aligned); x is staged per 128-byte K atom
@@ -285,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
       uint32_t w = 0;
 #pragma unroll
       for (int i = 0; i < CQ; ++i) w |= (z[i] >= 0.f ? 1u : 0u) << i;
-      if (pend_n == 0.f) w = (CQ == 32) ? 0xFFFFFFFFu : 0xFFFFu;
+      if (pend_n == 0.f) w = (CQ == 32) ? 0xFFFFFFFFu : 0xFFFFu;   // zero vector: all signs +1
       float rn2 = 0.f;
       if (wg == 0) {
         if (!wait(xr + par, (uint32_t)((t >> 1) & 1))) { fail(107); return false; }
@@ -319,26 +322,63 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
 #pragma unroll
       for (int g = 0; g < 4; ++g) n2 += s_n[(par * 4 + g) * kTileM + row];
       const float nrm = sqrtf(n2);
-      const float inv = nrm > 0.f ? 1.f / nrm : 0.f;
-      uint32_t planes[P];
+      // nearest centroid by sign and magnitude: y = D / ||x|| > 0 picks the upper half of the
+      // (odd-symmetric) codebook; the magnitude index is a binary search of |D| against the
+      // positive boundaries scaled by ||x|| (so no division per coordinate)
+      float pn[8];
 #pragma unroll
-      for (int p = 0; p < P; ++p) planes[p] = 0u;
+      for (int j = 0; j < LEVELS / 2 - 1; ++j) pn[j] = nrm * A.pos_t[j];
+      const float s256 = nrm > 0.f ? kRScale / nrm : 0.f;   // residual scale r * 2^8 = D s256 - 2^8 c
+      uint32_t S = 0u, B0 = 0u, B1 = 0u, B2 = 0u;
       float rn2p = 0.f;
       float rs[CQ];
 #pragma unroll
       for (int i = 0; i < CQ; ++i) {
-        const float yy = y[i] * inv;
-        int idx = 0;
+        const float Dv = y[i], a = fabsf(Dv);
+        const bool sp = Dv > 0.f;
+        bool b0 = false, b1 = false, b2 = false;
+        float m = 0.f;
+        if constexpr (K == 1) {
+          if (PROD) m = A.mag[0];
+        } else if constexpr (K == 2) {
+          b0 = a > pn[0];
+          if (PROD) m = b0 ? A.mag[1] : A.mag[0];
+        } else if constexpr (K == 3) {
+          b1 = a > pn[1];
+          b0 = a > (b1 ? pn[2] : pn[0]);
+          if (PROD) m = b1 ? (b0 ? A.mag[3] : A.mag[2]) : (b0 ? A.mag[1] : A.mag[0]);
+        } else {
+          b2 = a > pn[3];
+          b1 = a > (b2 ? pn[5] : pn[1]);
+          b0 = a > (b2 ? (b1 ? pn[6] : pn[4]) : (b1 ? pn[2] : pn[0]));
+          if (PROD)
+            m = b2 ? (b1 ? (b0 ? A.mag[7] : A.mag[6]) : (b0 ? A.mag[5] : A.mag[4]))
+                   : (b1 ? (b0 ? A.mag[3] : A.mag[2]) : (b0 ? A.mag[1] : A.mag[0]));
+        }
+        S |= (uint32_t)sp << i;
+        B0 |= (uint32_t)b0 << i;
+        B1 |= (uint32_t)b1 << i;
+        B2 |= (uint32_t)b2 << i;
+        if (PROD) {
+          const float r = fmaf(Dv, s256, sp ? -kRScale * m : kRScale * m);   // 2^8 (y - c[idx])
+          rn2p = fmaf(r, r, rn2p);
+          rs[i] = r;
+        }
+      }
+      rn2p *= 1.f / (kRScale * kRScale);
+      // idx = L/2 + |idx| (y > 0) or L/2 - 1 - |idx| = (L/2 - 1) ^ |idx| (y <= 0):
+      // bit K-1 is the sign, the lower bits are the magnitude bits, flipped when y <= 0
+      uint32_t planes[P];
+      {
+        const uint32_t nS = ~S;
+        if constexpr (K >= 2) planes[0] = B0 ^ nS;
+        if constexpr (K >= 3) planes[1] = B1 ^ nS;
+        if constexpr (K >= 4) planes[2] = B2 ^ nS;
+        planes[K - 1] = S;
+        if constexpr (CQ == 16) {
 #pragma unroll
-        for (int j = 0; j < LEVELS - 1; ++j) idx += (yy > A.t[j]) ? 1 : 0;
-        float cv = A.c[0];
-#pragma unroll
-        for (int j = 1; j < LEVELS; ++j) cv = (idx == j) ? A.c[j] : cv;
-        const float rr = yy - cv;
-        rn2p = fmaf(rr, rr, rn2p);
-        rs[i] = rr * kRScale;
-#pragma unroll
-        for (int p = 0; p < K; ++p) planes[p] |= (uint32_t)((idx >> p) & 1) << i;
+          for (int p = 0; p < K; ++p) planes[p] &= 0xFFFFu;
+        }
       }
       const int64_t v = tile * kTileM + row;
       if (PROD) {
@@ -440,9 +480,10 @@ int launch_tc_t(const tq_ctx* ctx, const void* x, int64_t n, int64_t ld, const t
   a.norm = dst->norm;
   a.rnorm = dst->rnorm;
   a.err = ctx->dev_err;
-  for (int j = 0; j < 16; ++j) {
-    a.c[j] = ctx->cb.c[j];
-    a.t[j] = ctx->cb.t[j];
+  const int L = ctx->cb.K;
+  for (int j = 0; j < 8; ++j) {
+    a.pos_t[j] = (j + 1 < L / 2) ? ctx->cb.t[L / 2 - 1 + j + 1] : INFINITY;
+    a.mag[j] = (j < L / 2) ? ctx->cb.c[L / 2 + j] : 0.f;
   }
   auto kern = quantize_tc_kernel<D, PROD, K>;
   // one CTA per SM: it owns all 512 TMEM columns (more than half the shared memory forces it)
