@@ -26,9 +26,12 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "sm100.cuh"
 
 namespace tq {
 namespace {
+
+using namespace sm100;
 
 constexpr int kWarps = 4;
 constexpr int kRep = 4;   // query heads per kv head handled by this kernel
@@ -94,6 +97,37 @@ __device__ __forceinline__ void load_quarter(const uint8_t* rec, int l, uint32_t
   }
 }
 
+// Same, from a record staged in shared memory (byte offset of the record arbitrary: the
+// staged copy keeps the global alignment of each record modulo 16).
+template <int Q, int P>
+__device__ __forceinline__ void lds_quarter(const uint8_t* rec, int l, uint32_t (&w)[P]) {
+  if constexpr (Q == 32) {
+    const uint8_t* p = rec + l * (4 * P);
+    if constexpr (P == 4) {
+      uint4 v = *reinterpret_cast<const uint4*>(p);
+      w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    } else if constexpr (P == 2) {
+      uint2 v = *reinterpret_cast<const uint2*>(p);
+      w[0] = v.x; w[1] = v.y;
+    } else {
+#pragma unroll
+      for (int i = 0; i < P; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
+    }
+  } else {
+    const uint8_t* p = rec + l * (2 * P);
+    if constexpr (P == 4) {
+      uint2 v = *reinterpret_cast<const uint2*>(p);
+      w[0] = v.x & 0xFFFFu; w[1] = v.x >> 16; w[2] = v.y & 0xFFFFu; w[3] = v.y >> 16;
+    } else if constexpr (P == 2) {
+      uint32_t v = *reinterpret_cast<const uint32_t*>(p);
+      w[0] = v & 0xFFFFu; w[1] = v >> 16;
+    } else {
+#pragma unroll
+      for (int i = 0; i < P; ++i) w[i] = reinterpret_cast<const unsigned short*>(p)[i];
+    }
+  }
+}
+
 // prmt selector nibbles (3 index bits) for coordinates 4k + qq of a quarter.
 template <int NB, uint32_t M1>
 __device__ __forceinline__ uint32_t selector(const uint32_t* w, int qq) {
@@ -140,6 +174,7 @@ struct MmaGroup {
   float coef;          // sqrt(pi/2)/m
   int off;             // first channel of the group
   int kbytes, vbytes;  // record sizes
+  int64_t kcap, vcap;  // slots allocated in the key / value caches
 };
 
 struct MmaArgs {
@@ -150,8 +185,8 @@ struct MmaArgs {
   const int32_t* seq_lens;
   const float* qprep;  // [B*Hq][G][2*qp_ld]: (Pi q, S q) of each group
   float* part;         // [B*Hq][nsplit][D+2]: (m, l, acc) per split
-  int* done;           // [B*Hkv] finished-split counters (zeroed by the prep kernel)
   float* out;          // [B*Hq][D]
+  int* err;            // device error word (a pipeline wait that timed out)
 };
 
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
@@ -281,13 +316,52 @@ __device__ __forceinline__ void tile_logits(const TileData<GC>& t, const QFrag<G
   lb += h2f(t.nkb) * fmaf(cb, sgn[2] + sgn[3], mse[2] + mse[3]);
 }
 
+constexpr int kStageTok = kWarps * 16;  // tokens per pipeline stage: one 16-token tile per consumer warp
+constexpr int kNStage = 4;
+constexpr uint64_t kDecWaitNs = 2000000000ull;
+
+// Shared-memory layout of one pipeline stage: per group the K and V code bytes of 64
+// consecutive slots (copied with 16-byte granularity, hence 32 bytes of slack) and the
+// three fp16 norm arrays.
+template <class G0, class G1c, bool TWO>
+struct Stage {
+  static constexpr int KB0 = G0::PK * G0::DG / 8, VB0 = G0::PV * G0::DG / 8;
+  static constexpr int KB1 = G1c::PK * G1c::DG / 8, VB1 = G1c::PV * G1c::DG / 8;
+  static constexpr int OFF_K0 = 0;
+  static constexpr int OFF_V0 = OFF_K0 + kStageTok * KB0 + 32;
+  static constexpr int OFF_K1 = OFF_V0 + kStageTok * VB0 + 32;
+  static constexpr int OFF_V1 = OFF_K1 + (TWO ? kStageTok * KB1 + 32 : 0);
+  static constexpr int OFF_N = OFF_V1 + (TWO ? kStageTok * VB1 + 32 : 0);   // uint16 [G][3][64]
+  static constexpr int BYTES = ((OFF_N + (TWO ? 2 : 1) * 3 * kStageTok * 2) + 127) / 128 * 128;
+};
+
+// Copy bytes [b0, b1) of a packed array into shared memory at dst + (b0 & 15): one bulk copy
+// of the 16-byte aligned span inside the allocation, plain loads for a ragged end beyond
+// the last full 16 bytes of the allocation.  Returns the bulk byte count (for expect_tx).
+__device__ __forceinline__ uint32_t stage_span(uint8_t* dst, const uint8_t* src, int64_t b0, int64_t b1, int64_t total,
+                                               uint64_t* bar, bool issue) {
+  const int64_t a0 = b0 & ~int64_t(15);
+  const int64_t cap16 = total & ~int64_t(15);
+  int64_t a1 = (b1 + 15) & ~int64_t(15);
+  if (a1 > cap16) a1 = cap16;
+  uint32_t bytes = a1 > a0 ? (uint32_t)(a1 - a0) : 0u;
+  if (issue) {
+    if (bytes) bulk_load(dst, src + a0, bytes, bar);
+    for (int64_t x = (a1 > a0 ? a1 : a0); x < b1; ++x) dst[x - a0] = src[x];
+  }
+  return bytes;
+}
+
 template <class G0, class G1>
-__global__ void __launch_bounds__(kWarps * 32) decode_mma_kernel(MmaArgs A) {
+__global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArgs A) {
   constexpr bool TWO = !std::is_same<G1, void>::value;
   using G1c = typename std::conditional<TWO, G1, G0>::type;
+  using ST = Stage<G0, G1c, TWO>;
+  extern __shared__ __align__(128) uint8_t dsm[];
   __shared__ float s_m[kWarps][kRep], s_l[kWarps][kRep];
   __shared__ float s_acc[kWarps][kRep][256];
-  __shared__ int s_last;
+  __shared__ __align__(8) uint64_t full[kNStage], empty[kNStage];
+  __shared__ int s_abort;
   const int split = blockIdx.x, bh = blockIdx.y;
   const int b = bh / A.Hkv, hk = bh % A.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -296,110 +370,186 @@ __global__ void __launch_bounds__(kWarps * 32) decode_mma_kernel(MmaArgs A) {
   const int t_begin = split * A.chunk;
   const int t_end = min(T, t_begin + A.chunk);
   const int64_t slot0 = (int64_t)bh * A.max_len;
-  constexpr int kStride = kWarps * 16;
-
-  // The first tile's codes are inputs of this call: fetch them before waiting for the
-  // query-preparation kernel that precedes this one on the stream.
-  TileData<G0> c0;
-  TileData<G1c> c1;
-  int ts = t_begin + warp * 16;
-  if (ts < t_end) {
-    const int64_t sa = slot0 + min(ts + g, T - 1), sb = slot0 + min(ts + g + 8, T - 1);
-    load_tile<G0>(c0, A.g[0], sa, sb, l);
-    if constexpr (TWO) load_tile<G1c>(c1, A.g[1], sa, sb, l);
-  }
-  const Lut kl0 = A.g[0].klut, vl0 = A.g[0].vlut;
-  const Lut kl1 = A.g[TWO ? 1 : 0].klut, vl1 = A.g[TWO ? 1 : 0].vlut;
-  grid_dependency_wait();
-  QFrag<G0> qf0;
-  load_qfrag<G0>(qf0, A, 0, b, hk, lane);
-  QFrag<G1c> qf1;
-  if constexpr (TWO) load_qfrag<G1c>(qf1, A, 1, b, hk, lane);
-
-  float acc0[G0::NKB][4];
-  float acc1[G1c::NKB][4];
-#pragma unroll
-  for (int i = 0; i < G0::NKB; ++i) acc0[i][0] = acc0[i][1] = acc0[i][2] = acc0[i][3] = 0.f;
-#pragma unroll
-  for (int i = 0; i < G1c::NKB; ++i) acc1[i][0] = acc1[i][1] = acc1[i][2] = acc1[i][3] = 0.f;
-  // softmax state of head l (log2 domain); l_run is this lane's partial sum over its tokens
-  float m_run = -INFINITY, l_run = 0.f;
-
-  for (; ts < t_end; ts += kStride) {
-    // prefetch the next tile while this one is computed
-    TileData<G0> n0;
-    TileData<G1c> n1;
-    const int tn = ts + kStride;
-    if (tn < t_end) {
-      const int64_t sa = slot0 + min(tn + g, T - 1), sb = slot0 + min(tn + g + 8, T - 1);
-      load_tile<G0>(n0, A.g[0], sa, sb, l);
-      if constexpr (TWO) load_tile<G1c>(n1, A.g[1], sa, sb, l);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNStage; ++i) {
+      mbar_init(full + i, 32);
+      mbar_init(empty + i, kWarps);
     }
-    float la = 0.f, lb = 0.f;
-    tile_logits<G0>(c0, qf0, kl0, A.g[0], la, lb);
-    if constexpr (TWO) tile_logits<G1c>(c1, qf1, kl1, A.g[1], la, lb);
-    // online softmax (log2 domain) of head l over tokens g, g+8 of the tile
-    la = (ts + g < t_end) ? la * A.scale_log2 : -INFINITY;
-    lb = (ts + g + 8 < t_end) ? lb * A.scale_log2 : -INFINITY;
-    float mt = fmaxf(la, lb);
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
-    if (mt > m_run) {
-      const float alpha = exp2f(m_run - mt);
-      m_run = mt;
-      l_run *= alpha;
-#pragma unroll
-      for (int i = 0; i < G0::NKB; ++i) {
-        acc0[i][0] *= alpha; acc0[i][1] *= alpha; acc0[i][2] *= alpha; acc0[i][3] *= alpha;
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const volatile int* abort_v = &s_abort;
+  auto fail = [&](int code) {
+    atomicExch(&s_abort, 1);
+    if (A.err) atomicCAS(A.err, 0, code);
+  };
+
+  if (warp == kWarps) {
+    // ---------------------------------------------------------------- producer warp
+    int it = 0;
+    int pending[kNStage];
+    for (int i = 0; i < kNStage; ++i) pending[i] = -1;
+    for (int ts = t_begin; ts < t_end; ts += kStageTok, ++it) {
+      const int s = it % kNStage;
+      const uint32_t ph = (it / kNStage) & 1;
+      if (!mbar_wait(empty + s, ph ^ 1, abort_v, kDecWaitNs)) { fail(201); break; }
+      const int ntok = min(kStageTok, t_end - ts);
+      uint8_t* st = dsm + s * ST::BYTES;
+      const int64_t first = slot0 + ts, last = slot0 + ts + ntok;
+      auto spans = [&](bool issue) {
+        uint32_t tx = 0;
+        const MmaGroup& g0 = A.g[0];
+        tx += stage_span(st + ST::OFF_K0, g0.kcodes, first * ST::KB0, last * ST::KB0, g0.kcap * ST::KB0, full + s, issue);
+        tx += stage_span(st + ST::OFF_V0, g0.vcodes, first * ST::VB0, last * ST::VB0, g0.vcap * ST::VB0, full + s, issue);
+        if constexpr (TWO) {
+          const MmaGroup& g1 = A.g[1];
+          tx += stage_span(st + ST::OFF_K1, g1.kcodes, first * ST::KB1, last * ST::KB1, g1.kcap * ST::KB1, full + s, issue);
+          tx += stage_span(st + ST::OFF_V1, g1.vcodes, first * ST::VB1, last * ST::VB1, g1.vcap * ST::VB1, full + s, issue);
+        }
+        return tx;
+      };
+      if (lane == 0) {
+        mbar_expect_tx(full + s, spans(false));
+        spans(true);
       }
-      if constexpr (TWO) {
+      uint16_t* nrm = reinterpret_cast<uint16_t*>(st + ST::OFF_N);
+      for (int j = lane; j < kStageTok; j += 32) {
+        const bool ok = j < ntok;
+        const int64_t sl = slot0 + ts + j;
 #pragma unroll
-        for (int i = 0; i < G1c::NKB; ++i) {
-          acc1[i][0] *= alpha; acc1[i][1] *= alpha; acc1[i][2] *= alpha; acc1[i][3] *= alpha;
+        for (int gi = 0; gi < (TWO ? 2 : 1); ++gi) {
+          const MmaGroup& gr = A.g[gi];
+          nrm[(gi * 3 + 0) * kStageTok + j] = ok ? __ldg(gr.knorm + sl) : (uint16_t)0;
+          nrm[(gi * 3 + 1) * kStageTok + j] = ok ? __ldg(gr.krnorm + sl) : (uint16_t)0;
+          nrm[(gi * 3 + 2) * kStageTok + j] = ok ? __ldg(gr.vnorm + sl) : (uint16_t)0;
         }
       }
+      __syncwarp();
+      mbar_arrive(full + s);
+      if (lane == 0) pending[s] = (int)ph;
     }
-    const float pa = exp2f(la - m_run), pb = exp2f(lb - m_run);
-    l_run += pa + pb;
-    // probability operand: columns 2l, 2l+1 = hi and lo halves of p * ||v|| for head l
-    auto pfrag = [&](float na, float nb, uint32_t& b0, uint32_t& b1) {
-      const float wa = pa * na, wb = pb * nb;
-      const float ha = __half2float(__float2half_rn(wa)), hb = __half2float(__float2half_rn(wb));
-      b0 = movT(pack_h2(ha, wa - ha));
-      b1 = movT(pack_h2(hb, wb - hb));
-    };
-    uint32_t pb0, pb1;
-    pfrag(h2f(c0.nva), h2f(c0.nvb), pb0, pb1);
-    group_values<G0>(vl0, c0.va, c0.vb, pb0, pb1, acc0);
-    if constexpr (TWO) {
-      pfrag(h2f(c1.nva), h2f(c1.nvb), pb0, pb1);
-      group_values<G1c>(vl1, c1.va, c1.vb, pb0, pb1, acc1);
-    }
-    c0 = n0;
-    if constexpr (TWO) c1 = n1;
+    // bulk copies still in flight land before the CTA exits
+    if (lane == 0)
+      for (int i = 0; i < kNStage; ++i)
+        if (pending[i] >= 0) mbar_wait(full + i, (uint32_t)pending[i], nullptr, kDecWaitNs);
   }
 
-  // ---- warp state -> shared memory (lane (g, l) holds head l)
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 4);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 8);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
-  if (g == 0) {
-    s_m[warp][l] = m_run;
-    s_l[warp][l] = l_run;
-  }
-  auto store_acc = [&](auto& acc, auto gc_tag, int off) {
-    using GC = decltype(gc_tag);
+  // ------------------------------------------------------------------ consumer warps
+  float acc0[G0::NKB][4];
+  float acc1[G1c::NKB][4];
+  float m_run = -INFINITY, l_run = 0.f;
+  if (warp < kWarps) {
+    const Lut kl0 = A.g[0].klut, vl0 = A.g[0].vlut;
+    const Lut kl1 = A.g[TWO ? 1 : 0].klut, vl1 = A.g[TWO ? 1 : 0].vlut;
+    grid_dependency_wait();   // prepared queries come from the preceding kernel
+    QFrag<G0> qf0;
+    load_qfrag<G0>(qf0, A, 0, b, hk, lane);
+    QFrag<G1c> qf1;
+    if constexpr (TWO) load_qfrag<G1c>(qf1, A, 1, b, hk, lane);
 #pragma unroll
-    for (int mb = 0; mb < GC::NKB; ++mb) {
-      const int qq = mb & 3, hh = mb >> 2;
-      const int c0_ = GC::Q * (g >> 1) + qq + 16 * hh + 4 * (g & 1);   // row g: block f = 0
-      s_acc[warp][l][off + c0_] = acc[mb][0] + acc[mb][1];
-      s_acc[warp][l][off + c0_ + 8] = acc[mb][2] + acc[mb][3];          // row g+8: block f = 1
+    for (int i = 0; i < G0::NKB; ++i) acc0[i][0] = acc0[i][1] = acc0[i][2] = acc0[i][3] = 0.f;
+#pragma unroll
+    for (int i = 0; i < G1c::NKB; ++i) acc1[i][0] = acc1[i][1] = acc1[i][2] = acc1[i][3] = 0.f;
+    int it = 0;
+    for (int ts = t_begin; ts < t_end; ts += kStageTok, ++it) {
+      const int s = it % kNStage;
+      if (!mbar_wait(full + s, (it / kNStage) & 1, abort_v, kDecWaitNs)) { fail(202); break; }
+      const int tt = ts + warp * 16;           // this warp's 16-token tile
+      const bool live = tt < t_end;
+      const uint8_t* st = dsm + s * ST::BYTES;
+      const int64_t first = slot0 + ts;
+      const int ja = warp * 16 + g, jb = ja + 8;   // stage-local token rows of this lane
+      TileData<G0> c0;
+      TileData<G1c> c1;
+      if (live) {
+        const uint8_t* k0 = st + ST::OFF_K0 + ((first * ST::KB0) & 15);
+        const uint8_t* v0 = st + ST::OFF_V0 + ((first * ST::VB0) & 15);
+        lds_quarter<G0::Q, G0::PK>(k0 + ja * ST::KB0, l, c0.ka);
+        lds_quarter<G0::Q, G0::PK>(k0 + jb * ST::KB0, l, c0.kb);
+        lds_quarter<G0::Q, G0::PV>(v0 + ja * ST::VB0, l, c0.va);
+        lds_quarter<G0::Q, G0::PV>(v0 + jb * ST::VB0, l, c0.vb);
+        const uint16_t* nrm = reinterpret_cast<const uint16_t*>(st + ST::OFF_N);
+        c0.nka = nrm[ja]; c0.nkb = nrm[jb];
+        c0.rka = nrm[kStageTok + ja]; c0.rkb = nrm[kStageTok + jb];
+        c0.nva = nrm[2 * kStageTok + ja]; c0.nvb = nrm[2 * kStageTok + jb];
+        if constexpr (TWO) {
+          const uint8_t* k1 = st + ST::OFF_K1 + ((first * ST::KB1) & 15);
+          const uint8_t* v1 = st + ST::OFF_V1 + ((first * ST::VB1) & 15);
+          lds_quarter<G1c::Q, G1c::PK>(k1 + ja * ST::KB1, l, c1.ka);
+          lds_quarter<G1c::Q, G1c::PK>(k1 + jb * ST::KB1, l, c1.kb);
+          lds_quarter<G1c::Q, G1c::PV>(v1 + ja * ST::VB1, l, c1.va);
+          lds_quarter<G1c::Q, G1c::PV>(v1 + jb * ST::VB1, l, c1.vb);
+          c1.nka = nrm[3 * kStageTok + ja]; c1.nkb = nrm[3 * kStageTok + jb];
+          c1.rka = nrm[4 * kStageTok + ja]; c1.rkb = nrm[4 * kStageTok + jb];
+          c1.nva = nrm[5 * kStageTok + ja]; c1.nvb = nrm[5 * kStageTok + jb];
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty + s);   // the stage's data now sits in registers
+      if (!live) continue;
+      float la = 0.f, lb = 0.f;
+      tile_logits<G0>(c0, qf0, kl0, A.g[0], la, lb);
+      if constexpr (TWO) tile_logits<G1c>(c1, qf1, kl1, A.g[1], la, lb);
+      // online softmax (log2 domain) of head l over tokens g, g+8 of the tile
+      la = (tt + g < t_end) ? la * A.scale_log2 : -INFINITY;
+      lb = (tt + g + 8 < t_end) ? lb * A.scale_log2 : -INFINITY;
+      float mt = fmaxf(la, lb);
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+      if (mt > m_run) {
+        const float alpha = exp2f(m_run - mt);
+        m_run = mt;
+        l_run *= alpha;
+#pragma unroll
+        for (int i = 0; i < G0::NKB; ++i) {
+          acc0[i][0] *= alpha; acc0[i][1] *= alpha; acc0[i][2] *= alpha; acc0[i][3] *= alpha;
+        }
+        if constexpr (TWO) {
+#pragma unroll
+          for (int i = 0; i < G1c::NKB; ++i) {
+            acc1[i][0] *= alpha; acc1[i][1] *= alpha; acc1[i][2] *= alpha; acc1[i][3] *= alpha;
+          }
+        }
+      }
+      const float pa = exp2f(la - m_run), pb = exp2f(lb - m_run);
+      l_run += pa + pb;
+      auto pfrag = [&](float na, float nb, uint32_t& b0, uint32_t& b1) {
+        const float wa = pa * na, wb = pb * nb;
+        const float ha = __half2float(__float2half_rn(wa)), hb = __half2float(__float2half_rn(wb));
+        b0 = movT(pack_h2(ha, wa - ha));
+        b1 = movT(pack_h2(hb, wb - hb));
+      };
+      uint32_t pb0, pb1;
+      pfrag(h2f(c0.nva), h2f(c0.nvb), pb0, pb1);
+      group_values<G0>(vl0, c0.va, c0.vb, pb0, pb1, acc0);
+      if constexpr (TWO) {
+        pfrag(h2f(c1.nva), h2f(c1.nvb), pb0, pb1);
+        group_values<G1c>(vl1, c1.va, c1.vb, pb0, pb1, acc1);
+      }
     }
-  };
-  store_acc(acc0, G0{}, A.g[0].off);
-  if constexpr (TWO) store_acc(acc1, G1c{}, A.g[1].off);
+    // ---- warp state -> shared memory (lane (g, l) holds head l)
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 4);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 8);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
+    if (g == 0) {
+      s_m[warp][l] = m_run;
+      s_l[warp][l] = l_run;
+    }
+    auto store_acc = [&](auto& acc, auto gc_tag, int off) {
+      using GC = decltype(gc_tag);
+#pragma unroll
+      for (int mb = 0; mb < GC::NKB; ++mb) {
+        const int qq = mb & 3, hh = mb >> 2;
+        const int c0_ = GC::Q * (g >> 1) + qq + 16 * hh + 4 * (g & 1);   // row g: block f = 0
+        s_acc[warp][l][off + c0_] = acc[mb][0] + acc[mb][1];
+        s_acc[warp][l][off + c0_ + 8] = acc[mb][2] + acc[mb][3];          // row g+8: block f = 1
+      }
+    };
+    store_acc(acc0, G0{}, A.g[0].off);
+    if constexpr (TWO) store_acc(acc1, G1c{}, A.g[1].off);
+  }
   __syncthreads();
   // ---- merge the warps: one partial per (query head, split); m in natural-log units
   const float ln2 = 0.69314718055994531f;
@@ -422,115 +572,143 @@ __global__ void __launch_bounds__(kWarps * 32) decode_mma_kernel(MmaArgs A) {
     }
     dst[2 + c] = acc;
   }
-  // ---- the last split of this (sequence, kv head) to finish merges all splits
-  __threadfence();
+  // the merge kernel (launched programmatically behind this one) may start once every
+  // CTA has written its partial
   __syncthreads();
-  if (threadIdx.x == 0) s_last = (atomicAdd(A.done + bh, 1) == A.nsplit - 1) ? 1 : 0;
+  allow_dependent_launch();
+}
+
+// (Pi q, S q) of the kRep query heads of one (sequence, kv head), 64 outputs per CTA
+// (blockIdx.y selects them; outputs o < d_g are Pi q, the rest S q): the 64 needed
+// columns of Pi^T or S^T are staged in shared memory with 16-byte loads, then thread
+// (head, o) takes its dot product from shared memory.
+template <typename T>
+__global__ void __launch_bounds__(256) decode_prep_kernel(const T* __restrict__ q, int D, int off, int dg,
+                                                          const float* __restrict__ PiT, const float* __restrict__ ST,
+                                                          float* __restrict__ qprep, int G, int gi, int qp_ld) {
+  __shared__ __align__(16) float ms[128 * 64];
+  __shared__ float qs[kRep][128];
+  allow_dependent_launch();
+  const int grp = blockIdx.x;                    // = b * Hkv + hk; rows grp*kRep .. +kRep-1
+  const int o0 = blockIdx.y * 64;                // first output of this CTA
+  const float* M = o0 < dg ? PiT + o0 : ST + (o0 - dg);
+  float4* m4 = reinterpret_cast<float4*>(ms);
+#pragma unroll 8
+  for (int e = threadIdx.x; e < dg * 16; e += blockDim.x) {     // dg rows x 16 float4
+    const int j = e >> 4, c4 = e & 15;
+    m4[e] = __ldg(reinterpret_cast<const float4*>(M + (size_t)j * dg) + c4);
+  }
+  for (int e = threadIdx.x; e < kRep * dg; e += blockDim.x) {
+    const int h = e / dg, j = e % dg;
+    const size_t at = (size_t)(grp * kRep + h) * D + off + j;
+    if constexpr (std::is_same<T, float>::value) qs[h][j] = q[at];
+    else qs[h][j] = __bfloat162float(q[at]);
+  }
   __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  float* wts = &s_acc[0][0][0];                  // reuse: [kRep][nsplit] weights (nsplit <= 512)
-  float* rot = &s_acc[2][0][0];                  // [kRep][D] merged rotated-basis accumulators
-  for (int h = warp; h < kRep; h += kWarps) {
-    const float* P = A.part + (size_t)(b * A.Hq + hk * kRep + h) * A.nsplit * (A.D + 2);
+  const int h = threadIdx.x >> 6, oc = threadIdx.x & 63;
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll 8
+  for (int j = 0; j < dg; j += 2) {
+    a0 = fmaf(ms[j * 64 + oc], qs[h][j], a0);
+    a1 = fmaf(ms[(j + 1) * 64 + oc], qs[h][j + 1], a1);
+  }
+  qprep[((size_t)(grp * kRep + h) * G + gi) * 2 * qp_ld + o0 + oc] = a0 + a1;
+}
+
+// Log-sum-exp merge of the context splits and the inverse rotation of the value groups:
+// one CTA per (query row, 64 output channels).  The merged rotated-basis accumulator of
+// the row is built in shared memory (all splits' loads independent), then thread
+// (output, quarter) sums a quarter of o[c] = sum_i Pi_v[i][c - off] acc[off + i].
+struct Merge2Args {
+  const float* part;
+  int nsplit, D, G;
+  int off[3];
+  const float* PiV[2];
+  float* out;
+};
+
+__global__ void __launch_bounds__(256) decode_merge_mma_kernel(Merge2Args A) {
+  __shared__ float w[512];
+  __shared__ float acc[256];
+  __shared__ float red[4][64];
+  __shared__ float part2[2][256];
+  grid_dependency_wait();
+  const int row = blockIdx.x, c0 = blockIdx.y * 64;
+  const int D = A.D, ns = A.nsplit;
+  const float* P = A.part + (size_t)row * ns * (D + 2);
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
     float M = -INFINITY;
-    for (int s = lane; s < A.nsplit; s += 32) M = fmaxf(M, __ldcg(P + (size_t)s * (A.D + 2)));
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, P[(size_t)s * (D + 2)]);
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.f;
-    for (int s = lane; s < A.nsplit; s += 32) {
-      const float ms = __ldcg(P + (size_t)s * (A.D + 2));
-      const float w = (ms == -INFINITY) ? 0.f : __expf(ms - M);
-      wts[h * 512 + s] = w;
-      L += w * __ldcg(P + (size_t)s * (A.D + 2) + 1);
+    for (int s = lane; s < ns; s += 32) {
+      const float ms = P[(size_t)s * (D + 2)];
+      const float f = (ms == -INFINITY) ? 0.f : __expf(ms - M);
+      w[s] = f;
+      L += f * P[(size_t)s * (D + 2) + 1];
     }
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
     const float inv = L > 0.f ? 1.f / L : 0.f;
     __syncwarp();
-    for (int s = lane; s < A.nsplit; s += 32) wts[h * 512 + s] *= inv;
+    for (int s = lane; s < ns; s += 32) w[s] *= inv;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < kRep * A.D; e += blockDim.x) {
-    const int h = e / A.D, c = e % A.D;
-    const float* P = A.part + (size_t)(b * A.Hq + hk * kRep + h) * A.nsplit * (A.D + 2) + 2 + c;
-    float a0 = 0.f, a1 = 0.f;
-    int s = 0;
-    for (; s + 1 < A.nsplit; s += 2) {
-      a0 = fmaf(wts[h * 512 + s], __ldcg(P + (size_t)s * (A.D + 2)), a0);
-      a1 = fmaf(wts[h * 512 + s + 1], __ldcg(P + (size_t)(s + 1) * (A.D + 2)), a1);
+  // every split's contribution is an independent load: keep 16 of them in flight per thread
+  {
+    const int nthr = blockDim.x;
+    const int halves = nthr / D > 1 ? nthr / D : 1;     // threads per coordinate
+    const int i = threadIdx.x % D, hsel = threadIdx.x / D;
+    float a[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) a[u] = 0.f;
+    if (hsel < halves) {
+      for (int s0 = hsel * 16; s0 < ns; s0 += 16 * halves) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (s0 + u < ns) a[u] = fmaf(w[s0 + u], P[(size_t)(s0 + u) * (D + 2) + 2 + i], a[u]);
+      }
     }
-    if (s < A.nsplit) a0 = fmaf(wts[h * 512 + s], __ldcg(P + (size_t)s * (A.D + 2)), a0);
-    rot[h * 256 + c] = a0 + a1;
+    float t = 0.f;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) t += a[u];
+    if (hsel < halves) part2[hsel][i] = t;
+    __syncthreads();
+    if (hsel == 0) {
+      float sum = 0.f;
+      for (int h = 0; h < halves; ++h) sum += part2[h][i];
+      acc[i] = sum;
+    }
   }
   __syncthreads();
-  // o = Pi_v^T acc per group: o[off+j] = sum_i Pi_v[i][j] acc[off+i]
-  for (int c = threadIdx.x; c < A.D; c += blockDim.x) {
-    const int gi = (A.G > 1 && c >= A.g[1].off) ? 1 : 0;
-    const MmaGroup& gr = A.g[gi];
-    const int dg = (gi == 0) ? (A.G > 1 ? A.g[1].off : A.D) : A.D - gr.off;
-    const int j = c - gr.off;
-    float o[kRep] = {0.f, 0.f, 0.f, 0.f};
-    const float* Pi = gr.PiV + j;
+  const int oc = threadIdx.x & 63, qtr = threadIdx.x >> 6;
+  const int c = c0 + oc;
+  float o = 0.f;
+  if (c < D) {
+    const int gi = (A.G > 1 && c >= A.off[1]) ? 1 : 0;
+    const int off = A.off[gi], dg = A.off[gi + 1] - off, j = c - off;
+    const float* Pi = A.PiV[gi] + j;
+    const int i0 = qtr * (dg / 4), i1 = i0 + dg / 4;
 #pragma unroll 8
-    for (int i = 0; i < dg; ++i) {
-      const float p = __ldg(Pi + (size_t)i * dg);
-#pragma unroll
-      for (int h = 0; h < kRep; ++h) o[h] = fmaf(p, rot[h * 256 + gr.off + i], o[h]);
-    }
-#pragma unroll
-    for (int h = 0; h < kRep; ++h) A.out[(size_t)(b * A.Hq + hk * kRep + h) * A.D + c] = o[h];
+    for (int i = i0; i < i1; ++i) o = fmaf(__ldg(Pi + (size_t)i * dg), acc[off + i], o);
   }
-}
-
-// (Pi q, S q) for a 32-row x 32-output tile of the prepared-query matrix per CTA (the
-// rows are the B*Hq query rows, the outputs the 2*d_g coordinates of Pi q and S q);
-// CTA (0, 0) of group 0 also clears the completion counters.
-template <typename T>
-__global__ void __launch_bounds__(256) decode_prep_kernel(const T* __restrict__ q, int rows, int D, int off, int dg,
-                                                          const float* __restrict__ PiT, const float* __restrict__ ST,
-                                                          float* __restrict__ qprep, int G, int gi, int qp_ld,
-                                                          int* __restrict__ done, int ndone) {
-  __shared__ float qs[32][129];
-  __shared__ float ms[128][33];
-  allow_dependent_launch();
-  const int o0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
-  if (blockIdx.x == 0 && blockIdx.y == 0 && gi == 0)
-    for (int i = threadIdx.x; i < ndone; i += blockDim.x) done[i] = 0;
-  for (int e = threadIdx.x; e < 32 * dg; e += blockDim.x) {
-    const int r = e / dg, j = e % dg;
-    float v = 0.f;
-    if (r0 + r < rows) {
-      if constexpr (std::is_same<T, float>::value) v = q[(size_t)(r0 + r) * D + off + j];
-      else v = __bfloat162float(q[(size_t)(r0 + r) * D + off + j]);
-    }
-    qs[r][j] = v;
-  }
-  for (int e = threadIdx.x; e < 32 * dg; e += blockDim.x) {
-    const int j = e / 32, c = e % 32, o = o0 + c;
-    float v = 0.f;
-    if (o < dg) v = __ldg(PiT + (size_t)j * dg + o);
-    else if (o < 2 * dg) v = __ldg(ST + (size_t)j * dg + (o - dg));
-    ms[j][c] = v;
-  }
+  red[qtr][oc] = o;
   __syncthreads();
-  const int r = threadIdx.x >> 3, c0 = (threadIdx.x & 7) * 4;
-  float a[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int j = 0; j < dg; ++j) {
-    const float x = qs[r][j];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] = fmaf(ms[j][c0 + i], x, a[i]);
-  }
-  if (r0 + r < rows)
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (o0 + c0 + i < 2 * dg) qprep[((size_t)(r0 + r) * G + gi) * 2 * qp_ld + o0 + c0 + i] = a[i];
+  if (qtr == 0 && c < D)
+    A.out[(size_t)row * D + c] = (red[0][oc] + red[1][oc]) + (red[2][oc] + red[3][oc]);
 }
 
 template <class G0, class G1>
 int launch_mma_t(const MmaArgs& A, int nsplit, int BHkv, cudaStream_t st) {
+  constexpr bool TWO = !std::is_same<G1, void>::value;
+  using G1c = typename std::conditional<TWO, G1, G0>::type;
+  const int dyn = kNStage * Stage<G0, G1c, TWO>::BYTES;
+  cudaError_t ea = cudaFuncSetAttribute(decode_mma_kernel<G0, G1>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+  if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncSetAttribute(decode_mma_kernel)");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nsplit, BHkv);
-  cfg.blockDim = dim3(kWarps * 32);
-  cfg.dynamicSmemBytes = 0;
+  cfg.blockDim = dim3((kWarps + 1) * 32);
+  cfg.dynamicSmemBytes = dyn;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -585,17 +763,15 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
   char* base = static_cast<char*>(ws);
   float* qprep = reinterpret_cast<float*>(base + W.qp);
   float* part = reinterpret_cast<float*>(base + W.part);
-  int* done = reinterpret_cast<int*>(base + W.cnt);
   for (int g = 0; g < G; ++g) {
     const int dg = kctx[g]->lay.d;
-    const dim3 pgrid(div_up(2 * dg, 32), div_up(B * Hq, 32));
+    const dim3 pgrid(B * Hkv, 2 * dg / 64);
     if (q_dtype == TQ_DTYPE_F32)
-      decode_prep_kernel<float><<<pgrid, 256, 0, st>>>(static_cast<const float*>(q), B * Hq, D, off[g], dg,
-                                                       kctx[g]->PiT, kctx[g]->ST, qprep, G, g, D, done, B * Hkv);
+      decode_prep_kernel<float><<<pgrid, 256, 0, st>>>(static_cast<const float*>(q), D, off[g], dg, kctx[g]->PiT,
+                                                       kctx[g]->ST, qprep, G, g, D);
     else
-      decode_prep_kernel<__nv_bfloat16><<<pgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), B * Hq, D, off[g],
-                                                               dg, kctx[g]->PiT, kctx[g]->ST, qprep, G, g, D, done,
-                                                               B * Hkv);
+      decode_prep_kernel<__nv_bfloat16><<<pgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), D, off[g], dg,
+                                                               kctx[g]->PiT, kctx[g]->ST, qprep, G, g, D);
     count_launch();
     int r = check_launch("decode_prep_kernel");
     if (r != TQ_OK) return r;
@@ -603,7 +779,7 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
   MmaArgs A{};
   A.B = B; A.Hq = Hq; A.Hkv = Hkv; A.D = D; A.nsplit = W.nsplit; A.chunk = W.chunk; A.qp_ld = D; A.G = G;
   A.max_len = max_len; A.scale_log2 = scale * 1.4426950408889634f; A.seq_lens = seq_lens; A.qprep = qprep;
-  A.part = part; A.done = done; A.out = out;
+  A.part = part; A.out = out;
   for (int g = 0; g < G; ++g) {
     MmaGroup& gr = A.g[g];
     gr.kcodes = kc[g].codes; gr.knorm = kc[g].norm; gr.krnorm = kc[g].rnorm;
@@ -615,11 +791,33 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
     gr.off = off[g];
     gr.kbytes = kctx[g]->lay.code_bytes;
     gr.vbytes = vctx[g]->lay.code_bytes;
+    gr.kcap = kc[g].cap;
+    gr.vcap = vc[g].cap;
   }
-  if (G == 1 && sig[0] == 12834) return launch_mma_t<C128_34, void>(A, W.nsplit, B * Hkv, st);
-  if (G == 1) return launch_mma_t<C128_23, void>(A, W.nsplit, B * Hkv, st);
-  if (is(6434, 6423)) return launch_mma_t<C64_34, C64_23>(A, W.nsplit, B * Hkv, st);
-  return launch_mma_t<C64_23, C64_12>(A, W.nsplit, B * Hkv, st);
+  A.err = kctx[0]->dev_err;
+  int r;
+  if (G == 1 && sig[0] == 12834) r = launch_mma_t<C128_34, void>(A, W.nsplit, B * Hkv, st);
+  else if (G == 1) r = launch_mma_t<C128_23, void>(A, W.nsplit, B * Hkv, st);
+  else if (is(6434, 6423)) r = launch_mma_t<C64_34, C64_23>(A, W.nsplit, B * Hkv, st);
+  else r = launch_mma_t<C64_23, C64_12>(A, W.nsplit, B * Hkv, st);
+  if (r != TQ_OK) return r;
+  Merge2Args M{};
+  M.part = part; M.nsplit = W.nsplit; M.D = D; M.G = G; M.out = out;
+  for (int g = 0; g < G; ++g) { M.off[g] = off[g]; M.PiV[g] = vctx[g]->Pi; }
+  M.off[G] = D;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(B * Hq, div_up(D, 64));
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_merge_mma_kernel, M);
+  count_launch();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(decode_merge_mma_kernel)");
+  return check_launch("decode_merge_mma_kernel");
 }
 
 }  // namespace tq
