@@ -33,21 +33,28 @@
  * Packed code layout (produced by tq_quantize_kv, read by every other call)
  *   A context with dimension d, MSE bits k (k = bits-1 in prod mode, k = bits in MSE
  *   mode) stores each vector as
- *     - P bit planes over d_pad = 32*ceil(d/32) coordinate positions, P = k+1 in prod
- *       mode (k index planes, then 1 sign plane), P = k in MSE mode;
+ *     - a P-bit code per coordinate, P = k+1 in prod mode, P = k in MSE mode, packed
+ *       into code_bytes = P*d_pad/8 bytes with d_pad = 32*ceil(d/32);
  *     - fp16 norm ||x|| (and, prod mode, fp16 residual norm ||r||) in separate arrays.
- *   The code record of one vector is code_bytes = P*d_pad/8 bytes, divided into 4
- *   quarters of P*d_pad/32 bytes.  Quarter q holds coordinate positions
- *   [q*d_pad/4, (q+1)*d_pad/4); inside a quarter, plane p occupies the d_pad/32 bytes at
- *   offset p*d_pad/32, and bit b of that chunk (bit b%8 of byte b/8, LSB first) belongs
- *   to position q*d_pad/4 + b.  So for plane p and position i:
- *       byte = (i / (d_pad/4)) * (P*d_pad/32) + p*(d_pad/32) + (i % (d_pad/4)) / 8
- *       bit  = (i % (d_pad/4)) % 8
- *   Index plane p (p < k) holds bit p of idx_i, the codebook index of rotated
- *   coordinate y_i (binary, LSB = plane 0; centroids are sorted ascending).  The sign
- *   plane (p = k, prod mode) holds s_j = [(S r)_j >= 0] for projection row j.
- *   Positions i >= d are zero.  Slot t of a tq_packed buffer starts at
- *   codes + t*code_bytes.
+ *   Code of coordinate i.  With K = 2^k levels (centroids sorted ascending, c[K-1-j] =
+ *   -c[j]) the index idx_i of rotated coordinate y_i is stored in sign-magnitude form:
+ *   bit k-1 is the negative-half flag n = [idx < K/2], bits 0..k-2 the magnitude rank
+ *   m = n ? K/2-1-idx : idx-K/2 (so c[idx] = (n ? -1 : +1) * c[K/2+m]).  For k = 1 the
+ *   code is n alone.  In prod mode bit k holds the QJL sign s_i = [(S r)_i >= 0].  Bit
+ *   P-1 is called the top bit.
+ *   Record.  d_pad/32 groups of P little-endian 32-bit words; group g holds coordinates
+ *   32g .. 32g+31.  Inside a group, coordinate e = 8s + j (slice s = 0..3, j = 4h + t
+ *   with half h = 0..1, t = 0..3) keeps code bit b at (word, bit):
+ *       P = 1:  top        -> (0, E)          E = 8t + 7 - (2s + h)
+ *       P = 2:  bit 0      -> (0, 4j + s);                     top -> (1, E)
+ *       P = 3:  bits 0, 1  -> (s & 1, 4j + 2*(s >> 1) + b);    top -> (2, E)
+ *       P = 4:  bits 0..2  -> (s, 4j + b);   top -> (s, 8t + 7) if h = 0, (s, 8t + 3) if h = 1
+ *       P = 5:  bits 0..3 as for P = 4 (bit 3 in the P = 4 top place);  top -> (4, E)
+ *   This places, for every slice, the low code bits of four consecutive coordinates as
+ *   nibbles of one 16-bit half-word and their top bits as the most significant bits of
+ *   four bytes (after one left shift), which is what the decode kernels' byte-permute
+ *   table lookups consume.  Coordinates i >= d have code 0.  Slot t of a tq_packed buffer
+ *   starts at codes + t*code_bytes.
  */
 #ifndef TQ_H
 #define TQ_H
@@ -95,7 +102,7 @@ typedef struct tq_info {
   int k;          /* MSE index bits: bits-1 (prod) or bits (MSE) */
   int m;          /* QJL projection rows (= d in prod mode, 0 in MSE mode) */
   int mode;       /* TQ_MODE_* */
-  int planes;     /* P: bit planes per vector */
+  int planes;     /* P: code bits per coordinate */
   int d_pad;      /* 32*ceil(d/32) */
   int code_bytes; /* P*d_pad/8 */
   uint64_t seed;

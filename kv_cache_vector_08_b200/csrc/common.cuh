@@ -20,21 +20,49 @@ constexpr int kMaxLevels = 16;  // 2^k for k <= 4
 struct Codebook {
   float c[kMaxLevels];      // centroids, ascending
   float t[kMaxLevels];      // boundaries (K-1 used); t[K-1..] = +inf
+  float cc[kMaxLevels];     // centroid of each sign-magnitude index code (see index_code)
   int K;                    // 2^k
 };
 
 struct Layout {
-  int d, d_pad, k, planes, code_bytes;
-  int quarter;              // d_pad / 4 coordinate positions per quarter
-  int chunk;                // d_pad / 32 bytes per plane inside a quarter
-  int qbytes;               // planes * chunk bytes per quarter
+  int d, d_pad, k, planes, code_bytes;   // planes = P code bits per coordinate
 };
 
-// Byte offset, inside one vector's record, of the byte holding plane p of positions
-// [i, i+8) (i a multiple of 8).
-__host__ __device__ inline int plane_byte(const Layout& L, int p, int i) {
-  int q = i / L.quarter;
-  return q * L.qbytes + p * L.chunk + (i - q * L.quarter) / 8;
+// Sign-magnitude code of a k-bit codebook index (the packed-code convention): bit k-1 is
+// the negative-half flag [idx < K/2], the low bits the magnitude rank counted from the
+// centre of the (odd-symmetric) codebook; for k = 1 the code is the flag alone.
+__host__ __device__ inline uint32_t index_code(int idx, int k) {
+  const int half = 1 << (k - 1);
+  if (k == 1) return idx == 0 ? 1u : 0u;
+  const bool neg = idx < half;
+  return ((neg ? 1u : 0u) << (k - 1)) | (uint32_t)(neg ? half - 1 - idx : idx - half);
+}
+__host__ __device__ inline int code_index(uint32_t code, int k) {
+  const int half = 1 << (k - 1);
+  if (k == 1) return (code & 1u) ? 0 : 1;
+  const int m = (int)(code & (uint32_t)(half - 1));
+  return ((code >> (k - 1)) & 1u) ? half - 1 - m : half + m;
+}
+
+// Position of code bit b of coordinate e (0..31) of a 32-coordinate group with P-bit
+// codes, as 32 * word + bit (the record layout stated with the packed format).
+__host__ __device__ constexpr int code_bit_pos(int P, int e, int b) {
+  return P == 1 ? (8 * ((e & 7) & 3) + 7 - (2 * (e >> 3) + ((e & 7) >> 2)))
+       : (b == P - 1 && P != 4) ? 32 * (P - 1) + (8 * ((e & 7) & 3) + 7 - (2 * (e >> 3) + ((e & 7) >> 2)))
+       : P == 2 ? 4 * (e & 7) + (e >> 3)
+       : P == 3 ? 32 * ((e >> 3) & 1) + 4 * (e & 7) + 2 * (e >> 4) + b
+       : b == 3 ? 32 * (e >> 3) + ((((e & 7) >> 2) == 0) ? 8 * (e & 3) + 7 : 8 * (e & 3) + 3)
+       : 32 * (e >> 3) + 4 * (e & 7) + b;
+}
+
+// P-bit code of coordinate e of a group whose P words are in w.
+__device__ __forceinline__ uint32_t group_code(const uint32_t* w, int P, int e) {
+  uint32_t c = 0;
+  for (int b = 0; b < P; ++b) {
+    const int q = code_bit_pos(P, e, b);
+    c |= ((w[q >> 5] >> (q & 31)) & 1u) << b;
+  }
+  return c;
 }
 
 }  // namespace tq
@@ -46,6 +74,7 @@ struct tq_ctx {
   tq::Codebook cb{};
   int m = 0, mode = 0, bits = 0;
   float sqrt_pi_over_2_over_m = 0.f;  // QJL unbiasing constant sqrt(pi/2)/m
+  float s_rowmax = 0.f;               // max_j ||S_j||: bounds |(S q)_j| by s_rowmax * ||q||
   // device float32 copies (row-major)
   float* Pi = nullptr;    // [d][d]    y = Pi x
   float* PiT = nullptr;   // [d][d]    Pi^T (coalesced column access)

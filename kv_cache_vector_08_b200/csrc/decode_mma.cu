@@ -3,24 +3,32 @@
 // turboquant.net "集成到 Attention": keys and values stay quantized and attention reads
 // them directly; admirer.cn (H100 paragraph): the attention-logit computation on 4-bit
 // keys is where the speed-up is measured.  Per cached token and GQA group of query heads
-// the work is a small dense contraction (4 heads x 128 coordinates for the MSE term, the
-// QJL sign term and the value accumulation), so each warp runs it on mma.sync m16n8k16:
+// the work is a small contraction (4 heads x d coordinates for the MSE term, the QJL sign
+// term and the value accumulation), so each warp runs it on mma.sync over 16-token tiles:
 //
-//   logits^T [16 tokens x 8] = Ck [16 x 16k] * [q~_hi | q~_lo]      (MSE term, 4 heads)
-//                            + Sk [16 x 16k] * [q^_hi | q^_lo]      (QJL term, +-1 signs)
-//   out^T   [16 coords x 8]  += Cv^T [16 x 16 tokens] * [P_hi | P_lo]
+//   keys (int8, m16n8k32):  [16 tokens x 32 coords] x [32 coords x 8]
+//      MSE term  C_hi * Q~ + C_lo * Q~    centroids as two int8 digits of a 16-bit fixed
+//                                          point, the prepared query Pi q as two int8
+//                                          digits in the 8 columns (4 heads x hi/lo)
+//      QJL term  A_s * Q^                 A_s = -[sign bit], from one sign-replicating
+//                                          byte permute per 4 coordinates
+//   values (fp16, m16n8k16): out^T [16 coords x 8] += Cv^T [16 x 16 tokens] * [P_hi | P_lo]
 //
-// The A operands are produced straight from the packed bit planes in registers: the
-// bit planes of four coordinates form a prmt selector that looks the fp16 centroid
-// bytes up in register-resident tables (4 lookups per prmt); signs become +-1.0 with one
-// shift and one LOP3 per pair; the value tile is turned around with movmatrix.  The hi/lo
-// halves of the queries and of the probabilities ride in the 8 columns of each MMA, so the
-// fp16 rounding of the queries and probabilities costs no extra MMA.  Centroids are used
-// at fp16 precision (relative error <= 2^-11), well inside the output tolerance.
+// The A operands come straight from the packed words: for every 8-coordinate slice the
+// low code bits are nibbles of one word (one AND gives four byte-permute selectors) and
+// the top bits sit at byte msbs after at most one shift, so a 4-entry byte lookup costs
+// one prmt.  Keys: the two centroid digits are two lookups, the sign bytes one prmt.
+// Values: magnitude bytes are looked up (low and high byte of the fp16 magnitude), the
+// negative flag is XORed into the sign bit, two prmt interleave the bytes, movmatrix turns
+// the 8x8 blocks around.  Integer products are exact; the fixed-point scales (|q| bound
+// for the query, max |c| for the centroids) keep every digit in range, so the logits carry
+// only the 2^-15 rounding of the two fixed-point operands.
 //
-// One CTA (4 warps) handles one (sequence, kv head, context split); warps take 16-token
-// tiles in turn, keep an online softmax (log2 domain) per head, and merge their states in
-// shared memory before writing one partial (m, l, acc) per query head and split.
+// One CTA (4 consumer warps + 1 producer warp) handles one (sequence, kv head, context
+// split).  The producer stages 64 tokens of K/V code bytes and norms per pipeline stage
+// with bulk copies; consumer warps take one 16-token tile of every stage, keep an online
+// softmax (log2 domain) per head, and merge their states in shared memory before writing
+// one partial (m, l, acc) per query head and split.
 #include <cfloat>
 #include <type_traits>
 
@@ -34,7 +42,15 @@ namespace {
 using namespace sm100;
 
 constexpr int kWarps = 4;
-constexpr int kRep = 4;   // query heads per kv head handled by this kernel
+constexpr int kRep = 4;            // query heads per kv head handled by this kernel
+constexpr float kFix = 32000.f;    // fixed-point range of queries and key centroids (< 2^15)
+
+__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -49,118 +65,91 @@ __device__ __forceinline__ uint32_t movT(uint32_t x) {
   return y;
 }
 
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// 0xFF in every byte whose msb is set, 0x00 elsewhere (prmt sign replication)
+__device__ __forceinline__ uint32_t msb_bytes(uint32_t x) { return prmt(x, x, 0xBA98u); }
+
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
 // Static description of one channel group handled by the kernel.
-template <int DG_, int KK_, int KV_>
+template <int DG_, int PK_, int PV_>
 struct GroupCfg {
   static constexpr int DG = DG_;            // group width (64 or 128)
-  static constexpr int Q = DG_ / 4;         // coordinates per quarter
-  static constexpr int KK = KK_;            // key index bits (prod mode)
-  static constexpr int KV = KV_;            // value index bits (MSE mode)
-  static constexpr int PK = KK_ + 1;        // key planes
-  static constexpr int PV = KV_;            // value planes
-  static constexpr int NKB = DG_ / 16;      // 16-coordinate k-blocks
-  static constexpr uint32_t M1 = (Q == 32) ? 0x11111111u : 0x1111u;
+  static constexpr int PK = PK_;            // key code bits (MSE index bits + QJL sign)
+  static constexpr int PV = PV_;            // value code bits
+  static constexpr int NS = DG_ / 32;       // 8-coordinate slices per thread
+  static constexpr int CQ = DG_ / 4;        // coordinates per thread
+  static constexpr int KB = PK_ * DG_ / 8;  // key record bytes
+  static constexpr int VB = PV_ * DG_ / 8;  // value record bytes
 };
 
-// Quarter l of one record: planes as 32-bit words (16 valid bits when Q = 16).
-template <int Q, int P>
-__device__ __forceinline__ void load_quarter(const uint8_t* rec, int l, uint32_t (&w)[P]) {
-  if constexpr (Q == 32) {
-    const uint8_t* p = rec + l * (4 * P);
-    if constexpr (P == 4) {
-      uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-      w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-    } else if constexpr (P == 2) {
-      uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
-      w[0] = v.x; w[1] = v.y;
-    } else {
-#pragma unroll
-      for (int i = 0; i < P; ++i) w[i] = __ldg(reinterpret_cast<const uint32_t*>(p) + i);
-    }
-  } else {
-    const uint8_t* p = rec + l * (2 * P);
-    if constexpr (P == 4) {
-      uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
-      w[0] = v.x & 0xFFFFu; w[1] = v.x >> 16; w[2] = v.y & 0xFFFFu; w[3] = v.y >> 16;
-    } else if constexpr (P == 2) {
-      uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(p));
-      w[0] = v & 0xFFFFu; w[1] = v >> 16;
-    } else {
-#pragma unroll
-      for (int i = 0; i < P; ++i) w[i] = __ldg(reinterpret_cast<const unsigned short*>(p) + i);
-    }
-  }
-}
-
-// Same, from a record staged in shared memory (byte offset of the record arbitrary: the
-// staged copy keeps the global alignment of each record modulo 16).
-template <int Q, int P>
-__device__ __forceinline__ void lds_quarter(const uint8_t* rec, int l, uint32_t (&w)[P]) {
-  if constexpr (Q == 32) {
-    const uint8_t* p = rec + l * (4 * P);
-    if constexpr (P == 4) {
-      uint4 v = *reinterpret_cast<const uint4*>(p);
-      w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-    } else if constexpr (P == 2) {
-      uint2 v = *reinterpret_cast<const uint2*>(p);
-      w[0] = v.x; w[1] = v.y;
-    } else {
-#pragma unroll
-      for (int i = 0; i < P; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
-    }
-  } else {
-    const uint8_t* p = rec + l * (2 * P);
-    if constexpr (P == 4) {
-      uint2 v = *reinterpret_cast<const uint2*>(p);
-      w[0] = v.x & 0xFFFFu; w[1] = v.x >> 16; w[2] = v.y & 0xFFFFu; w[3] = v.y >> 16;
-    } else if constexpr (P == 2) {
-      uint32_t v = *reinterpret_cast<const uint32_t*>(p);
-      w[0] = v & 0xFFFFu; w[1] = v >> 16;
-    } else {
-#pragma unroll
-      for (int i = 0; i < P; ++i) w[i] = reinterpret_cast<const unsigned short*>(p)[i];
-    }
-  }
-}
-
-// prmt selector nibbles (3 index bits) for coordinates 4k + qq of a quarter.
-template <int NB, uint32_t M1>
-__device__ __forceinline__ uint32_t selector(const uint32_t* w, int qq) {
-  uint32_t s = (w[0] >> qq) & M1;
-  if constexpr (NB > 1) s |= ((w[1] >> qq) & M1) << 1;
-  if constexpr (NB > 2) s |= ((w[2] >> qq) & M1) << 2;
-  return s;
-}
-
-// fp16 centroid table split into low/high bytes, 8 entries per register pair (built on
-// the host from the context's codebook).
-struct Lut {
-  uint32_t lo[4], hi[4];  // lo[0..1]: low bytes of c[0..7], lo[2..3]: of c[8..15]
+// The words of one record a thread needs: d = 128, its own 32-coordinate block (P words);
+// d = 64 with P = 4, its two slices' words; d = 64 otherwise, the block it shares with its
+// neighbour (P words), pre-shifted so that slice u of this thread reads like slice u of a
+// d = 128 block (the shared words interleave the two threads' slices).
+template <int DG, int P>
+struct Words {
+  static constexpr int N = (DG == 64 && P == 4) ? 2 : P;
+  uint32_t w[N];
 };
 
-// Two half2 registers: fp16 centroids of the coordinates selected by the 4 nibbles of
-// `sel` (pairs nibble 0,1 and nibble 2,3).  NB index bits; the 4th bit (NB == 4) chooses
-// between the two 8-entry tables through `sel4` (nibble k = k + 4*b3_k).
-template <int NB>
-__device__ __forceinline__ void lookup(const Lut& t, uint32_t sel, uint32_t sel4, uint32_t& x01, uint32_t& x23) {
-  uint32_t L, H;
-  if constexpr (NB <= 3) {
-    L = __byte_perm(t.lo[0], t.lo[1], sel);
-    H = __byte_perm(t.hi[0], t.hi[1], sel);
+template <int DG, int P>
+__device__ __forceinline__ void lds_words(Words<DG, P>& r, const uint8_t* rec, int l) {
+  if constexpr (DG == 128 && P == 4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(rec + 16 * l);
+    r.w[0] = v.x; r.w[1] = v.y; r.w[2] = v.z; r.w[3] = v.w;
+  } else if constexpr (DG == 64 && P == 4) {
+    const uint2 v = *reinterpret_cast<const uint2*>(rec + 8 * l);
+    r.w[0] = v.x; r.w[1] = v.y;
+  } else if constexpr (DG == 128) {
+    const uint32_t* p = reinterpret_cast<const uint32_t*>(rec + 4 * P * l);
+#pragma unroll
+    for (int i = 0; i < P; ++i) r.w[i] = p[i];
   } else {
-    uint32_t La = __byte_perm(t.lo[0], t.lo[1], sel), Lb = __byte_perm(t.lo[2], t.lo[3], sel);
-    uint32_t Ha = __byte_perm(t.hi[0], t.hi[1], sel), Hb = __byte_perm(t.hi[2], t.hi[3], sel);
-    L = __byte_perm(La, Lb, sel4);
-    H = __byte_perm(Ha, Hb, sel4);
+    const uint32_t* p = reinterpret_cast<const uint32_t*>(rec + 4 * P * (l >> 1));
+#pragma unroll
+    for (int i = 0; i < P; ++i) r.w[i] = p[i];
+    const int odd = l & 1;                    // this thread's slices are 2*odd, 2*odd+1
+    if constexpr (P == 3) {
+      r.w[0] >>= 2 * odd;
+      r.w[1] >>= 2 * odd;
+    } else {
+      r.w[0] >>= 2 * odd;
+    }
+    r.w[P - 1] <<= 4 * odd;
   }
-  x01 = __byte_perm(L, H, 0x5140);
-  x23 = __byte_perm(L, H, 0x7362);
 }
+
+// Byte-permute selectors (low code bits) of slice u: nibbles 0-3 = coordinates 8u..8u+3,
+// nibbles 4-7 = 8u+4..8u+7 of this thread.
+template <int DG, int P>
+__device__ __forceinline__ uint32_t low_sel(const Words<DG, P>& r, int u) {
+  if constexpr (P == 4) return r.w[u] & 0x77777777u;
+  else if constexpr (P == 3) return (r.w[u & 1] >> (2 * (u >> 1))) & 0x33333333u;
+  else return (r.w[0] >> u) & 0x11111111u;
+}
+
+// Top code bits of slice u, half h (coordinates 8u + 4h + t) at the msbs of bytes t.
+template <int DG, int P>
+__device__ __forceinline__ uint32_t top_bits(const Words<DG, P>& r, int u, int h) {
+  if constexpr (P == 4) return h ? (r.w[u] << 4) : r.w[u];
+  else return r.w[P - 1] << (2 * u + h);
+}
+
+// Lookup tables, built on the host from the contexts' codebooks: key centroids by code as
+// two int8 digits of round(c * kc_scale) (hi = floor((C+128)/256), lo = C - 256 hi), value
+// magnitudes c[K/2 + m] as fp16 low / high bytes.  8 entries = 2 registers per table.
+struct Luts {
+  uint32_t kh[2], kl[2], vlo[2], vhi[2];
+};
 
 // Per-group kernel arguments.
 struct MmaGroup {
@@ -169,151 +158,143 @@ struct MmaGroup {
   const uint16_t* krnorm;
   const uint8_t* vcodes;
   const uint16_t* vnorm;
-  const float* PiV;    // value rotation [d_g][d_g] row-major (float32)
-  Lut klut, vlut;      // fp16 key / value centroid tables
+  Luts lut;
+  float kc_inv;        // 1 / key-centroid fixed-point scale
   float coef;          // sqrt(pi/2)/m
   int off;             // first channel of the group
-  int kbytes, vbytes;  // record sizes
   int64_t kcap, vcap;  // slots allocated in the key / value caches
 };
 
 struct MmaArgs {
   MmaGroup g[2];
-  int B, Hq, Hkv, D, nsplit, chunk, qp_ld, G;
+  int B, Hq, Hkv, D, nsplit, chunk, G;
   int64_t max_len;
-  float scale_log2;    // softmax scale * log2(e)
+  float scale_log2;        // softmax scale * log2(e)
   const int32_t* seq_lens;
-  const float* qprep;  // [B*Hq][G][2*qp_ld]: (Pi q, S q) of each group
-  float* part;         // [B*Hq][nsplit][D+2]: (m, l, acc) per split
-  float* out;          // [B*Hq][D]
-  int* err;            // device error word (a pipeline wait that timed out)
+  const int16_t* qfix;     // [B*Hq][G][2][D]: round(Pi q * s_m), round(S q * s_s)
+  const float* qinv;       // [B*Hq][G][2]: 1/s_m, 1/s_s
+  float* part;             // [B*Hq][nsplit][D+2]: (m, l, acc) per split
+  int* err;                // device error word (a pipeline wait that timed out)
 };
 
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void allow_dependent_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
-// Query fragments of one group for this thread, built once per CTA.
+// Query operands of one group for this thread: B fragments (column g = head g/2, digit
+// g&1; k-slots = this thread's coordinates 8u + 4h + t), and, for the thread's own
+// accumulator head l, the fixed-point scales and sum_j Q^_j (for the QJL identity).
 template <class GC>
-struct QFrag {
-  uint32_t mse[GC::NKB][2];
-  uint32_t sgn[GC::NKB][2];
+struct QOps {
+  uint32_t bm[GC::NS][2], bs[GC::NS][2];
+  float inv_m, inv_s, sum_s;
 };
 
 template <class GC>
-__device__ __forceinline__ void load_qfrag(QFrag<GC>& f, const MmaArgs& A, int gi, int b, int hk, int lane) {
+__device__ __forceinline__ void load_qops(QOps<GC>& f, const MmaArgs& A, int gi, int b, int hk, int lane) {
   const int g = lane >> 2, l = lane & 3;
-  const int head = hk * kRep + (g >> 1);   // column n = g: head n/2, hi (n even) or lo (n odd) half
-  const bool lo_part = (g & 1) != 0;
-  const float* src = A.qprep + ((size_t)(b * A.Hq + head) * A.G + gi) * 2 * A.qp_ld;
-  const float* qt = src;
-  const float* qs = src + GC::DG;
-  auto part = [&](float v) {
-    float h = __half2float(__float2half_rn(v));
-    return lo_part ? v - h : v;
+  const int head = hk * kRep + (g >> 1);
+  const bool lo = (g & 1) != 0;
+  const int16_t* qm = A.qfix + ((size_t)(b * A.Hq + head) * A.G + gi) * 2 * A.D + GC::CQ * l;
+  const int16_t* qs = qm + A.D;
+  auto digit = [&](int v) -> uint32_t {
+    const int hi = (v + 128) >> 8;
+    return (uint32_t)(uint8_t)(lo ? v - (hi << 8) : hi);
   };
+  int ssum = 0;
 #pragma unroll
-  for (int kb = 0; kb < GC::NKB; ++kb) {
-    const int qq = kb & 3, hh = kb >> 2;
-    const int base = GC::Q * l + qq + 16 * hh;
-    f.mse[kb][0] = pack_h2(part(qt[base]), part(qt[base + 4]));
-    f.mse[kb][1] = pack_h2(part(qt[base + 8]), part(qt[base + 12]));
-    const int sb = GC::Q * l + 2 * kb;
-    f.sgn[kb][0] = pack_h2(part(qs[sb]), part(qs[sb + GC::Q / 2]));
-    f.sgn[kb][1] = pack_h2(part(qs[sb + 1]), part(qs[sb + 1 + GC::Q / 2]));
-  }
-}
-
-// MSE + QJL logits of one group for tokens (g, g+8) of a tile, columns 2l, 2l+1.
-template <class GC>
-__device__ __forceinline__ void group_logits(const QFrag<GC>& qf, const Lut& kl, const uint32_t (&w0)[GC::PK],
-                                             const uint32_t (&w1)[GC::PK], float (&mse)[4], float (&sgn)[4]) {
+  for (int u = 0; u < GC::NS; ++u) {
+    const uint4 vm = *reinterpret_cast<const uint4*>(qm + 8 * u);
+    const uint4 vs = *reinterpret_cast<const uint4*>(qs + 8 * u);
+    const uint32_t wm[4] = {vm.x, vm.y, vm.z, vm.w}, ws[4] = {vs.x, vs.y, vs.z, vs.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) mse[i] = sgn[i] = 0.f;
-  uint32_t nw0 = ~w0[GC::KK], nw1 = ~w1[GC::KK];
-  if constexpr (GC::Q == 16) {
-    nw0 = (nw0 & 0xFFu) | ((nw0 & 0xFF00u) << 8);
-    nw1 = (nw1 & 0xFFu) | ((nw1 & 0xFF00u) << 8);
-  }
+    for (int h = 0; h < 2; ++h) {
+      uint32_t dm = 0, ds = 0;
 #pragma unroll
-  for (int qq = 0; qq < 4; ++qq) {
-    const uint32_t s0 = selector<GC::KK, GC::M1>(w0, qq), s1 = selector<GC::KK, GC::M1>(w1, qq);
-#pragma unroll
-    for (int hh = 0; hh < GC::DG / 64; ++hh) {
-      const int kb = qq + 4 * hh;
-      uint32_t a0, a2, a1, a3;
-      lookup<GC::KK>(kl, s0 >> (16 * hh), 0, a0, a2);
-      lookup<GC::KK>(kl, s1 >> (16 * hh), 0, a1, a3);
-      mma16816(mse, a0, a1, a2, a3, qf.mse[kb][0], qf.mse[kb][1]);
+      for (int t = 0; t < 4; ++t) {
+        const int j = 4 * h + t;
+        const int vmj = (int)(int16_t)(wm[j >> 1] >> (16 * (j & 1)));
+        const int vsj = (int)(int16_t)(ws[j >> 1] >> (16 * (j & 1)));
+        dm |= digit(vmj) << (8 * t);
+        ds |= digit(vsj) << (8 * t);
+        ssum += vsj;
+      }
+      f.bm[u][h] = dm;
+      f.bs[u][h] = ds;
     }
   }
-#pragma unroll
-  for (int kb = 0; kb < GC::NKB; ++kb) {
-    const int j0 = 2 * kb;
-    uint32_t a0 = ((nw0 << (15 - j0)) & 0x80008000u) | 0x3C003C00u;
-    uint32_t a2 = ((nw0 << (14 - j0)) & 0x80008000u) | 0x3C003C00u;
-    uint32_t a1 = ((nw1 << (15 - j0)) & 0x80008000u) | 0x3C003C00u;
-    uint32_t a3 = ((nw1 << (14 - j0)) & 0x80008000u) | 0x3C003C00u;
-    mma16816(sgn, a0, a1, a2, a3, qf.sgn[kb][0], qf.sgn[kb][1]);
-  }
+  // sum over the head's coordinates: the four threads of a quad hold head g/2; the
+  // accumulator head of this thread is l, held by quad 2l
+  ssum += __shfl_xor_sync(0xffffffffu, ssum, 1);
+  ssum += __shfl_xor_sync(0xffffffffu, ssum, 2);
+  ssum = __shfl_sync(0xffffffffu, ssum, 8 * l);
+  const float* inv = A.qinv + ((size_t)(b * A.Hq + hk * kRep + l) * A.G + gi) * 2;
+  f.inv_m = inv[0];
+  f.inv_s = inv[1];
+  f.sum_s = (float)ssum;
 }
 
-// Value accumulation of one group: acc[mb] (rows: coordinates, cols: [P_hi | P_lo] heads).
+// One group's key codes of the tile's two token rows (g, g+8) and their norms.
 template <class GC>
-__device__ __forceinline__ void group_values(const Lut& vl, const uint32_t (&w0)[GC::PV], const uint32_t (&w1)[GC::PV],
-                                             uint32_t pb0, uint32_t pb1, float (&acc)[GC::NKB][4]) {
-#pragma unroll
-  for (int qq = 0; qq < 4; ++qq) {
-    const uint32_t s0 = selector<(GC::KV < 3 ? GC::KV : 3), GC::M1>(w0, qq);
-    const uint32_t s1 = selector<(GC::KV < 3 ? GC::KV : 3), GC::M1>(w1, qq);
-    uint32_t b40 = 0, b41 = 0;
-    if constexpr (GC::KV == 4) {
-      b40 = ((w0[3] >> qq) & GC::M1) << 2;
-      b41 = ((w1[3] >> qq) & GC::M1) << 2;
-    }
-#pragma unroll
-    for (int hh = 0; hh < GC::DG / 64; ++hh) {
-      const int mb = qq + 4 * hh;
-      uint32_t x0f, x0s, x1f, x1s;  // token g / g+8, coordinate blocks f = 0 (first) and 1 (second)
-      lookup<GC::KV>(vl, s0 >> (16 * hh), ((b40 >> (16 * hh)) & 0xFFFFu) | 0x3210u, x0f, x0s);
-      lookup<GC::KV>(vl, s1 >> (16 * hh), ((b41 >> (16 * hh)) & 0xFFFFu) | 0x3210u, x1f, x1s);
-      // rows (coordinates) g: block f = 0, g+8: block f = 1; k (tokens) 2l.. from token g, 2l+8.. from g+8
-      mma16816(acc[mb], movT(x0f), movT(x0s), movT(x1f), movT(x1s), pb0, pb1);
-    }
-  }
-}
-
-// Everything a thread loads for one 16-token tile of one group.
-template <class GC>
-struct TileData {
-  uint32_t ka[GC::PK], kb[GC::PK], va[GC::PV], vb[GC::PV];
-  unsigned short nka, nkb, rka, rkb, nva, nvb;
+struct KeyTile {
+  Words<GC::DG, GC::PK> a, b;
+  float na, nb, ra, rb;
 };
-
 template <class GC>
-__device__ __forceinline__ void load_tile(TileData<GC>& t, const MmaGroup& gr, int64_t sa, int64_t sb, int l) {
-  load_quarter<GC::Q, GC::PK>(gr.kcodes + sa * gr.kbytes, l, t.ka);
-  load_quarter<GC::Q, GC::PK>(gr.kcodes + sb * gr.kbytes, l, t.kb);
-  load_quarter<GC::Q, GC::PV>(gr.vcodes + sa * gr.vbytes, l, t.va);
-  load_quarter<GC::Q, GC::PV>(gr.vcodes + sb * gr.vbytes, l, t.vb);
-  t.nka = __ldg(gr.knorm + sa);
-  t.nkb = __ldg(gr.knorm + sb);
-  t.rka = __ldg(gr.krnorm + sa);
-  t.rkb = __ldg(gr.krnorm + sb);
-  t.nva = __ldg(gr.vnorm + sa);
-  t.nvb = __ldg(gr.vnorm + sb);
-}
+struct ValTile {
+  Words<GC::DG, GC::PV> a, b;
+  float na, nb;
+};
 
 __device__ __forceinline__ float h2f(unsigned short h) { return __half2float(__ushort_as_half(h)); }
 
+// MSE + QJL logits of one group for tokens (g, g+8) of a tile, head l.
 template <class GC>
-__device__ __forceinline__ void tile_logits(const TileData<GC>& t, const QFrag<GC>& qf, const Lut& kl,
-                                            const MmaGroup& gr, float& la, float& lb) {
-  float mse[4], sgn[4];
-  group_logits<GC>(qf, kl, t.ka, t.kb, mse, sgn);
-  // columns 2l, 2l+1 are the hi and lo halves of head l
-  const float ca = gr.coef * h2f(t.rka), cb = gr.coef * h2f(t.rkb);
-  la += h2f(t.nka) * fmaf(ca, sgn[0] + sgn[1], mse[0] + mse[1]);
-  lb += h2f(t.nkb) * fmaf(cb, sgn[2] + sgn[3], mse[2] + mse[3]);
+__device__ __forceinline__ void group_logits(const QOps<GC>& q, const Luts& t, const KeyTile<GC>& k, float coef,
+                                             float kc_inv, float& la, float& lb) {
+  int dh[4] = {0, 0, 0, 0}, dl[4] = {0, 0, 0, 0}, ds[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int u = 0; u < GC::NS; ++u) {
+    const uint32_t sa = low_sel(k.a, u), sb = low_sel(k.b, u);
+    const uint32_t sa1 = sa >> 16, sb1 = sb >> 16;
+    mma_s8(dh, prmt(t.kh[0], t.kh[1], sa), prmt(t.kh[0], t.kh[1], sb), prmt(t.kh[0], t.kh[1], sa1),
+           prmt(t.kh[0], t.kh[1], sb1), q.bm[u][0], q.bm[u][1]);
+    mma_s8(dl, prmt(t.kl[0], t.kl[1], sa), prmt(t.kl[0], t.kl[1], sb), prmt(t.kl[0], t.kl[1], sa1),
+           prmt(t.kl[0], t.kl[1], sb1), q.bm[u][0], q.bm[u][1]);
+    mma_s8(ds, msb_bytes(top_bits(k.a, u, 0)), msb_bytes(top_bits(k.b, u, 0)), msb_bytes(top_bits(k.a, u, 1)),
+           msb_bytes(top_bits(k.b, u, 1)), q.bs[u][0], q.bs[u][1]);
+  }
+  // columns 2l (query hi digit), 2l+1 (lo digit); rows g (d[0..1]) and g+8 (d[2..3])
+  const float cm = kc_inv * q.inv_m;
+  auto logit = [&](int i, float n, float r) {
+    const float mse = fmaf(65536.f, (float)dh[i], (float)(256 * (dh[i + 1] + dl[i]) + dl[i + 1])) * cm;
+    // sum_j s_j Q^_j = -2 sum_j a_j Q^_j - sum_j Q^_j  (a_j = -1 where the sign bit is set)
+    const float sq = (-2.f * (float)(256 * ds[i] + ds[i + 1]) - q.sum_s) * q.inv_s;
+    return n * fmaf(coef * r, sq, mse);
+  };
+  la += logit(0, k.na, k.ra);
+  lb += logit(2, k.nb, k.rb);
+}
+
+// Value accumulation of one group: acc[u][h] (rows: the 16 coordinates 8u + 4h + t of the
+// four threads of a row quad, cols: [P_hi | P_lo] heads).
+template <class GC>
+__device__ __forceinline__ void group_values(const Luts& t, const ValTile<GC>& v, uint32_t pb0, uint32_t pb1,
+                                             float (&acc)[GC::NS][2][4]) {
+#pragma unroll
+  for (int u = 0; u < GC::NS; ++u) {
+    const uint32_t sa = low_sel(v.a, u), sb = low_sel(v.b, u);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t xa = h ? sa >> 16 : sa, xb = h ? sb >> 16 : sb;
+      const uint32_t la = prmt(t.vlo[0], t.vlo[1], xa), lb = prmt(t.vlo[0], t.vlo[1], xb);
+      const uint32_t ha = prmt(t.vhi[0], t.vhi[1], xa) ^ (top_bits(v.a, u, h) & 0x80808080u);
+      const uint32_t hb = prmt(t.vhi[0], t.vhi[1], xb) ^ (top_bits(v.b, u, h) & 0x80808080u);
+      // token g: coordinates (4h, 4h+1) and (4h+2, 4h+3); token g+8 likewise
+      const uint32_t a01 = prmt(la, ha, 0x5140u), a23 = prmt(la, ha, 0x7362u);
+      const uint32_t b01 = prmt(lb, hb, 0x5140u), b23 = prmt(lb, hb, 0x7362u);
+      mma16816(acc[u][h], movT(a01), movT(a23), movT(b01), movT(b23), pb0, pb1);
+    }
+  }
 }
 
 constexpr int kStageTok = kWarps * 16;  // tokens per pipeline stage: one 16-token tile per consumer warp
@@ -325,8 +306,8 @@ constexpr uint64_t kDecWaitNs = 2000000000ull;
 // three fp16 norm arrays.
 template <class G0, class G1c, bool TWO>
 struct Stage {
-  static constexpr int KB0 = G0::PK * G0::DG / 8, VB0 = G0::PV * G0::DG / 8;
-  static constexpr int KB1 = G1c::PK * G1c::DG / 8, VB1 = G1c::PV * G1c::DG / 8;
+  static constexpr int KB0 = G0::KB, VB0 = G0::VB;
+  static constexpr int KB1 = G1c::KB, VB1 = G1c::VB;
   static constexpr int OFF_K0 = 0;
   static constexpr int OFF_V0 = OFF_K0 + kStageTok * KB0 + 32;
   static constexpr int OFF_K1 = OFF_V0 + kStageTok * VB0 + 32;
@@ -436,21 +417,25 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
   }
 
   // ------------------------------------------------------------------ consumer warps
-  float acc0[G0::NKB][4];
-  float acc1[G1c::NKB][4];
+  float acc0[G0::NS][2][4];
+  float acc1[G1c::NS][2][4];
   float m_run = -INFINITY, l_run = 0.f;
   if (warp < kWarps) {
-    const Lut kl0 = A.g[0].klut, vl0 = A.g[0].vlut;
-    const Lut kl1 = A.g[TWO ? 1 : 0].klut, vl1 = A.g[TWO ? 1 : 0].vlut;
+    const Luts t0 = A.g[0].lut;
+    const Luts t1 = A.g[TWO ? 1 : 0].lut;
     grid_dependency_wait();   // prepared queries come from the preceding kernel
-    QFrag<G0> qf0;
-    load_qfrag<G0>(qf0, A, 0, b, hk, lane);
-    QFrag<G1c> qf1;
-    if constexpr (TWO) load_qfrag<G1c>(qf1, A, 1, b, hk, lane);
+    QOps<G0> q0;
+    load_qops<G0>(q0, A, 0, b, hk, lane);
+    QOps<G1c> q1;
+    if constexpr (TWO) load_qops<G1c>(q1, A, 1, b, hk, lane);
 #pragma unroll
-    for (int i = 0; i < G0::NKB; ++i) acc0[i][0] = acc0[i][1] = acc0[i][2] = acc0[i][3] = 0.f;
+    for (int u = 0; u < G0::NS; ++u)
 #pragma unroll
-    for (int i = 0; i < G1c::NKB; ++i) acc1[i][0] = acc1[i][1] = acc1[i][2] = acc1[i][3] = 0.f;
+      for (int h = 0; h < 2; ++h) acc0[u][h][0] = acc0[u][h][1] = acc0[u][h][2] = acc0[u][h][3] = 0.f;
+#pragma unroll
+    for (int u = 0; u < G1c::NS; ++u)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) acc1[u][h][0] = acc1[u][h][1] = acc1[u][h][2] = acc1[u][h][3] = 0.f;
     int it = 0;
     for (int ts = t_begin; ts < t_end; ts += kStageTok, ++it) {
       const int s = it % kNStage;
@@ -460,37 +445,39 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
       const uint8_t* st = dsm + s * ST::BYTES;
       const int64_t first = slot0 + ts;
       const int ja = warp * 16 + g, jb = ja + 8;   // stage-local token rows of this lane
-      TileData<G0> c0;
-      TileData<G1c> c1;
+      KeyTile<G0> k0;
+      ValTile<G0> v0;
+      KeyTile<G1c> k1;
+      ValTile<G1c> v1;
       if (live) {
-        const uint8_t* k0 = st + ST::OFF_K0 + ((first * ST::KB0) & 15);
-        const uint8_t* v0 = st + ST::OFF_V0 + ((first * ST::VB0) & 15);
-        lds_quarter<G0::Q, G0::PK>(k0 + ja * ST::KB0, l, c0.ka);
-        lds_quarter<G0::Q, G0::PK>(k0 + jb * ST::KB0, l, c0.kb);
-        lds_quarter<G0::Q, G0::PV>(v0 + ja * ST::VB0, l, c0.va);
-        lds_quarter<G0::Q, G0::PV>(v0 + jb * ST::VB0, l, c0.vb);
+        const uint8_t* kp = st + ST::OFF_K0 + ((first * ST::KB0) & 15);
+        const uint8_t* vp = st + ST::OFF_V0 + ((first * ST::VB0) & 15);
+        lds_words(k0.a, kp + ja * ST::KB0, l);
+        lds_words(k0.b, kp + jb * ST::KB0, l);
+        lds_words(v0.a, vp + ja * ST::VB0, l);
+        lds_words(v0.b, vp + jb * ST::VB0, l);
         const uint16_t* nrm = reinterpret_cast<const uint16_t*>(st + ST::OFF_N);
-        c0.nka = nrm[ja]; c0.nkb = nrm[jb];
-        c0.rka = nrm[kStageTok + ja]; c0.rkb = nrm[kStageTok + jb];
-        c0.nva = nrm[2 * kStageTok + ja]; c0.nvb = nrm[2 * kStageTok + jb];
+        k0.na = h2f(nrm[ja]); k0.nb = h2f(nrm[jb]);
+        k0.ra = h2f(nrm[kStageTok + ja]); k0.rb = h2f(nrm[kStageTok + jb]);
+        v0.na = h2f(nrm[2 * kStageTok + ja]); v0.nb = h2f(nrm[2 * kStageTok + jb]);
         if constexpr (TWO) {
-          const uint8_t* k1 = st + ST::OFF_K1 + ((first * ST::KB1) & 15);
-          const uint8_t* v1 = st + ST::OFF_V1 + ((first * ST::VB1) & 15);
-          lds_quarter<G1c::Q, G1c::PK>(k1 + ja * ST::KB1, l, c1.ka);
-          lds_quarter<G1c::Q, G1c::PK>(k1 + jb * ST::KB1, l, c1.kb);
-          lds_quarter<G1c::Q, G1c::PV>(v1 + ja * ST::VB1, l, c1.va);
-          lds_quarter<G1c::Q, G1c::PV>(v1 + jb * ST::VB1, l, c1.vb);
-          c1.nka = nrm[3 * kStageTok + ja]; c1.nkb = nrm[3 * kStageTok + jb];
-          c1.rka = nrm[4 * kStageTok + ja]; c1.rkb = nrm[4 * kStageTok + jb];
-          c1.nva = nrm[5 * kStageTok + ja]; c1.nvb = nrm[5 * kStageTok + jb];
+          const uint8_t* kq = st + ST::OFF_K1 + ((first * ST::KB1) & 15);
+          const uint8_t* vq = st + ST::OFF_V1 + ((first * ST::VB1) & 15);
+          lds_words(k1.a, kq + ja * ST::KB1, l);
+          lds_words(k1.b, kq + jb * ST::KB1, l);
+          lds_words(v1.a, vq + ja * ST::VB1, l);
+          lds_words(v1.b, vq + jb * ST::VB1, l);
+          k1.na = h2f(nrm[3 * kStageTok + ja]); k1.nb = h2f(nrm[3 * kStageTok + jb]);
+          k1.ra = h2f(nrm[4 * kStageTok + ja]); k1.rb = h2f(nrm[4 * kStageTok + jb]);
+          v1.na = h2f(nrm[5 * kStageTok + ja]); v1.nb = h2f(nrm[5 * kStageTok + jb]);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty + s);   // the stage's data now sits in registers
       if (!live) continue;
       float la = 0.f, lb = 0.f;
-      tile_logits<G0>(c0, qf0, kl0, A.g[0], la, lb);
-      if constexpr (TWO) tile_logits<G1c>(c1, qf1, kl1, A.g[1], la, lb);
+      group_logits<G0>(q0, t0, k0, A.g[0].coef, A.g[0].kc_inv, la, lb);
+      if constexpr (TWO) group_logits<G1c>(q1, t1, k1, A.g[1].coef, A.g[1].kc_inv, la, lb);
       // online softmax (log2 domain) of head l over tokens g, g+8 of the tile
       la = (tt + g < t_end) ? la * A.scale_log2 : -INFINITY;
       lb = (tt + g + 8 < t_end) ? lb * A.scale_log2 : -INFINITY;
@@ -503,14 +490,18 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
         m_run = mt;
         l_run *= alpha;
 #pragma unroll
-        for (int i = 0; i < G0::NKB; ++i) {
-          acc0[i][0] *= alpha; acc0[i][1] *= alpha; acc0[i][2] *= alpha; acc0[i][3] *= alpha;
-        }
+        for (int u = 0; u < G0::NS; ++u)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc0[u][h][i] *= alpha;
         if constexpr (TWO) {
 #pragma unroll
-          for (int i = 0; i < G1c::NKB; ++i) {
-            acc1[i][0] *= alpha; acc1[i][1] *= alpha; acc1[i][2] *= alpha; acc1[i][3] *= alpha;
-          }
+          for (int u = 0; u < G1c::NS; ++u)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) acc1[u][h][i] *= alpha;
         }
       }
       const float pa = exp2f(la - m_run), pb = exp2f(lb - m_run);
@@ -522,11 +513,11 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
         b1 = movT(pack_h2(hb, wb - hb));
       };
       uint32_t pb0, pb1;
-      pfrag(h2f(c0.nva), h2f(c0.nvb), pb0, pb1);
-      group_values<G0>(vl0, c0.va, c0.vb, pb0, pb1, acc0);
+      pfrag(v0.na, v0.nb, pb0, pb1);
+      group_values<G0>(t0, v0, pb0, pb1, acc0);
       if constexpr (TWO) {
-        pfrag(h2f(c1.nva), h2f(c1.nvb), pb0, pb1);
-        group_values<G1c>(vl1, c1.va, c1.vb, pb0, pb1, acc1);
+        pfrag(v1.na, v1.nb, pb0, pb1);
+        group_values<G1c>(t1, v1, pb0, pb1, acc1);
       }
     }
     // ---- warp state -> shared memory (lane (g, l) holds head l)
@@ -537,15 +528,17 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
       s_m[warp][l] = m_run;
       s_l[warp][l] = l_run;
     }
+    // row g of block (u, h) is coordinate CQ (g>>1) + 8u + 4h + (g&1), row g+8 adds 2
     auto store_acc = [&](auto& acc, auto gc_tag, int off) {
       using GC = decltype(gc_tag);
 #pragma unroll
-      for (int mb = 0; mb < GC::NKB; ++mb) {
-        const int qq = mb & 3, hh = mb >> 2;
-        const int c0_ = GC::Q * (g >> 1) + qq + 16 * hh + 4 * (g & 1);   // row g: block f = 0
-        s_acc[warp][l][off + c0_] = acc[mb][0] + acc[mb][1];
-        s_acc[warp][l][off + c0_ + 8] = acc[mb][2] + acc[mb][3];          // row g+8: block f = 1
-      }
+      for (int u = 0; u < GC::NS; ++u)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int c = GC::CQ * (g >> 1) + 8 * u + 4 * h + (g & 1);
+          s_acc[warp][l][off + c] = acc[u][h][0] + acc[u][h][1];
+          s_acc[warp][l][off + c + 2] = acc[u][h][2] + acc[u][h][3];
+        }
     };
     store_acc(acc0, G0{}, A.g[0].off);
     if constexpr (TWO) store_acc(acc1, G1c{}, A.g[1].off);
@@ -578,25 +571,37 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
   allow_dependent_launch();
 }
 
-// (Pi q, S q) of the kRep query heads of one (sequence, kv head), 64 outputs per CTA
-// (blockIdx.y selects them; outputs o < d_g are Pi q, the rest S q): the 64 needed
-// columns of Pi^T or S^T are staged in shared memory with 16-byte loads, then thread
-// (head, o) takes its dot product from shared memory.
+// Prepared queries of the kRep query heads of one (sequence, kv head) for one group, 64
+// outputs per CTA (blockIdx.y selects them; outputs o < d_g are Pi q, the rest S q), as
+// 16-bit fixed point: round(Pi q * 32000/|q_g|) and round(S q * 32000/(|q_g| max_j |S_j|)),
+// both bounded by 32000 in magnitude (|(Pi q)_o| <= |q_g|, |(S q)_o| <= |S_o| |q_g|).  The
+// 64 needed columns of Pi^T or S^T are staged in shared memory with 16-byte loads, all in
+// flight at once; thread (head, o) takes its dot product from shared memory.
 template <typename T>
 __global__ void __launch_bounds__(256) decode_prep_kernel(const T* __restrict__ q, int D, int off, int dg,
                                                           const float* __restrict__ PiT, const float* __restrict__ ST,
-                                                          float* __restrict__ qprep, int G, int gi, int qp_ld) {
+                                                          float s_rowmax, int16_t* __restrict__ qfix,
+                                                          float* __restrict__ qinv, int G, int gi) {
   __shared__ __align__(16) float ms[128 * 64];
   __shared__ float qs[kRep][128];
+  __shared__ float qn[kRep];
   allow_dependent_launch();
   const int grp = blockIdx.x;                    // = b * Hkv + hk; rows grp*kRep .. +kRep-1
   const int o0 = blockIdx.y * 64;                // first output of this CTA
   const float* M = o0 < dg ? PiT + o0 : ST + (o0 - dg);
   float4* m4 = reinterpret_cast<float4*>(ms);
-#pragma unroll 8
-  for (int e = threadIdx.x; e < dg * 16; e += blockDim.x) {     // dg rows x 16 float4
-    const int j = e >> 4, c4 = e & 15;
-    m4[e] = __ldg(reinterpret_cast<const float4*>(M + (size_t)j * dg) + c4);
+  {
+    float4 r[8];                                 // dg <= 128: at most 8 loads per thread
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = threadIdx.x + u * 256;
+      if (e < dg * 16) r[u] = __ldg(reinterpret_cast<const float4*>(M + (size_t)(e >> 4) * dg) + (e & 15));
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = threadIdx.x + u * 256;
+      if (e < dg * 16) m4[e] = r[u];
+    }
   }
   for (int e = threadIdx.x; e < kRep * dg; e += blockDim.x) {
     const int h = e / dg, j = e % dg;
@@ -605,6 +610,13 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const T* __restrict__ 
     else qs[h][j] = __bfloat162float(q[at]);
   }
   __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < kRep) {
+    float s = 0.f;
+    for (int j = lane; j < dg; j += 32) s = fmaf(qs[warp][j], qs[warp][j], s);
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) qn[warp] = sqrtf(s);
+  }
   const int h = threadIdx.x >> 6, oc = threadIdx.x & 63;
   float a0 = 0.f, a1 = 0.f;
 #pragma unroll 8
@@ -612,13 +624,19 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const T* __restrict__ 
     a0 = fmaf(ms[j * 64 + oc], qs[h][j], a0);
     a1 = fmaf(ms[(j + 1) * 64 + oc], qs[h][j + 1], a1);
   }
-  qprep[((size_t)(grp * kRep + h) * G + gi) * 2 * qp_ld + o0 + oc] = a0 + a1;
+  __syncthreads();
+  const bool sq = o0 >= dg;
+  const float bound = sq ? qn[h] * s_rowmax : qn[h];
+  const float sc = bound > 0.f ? kFix / bound : 0.f;
+  const size_t row = (size_t)(grp * kRep + h) * G + gi;
+  qfix[row * 2 * D + (sq ? D + o0 - dg : o0) + oc] = (int16_t)__float2int_rn((a0 + a1) * sc);
+  if (oc == 0 && (o0 == 0 || o0 == dg)) qinv[row * 2 + (sq ? 1 : 0)] = bound / kFix;
 }
 
 // Log-sum-exp merge of the context splits and the inverse rotation of the value groups:
-// one CTA per (query row, 64 output channels).  The merged rotated-basis accumulator of
-// the row is built in shared memory (all splits' loads independent), then thread
-// (output, quarter) sums a quarter of o[c] = sum_i Pi_v[i][c - off] acc[off + i].
+// one CTA per (query row, 64 output channels).  The rotation entries are fetched before
+// the dependency wait; after it, every split's (m, l, acc) is loaded at once and merged
+// with a running maximum, so the merge costs one dependent round trip.
 struct Merge2Args {
   const float* part;
   int nsplit, D, G;
@@ -628,69 +646,84 @@ struct Merge2Args {
 };
 
 __global__ void __launch_bounds__(256) decode_merge_mma_kernel(Merge2Args A) {
-  __shared__ float w[512];
-  __shared__ float acc[256];
+  __shared__ float s_acc[4][256];
+  __shared__ float s_ml[4][256][2];
   __shared__ float red[4][64];
-  __shared__ float part2[2][256];
-  grid_dependency_wait();
   const int row = blockIdx.x, c0 = blockIdx.y * 64;
   const int D = A.D, ns = A.nsplit;
-  const float* P = A.part + (size_t)row * ns * (D + 2);
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    float M = -INFINITY;
-    for (int s = lane; s < ns; s += 32) M = fmaxf(M, P[(size_t)s * (D + 2)]);
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.f;
-    for (int s = lane; s < ns; s += 32) {
-      const float ms = P[(size_t)s * (D + 2)];
-      const float f = (ms == -INFINITY) ? 0.f : __expf(ms - M);
-      w[s] = f;
-      L += f * P[(size_t)s * (D + 2) + 1];
-    }
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    __syncwarp();
-    for (int s = lane; s < ns; s += 32) w[s] *= inv;
-  }
-  __syncthreads();
-  // every split's contribution is an independent load: keep 16 of them in flight per thread
-  {
-    const int nthr = blockDim.x;
-    const int halves = nthr / D > 1 ? nthr / D : 1;     // threads per coordinate
-    const int i = threadIdx.x % D, hsel = threadIdx.x / D;
-    float a[16];
-#pragma unroll
-    for (int u = 0; u < 16; ++u) a[u] = 0.f;
-    if (hsel < halves) {
-      for (int s0 = hsel * 16; s0 < ns; s0 += 16 * halves) {
-#pragma unroll
-        for (int u = 0; u < 16; ++u)
-          if (s0 + u < ns) a[u] = fmaf(w[s0 + u], P[(size_t)(s0 + u) * (D + 2) + 2 + i], a[u]);
-      }
-    }
-    float t = 0.f;
-#pragma unroll
-    for (int u = 0; u < 16; ++u) t += a[u];
-    if (hsel < halves) part2[hsel][i] = t;
-    __syncthreads();
-    if (hsel == 0) {
-      float sum = 0.f;
-      for (int h = 0; h < halves; ++h) sum += part2[h][i];
-      acc[i] = sum;
-    }
-  }
-  __syncthreads();
+  // rotation column of this thread's output, quarter qtr of its rows (before the wait)
   const int oc = threadIdx.x & 63, qtr = threadIdx.x >> 6;
   const int c = c0 + oc;
+  float pv[32];
+  int gsel = 0, goff = 0, gd = 0;
+  if (c < D) {
+    gsel = (A.G > 1 && c >= A.off[1]) ? 1 : 0;
+    goff = A.off[gsel];
+    gd = A.off[gsel + 1] - goff;
+    const float* Pi = A.PiV[gsel] + (c - goff);
+    const int i0 = qtr * (gd / 4), n = gd / 4;   // n <= 32
+#pragma unroll
+    for (int u = 0; u < 32; ++u) pv[u] = (u < n) ? __ldg(Pi + (size_t)(i0 + u) * gd) : 0.f;
+  }
+  grid_dependency_wait();
+  // merged rotated-basis accumulator: thread (coordinate i, half hs) runs over splits
+  // hs, hs + halves, ... with a running maximum
+  const float* P = A.part + (size_t)row * ns * (D + 2);
+  int halves = blockDim.x / D;
+  halves = halves < 1 ? 1 : (halves > 4 ? 4 : halves);
+  const int i = threadIdx.x % D, hs = threadIdx.x / D;
+  if (hs < halves) {
+    float M = -INFINITY, L = 0.f, acc = 0.f;
+    for (int s0 = hs; s0 < ns; s0 += 16 * halves) {
+      float m16[16], l16[16], a16[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int s = s0 + u * halves;
+        const float* ps = P + (size_t)s * (D + 2);
+        m16[u] = s < ns ? ps[0] : -INFINITY;
+        l16[u] = s < ns ? ps[1] : 0.f;
+        a16[u] = s < ns ? ps[2 + i] : 0.f;
+      }
+      float mx = M;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) mx = fmaxf(mx, m16[u]);
+      if (mx > -INFINITY) {
+        const float f = M == -INFINITY ? 0.f : __expf(M - mx);
+        L *= f;
+        acc *= f;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const float w = m16[u] == -INFINITY ? 0.f : __expf(m16[u] - mx);
+          L = fmaf(w, l16[u], L);
+          acc = fmaf(w, a16[u], acc);
+        }
+        M = mx;
+      }
+    }
+    s_acc[hs][i] = acc;
+    s_ml[hs][i][0] = M;
+    s_ml[hs][i][1] = L;
+  }
+  __syncthreads();
+  // thread i combines the partial states of coordinate i (only it touches index i)
+  if (threadIdx.x < D) {
+    float M = -INFINITY;
+    for (int h = 0; h < halves; ++h) M = fmaxf(M, s_ml[h][i][0]);
+    float L = 0.f, acc = 0.f;
+    for (int h = 0; h < halves; ++h) {
+      const float f = s_ml[h][i][0] == -INFINITY ? 0.f : __expf(s_ml[h][i][0] - M);
+      L = fmaf(f, s_ml[h][i][1], L);
+      acc = fmaf(f, s_acc[h][i], acc);
+    }
+    s_acc[0][i] = L > 0.f ? acc / L : 0.f;
+  }
+  __syncthreads();
   float o = 0.f;
   if (c < D) {
-    const int gi = (A.G > 1 && c >= A.off[1]) ? 1 : 0;
-    const int off = A.off[gi], dg = A.off[gi + 1] - off, j = c - off;
-    const float* Pi = A.PiV[gi] + j;
-    const int i0 = qtr * (dg / 4), i1 = i0 + dg / 4;
-#pragma unroll 8
-    for (int i = i0; i < i1; ++i) o = fmaf(__ldg(Pi + (size_t)i * dg), acc[off + i], o);
+    const int i0 = qtr * (gd / 4), n = gd / 4;
+#pragma unroll
+    for (int u = 0; u < 32; ++u)
+      if (u < n) o = fmaf(pv[u], s_acc[0][goff + i0 + u], o);
   }
   red[qtr][oc] = o;
   __syncthreads();
@@ -723,18 +756,28 @@ int launch_mma_t(const MmaArgs& A, int nsplit, int BHkv, cudaStream_t st) {
 
 }  // namespace
 
-Lut host_lut(const Codebook& cb) {
-  Lut t{};
-  for (int j = 0; j < 16; ++j) {
-    uint16_t b = 0;
-    if (j < cb.K) {
-      __half h = __float2half_rn(cb.c[j]);
-      b = *reinterpret_cast<uint16_t*>(&h);
-    }
-    t.lo[j / 4] |= (uint32_t)(b & 0xFF) << (8 * (j % 4));
-    t.hi[j / 4] |= (uint32_t)(b >> 8) << (8 * (j % 4));
+// Tables of one (key context, value context) pair; returns the key-centroid scale inverse.
+float host_luts(const tq_ctx* kc, const tq_ctx* vc, Luts* t) {
+  *t = Luts{};
+  const Codebook& kb = kc->cb;
+  float cmax = 0.f;
+  for (int j = 0; j < kb.K; ++j) cmax = fmaxf(cmax, fabsf(kb.c[j]));
+  const float sc = cmax > 0.f ? kFix / cmax : 0.f;
+  for (int code = 0; code < kb.K && code < 8; ++code) {
+    const int C = (int)lrintf(kb.cc[code] * sc);
+    const int hi = (C + 128) >> 8, lo = C - (hi << 8);
+    t->kh[code / 4] |= (uint32_t)(uint8_t)hi << (8 * (code % 4));
+    t->kl[code / 4] |= (uint32_t)(uint8_t)lo << (8 * (code % 4));
   }
-  return t;
+  const Codebook& vb = vc->cb;
+  const int half = vb.K / 2;
+  for (int m = 0; m < half && m < 8; ++m) {
+    __half hv = __float2half_rn(vb.c[half + m]);
+    const uint16_t bits = *reinterpret_cast<uint16_t*>(&hv);
+    t->vlo[m / 4] |= (uint32_t)(bits & 0xFF) << (8 * (m % 4));
+    t->vhi[m / 4] |= (uint32_t)(bits >> 8) << (8 * (m % 4));
+  }
+  return sc > 0.f ? 1.f / sc : 0.f;
 }
 
 // Returns kNotHandled when the shape is outside this kernel's instantiations.
@@ -746,60 +789,57 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
   for (int g = 0; g < G; ++g) {
     const int dg = kctx[g]->lay.d;
     if (dg != 64 && dg != 128) return kNotHandled;
-    if (vctx[g]->lay.k < 2) return kNotHandled;
-    sig[g] = dg * 100 + kctx[g]->lay.k * 10 + vctx[g]->lay.k;
+    sig[g] = dg * 100 + kctx[g]->lay.planes * 10 + vctx[g]->lay.planes;
   }
   auto is = [&](int a, int bsig) { return sig[0] == a && sig[1] == bsig; };
-  using C128_34 = GroupCfg<128, 3, 4>;
-  using C64_34 = GroupCfg<64, 3, 4>;
-  using C64_23 = GroupCfg<64, 2, 3>;
-  using C64_12 = GroupCfg<64, 1, 2>;
-  using C128_23 = GroupCfg<128, 2, 3>;
-  const bool ok = (G == 1 && (sig[0] == 12834 || sig[0] == 12823)) || is(6434, 6423) || is(6423, 6412);
+  using C128_44 = GroupCfg<128, 4, 4>;
+  using C128_33 = GroupCfg<128, 3, 3>;
+  using C64_44 = GroupCfg<64, 4, 4>;
+  using C64_33 = GroupCfg<64, 3, 3>;
+  using C64_22 = GroupCfg<64, 2, 2>;
+  const bool ok = (G == 1 && (sig[0] == 12844 || sig[0] == 12833)) || is(6444, 6433) || is(6433, 6422);
   if (!ok) return kNotHandled;
 
   const DecodeWs W = decode_ws(B, Hq, Hkv, D, G, max_len);
   if (W.nsplit > 512) return kNotHandled;
   char* base = static_cast<char*>(ws);
-  float* qprep = reinterpret_cast<float*>(base + W.qp);
+  int16_t* qfix = reinterpret_cast<int16_t*>(base + W.qp);
+  float* qinv = reinterpret_cast<float*>(base + W.qp + (((size_t)B * Hq * G * 2 * D * 2 + 255) / 256) * 256);
   float* part = reinterpret_cast<float*>(base + W.part);
   for (int g = 0; g < G; ++g) {
     const int dg = kctx[g]->lay.d;
     const dim3 pgrid(B * Hkv, 2 * dg / 64);
     if (q_dtype == TQ_DTYPE_F32)
       decode_prep_kernel<float><<<pgrid, 256, 0, st>>>(static_cast<const float*>(q), D, off[g], dg, kctx[g]->PiT,
-                                                       kctx[g]->ST, qprep, G, g, D);
+                                                       kctx[g]->ST, kctx[g]->s_rowmax, qfix, qinv, G, g);
     else
       decode_prep_kernel<__nv_bfloat16><<<pgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), D, off[g], dg,
-                                                               kctx[g]->PiT, kctx[g]->ST, qprep, G, g, D);
+                                                               kctx[g]->PiT, kctx[g]->ST, kctx[g]->s_rowmax, qfix,
+                                                               qinv, G, g);
     count_launch();
     int r = check_launch("decode_prep_kernel");
     if (r != TQ_OK) return r;
   }
   MmaArgs A{};
-  A.B = B; A.Hq = Hq; A.Hkv = Hkv; A.D = D; A.nsplit = W.nsplit; A.chunk = W.chunk; A.qp_ld = D; A.G = G;
-  A.max_len = max_len; A.scale_log2 = scale * 1.4426950408889634f; A.seq_lens = seq_lens; A.qprep = qprep;
-  A.part = part; A.out = out;
+  A.B = B; A.Hq = Hq; A.Hkv = Hkv; A.D = D; A.nsplit = W.nsplit; A.chunk = W.chunk; A.G = G;
+  A.max_len = max_len; A.scale_log2 = scale * 1.4426950408889634f; A.seq_lens = seq_lens;
+  A.qfix = qfix; A.qinv = qinv; A.part = part;
   for (int g = 0; g < G; ++g) {
     MmaGroup& gr = A.g[g];
     gr.kcodes = kc[g].codes; gr.knorm = kc[g].norm; gr.krnorm = kc[g].rnorm;
     gr.vcodes = vc[g].codes; gr.vnorm = vc[g].norm;
-    gr.PiV = vctx[g]->Pi;
-    gr.klut = host_lut(kctx[g]->cb);
-    gr.vlut = host_lut(vctx[g]->cb);
+    gr.kc_inv = host_luts(kctx[g], vctx[g], &gr.lut);
     gr.coef = kctx[g]->sqrt_pi_over_2_over_m;
     gr.off = off[g];
-    gr.kbytes = kctx[g]->lay.code_bytes;
-    gr.vbytes = vctx[g]->lay.code_bytes;
     gr.kcap = kc[g].cap;
     gr.vcap = vc[g].cap;
   }
   A.err = kctx[0]->dev_err;
   int r;
-  if (G == 1 && sig[0] == 12834) r = launch_mma_t<C128_34, void>(A, W.nsplit, B * Hkv, st);
-  else if (G == 1) r = launch_mma_t<C128_23, void>(A, W.nsplit, B * Hkv, st);
-  else if (is(6434, 6423)) r = launch_mma_t<C64_34, C64_23>(A, W.nsplit, B * Hkv, st);
-  else r = launch_mma_t<C64_23, C64_12>(A, W.nsplit, B * Hkv, st);
+  if (G == 1 && sig[0] == 12844) r = launch_mma_t<C128_44, void>(A, W.nsplit, B * Hkv, st);
+  else if (G == 1) r = launch_mma_t<C128_33, void>(A, W.nsplit, B * Hkv, st);
+  else if (is(6444, 6433)) r = launch_mma_t<C64_44, C64_33>(A, W.nsplit, B * Hkv, st);
+  else r = launch_mma_t<C64_33, C64_22>(A, W.nsplit, B * Hkv, st);
   if (r != TQ_OK) return r;
   Merge2Args M{};
   M.part = part; M.nsplit = W.nsplit; M.D = D; M.G = G; M.out = out;

@@ -42,12 +42,22 @@ __device__ __forceinline__ int nearest(float y, const float* t, int K) {
   return idx;
 }
 
-// Read the k-bit index and (prod) sign of coordinate i of a record.
-__device__ __forceinline__ int read_index(const uint8_t* rec, const Layout& L, int i) {
-  int base = (i / L.quarter) * L.qbytes + (i % L.quarter) / 8;
-  int bit = (i % L.quarter) % 8, idx = 0;
-  for (int p = 0; p < L.k; ++p) idx |= ((rec[base + p * L.chunk] >> bit) & 1) << p;
-  return idx;
+// The P-bit code of coordinate i of a record (index code in bits 0..k-1, the QJL sign
+// in bit k in prod mode).
+__device__ __forceinline__ uint32_t read_code(const uint8_t* rec, const Layout& L, int i) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(rec) + (i >> 5) * L.planes;
+  uint32_t c = 0;
+  for (int b = 0; b < L.planes; ++b) {
+    const int q = code_bit_pos(L.planes, i & 31, b);
+    c |= ((w[q >> 5] >> (q & 31)) & 1u) << b;
+  }
+  return c;
+}
+
+// The P words of group g of a record, into registers (P <= 5).
+__device__ __forceinline__ void load_group(const uint8_t* rec, const Layout& L, int g, uint32_t (&w)[5]) {
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(rec) + g * L.planes;
+  for (int b = 0; b < L.planes; ++b) w[b] = src[b];
 }
 
 // ---------------------------------------------------------------------------- quantize
@@ -140,21 +150,22 @@ __global__ void __launch_bounds__(128) quantize_simt_kernel(
     norm[slot] = f16_bits(nrm[v]);
     if (PROD) rnorm[slot] = zero ? (uint16_t)0 : f16_bits(rn[v]);
   }
-  // pack: one thread per output byte
-  const int nb = L.code_bytes;
-  for (int e = threadIdx.x; e < nv * nb; e += blockDim.x) {
-    int v = e / nb, B = e % nb;
-    int q = B / L.qbytes, r = B % L.qbytes;
-    int p = r / L.chunk, i0 = q * L.quarter + (r % L.chunk) * 8;
-    uint32_t byte = 0;
-#pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      int i = i0 + b;
-      uint32_t bit = (p < L.k) ? ((ids[v * dp + i] >> p) & 1u) : sg[v * dp + i];
-      byte |= (i < d ? bit : 0u) << b;
+  // pack: one thread per output word (every code bit has one place in its group's words)
+  const int P = L.planes, nwords = L.code_bytes / 4;
+  for (int e = threadIdx.x; e < nv * nwords; e += blockDim.x) {
+    const int v = e / nwords, W = e % nwords, g = W / P, wi = W % P;
+    uint32_t word = 0;
+    for (int c = 0; c < 32; ++c) {
+      const int i = g * 32 + c;
+      if (i >= d) break;
+      const uint32_t code = index_code(ids[v * dp + i], L.k) | ((uint32_t)sg[v * dp + i] << L.k);
+      for (int b = 0; b < P; ++b) {
+        const int q = code_bit_pos(P, c, b);
+        if ((q >> 5) == wi) word |= ((code >> b) & 1u) << (q & 31);
+      }
     }
     int64_t slot = slots ? slots[v0 + v] : v0 + v;
-    codes[slot * nb + B] = (uint8_t)byte;
+    reinterpret_cast<uint32_t*>(codes + slot * L.code_bytes)[W] = word;
   }
 }
 
@@ -201,7 +212,7 @@ __global__ void __launch_bounds__(128) dequantize_simt_kernel(
     float val = 0.f;
     if (v < nv && i < d) {
       int64_t slot = slots ? slots[v0 + v] : v0 + v;
-      val = cb.c[read_index(codes + slot * L.code_bytes, L, i)];
+      val = cb.cc[read_code(codes + slot * L.code_bytes, L, i) & (uint32_t)(cb.K - 1)];
     }
     cv[e] = val;
   }
@@ -265,7 +276,7 @@ __global__ void __launch_bounds__(128) logits_simt_kernel(
     qt[e] = ok ? qprep[(a0 + a) * qld + i] : 0.f;
     qs[e] = (ok && prod) ? qprep[(a0 + a) * qld + d + i] : 0.f;
   }
-  if (threadIdx.x < 16) ct[threadIdx.x] = cb.c[threadIdx.x];
+  if (threadIdx.x < 16) ct[threadIdx.x] = cb.cc[threadIdx.x];
   __syncthreads();
   int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= n) return;
@@ -273,15 +284,15 @@ __global__ void __launch_bounds__(128) logits_simt_kernel(
   float mse[QT], qjl[QT];
 #pragma unroll
   for (int a = 0; a < QT; ++a) mse[a] = qjl[a] = 0.f;
-  for (int i0 = 0; i0 < d; i0 += 8) {
-    int base = plane_byte(L, 0, i0);
-    uint32_t pl[5];
-    for (int p = 0; p < L.planes; ++p) pl[p] = rec[base + p * L.chunk];
-    for (int bb = 0; bb < 8 && i0 + bb < d; ++bb) {
-      int i = i0 + bb, idx = 0;
-      for (int p = 0; p < L.k; ++p) idx |= ((pl[p] >> bb) & 1) << p;
-      float c = ct[idx];
-      bool s = prod ? ((pl[L.k] >> bb) & 1) : false;
+  const uint32_t kmask = (uint32_t)(cb.K - 1);
+  for (int g = 0; g * 32 < d; ++g) {
+    uint32_t w[5];
+    load_group(rec, L, g, w);
+    for (int e = 0; e < 32 && g * 32 + e < d; ++e) {
+      const int i = g * 32 + e;
+      const uint32_t code = group_code(w, L.planes, e);
+      float c = ct[code & kmask];
+      bool s = prod ? ((code >> L.k) & 1u) : false;
 #pragma unroll
       for (int a = 0; a < QT; ++a) {
         mse[a] = fmaf(qt[a * dp + i], c, mse[a]);
@@ -353,8 +364,8 @@ __global__ void __launch_bounds__(kDecTile) decode_split_simt_kernel(DecodeArgs 
   }
   if (tid < 16)
     for (int g = 0; g < G; ++g) {
-      cvt[g * 16 + tid] = A.g[g].vcb.c[tid];
-      ckt[g * 16 + tid] = A.g[g].kcb.c[tid];
+      cvt[g * 16 + tid] = A.g[g].vcb.cc[tid];
+      ckt[g * 16 + tid] = A.g[g].kcb.cc[tid];
     }
   float m_run[kMaxRep], l_run[kMaxRep], acc[kMaxRep][2];
 #pragma unroll
@@ -380,16 +391,15 @@ __global__ void __launch_bounds__(kDecTile) decode_split_simt_kernel(DecodeArgs 
         float mse[kMaxRep], qjl[kMaxRep];
 #pragma unroll
         for (int h = 0; h < kMaxRep; ++h) mse[h] = qjl[h] = 0.f;
-        for (int i0 = 0; i0 < L.d; i0 += 8) {
-          int base = plane_byte(L, 0, i0);
-          uint32_t pl[5];
-          for (int p = 0; p < L.planes; ++p) pl[p] = rec[base + p * L.chunk];
-          for (int bb = 0; bb < 8 && i0 + bb < L.d; ++bb) {
-            int idx = 0;
-            for (int p = 0; p < L.k; ++p) idx |= ((pl[p] >> bb) & 1) << p;
-            float c = ckt[g * 16 + idx];
-            bool s = (pl[L.k] >> bb) & 1;
-            int col = gr.off + i0 + bb;
+        const uint32_t kmask = (uint32_t)(gr.kcb.K - 1);
+        for (int gg = 0; gg * 32 < L.d; ++gg) {
+          uint32_t w[5];
+          load_group(rec, L, gg, w);
+          for (int e = 0; e < 32 && gg * 32 + e < L.d; ++e) {
+            const uint32_t code = group_code(w, L.planes, e);
+            float c = ckt[g * 16 + (code & kmask)];
+            bool s = (code >> L.k) & 1u;
+            int col = gr.off + gg * 32 + e;
 #pragma unroll
             for (int h = 0; h < kMaxRep; ++h) {
               if (h < rep) {
@@ -462,13 +472,12 @@ __global__ void __launch_bounds__(kDecTile) decode_split_simt_kernel(DecodeArgs 
       const Layout& L = gr.vl;
       const uint8_t* tile = vcs;
       for (int gg = 0; gg < g; ++gg) tile += kDecTile * A.g[gg].vl.code_bytes;
-      int i = col - gr.off;
-      int base = (i / L.quarter) * L.qbytes + (i % L.quarter) / 8, bit = (i % L.quarter) % 8;
+      const int i = col - gr.off;
+      const uint32_t vmask = (uint32_t)(gr.vcb.K - 1);
       for (int tt = 0; tt < ntok; ++tt) {
         const uint8_t* rec = tile + tt * L.code_bytes;
-        int idx = 0;
-        for (int p = 0; p < L.k; ++p) idx |= ((rec[base + p * L.chunk] >> bit) & 1) << p;
-        float cv = cvt[g * 16 + idx] * vn[g * kDecTile + tt];
+        const uint32_t code = read_code(rec, L, i);
+        float cv = cvt[g * 16 + (code & vmask)] * vn[g * kDecTile + tt];
 #pragma unroll
         for (int h = 0; h < kMaxRep; ++h)
           if (h < rep) acc[h][cc] = fmaf(lg[h * kDecTile + tt], cv, acc[h][cc]);
@@ -567,7 +576,7 @@ __global__ void __launch_bounds__(256) search_block_kernel(
     qt[e] = ok ? qprep[(a0 + a) * qld + i] : 0.f;
     qs[e] = ok ? qprep[(a0 + a) * qld + d + i] : 0.f;
   }
-  if (threadIdx.x < 16) ct[threadIdx.x] = cb.c[threadIdx.x];
+  if (threadIdx.x < 16) ct[threadIdx.x] = cb.cc[threadIdx.x];
   __syncthreads();
   for (int r = threadIdx.x; r < kSearchBlock; r += blockDim.x) {
     int64_t b = n0 + r;
@@ -576,15 +585,15 @@ __global__ void __launch_bounds__(256) search_block_kernel(
     for (int a = 0; a < kSearchQT; ++a) mse[a] = qjl[a] = 0.f;
     if (b < N) {
       const uint8_t* rec = codes + b * L.code_bytes;
-      for (int i0 = 0; i0 < d; i0 += 8) {
-        int base = plane_byte(L, 0, i0);
-        uint32_t pl[5];
-        for (int p = 0; p < L.planes; ++p) pl[p] = rec[base + p * L.chunk];
-        for (int bb = 0; bb < 8 && i0 + bb < d; ++bb) {
-          int i = i0 + bb, idx = 0;
-          for (int p = 0; p < L.k; ++p) idx |= ((pl[p] >> bb) & 1) << p;
-          float c = ct[idx];
-          bool s = (pl[L.k] >> bb) & 1;
+      const uint32_t kmask = (uint32_t)(cb.K - 1);
+      for (int g = 0; g * 32 < d; ++g) {
+        uint32_t w[5];
+        load_group(rec, L, g, w);
+        for (int e = 0; e < 32 && g * 32 + e < d; ++e) {
+          const int i = g * 32 + e;
+          const uint32_t code = group_code(w, L.planes, e);
+          float c = ct[code & kmask];
+          bool s = (code >> L.k) & 1u;
 #pragma unroll
           for (int a = 0; a < kSearchQT; ++a) {
             mse[a] = fmaf(qt[a * dp + i], c, mse[a]);

@@ -15,9 +15,10 @@
 // Roles (576 threads, one persistent CTA per SM): warp 0 issues TMA loads (constants
 // once, then the x tiles one 128-byte K atom at a time), warp 1 allocates TMEM and issues
 // the MMAs, warps 2-17 are the epilogue: thread (row, w) owns vector `row` of the tile and
-// coordinates [w d/4, (w+1) d/4), i.e. exactly one quarter of its packed record.  Two TMEM
-// accumulator buffers (each holding a tile's Pi x, then its QJL projection) and two
-// residual buffers let the MMAs of the next tile run under the epilogue of this one.
+// coordinates [w d/4, (w+1) d/4), i.e. exactly one quarter of its packed record.  TMEM
+// holds two Pi x accumulators (each released as soon as the epilogue has read it, so the
+// Pi x GEMM runs two tiles ahead), one QJL accumulator and one residual operand: the QJL
+// GEMM of tile t runs under the epilogue of tile t + 1, which collects its signs.
 // Every mbarrier wait is bounded; a timeout sets the context's error word and the CTA
 // winds down (in-flight copies and MMAs are drained and TMEM is always released).
 #include <cuda.h>
@@ -35,8 +36,7 @@ using namespace sm100;
 
 constexpr int kTileM = 128;
 constexpr uint64_t kWaitNs = 2000000000ull;   // a pipeline wait longer than 2 s is declared stuck
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColBuf0 = 0, kColR0 = 256;  // accumulators [2] x 128 cols, residuals [2] x 128 cols
+constexpr uint32_t kTmemCols = 512;   // columns [0, 2d): Pi x [2]; [2d, 3d): QJL projection; [3d, 4d): residual
 constexpr float kRScale = 256.f;              // the residual enters the QJL GEMM as r * 2^8 (M as 16 * M)
 constexpr int kEpiWarps = 16;                 // 4 warpgroups: thread = (vector row, quarter of its coords)
 constexpr int kThreads = 64 + 32 * kEpiWarps;
@@ -77,6 +77,44 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// The epilogue's comparisons and bit packing run on the FMA pipe (the integer / compare
+// pipe has half its issue rate): with B = 2^64, sat(|y| B - t B) is exactly [|y| > t]
+// (every nonzero difference of floats near t is far above 2^-64), a selected threshold is
+// an FMA of 0/1 values, and packed bits accumulate exactly as sums of powers of two in
+// 16-bit halves of each word.
+constexpr float kBig = 18446744073709551616.f;   // 2^64
+
+__device__ __forceinline__ float above(float y, float nt) {   // [|y| > t], nt = -t 2^64
+  float d;
+  asm("{\n .reg .f32 a;\n abs.f32 a, %1;\n fma.rn.sat.f32 %0, a, %2, %3;\n}\n" : "=f"(d) : "f"(y), "f"(kBig), "f"(nt));
+  return d;
+}
+__device__ __forceinline__ float positive(float y) {           // [y > 0] for every finite y
+  float u, d;
+  asm("mul.rn.f32 %0, %1, %2;\n" : "=f"(u) : "f"(y), "f"(8.5070591730234616e37f));   // 2^126
+  asm("mul.rn.sat.f32 %0, %1, %2;\n" : "=f"(d) : "f"(u), "f"(8.5070591730234616e37f));
+  return d;
+}
+
+// Bit-packing accumulators: half-words of PW words as exact float sums.
+template <int PW>
+struct PackAcc {
+  float h[2 * PW];
+  __device__ __forceinline__ void clear() {
+#pragma unroll
+    for (int i = 0; i < 2 * PW; ++i) h[i] = 0.f;
+  }
+  // add v (0 or 1) at bit q = 32 word + bit
+  __device__ __forceinline__ void add(int q, float v) { h[q >> 4] = fmaf(v, (float)(1u << (q & 15)), h[q >> 4]); }
+  __device__ __forceinline__ void to_words(uint32_t (&w)[PW]) const {
+#pragma unroll
+    for (int i = 0; i < PW; ++i) {
+      const uint32_t lo = __float_as_uint(h[2 * i] + 8388608.f), hi = __float_as_uint(h[2 * i + 1] + 8388608.f);
+      w[i] = __byte_perm(lo, hi, 0x5410);
+    }
+  }
+};
+
 template <int D, bool PROD, int K>
 __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                                                                   const __grid_constant__ CUtensorMap tm_pi,
@@ -86,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
   constexpr int NK = D / 16;             // k-steps per product
   constexpr int CQ = D / 4;              // coordinates per epilogue thread (one record quarter)
   constexpr int LEVELS = 1 << K;
-  constexpr int P = K + (PROD ? 1 : 0);  // bit planes
+  constexpr int P = K + (PROD ? 1 : 0);  // code bits per coordinate
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* s_n = reinterpret_cast<float*>(smem + SM::OFF_XCH);          // [2][4][128] partial ||y||^2
@@ -95,14 +133,15 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
   uint64_t* full_x = bars;                  // [NSLOT] TMA -> MMA
   uint64_t* empty_x = bars + NSLOT;         // [NSLOT] MMA -> TMA
   uint64_t* const_full = bars + 2 * NSLOT;  // constant operands landed
-  // Every barrier below exists once per accumulator buffer: a barrier completes its next
-  // phase only after each of its waiters has seen the previous one, so parity waits never
-  // skip a phase even when one role runs a whole tile ahead of another.
+  // A barrier completes its next phase only after each of its waiters has seen the
+  // previous one (every chain below closes through the other role), so parity waits never
+  // skip a phase even when one role runs ahead of another.
   uint64_t* y_full = const_full + 1;        // [2] MMA -> epilogue (Pi x ready)
-  uint64_t* z_full = y_full + 2;            // [2] MMA -> epilogue (QJL projection ready)
-  uint64_t* r_full = z_full + 2;            // [2] epilogue -> MMA (residual in TMEM)
-  uint64_t* buf_empty = r_full + 2;         // [2] epilogue -> MMA (accumulator buffer free)
-  uint64_t* xn = buf_empty + 2;             // [2] norm partials written
+  uint64_t* y_empty = y_full + 2;           // [2] epilogue -> MMA (Pi x read into registers)
+  uint64_t* z_full = y_empty + 2;           // MMA -> epilogue (QJL projection ready, residual consumed)
+  uint64_t* z_empty = z_full + 1;           // epilogue -> MMA (QJL projection read)
+  uint64_t* r_full = z_empty + 1;           // epilogue -> MMA (residual in TMEM)
+  uint64_t* xn = r_full + 1;                // [2] norm partials written
   uint64_t* xr = xn + 2;                    // [2] residual-norm partials written
   uint64_t* drain = xr + 2;                 // MMA issuer: every issued MMA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -110,6 +149,9 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ntiles = (A.n + kTileM - 1) / kTileM;
+  // this CTA's tiles: blockIdx.x + t * gridDim.x for t < nloc
+  const int nloc = (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
+  constexpr uint32_t kColZ = 2 * D, kColR = 3 * D;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSLOT; ++s) {
@@ -119,12 +161,13 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
     mbar_init(const_full, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(y_full + b, 1);
-      mbar_init(z_full + b, 1);
-      mbar_init(r_full + b, kEpiThreads);
-      mbar_init(buf_empty + b, kEpiThreads);
+      mbar_init(y_empty + b, kEpiThreads);
       mbar_init(xn + b, kEpiThreads);
       mbar_init(xr + b, kEpiThreads);
     }
+    mbar_init(z_full, 1);
+    mbar_init(z_empty, kEpiThreads);
+    mbar_init(r_full, kEpiThreads);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -183,33 +226,16 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
       const uint32_t pi_addr = smem_u32(smem + SM::OFF_PI), m_addr = smem_u32(smem + SM::OFF_M);
       bool ok = wait(const_full, 0);
       if (!ok) fail(102);
-      // z = (R_hi + R_lo)(M_hi + M_lo) without the lo*lo term, into the tile's buffer
-      auto issue_z = [&](int t) -> bool {
-        const int par = t & 1;
-        if (!wait(r_full + par, (uint32_t)((t >> 1) & 1))) { fail(104); return false; }
+      // Pi x of local tile t into accumulator t & 1 (three bf16 splits of Pi)
+      int64_t q = 0;                      // x atoms consumed
+      auto issue_y = [&](int t) -> bool {
+        const int b = t & 1;
+        if (!wait(y_empty + b, (uint32_t)(((t >> 1) & 1) ^ 1))) { fail(103); return false; }
         tc_fence_after();
-        const uint32_t dz = tmem + kColBuf0 + 128 * par, rz = tmem + kColR0 + 128 * par;
-        for (int sp = 0; sp < 3; ++sp) {
-          const uint32_t a_col = rz + (sp == 2 ? D / 2 : 0);
-          const int msp = (sp == 1) ? 1 : 0;
-          for (int ks = 0; ks < NK; ++ks) {
-            const uint64_t db = desc_sw128(m_addr + msp * SM::M_SPLIT + (ks >> 2) * D * 128 + (ks & 3) * 32);
-            mma_ts(dz, a_col + ks * 8, db, idz, (sp | ks) ? 1u : 0u);
-          }
-        }
-        mma_commit(z_full + par);
-        return true;
-      };
-      int it = 0;
-      int64_t q = 0;
-      for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
-        const int par = it & 1;
-        if (!wait(buf_empty + par, (uint32_t)(((it >> 1) & 1) ^ 1))) { fail(103); ok = false; break; }
-        tc_fence_after();
-        const uint32_t dy = tmem + kColBuf0 + 128 * par;
+        const uint32_t dy = tmem + (uint32_t)(b * D);
         for (int a = 0; a < KA; ++a, ++q) {
           const int s = (int)(q % NSLOT);
-          if (!wait(full_x + s, (uint32_t)((q / NSLOT) & 1))) { fail(103); ok = false; break; }
+          if (!wait(full_x + s, (uint32_t)((q / NSLOT) & 1))) { fail(103); return false; }
           tc_fence_after();
           const uint32_t x_addr = smem_u32(smem + SM::OFF_X + s * SM::ATOM);
           for (int sp = 0; sp < 3; ++sp)
@@ -220,11 +246,33 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
             }
           mma_commit(empty_x + s);
         }
-        if (!ok) break;
-        mma_commit(y_full + par);
-        if (PROD && it >= 1 && !issue_z(it - 1)) { ok = false; break; }
+        mma_commit(y_full + b);
+        return true;
+      };
+      // QJL projection of tile t: (R_hi + R_lo)(M_hi + M_lo) without the lo*lo term
+      auto issue_z = [&](int t) -> bool {
+        if (!wait(r_full, (uint32_t)(t & 1))) { fail(104); return false; }
+        if (!wait(z_empty, (uint32_t)((t & 1) ^ 1))) { fail(104); return false; }
+        tc_fence_after();
+        const uint32_t dz = tmem + kColZ, rz = tmem + kColR;
+        for (int sp = 0; sp < 3; ++sp) {
+          const uint32_t a_col = rz + (sp == 2 ? D / 2 : 0);
+          const int msp = (sp == 1) ? 1 : 0;
+          for (int ks = 0; ks < NK; ++ks) {
+            const uint64_t db = desc_sw128(m_addr + msp * SM::M_SPLIT + (ks >> 2) * D * 128 + (ks & 3) * 32);
+            mma_ts(dz, a_col + ks * 8, db, idz, (sp | ks) ? 1u : 0u);
+          }
+        }
+        mma_commit(z_full);
+        return true;
+      };
+      // Pi x runs two tiles ahead of the epilogue; the QJL GEMM of tile t waits for its
+      // residual (the end of tile t's epilogue)
+      for (int t = 0; ok && t < 2 && t < nloc; ++t) ok = issue_y(t);
+      for (int t = 0; ok && t < nloc; ++t) {
+        if (t + 2 < nloc) ok = issue_y(t + 2);
+        if (ok && PROD) ok = issue_z(t);
       }
-      if (PROD && ok && it >= 1) issue_z(it - 1);
       // every MMA issued above completes before TMEM is released
       mma_commit(drain);
       mbar_wait(drain, 0, nullptr, kWaitNs);
@@ -236,8 +284,15 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
     const int row = tq * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(tq * 32) << 16);
     const int c0 = wg * CQ;
+    // this thread's words of the packed record (the code bit places of the packed format
+    // depend only on the coordinate's place inside its 32-coordinate group)
+    constexpr int PW = P * CQ / 32;
+    auto put = [](uint32_t (&w)[PW], int i, int b, bool bit) {
+      const int q = code_bit_pos(P, i, b);
+      w[q >> 5] |= (bit ? 1u : 0u) << (q & 31);
+    };
     // state of the tile whose QJL signs are still to come
-    uint32_t pend_planes[K];
+    uint32_t pend_words[PW];
     float pend_n = 0.f;
     int64_t pend_v = -1;
     auto load_cols = [&](uint32_t col, float (&v)[CQ]) {
@@ -255,131 +310,131 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
         for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
       }
     };
-    // one record quarter: planes[0..P-1] of this thread's CQ coordinates
-    auto store_quarter = [&](int64_t v, const uint32_t* pl, float nrm, float rn2) {
+    // this thread's PW words of the record (bytes [wg P D/32, (wg+1) P D/32))
+    auto store_quarter = [&](int64_t v, const uint32_t (&pl)[PW], float nrm, float rn2) {
       if (v >= A.n) return;
       const int64_t slot = A.slots ? A.slots[v] : v;
       uint8_t* rec = A.codes + slot * (int64_t)(P * D / 8) + wg * (P * D / 32);
-      if constexpr (CQ == 32) {
-        if constexpr (P == 4) *reinterpret_cast<uint4*>(rec) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
-        else if constexpr (P == 2) *reinterpret_cast<uint2*>(rec) = make_uint2(pl[0], pl[1]);
-        else
+      if constexpr (PW == 4) *reinterpret_cast<uint4*>(rec) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+      else if constexpr (PW == 2) *reinterpret_cast<uint2*>(rec) = make_uint2(pl[0], pl[1]);
+      else {
 #pragma unroll
-          for (int p = 0; p < P; ++p) reinterpret_cast<uint32_t*>(rec)[p] = pl[p];
-      } else {
-        if constexpr (P == 4) *reinterpret_cast<uint2*>(rec) = make_uint2(pl[0] | (pl[1] << 16), pl[2] | (pl[3] << 16));
-        else if constexpr (P == 2) *reinterpret_cast<uint32_t*>(rec) = pl[0] | (pl[1] << 16);
-        else
-#pragma unroll
-          for (int p = 0; p < P; ++p) reinterpret_cast<uint16_t*>(rec)[p] = (uint16_t)pl[p];
+        for (int p = 0; p < PW; ++p) reinterpret_cast<uint32_t*>(rec)[p] = pl[p];
       }
       if (wg == 0) {
         A.norm[slot] = __half_as_ushort(__float2half_rn(nrm));
         if (PROD) A.rnorm[slot] = nrm > 0.f ? __half_as_ushort(__float2half_rn(sqrtf(rn2))) : (uint16_t)0;
       }
     };
-    // signs of tile t's QJL projection, then its record quarter
-    auto finish_z = [&](int t) -> bool {
-      const int par = t & 1;
-      if (!wait(z_full + par, (uint32_t)((t >> 1) & 1))) { fail(106); return false; }
+    // signs of the pending tile's QJL projection (z_full already waited) into the top code
+    // bits of its words; the projection buffer is handed back to the MMA issuer
+    auto take_signs = [&]() {
       tc_fence_after();
       float z[CQ];
-      load_cols(kColBuf0 + 128 * par + c0, z);
-      uint32_t w = 0;
+      load_cols(kColZ + c0, z);
+      tc_fence_before();
+      mbar_arrive(z_empty);
+      PackAcc<PW> pk;
+      pk.clear();
 #pragma unroll
-      for (int i = 0; i < CQ; ++i) w |= (z[i] >= 0.f ? 1u : 0u) << i;
-      if (pend_n == 0.f) w = (CQ == 32) ? 0xFFFFFFFFu : 0xFFFFu;   // zero vector: all signs +1
+      for (int i = 0; i < CQ; ++i) pk.add(code_bit_pos(P, i, P - 1), positive(z[i]));
+      uint32_t sw[PW];
+      pk.to_words(sw);
+      // a projection exactly 0 sits on the sign boundary (counted positive); a zero vector
+      // has all signs +1
+      uint32_t topmask[PW];
+#pragma unroll
+      for (int p = 0; p < PW; ++p) topmask[p] = 0u;
+#pragma unroll
+      for (int i = 0; i < CQ; ++i) put(topmask, i, P - 1, true);
+      const bool zero = pend_n == 0.f;
+#pragma unroll
+      for (int p = 0; p < PW; ++p) pend_words[p] |= zero ? topmask[p] : sw[p];
+    };
+    // the pending tile t's record words, norms last
+    auto finish = [&](int t) -> bool {
       float rn2 = 0.f;
       if (wg == 0) {
-        if (!wait(xr + par, (uint32_t)((t >> 1) & 1))) { fail(107); return false; }
+        const int b = t & 1;
+        if (!wait(xr + b, (uint32_t)((t >> 1) & 1))) { fail(107); return false; }
 #pragma unroll
-        for (int g = 0; g < 4; ++g) rn2 += s_rn[(par * 4 + g) * kTileM + row];
+        for (int g = 0; g < 4; ++g) rn2 += s_rn[(b * 4 + g) * kTileM + row];
       }
-      tc_fence_before();
-      mbar_arrive(buf_empty + par);
-      uint32_t pl[P];
-#pragma unroll
-      for (int p = 0; p < K; ++p) pl[p] = pend_planes[p];
-      pl[P - 1] = w;
-      store_quarter(pend_v, pl, pend_n, rn2);
+      store_quarter(pend_v, pend_words, pend_n, rn2);
       return true;
     };
-    int it = 0;
     bool ok = true;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-      const int par = it & 1;
-      if (!wait(y_full + par, (uint32_t)((it >> 1) & 1))) { fail(105); ok = false; break; }
+    for (int t = 0; t < nloc; ++t) {
+      const int b = t & 1;
+      const int64_t tile = blockIdx.x + (int64_t)t * gridDim.x;
+      if (!wait(y_full + b, (uint32_t)((t >> 1) & 1))) { fail(105); ok = false; break; }
       tc_fence_after();
       float y[CQ];
-      load_cols(kColBuf0 + 128 * par + c0, y);
+      load_cols((uint32_t)(b * D) + c0, y);
+      tc_fence_before();
+      mbar_arrive(y_empty + b);
       float n2p = 0.f;
 #pragma unroll
       for (int i = 0; i < CQ; ++i) n2p = fmaf(y[i], y[i], n2p);
-      s_n[(par * 4 + wg) * kTileM + row] = n2p;
-      mbar_arrive(xn + par);
-      if (!wait(xn + par, (uint32_t)((it >> 1) & 1))) { fail(108); ok = false; break; }
+      s_n[(b * 4 + wg) * kTileM + row] = n2p;
+      mbar_arrive(xn + b);
+      if (!wait(xn + b, (uint32_t)((t >> 1) & 1))) { fail(108); ok = false; break; }
       float n2 = 0.f;
 #pragma unroll
-      for (int g = 0; g < 4; ++g) n2 += s_n[(par * 4 + g) * kTileM + row];
+      for (int g = 0; g < 4; ++g) n2 += s_n[(b * 4 + g) * kTileM + row];
       const float nrm = sqrtf(n2);
-      // nearest centroid by sign and magnitude: y = D / ||x|| > 0 picks the upper half of the
-      // (odd-symmetric) codebook; the magnitude index is a binary search of |D| against the
-      // positive boundaries scaled by ||x|| (so no division per coordinate)
-      float pn[8];
+      // nearest centroid by sign and magnitude on Y = 2^8 D / ||x|| = 2^8 y: Y > 0 picks the
+      // upper half of the (odd-symmetric) codebook, a binary search of |Y| over the positive
+      // boundaries gives the magnitude bits (thresholds selected by FMAs of earlier bits)
+      const float s256 = nrm > 0.f ? kRScale / nrm : 0.f;
+      float nt[7];
 #pragma unroll
-      for (int j = 0; j < LEVELS / 2 - 1; ++j) pn[j] = nrm * A.pos_t[j];
-      const float s256 = nrm > 0.f ? kRScale / nrm : 0.f;   // residual scale r * 2^8 = D s256 - 2^8 c
-      uint32_t S = 0u, B0 = 0u, B1 = 0u, B2 = 0u;
+      for (int j = 0; j < LEVELS / 2 - 1; ++j) nt[j] = -kRScale * kBig * A.pos_t[j];
+      float m2[4];                                   // 2^9 c[L/2 + m] (prod: residual table)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) m2[j] = (j < LEVELS / 2) ? 2.f * kRScale * A.mag[j] : 0.f;
+      PackAcc<PW> pk;
+      pk.clear();
       float rn2p = 0.f;
       float rs[CQ];
 #pragma unroll
       for (int i = 0; i < CQ; ++i) {
-        const float Dv = y[i], a = fabsf(Dv);
-        const bool sp = Dv > 0.f;
-        bool b0 = false, b1 = false, b2 = false;
-        float m = 0.f;
-        if constexpr (K == 1) {
-          if (PROD) m = A.mag[0];
-        } else if constexpr (K == 2) {
-          b0 = a > pn[0];
-          if (PROD) m = b0 ? A.mag[1] : A.mag[0];
+        const float Y = y[i] * s256;
+        const float sp = positive(Y);
+        float b0 = 0.f, b1 = 0.f, b2 = 0.f;
+        if constexpr (K == 2) {
+          b0 = above(Y, nt[0]);
         } else if constexpr (K == 3) {
-          b1 = a > pn[1];
-          b0 = a > (b1 ? pn[2] : pn[0]);
-          if (PROD) m = b1 ? (b0 ? A.mag[3] : A.mag[2]) : (b0 ? A.mag[1] : A.mag[0]);
-        } else {
-          b2 = a > pn[3];
-          b1 = a > (b2 ? pn[5] : pn[1]);
-          b0 = a > (b2 ? (b1 ? pn[6] : pn[4]) : (b1 ? pn[2] : pn[0]));
-          if (PROD)
-            m = b2 ? (b1 ? (b0 ? A.mag[7] : A.mag[6]) : (b0 ? A.mag[5] : A.mag[4]))
-                   : (b1 ? (b0 ? A.mag[3] : A.mag[2]) : (b0 ? A.mag[1] : A.mag[0]));
+          b1 = above(Y, nt[1]);
+          b0 = above(Y, fmaf(b1, nt[2] - nt[0], nt[0]));
+        } else if constexpr (K == 4) {
+          b2 = above(Y, nt[3]);
+          b1 = above(Y, fmaf(b2, nt[5] - nt[1], nt[1]));
+          const float e0 = fmaf(b2, nt[4] - nt[0], nt[0]), e1 = fmaf(b2, nt[6] - nt[2], nt[2]);
+          b0 = above(Y, fmaf(b1, e1, fmaf(-b1, e0, e0)));
         }
-        S |= (uint32_t)sp << i;
-        B0 |= (uint32_t)b0 << i;
-        B1 |= (uint32_t)b1 << i;
-        B2 |= (uint32_t)b2 << i;
-        if (PROD) {
-          const float r = fmaf(Dv, s256, sp ? -kRScale * m : kRScale * m);   // 2^8 (y - c[idx])
+        // sign-magnitude index code: magnitude bits, then the negative-half flag 1 - sp
+        if constexpr (K >= 2) pk.add(code_bit_pos(P, i, 0), b0);
+        if constexpr (K >= 3) pk.add(code_bit_pos(P, i, 1), b1);
+        if constexpr (K >= 4) pk.add(code_bit_pos(P, i, 2), b2);
+        pk.add(code_bit_pos(P, i, K - 1), 1.f - sp);
+        if constexpr (PROD) {
+          // M2 = 2^9 |c|, then r = Y - (2 sp - 1) M2 / 2 = (Y + M2/2) - sp M2
+          float M2 = m2[0];
+          if constexpr (K == 2) {
+            M2 = fmaf(b0, m2[1] - m2[0], m2[0]);
+          } else if constexpr (K == 3) {
+            const float lo = fmaf(b0, m2[1] - m2[0], m2[0]), hi = fmaf(b0, m2[3] - m2[2], m2[2]);
+            M2 = fmaf(b1, hi, fmaf(-b1, lo, lo));
+          }
+          const float r = fmaf(-sp, M2, fmaf(0.5f, M2, Y));
           rn2p = fmaf(r, r, rn2p);
           rs[i] = r;
         }
       }
+      uint32_t words[PW];
+      pk.to_words(words);
       rn2p *= 1.f / (kRScale * kRScale);
-      // idx = L/2 + |idx| (y > 0) or L/2 - 1 - |idx| = (L/2 - 1) ^ |idx| (y <= 0):
-      // bit K-1 is the sign, the lower bits are the magnitude bits, flipped when y <= 0
-      uint32_t planes[P];
-      {
-        const uint32_t nS = ~S;
-        if constexpr (K >= 2) planes[0] = B0 ^ nS;
-        if constexpr (K >= 3) planes[1] = B1 ^ nS;
-        if constexpr (K >= 4) planes[2] = B2 ^ nS;
-        planes[K - 1] = S;
-        if constexpr (CQ == 16) {
-#pragma unroll
-          for (int p = 0; p < K; ++p) planes[p] &= 0xFFFFu;
-        }
-      }
       const int64_t v = tile * kTileM + row;
       if (PROD) {
         uint32_t hi[CQ / 2], lo[CQ / 2];
@@ -390,7 +445,13 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
           hi[i] = pack_h2(h0, h1);
           lo[i] = pack_h2(a0 - h0, a1 - h1);
         }
-        const uint32_t rz = lane_base + kColR0 + 128 * par + c0 / 2;
+        // the QJL GEMM of tile t - 1 has consumed the residual operand once its projection
+        // is complete: collect those signs, then hand over this tile's residual
+        if (t >= 1) {
+          if (!wait(z_full, (uint32_t)((t - 1) & 1))) { fail(106); ok = false; break; }
+          take_signs();
+        }
+        const uint32_t rz = lane_base + kColR + c0 / 2;
         if constexpr (CQ == 32) {
           tmem_st16(rz, hi);
           tmem_st16(rz + D / 2, lo);
@@ -400,21 +461,26 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(r_full + par);
-        s_rn[(par * 4 + wg) * kTileM + row] = rn2p;
-        mbar_arrive(xr + par);
-        if (it >= 1 && !finish_z(it - 1)) { ok = false; break; }
+        mbar_arrive(r_full);
+        s_rn[(b * 4 + wg) * kTileM + row] = rn2p;
+        mbar_arrive(xr + b);
+        if (t >= 1 && !finish(t - 1)) { ok = false; break; }
 #pragma unroll
-        for (int p = 0; p < K; ++p) pend_planes[p] = planes[p];
+        for (int p = 0; p < PW; ++p) pend_words[p] = words[p];
         pend_n = nrm;
         pend_v = v;
       } else {
-        tc_fence_before();
-        mbar_arrive(buf_empty + par);
-        store_quarter(v, planes, nrm, 0.f);
+        store_quarter(v, words, nrm, 0.f);
       }
     }
-    if (PROD && ok && it >= 1) finish_z(it - 1);
+    if (PROD && ok && nloc >= 1) {
+      if (wait(z_full, (uint32_t)((nloc - 1) & 1))) {
+        take_signs();
+        finish(nloc - 1);
+      } else {
+        fail(106);
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -514,8 +580,9 @@ int launch_quantize_tc(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n,
   if (d == DD && prod == PP && k == KK) return launch_tc_t<DD, PP, KK>(ctx, x, n, ld, dst, slots, st);
   TQ_TC_CASE(128, true, 3) TQ_TC_CASE(128, true, 2) TQ_TC_CASE(128, true, 1)
   TQ_TC_CASE(128, false, 4) TQ_TC_CASE(128, false, 3) TQ_TC_CASE(128, false, 2)
-  TQ_TC_CASE(64, true, 3) TQ_TC_CASE(64, true, 2) TQ_TC_CASE(64, true, 1)
-  TQ_TC_CASE(64, false, 4) TQ_TC_CASE(64, false, 3) TQ_TC_CASE(64, false, 2)
+  // d = 64: a thread owns half of a 32-coordinate group, which is whole words only for
+  // 4-bit codes (every other code width shares a word between two threads)
+  TQ_TC_CASE(64, true, 3) TQ_TC_CASE(64, false, 4)
 #undef TQ_TC_CASE
   return kNotHandled;
 }

@@ -1,4 +1,5 @@
 // C ABI of libtq: argument checking, context construction and kernel dispatch.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -186,16 +187,19 @@ int tq_init(tq_ctx** out, int d, int bits, uint64_t seed, int mode) {
   L.d_pad = ((d + 31) / 32) * 32;
   L.planes = h.k + (mode == TQ_MODE_PROD ? 1 : 0);
   L.code_bytes = L.planes * L.d_pad / 8;
-  L.quarter = L.d_pad / 4;
-  L.chunk = L.d_pad / 32;
-  L.qbytes = L.planes * L.chunk;
   Codebook& cb = c->cb;
   cb.K = 1 << h.k;
   for (int j = 0; j < kMaxLevels; ++j) {
     cb.c[j] = j < cb.K ? (float)h.centroids[j] : 0.f;
     cb.t[j] = j < cb.K - 1 ? (float)h.boundaries[j] : INFINITY;
   }
+  for (int code = 0; code < kMaxLevels; ++code) cb.cc[code] = code < cb.K ? cb.c[code_index(code, h.k)] : 0.f;
   c->sqrt_pi_over_2_over_m = mode == TQ_MODE_PROD ? (float)(std::sqrt(M_PI / 2.0) / h.m) : 0.f;
+  for (int j = 0; j < h.m; ++j) {
+    double r = 0.0;
+    for (int i = 0; i < d; ++i) r += h.S[(size_t)j * d + i] * h.S[(size_t)j * d + i];
+    c->s_rowmax = std::max(c->s_rowmax, (float)(std::sqrt(r) * (1.0 + 1e-6)));
+  }
   if ((r = alloc_copy(&c->Pi, h.Pi)) != TQ_OK || (r = alloc_copy(&c->PiT, transpose(h.Pi, d, d))) != TQ_OK) {
     release(c);
     return r;
