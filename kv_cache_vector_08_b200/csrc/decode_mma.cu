@@ -301,19 +301,20 @@ constexpr int kStageTok = kWarps * 16;  // tokens per pipeline stage: one 16-tok
 constexpr int kNStage = 4;
 constexpr uint64_t kDecWaitNs = 2000000000ull;
 
-// Shared-memory layout of one pipeline stage: per group the K and V code bytes of 64
-// consecutive slots (copied with 16-byte granularity, hence 32 bytes of slack) and the
-// three fp16 norm arrays.
+// Shared-memory layout of one pipeline stage: per group the K and V code bytes and the
+// three fp16 norm arrays (key norm, residual norm, value norm) of 64 consecutive slots,
+// each copied with 16-byte granularity (hence 32 bytes of slack per array).
 template <class G0, class G1c, bool TWO>
 struct Stage {
   static constexpr int KB0 = G0::KB, VB0 = G0::VB;
   static constexpr int KB1 = G1c::KB, VB1 = G1c::VB;
+  static constexpr int NB = kStageTok * 2 + 32;                            // one norm array
   static constexpr int OFF_K0 = 0;
   static constexpr int OFF_V0 = OFF_K0 + kStageTok * KB0 + 32;
   static constexpr int OFF_K1 = OFF_V0 + kStageTok * VB0 + 32;
   static constexpr int OFF_V1 = OFF_K1 + (TWO ? kStageTok * KB1 + 32 : 0);
-  static constexpr int OFF_N = OFF_V1 + (TWO ? kStageTok * VB1 + 32 : 0);   // uint16 [G][3][64]
-  static constexpr int BYTES = ((OFF_N + (TWO ? 2 : 1) * 3 * kStageTok * 2) + 127) / 128 * 128;
+  static constexpr int OFF_N = OFF_V1 + (TWO ? kStageTok * VB1 + 32 : 0);   // [G][3] arrays of NB bytes
+  static constexpr int BYTES = ((OFF_N + (TWO ? 2 : 1) * 3 * NB) + 127) / 128 * 128;
 };
 
 // Copy bytes [b0, b1) of a packed array into shared memory at dst + (b0 & 15): one bulk copy
@@ -388,23 +389,22 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
           tx += stage_span(st + ST::OFF_K1, g1.kcodes, first * ST::KB1, last * ST::KB1, g1.kcap * ST::KB1, full + s, issue);
           tx += stage_span(st + ST::OFF_V1, g1.vcodes, first * ST::VB1, last * ST::VB1, g1.vcap * ST::VB1, full + s, issue);
         }
+#pragma unroll
+        for (int gi = 0; gi < (TWO ? 2 : 1); ++gi) {
+          const MmaGroup& gr = A.g[gi];
+          uint8_t* nb = st + ST::OFF_N + gi * 3 * ST::NB;
+          const uint8_t* kn = reinterpret_cast<const uint8_t*>(gr.knorm);
+          const uint8_t* kr = reinterpret_cast<const uint8_t*>(gr.krnorm);
+          const uint8_t* vn = reinterpret_cast<const uint8_t*>(gr.vnorm);
+          tx += stage_span(nb, kn, first * 2, last * 2, gr.kcap * 2, full + s, issue);
+          tx += stage_span(nb + ST::NB, kr, first * 2, last * 2, gr.kcap * 2, full + s, issue);
+          tx += stage_span(nb + 2 * ST::NB, vn, first * 2, last * 2, gr.vcap * 2, full + s, issue);
+        }
         return tx;
       };
       if (lane == 0) {
         mbar_expect_tx(full + s, spans(false));
         spans(true);
-      }
-      uint16_t* nrm = reinterpret_cast<uint16_t*>(st + ST::OFF_N);
-      for (int j = lane; j < kStageTok; j += 32) {
-        const bool ok = j < ntok;
-        const int64_t sl = slot0 + ts + j;
-#pragma unroll
-        for (int gi = 0; gi < (TWO ? 2 : 1); ++gi) {
-          const MmaGroup& gr = A.g[gi];
-          nrm[(gi * 3 + 0) * kStageTok + j] = ok ? __ldg(gr.knorm + sl) : (uint16_t)0;
-          nrm[(gi * 3 + 1) * kStageTok + j] = ok ? __ldg(gr.krnorm + sl) : (uint16_t)0;
-          nrm[(gi * 3 + 2) * kStageTok + j] = ok ? __ldg(gr.vnorm + sl) : (uint16_t)0;
-        }
       }
       __syncwarp();
       mbar_arrive(full + s);
@@ -456,10 +456,16 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
         lds_words(k0.b, kp + jb * ST::KB0, l);
         lds_words(v0.a, vp + ja * ST::VB0, l);
         lds_words(v0.b, vp + jb * ST::VB0, l);
-        const uint16_t* nrm = reinterpret_cast<const uint16_t*>(st + ST::OFF_N);
-        k0.na = h2f(nrm[ja]); k0.nb = h2f(nrm[jb]);
-        k0.ra = h2f(nrm[kStageTok + ja]); k0.rb = h2f(nrm[kStageTok + jb]);
-        v0.na = h2f(nrm[2 * kStageTok + ja]); v0.nb = h2f(nrm[2 * kStageTok + jb]);
+        // norms of slots past the context (staged bytes of other slots) read as 0
+        const bool va = tt + g < t_end, vb = tt + g + 8 < t_end;
+        const int nof = (int)((first * 2) & 15);
+        auto nrm = [&](int gi, int a, int j, bool ok) {
+          const uint16_t* p = reinterpret_cast<const uint16_t*>(st + ST::OFF_N + (gi * 3 + a) * ST::NB + nof);
+          return ok ? h2f(p[j]) : 0.f;
+        };
+        k0.na = nrm(0, 0, ja, va); k0.nb = nrm(0, 0, jb, vb);
+        k0.ra = nrm(0, 1, ja, va); k0.rb = nrm(0, 1, jb, vb);
+        v0.na = nrm(0, 2, ja, va); v0.nb = nrm(0, 2, jb, vb);
         if constexpr (TWO) {
           const uint8_t* kq = st + ST::OFF_K1 + ((first * ST::KB1) & 15);
           const uint8_t* vq = st + ST::OFF_V1 + ((first * ST::VB1) & 15);
@@ -467,9 +473,9 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
           lds_words(k1.b, kq + jb * ST::KB1, l);
           lds_words(v1.a, vq + ja * ST::VB1, l);
           lds_words(v1.b, vq + jb * ST::VB1, l);
-          k1.na = h2f(nrm[3 * kStageTok + ja]); k1.nb = h2f(nrm[3 * kStageTok + jb]);
-          k1.ra = h2f(nrm[4 * kStageTok + ja]); k1.rb = h2f(nrm[4 * kStageTok + jb]);
-          v1.na = h2f(nrm[5 * kStageTok + ja]); v1.nb = h2f(nrm[5 * kStageTok + jb]);
+          k1.na = nrm(1, 0, ja, va); k1.nb = nrm(1, 0, jb, vb);
+          k1.ra = nrm(1, 1, ja, va); k1.rb = nrm(1, 1, jb, vb);
+          v1.na = nrm(1, 2, ja, va); v1.nb = nrm(1, 2, jb, vb);
         }
       }
       __syncwarp();
@@ -799,6 +805,11 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
   using C64_22 = GroupCfg<64, 2, 2>;
   const bool ok = (G == 1 && (sig[0] == 12844 || sig[0] == 12833)) || is(6444, 6433) || is(6433, 6422);
   if (!ok) return kNotHandled;
+  // every staged array is read by bulk copies, which need 16-byte aligned sources
+  auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  for (int g = 0; g < G; ++g)
+    if (!a16(kc[g].codes) || !a16(vc[g].codes) || !a16(kc[g].norm) || !a16(kc[g].rnorm) || !a16(vc[g].norm))
+      return kNotHandled;
 
   const DecodeWs W = decode_ws(B, Hq, Hkv, D, G, max_len);
   if (W.nsplit > 512) return kNotHandled;

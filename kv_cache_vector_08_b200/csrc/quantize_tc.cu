@@ -12,9 +12,10 @@
 // rotated basis, and S r = (S Pi^T) y-residual = M r, so the QJL projection is a second
 // GEMM with A taken straight from tensor memory (hi*hi + hi*lo + lo*hi products).
 //
-// Roles (576 threads, one persistent CTA per SM): warp 0 issues TMA loads (constants
+// Roles (608 threads, one persistent CTA per SM): warp 0 issues TMA loads (constants
 // once, then the x tiles one 128-byte K atom at a time), warp 1 allocates TMEM and issues
-// the MMAs, warps 2-17 are the epilogue: thread (row, w) owns vector `row` of the tile and
+// the Pi x MMAs, warp 18 issues the QJL MMAs (so they wait only for their residual, never
+// for the next x tile), warps 2-17 are the epilogue: thread (row, w) owns vector `row` of the tile and
 // coordinates [w d/4, (w+1) d/4), i.e. exactly one quarter of its packed record.  TMEM
 // holds two Pi x accumulators (each released as soon as the epilogue has read it, so the
 // Pi x GEMM runs two tiles ahead), one QJL accumulator and one residual operand: the QJL
@@ -39,7 +40,8 @@ constexpr uint64_t kWaitNs = 2000000000ull;   // a pipeline wait longer than 2 s
 constexpr uint32_t kTmemCols = 512;   // columns [0, 2d): Pi x [2]; [2d, 3d): QJL projection; [3d, 4d): residual
 constexpr float kRScale = 256.f;              // the residual enters the QJL GEMM as r * 2^8 (M as 16 * M)
 constexpr int kEpiWarps = 16;                 // 4 warpgroups: thread = (vector row, quarter of its coords)
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kThreads = 96 + 32 * kEpiWarps;   // + TMA warp, Pi x issuer warp, QJL issuer warp (last)
+constexpr int kZWarp = 2 + kEpiWarps;
 constexpr int kEpiThreads = 32 * kEpiWarps;
 
 struct QtArgs {
@@ -63,10 +65,13 @@ struct Smem {
   static constexpr int ATOM = kTileM * 128;
   static constexpr int PI_SPLIT = D * D * 2;
   static constexpr int M_SPLIT = D * D * 2;
-  static constexpr int NSLOT = (D == 128 && PROD) ? 3 : 4;
   static constexpr int OFF_PI = 0;
   static constexpr int OFF_M = OFF_PI + 3 * PI_SPLIT;
   static constexpr int OFF_X = OFF_M + (PROD ? 2 * M_SPLIT : 0);
+  // as many x slots as the 227 KB of shared memory leave (the loads take microseconds, so
+  // every extra slot is prefetch depth), at most 8
+  static constexpr int FIXED = OFF_X + 2 * 2 * 4 * kTileM * 4 + 256 + 1024;
+  static constexpr int NSLOT = (232448 - FIXED) / ATOM > 8 ? 8 : (232448 - FIXED) / ATOM;
   static constexpr int OFF_XCH = OFF_X + NSLOT * ATOM;          // float [2][4][128] x 2 (norm partials)
   static constexpr int OFF_BAR = OFF_XCH + 2 * 2 * 4 * kTileM * 4;
   static constexpr int BYTES = OFF_BAR + 256 + 1024;            // barriers + alignment slack
@@ -89,12 +94,33 @@ __device__ __forceinline__ float above(float y, float nt) {   // [|y| > t], nt =
   asm("{\n .reg .f32 a;\n abs.f32 a, %1;\n fma.rn.sat.f32 %0, a, %2, %3;\n}\n" : "=f"(d) : "f"(y), "f"(kBig), "f"(nt));
   return d;
 }
-__device__ __forceinline__ float positive(float y) {           // [y > 0] for every finite y
-  float u, d;
-  asm("mul.rn.f32 %0, %1, %2;\n" : "=f"(u) : "f"(y), "f"(8.5070591730234616e37f));   // 2^126
-  asm("mul.rn.sat.f32 %0, %1, %2;\n" : "=f"(d) : "f"(u), "f"(8.5070591730234616e37f));
+// [y > 0] for every normal y; a denormal y (within 2^-126 of the sign boundary) counts as 0
+__device__ __forceinline__ float positive(float y) {
+  float d;
+  asm("mul.rn.ftz.sat.f32 %0, %1, %2;\n" : "=f"(d) : "f"(y), "f"(8.5070591730234616e37f));   // 2^126
   return d;
 }
+
+// Two fp32 lanes in one 64-bit register (Blackwell's packed f32x2 FMA: one issue slot
+// for two coordinates).
+using f2 = unsigned long long;
+__device__ __forceinline__ f2 f2pack(float a, float b) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2split(f2 r, float& a, float& b) { asm("mov.b64 {%0, %1}, %2;\n" : "=f"(a), "=f"(b) : "l"(r)); }
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+  f2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;\n" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 bcast2(float a) { return f2pack(a, a); }
 
 // Bit-packing accumulators: half-words of PW words as exact float sums.
 template <int PW>
@@ -104,6 +130,15 @@ struct PackAcc {
 #pragma unroll
     for (int i = 0; i < 2 * PW; ++i) h[i] = 0.f;
   }
+  // start from the bits in `mask` set (they are cleared with sub())
+  __device__ __forceinline__ void set(const uint32_t (&mask)[PW]) {
+#pragma unroll
+    for (int i = 0; i < PW; ++i) {
+      h[2 * i] = (float)(mask[i] & 0xFFFFu);
+      h[2 * i + 1] = (float)(mask[i] >> 16);
+    }
+  }
+  __device__ __forceinline__ void sub(int q, float v) { h[q >> 4] = fmaf(v, -(float)(1u << (q & 15)), h[q >> 4]); }
   // add v (0 or 1) at bit q = 32 word + bit
   __device__ __forceinline__ void add(int q, float v) { h[q >> 4] = fmaf(v, (float)(1u << (q & 15)), h[q >> 4]); }
   __device__ __forceinline__ void to_words(uint32_t (&w)[PW]) const {
@@ -143,8 +178,8 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
   uint64_t* r_full = z_empty + 1;           // epilogue -> MMA (residual in TMEM)
   uint64_t* xn = r_full + 1;                // [2] norm partials written
   uint64_t* xr = xn + 2;                    // [2] residual-norm partials written
-  uint64_t* drain = xr + 2;                 // MMA issuer: every issued MMA complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain = xr + 2;                 // [2] MMA issuers (Pi x, QJL): every issued MMA complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -169,6 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
     mbar_init(z_empty, kEpiThreads);
     mbar_init(r_full, kEpiThreads);
     mbar_init(drain, 1);
+    mbar_init(drain + 1, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -220,22 +256,23 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
         if (pending[s] >= 0) mbar_wait(full_x + s, (uint32_t)pending[s], nullptr, kWaitNs);
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------------------- MMA issuer
+    // ------------------------------------------------------------------ Pi x MMA issuer
     if (lane == 0) {
-      const uint32_t idy = idesc_f16(kTileM, D, 1), idz = idesc_f16(kTileM, D, 0);
-      const uint32_t pi_addr = smem_u32(smem + SM::OFF_PI), m_addr = smem_u32(smem + SM::OFF_M);
+      const uint32_t idy = idesc_f16(kTileM, D, 1);
+      const uint32_t pi_addr = smem_u32(smem + SM::OFF_PI);
       bool ok = wait(const_full, 0);
       if (!ok) fail(102);
-      // Pi x of local tile t into accumulator t & 1 (three bf16 splits of Pi)
+      // Pi x of local tile t into accumulator t & 1 (three bf16 splits of Pi); it runs
+      // two tiles ahead of the epilogue
       int64_t q = 0;                      // x atoms consumed
-      auto issue_y = [&](int t) -> bool {
+      for (int t = 0; ok && t < nloc; ++t) {
         const int b = t & 1;
-        if (!wait(y_empty + b, (uint32_t)(((t >> 1) & 1) ^ 1))) { fail(103); return false; }
+        if (!wait(y_empty + b, (uint32_t)(((t >> 1) & 1) ^ 1))) { fail(103); break; }
         tc_fence_after();
         const uint32_t dy = tmem + (uint32_t)(b * D);
         for (int a = 0; a < KA; ++a, ++q) {
           const int s = (int)(q % NSLOT);
-          if (!wait(full_x + s, (uint32_t)((q / NSLOT) & 1))) { fail(103); return false; }
+          if (!wait(full_x + s, (uint32_t)((q / NSLOT) & 1))) { fail(103); ok = false; break; }
           tc_fence_after();
           const uint32_t x_addr = smem_u32(smem + SM::OFF_X + s * SM::ATOM);
           for (int sp = 0; sp < 3; ++sp)
@@ -246,13 +283,25 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
             }
           mma_commit(empty_x + s);
         }
+        if (!ok) break;
         mma_commit(y_full + b);
-        return true;
-      };
-      // QJL projection of tile t: (R_hi + R_lo)(M_hi + M_lo) without the lo*lo term
-      auto issue_z = [&](int t) -> bool {
-        if (!wait(r_full, (uint32_t)(t & 1))) { fail(104); return false; }
-        if (!wait(z_empty, (uint32_t)((t & 1) ^ 1))) { fail(104); return false; }
+      }
+      // every MMA issued above completes before TMEM is released
+      mma_commit(drain);
+      mbar_wait(drain, 0, nullptr, kWaitNs);
+    }
+  } else if (warp == kZWarp) {
+    // ------------------------------------------------------------------- QJL MMA issuer
+    if (PROD && lane == 0) {
+      const uint32_t idz = idesc_f16(kTileM, D, 0);
+      const uint32_t m_addr = smem_u32(smem + SM::OFF_M);
+      bool ok = wait(const_full, 0);
+      if (!ok) fail(102);
+      // QJL projection of tile t: (R_hi + R_lo)(M_hi + M_lo) without the lo*lo term, as
+      // soon as the epilogue has written the residual and read the previous projection
+      for (int t = 0; ok && t < nloc; ++t) {
+        if (!wait(r_full, (uint32_t)(t & 1))) { fail(104); break; }
+        if (!wait(z_empty, (uint32_t)((t & 1) ^ 1))) { fail(104); break; }
         tc_fence_after();
         const uint32_t dz = tmem + kColZ, rz = tmem + kColR;
         for (int sp = 0; sp < 3; ++sp) {
@@ -264,18 +313,9 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
           }
         }
         mma_commit(z_full);
-        return true;
-      };
-      // Pi x runs two tiles ahead of the epilogue; the QJL GEMM of tile t waits for its
-      // residual (the end of tile t's epilogue)
-      for (int t = 0; ok && t < 2 && t < nloc; ++t) ok = issue_y(t);
-      for (int t = 0; ok && t < nloc; ++t) {
-        if (t + 2 < nloc) ok = issue_y(t + 2);
-        if (ok && PROD) ok = issue_z(t);
       }
-      // every MMA issued above completes before TMEM is released
-      mma_commit(drain);
-      mbar_wait(drain, 0, nullptr, kWaitNs);
+      mma_commit(drain + 1);
+      mbar_wait(drain + 1, 0, nullptr, kWaitNs);
     }
   } else {
     // ------------------------------------------------------------------------ epilogue
@@ -363,6 +403,25 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
       store_quarter(pend_v, pend_words, pend_n, rn2);
       return true;
     };
+    // per-kernel constants: scaled negative thresholds, the 2^9 magnitude table, and the
+    // places of the negative-half flags (set, then cleared for positive coordinates)
+    float nt[7];
+#pragma unroll
+    for (int j = 0; j < 7; ++j) nt[j] = (j < LEVELS / 2 - 1) ? -kRScale * kBig * A.pos_t[j] : 0.f;
+    float m2[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m2[j] = (j < LEVELS / 2) ? 2.f * kRScale * A.mag[j] : 0.f;
+    const f2 c_nt0 = bcast2(nt[0]), c_nt1 = bcast2(nt[1]), c_nt2 = bcast2(nt[2]);
+    const f2 c_d20 = bcast2(nt[2] - nt[0]), c_d51 = bcast2(nt[5] - nt[1]);
+    const f2 c_d40 = bcast2(nt[4] - nt[0]), c_d62 = bcast2(nt[6] - nt[2]);
+    const f2 c_m1 = bcast2(-1.f), c_mhalf = bcast2(-0.5f);
+    const f2 c_nm0 = bcast2(-m2[0]), c_nm2 = bcast2(-m2[2]);
+    const f2 c_nd10 = bcast2(m2[0] - m2[1]), c_nd32 = bcast2(m2[2] - m2[3]);
+    uint32_t nflags[PW];
+#pragma unroll
+    for (int p = 0; p < PW; ++p) nflags[p] = 0u;
+#pragma unroll
+    for (int i = 0; i < CQ; ++i) put(nflags, i, K - 1, true);
     bool ok = true;
     for (int t = 0; t < nloc; ++t) {
       const int b = t & 1;
@@ -373,9 +432,18 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
       load_cols((uint32_t)(b * D) + c0, y);
       tc_fence_before();
       mbar_arrive(y_empty + b);
-      float n2p = 0.f;
+      float n2p;
+      {
+        f2 n2 = 0ull;
 #pragma unroll
-      for (int i = 0; i < CQ; ++i) n2p = fmaf(y[i], y[i], n2p);
+        for (int i = 0; i < CQ; i += 2) {
+          const f2 v = f2pack(y[i], y[i + 1]);
+          n2 = fma2(v, v, n2);
+        }
+        float a, c;
+        f2split(n2, a, c);
+        n2p = a + c;
+      }
       s_n[(b * 4 + wg) * kTileM + row] = n2p;
       mbar_arrive(xn + b);
       if (!wait(xn + b, (uint32_t)((t >> 1) & 1))) { fail(108); ok = false; break; }
@@ -387,50 +455,67 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
       // upper half of the (odd-symmetric) codebook, a binary search of |Y| over the positive
       // boundaries gives the magnitude bits (thresholds selected by FMAs of earlier bits)
       const float s256 = nrm > 0.f ? kRScale / nrm : 0.f;
-      float nt[7];
-#pragma unroll
-      for (int j = 0; j < LEVELS / 2 - 1; ++j) nt[j] = -kRScale * kBig * A.pos_t[j];
-      float m2[4];                                   // 2^9 c[L/2 + m] (prod: residual table)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) m2[j] = (j < LEVELS / 2) ? 2.f * kRScale * A.mag[j] : 0.f;
       PackAcc<PW> pk;
-      pk.clear();
-      float rn2p = 0.f;
+      pk.set(nflags);
       float rs[CQ];
+      f2 rn2 = 0ull;
+      const f2 S2 = bcast2(s256);
 #pragma unroll
-      for (int i = 0; i < CQ; ++i) {
-        const float Y = y[i] * s256;
-        const float sp = positive(Y);
-        float b0 = 0.f, b1 = 0.f, b2 = 0.f;
+      for (int i = 0; i < CQ; i += 2) {
+        float Ya, Yb;
+        const f2 Y2 = mul2(f2pack(y[i], y[i + 1]), S2);
+        f2split(Y2, Ya, Yb);
+        const float spa = positive(Ya), spb = positive(Yb);
+        float b0a = 0.f, b0b = 0.f, b1a = 0.f, b1b = 0.f, b2a = 0.f, b2b = 0.f;
         if constexpr (K == 2) {
-          b0 = above(Y, nt[0]);
+          b0a = above(Ya, nt[0]);
+          b0b = above(Yb, nt[0]);
         } else if constexpr (K == 3) {
-          b1 = above(Y, nt[1]);
-          b0 = above(Y, fmaf(b1, nt[2] - nt[0], nt[0]));
+          b1a = above(Ya, nt[1]);
+          b1b = above(Yb, nt[1]);
+          float ta, tb;
+          f2split(fma2(f2pack(b1a, b1b), c_d20, c_nt0), ta, tb);
+          b0a = above(Ya, ta);
+          b0b = above(Yb, tb);
         } else if constexpr (K == 4) {
-          b2 = above(Y, nt[3]);
-          b1 = above(Y, fmaf(b2, nt[5] - nt[1], nt[1]));
-          const float e0 = fmaf(b2, nt[4] - nt[0], nt[0]), e1 = fmaf(b2, nt[6] - nt[2], nt[2]);
-          b0 = above(Y, fmaf(b1, e1, fmaf(-b1, e0, e0)));
+          b2a = above(Ya, nt[3]);
+          b2b = above(Yb, nt[3]);
+          const f2 B2 = f2pack(b2a, b2b);
+          float ta, tb;
+          f2split(fma2(B2, c_d51, c_nt1), ta, tb);
+          b1a = above(Ya, ta);
+          b1b = above(Yb, tb);
+          const f2 E0 = fma2(B2, c_d40, c_nt0), E1 = fma2(B2, c_d62, c_nt2);
+          f2split(fma2(f2pack(b1a, b1b), fma2(E0, c_m1, E1), E0), ta, tb);
+          b0a = above(Ya, ta);
+          b0b = above(Yb, tb);
         }
         // sign-magnitude index code: magnitude bits, then the negative-half flag 1 - sp
-        if constexpr (K >= 2) pk.add(code_bit_pos(P, i, 0), b0);
-        if constexpr (K >= 3) pk.add(code_bit_pos(P, i, 1), b1);
-        if constexpr (K >= 4) pk.add(code_bit_pos(P, i, 2), b2);
-        pk.add(code_bit_pos(P, i, K - 1), 1.f - sp);
+        if constexpr (K >= 2) { pk.add(code_bit_pos(P, i, 0), b0a); pk.add(code_bit_pos(P, i + 1, 0), b0b); }
+        if constexpr (K >= 3) { pk.add(code_bit_pos(P, i, 1), b1a); pk.add(code_bit_pos(P, i + 1, 1), b1b); }
+        if constexpr (K >= 4) { pk.add(code_bit_pos(P, i, 2), b2a); pk.add(code_bit_pos(P, i + 1, 2), b2b); }
+        pk.sub(code_bit_pos(P, i, K - 1), spa);
+        pk.sub(code_bit_pos(P, i + 1, K - 1), spb);
         if constexpr (PROD) {
-          // M2 = 2^9 |c|, then r = Y - (2 sp - 1) M2 / 2 = (Y + M2/2) - sp M2
-          float M2 = m2[0];
+          // -M = -2^9 |c| from the magnitude bits, then r = (Y + M/2) - sp M
+          f2 NM = c_nm0;
           if constexpr (K == 2) {
-            M2 = fmaf(b0, m2[1] - m2[0], m2[0]);
+            NM = fma2(f2pack(b0a, b0b), c_nd10, c_nm0);
           } else if constexpr (K == 3) {
-            const float lo = fmaf(b0, m2[1] - m2[0], m2[0]), hi = fmaf(b0, m2[3] - m2[2], m2[2]);
-            M2 = fmaf(b1, hi, fmaf(-b1, lo, lo));
+            const f2 B0 = f2pack(b0a, b0b);
+            const f2 NLO = fma2(B0, c_nd10, c_nm0), NHI = fma2(B0, c_nd32, c_nm2);
+            NM = fma2(f2pack(b1a, b1b), fma2(NLO, c_m1, NHI), NLO);
           }
-          const float r = fmaf(-sp, M2, fmaf(0.5f, M2, Y));
-          rn2p = fmaf(r, r, rn2p);
-          rs[i] = r;
+          const f2 R = fma2(f2pack(spa, spb), NM, fma2(c_mhalf, NM, Y2));
+          rn2 = fma2(R, R, rn2);
+          f2split(R, rs[i], rs[i + 1]);
         }
+      }
+      float rn2p;
+      {
+        float a, c;
+        f2split(rn2, a, c);
+        rn2p = a + c;
       }
       uint32_t words[PW];
       pk.to_words(words);
