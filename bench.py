@@ -345,10 +345,89 @@ def run_gpu(args):
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
+    line["rows"] = measure_rows(bench, peaks)
     line["cpu_baseline"] = cpu_baseline(w, w.kv_heads)
     print(json.dumps(line), flush=True)
     if ws > 1:
         torch.distributed.destroy_process_group()
+
+
+# ------------------------------------------------------------- the other path rows
+def _time_device(fn, flush, reps):
+    """Median device time (s) of fn() over reps, L2 flushed before every rep."""
+    import torch
+    st = torch.cuda.current_stream()
+    fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush(st)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        fn()
+        b.record(st)
+        b.synchronize()
+        ts.append(a.elapsed_time(b) / 1e3)
+    return float(np.median(ts))
+
+
+def fp32_fma_peak_tflops():
+    """CUDA-core fp32 peak from unit counts and clocks: 148 SMs x 128 FMA lanes x 2 flop x
+    the maximum SM clock (1965 MHz)."""
+    return 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def measure_rows(bench, peaks, reps=5):
+    """Time the hot-path rows that the decode step does not call (standalone logits,
+    dequantize, index + search) on bounded synthetic workloads, each against its roofline.
+    Runs after the timed step; not part of the step time."""
+    import torch
+    tq, dev = bench.tq, bench.dev
+    out = {}
+    flush = bench.flush_l2
+
+    def entry(t, bound, work, peak, unit, extra):
+        a = work / t / (1e9 if unit == "GB/s" else 1e12)
+        return dict(extra, us=t * 1e6, bound=bound, achieved=a, peak=peak, unit=unit, frac=a / peak)
+
+    # standalone logits of 4 queries against all 262,144 cached keys of the layer
+    kctx, kc = bench.kctx[0], bench.kc[0]
+    n = bench.vectors
+    q4 = torch.randn((4, bench.D), device=dev, generator=torch.Generator(device=dev).manual_seed(11))
+    lg = torch.empty((4, n), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(int(tq.lib().tq_attn_logits_workspace_size(kctx.handle, 4)), 1), dtype=torch.uint8,
+                     device=dev)
+    t = _time_device(lambda: tq.attn_logits(kctx, q4, kc, n, out=lg, workspace=ws), flush, reps)
+    nbytes = n * (kctx.code_bytes + 4) + 4 * n * 4
+    out["logits"] = entry(t, "hbm", nbytes, peaks["hbm"], "GB/s",
+                          {"work": "4 queries x 262144 keys (d=128, 4-bit prod)", "bytes": nbytes})
+    # dequantize the 262,144 value vectors of the layer (x = ||x|| Pi^T c[idx])
+    vctx, vc = bench.vctx[0], bench.vc[0]
+    xo = torch.empty((n, bench.D), dtype=torch.float32, device=dev)
+    t = _time_device(lambda: tq.dequantize(vctx, vc, n, out=xo), flush, reps)
+    flops = 2.0 * bench.D * bench.D * n
+    out["dequantize"] = entry(t, "alu", flops, fp32_fma_peak_tflops(), "TFLOP/s",
+                              {"work": "262144 value vectors (d=128, 4-bit MSE)", "flops": flops,
+                               "hbm_floor_us": (n * (vctx.code_bytes + 2) + n * bench.D * 4) / peaks["hbm"] / 1e3,
+                               "peak_source": "fp32 FMA lanes x clock (148 x 128 x 2 x 1.965 GHz)"})
+    # index + top-10 search at d = 1536 (200,000 database rows, 1000 queries) and
+    # d = 200 (1,000,000 rows, 1000 queries); unit-norm Gaussian vectors
+    for d, ndb in ((1536, 200_000), (200, 1_000_000)):
+        g = torch.Generator(device=dev).manual_seed(7)
+        db = torch.nn.functional.normalize(torch.randn((ndb, d), generator=g, device=dev), dim=1)
+        qs = torch.nn.functional.normalize(torch.randn((1000, d), generator=g, device=dev), dim=1)
+        ctx = tq.Context(d, 4, 12, tq.MODE_PROD)
+        pk = tq.alloc_packed(ctx, ndb, dev)
+        t_idx = _time_device(lambda: tq.quantize_kv(ctx, db, pk), flush, 2)
+        t_s = _time_device(lambda: tq.search_topk(ctx, qs, pk, ndb, 10), flush, 2)
+        fl = 4.0 * d * 1000 * ndb
+        out["search_d%d" % d] = entry(t_s, "tensor", fl, peaks["bf16"], "TFLOP/s",
+                                      {"work": "1000 queries x %d rows, top-10" % ndb, "flops": fl,
+                                       "index_us": t_idx * 1e6,
+                                       "index_vectors_per_s": ndb / t_idx,
+                                       "peak_source": "measured bf16 dense burst"})
+        del db, qs, pk, ctx
+    return out
 
 
 def run_e2e(bench, st, steps, warmup):

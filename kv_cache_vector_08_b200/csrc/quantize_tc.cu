@@ -70,11 +70,14 @@ struct Smem {
   static constexpr int OFF_X = OFF_M + (PROD ? 2 * M_SPLIT : 0);
   // as many x slots as the 227 KB of shared memory leave (the loads take microseconds, so
   // every extra slot is prefetch depth), at most 8
-  static constexpr int FIXED = OFF_X + 2 * 2 * 4 * kTileM * 4 + 256 + 1024;
+  // d = 64: code words shared by the two threads of a 32-coordinate group meet here
+  static constexpr int XW = D == 64 ? 2 * kTileM * 4 * 3 * 4 : 0;   // uint32 [2][128][4][3]
+  static constexpr int FIXED = OFF_X + 2 * 2 * 4 * kTileM * 4 + XW + 512 + 1024;
   static constexpr int NSLOT = (232448 - FIXED) / ATOM > 8 ? 8 : (232448 - FIXED) / ATOM;
   static constexpr int OFF_XCH = OFF_X + NSLOT * ATOM;          // float [2][4][128] x 2 (norm partials)
-  static constexpr int OFF_BAR = OFF_XCH + 2 * 2 * 4 * kTileM * 4;
-  static constexpr int BYTES = OFF_BAR + 256 + 1024;            // barriers + alignment slack
+  static constexpr int OFF_XW = OFF_XCH + 2 * 2 * 4 * kTileM * 4;
+  static constexpr int OFF_BAR = OFF_XW + XW;
+  static constexpr int BYTES = OFF_BAR + 512 + 1024;            // barriers + alignment slack
 };
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
@@ -179,7 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
   uint64_t* xn = r_full + 1;                // [2] norm partials written
   uint64_t* xr = xn + 2;                    // [2] residual-norm partials written
   uint64_t* drain = xr + 2;                 // [2] MMA issuers (Pi x, QJL): every issued MMA complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+  uint64_t* pairb = drain + 2;              // [8 pairs][2] d = 64: the two threads of a group met
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pairb + 16);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -205,6 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
     mbar_init(r_full, kEpiThreads);
     mbar_init(drain, 1);
     mbar_init(drain + 1, 1);
+    for (int i = 0; i < 16; ++i) mbar_init(pairb + i, 64);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -325,8 +330,13 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
     const uint32_t lane_base = tmem + ((uint32_t)(tq * 32) << 16);
     const int c0 = wg * CQ;
     // this thread's words of the packed record (the code bit places of the packed format
-    // depend only on the coordinate's place inside its 32-coordinate group)
-    constexpr int PW = P * CQ / 32;
+    // depend only on the coordinate's place inside its 32-coordinate group).  At d = 64 a
+    // thread holds half a group; for 4-bit codes that is two whole words, otherwise the
+    // two threads of a group share every word (SHARED): each builds the group's words
+    // from its own coordinates, as if they were slices 0-1, and the pair combines them.
+    constexpr bool SHARED = (D == 64 && P != 4);
+    constexpr int PW = SHARED ? P : P * CQ / 32;
+    uint32_t* s_xw = reinterpret_cast<uint32_t*>(smem + SM::OFF_XW);
     auto put = [](uint32_t (&w)[PW], int i, int b, bool bit) {
       const int q = code_bit_pos(P, i, b);
       w[q >> 5] |= (bit ? 1u : 0u) << (q & 31);
@@ -350,18 +360,48 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
         for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
       }
     };
-    // this thread's PW words of the record (bytes [wg P D/32, (wg+1) P D/32))
-    auto store_quarter = [&](int64_t v, const uint32_t (&pl)[PW], float nrm, float rn2) {
-      if (v >= A.n) return;
-      const int64_t slot = A.slots ? A.slots[v] : v;
-      uint8_t* rec = A.codes + slot * (int64_t)(P * D / 8) + wg * (P * D / 32);
-      if constexpr (PW == 4) *reinterpret_cast<uint4*>(rec) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
-      else if constexpr (PW == 2) *reinterpret_cast<uint2*>(rec) = make_uint2(pl[0], pl[1]);
-      else {
+    // this thread's PW words of the record (bytes [wg P D/32, (wg+1) P D/32)); SHARED: the
+    // even thread of the pair stores the group's P words.  Every thread of both warps of
+    // a pair reaches the pair barrier (rows past n only skip the global stores).
+    auto store_quarter = [&](int t, int64_t v, const uint32_t (&pl)[PW], float nrm, float rn2) {
+      const int tpar = t & 1;
+      const bool live = v < A.n;
+      const int64_t slot = live ? (A.slots ? A.slots[v] : v) : 0;
+      if constexpr (SHARED) {
+        const int odd = wg & 1;
+        uint32_t w[PW];
 #pragma unroll
-        for (int p = 0; p < PW; ++p) reinterpret_cast<uint32_t*>(rec)[p] = pl[p];
+        for (int p = 0; p < PW; ++p) w[p] = pl[p];
+        if (odd) {             // slices 2-3: low-bit words two places up, top bits 4 places down
+#pragma unroll
+          for (int p = 0; p < PW - 1; ++p) w[p] <<= 2;
+          w[PW - 1] >>= 4;
+        }
+        uint32_t* mine = s_xw + ((tpar * kTileM + row) * 4 + wg) * 3;
+#pragma unroll
+        for (int p = 0; p < PW; ++p) mine[p] = w[p];
+        uint64_t* pb = pairb + ((wg >> 1) * 4 + tq) * 2 + tpar;
+        mbar_arrive(pb);
+        if (!wait(pb, (uint32_t)((t >> 1) & 1))) {
+          fail(109);
+          return;
+        }
+        if (!odd && live) {
+          const uint32_t* other = mine + 3;
+          uint32_t* rec = reinterpret_cast<uint32_t*>(A.codes + slot * (int64_t)(P * D / 8)) + (wg >> 1) * P;
+#pragma unroll
+          for (int p = 0; p < PW; ++p) rec[p] = w[p] | other[p];
+        }
+      } else if (live) {
+        uint8_t* rec = A.codes + slot * (int64_t)(P * D / 8) + wg * (P * D / 32);
+        if constexpr (PW == 4) *reinterpret_cast<uint4*>(rec) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+        else if constexpr (PW == 2) *reinterpret_cast<uint2*>(rec) = make_uint2(pl[0], pl[1]);
+        else {
+#pragma unroll
+          for (int p = 0; p < PW; ++p) reinterpret_cast<uint32_t*>(rec)[p] = pl[p];
+        }
       }
-      if (wg == 0) {
+      if (live && wg == 0) {
         A.norm[slot] = __half_as_ushort(__float2half_rn(nrm));
         if (PROD) A.rnorm[slot] = nrm > 0.f ? __half_as_ushort(__float2half_rn(sqrtf(rn2))) : (uint16_t)0;
       }
@@ -400,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
 #pragma unroll
         for (int g = 0; g < 4; ++g) rn2 += s_rn[(b * 4 + g) * kTileM + row];
       }
-      store_quarter(pend_v, pend_words, pend_n, rn2);
+      store_quarter(t, pend_v, pend_words, pend_n, rn2);
       return true;
     };
     // per-kernel constants: scaled negative thresholds, the 2^9 magnitude table, and the
@@ -555,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
         pend_n = nrm;
         pend_v = v;
       } else {
-        store_quarter(v, words, nrm, 0.f);
+        store_quarter(t, v, words, nrm, 0.f);
       }
     }
     if (PROD && ok && nloc >= 1) {
@@ -665,9 +705,8 @@ int launch_quantize_tc(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n,
   if (d == DD && prod == PP && k == KK) return launch_tc_t<DD, PP, KK>(ctx, x, n, ld, dst, slots, st);
   TQ_TC_CASE(128, true, 3) TQ_TC_CASE(128, true, 2) TQ_TC_CASE(128, true, 1)
   TQ_TC_CASE(128, false, 4) TQ_TC_CASE(128, false, 3) TQ_TC_CASE(128, false, 2)
-  // d = 64: a thread owns half of a 32-coordinate group, which is whole words only for
-  // 4-bit codes (every other code width shares a word between two threads)
-  TQ_TC_CASE(64, true, 3) TQ_TC_CASE(64, false, 4)
+  TQ_TC_CASE(64, true, 3) TQ_TC_CASE(64, true, 2) TQ_TC_CASE(64, true, 1)
+  TQ_TC_CASE(64, false, 4) TQ_TC_CASE(64, false, 3) TQ_TC_CASE(64, false, 2)
 #undef TQ_TC_CASE
   return kNotHandled;
 }

@@ -77,6 +77,7 @@ def test_quantize_toy_config_fp32():
     (128, 2, 0, 700, "bf16"), (128, 3, 1, 700, "bf16"), (128, 2, 1, 700, "bf16"),   # tensor-core variants
     (64, 2, 1, 300, "bf16"), (128, 4, 0, 40000, "bf16"), (64, 4, 1, 40000, "bf16"),  # many tiles per CTA
     (128, 4, 1, 40000, "bf16"), (64, 3, 0, 40000, "bf16"), (128, 2, 0, 38000, "bf16"),
+    (64, 2, 0, 40000, "bf16"), (64, 3, 1, 40001, "bf16"), (64, 2, 1, 39999, "bf16"),   # d = 64 shared words
 ])
 def test_quantize_matches_oracle(d, bits, mode, n, dtype):
     seed = 1000 + 2 * bits + mode
