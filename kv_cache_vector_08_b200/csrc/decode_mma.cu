@@ -34,23 +34,17 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "mma_ops.cuh"
 #include "sm100.cuh"
 
 namespace tq {
 namespace {
 
 using namespace sm100;
+using namespace mmaops;
 
 constexpr int kWarps = 4;
 constexpr int kRep = 4;            // query heads per kv head handled by this kernel
-constexpr float kFix = 32000.f;    // fixed-point range of queries and key centroids (< 2^15)
-
-__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                       uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -64,15 +58,6 @@ __device__ __forceinline__ uint32_t movT(uint32_t x) {
   asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
   return y;
 }
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
-}
-
-// 0xFF in every byte whose msb is set, 0x00 elsewhere (prmt sign replication)
-__device__ __forceinline__ uint32_t msb_bytes(uint32_t x) { return prmt(x, x, 0xBA98u); }
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
@@ -143,13 +128,6 @@ __device__ __forceinline__ uint32_t top_bits(const Words<DG, P>& r, int u, int h
   if constexpr (P == 4) return h ? (r.w[u] << 4) : r.w[u];
   else return r.w[P - 1] << (2 * u + h);
 }
-
-// Lookup tables, built on the host from the contexts' codebooks: key centroids by code as
-// two int8 digits of round(c * kc_scale) (hi = floor((C+128)/256), lo = C - 256 hi), value
-// magnitudes c[K/2 + m] as fp16 low / high bytes.  8 entries = 2 registers per table.
-struct Luts {
-  uint32_t kh[2], kl[2], vlo[2], vhi[2];
-};
 
 // Per-group kernel arguments.
 struct MmaGroup {
@@ -577,66 +555,74 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
   allow_dependent_launch();
 }
 
-// Prepared queries of the kRep query heads of one (sequence, kv head) for one group, 64
-// outputs per CTA (blockIdx.y selects them; outputs o < d_g are Pi q, the rest S q), as
-// 16-bit fixed point: round(Pi q * 32000/|q_g|) and round(S q * 32000/(|q_g| max_j |S_j|)),
-// both bounded by 32000 in magnitude (|(Pi q)_o| <= |q_g|, |(S q)_o| <= |S_o| |q_g|).  The
-// 64 needed columns of Pi^T or S^T are staged in shared memory with 16-byte loads, all in
-// flight at once; thread (head, o) takes its dot product from shared memory.
+// Prepared queries of the kRep query rows grp*kRep .. +kRep-1 for one group and one part
+// (blockIdx.y = 0: Pi q, 1: S q), as 16-bit fixed point round(v * 32000 / max_o |v_o|) per
+// row, so every digit pair stays in range and the rounding is 2^-15 of the row's largest
+// output.  The d_g columns of Pi^T or S^T are staged in shared memory with 16-byte loads,
+// all in flight at once; thread (row, o) computes outputs o and o + 64.  Rows >= nrows
+// (padding of the last block) read as zero.
 template <typename T>
-__global__ void __launch_bounds__(256) decode_prep_kernel(const T* __restrict__ q, int D, int off, int dg,
-                                                          const float* __restrict__ PiT, const float* __restrict__ ST,
-                                                          float s_rowmax, int16_t* __restrict__ qfix,
-                                                          float* __restrict__ qinv, int G, int gi) {
-  __shared__ __align__(16) float ms[128 * 64];
+__global__ void __launch_bounds__(256) decode_prep_kernel(const T* __restrict__ q, int ldq, int off, int dg,
+                                                          int nrows, const float* __restrict__ PiT,
+                                                          const float* __restrict__ ST, int16_t* __restrict__ qfix,
+                                                          float* __restrict__ qinv, int D, int G, int gi) {
+  extern __shared__ float4 prep_smem[];
+  float* ms = reinterpret_cast<float*>(prep_smem);   // [dg][dg]
   __shared__ float qs[kRep][128];
-  __shared__ float qn[kRep];
+  __shared__ float red[8];
   allow_dependent_launch();
-  const int grp = blockIdx.x;                    // = b * Hkv + hk; rows grp*kRep .. +kRep-1
-  const int o0 = blockIdx.y * 64;                // first output of this CTA
-  const float* M = o0 < dg ? PiT + o0 : ST + (o0 - dg);
+  const int grp = blockIdx.x, part = blockIdx.y;
+  const float* M = part == 0 ? PiT : ST;
   float4* m4 = reinterpret_cast<float4*>(ms);
   {
-    float4 r[8];                                 // dg <= 128: at most 8 loads per thread
+    const int n4 = dg * dg / 4;                 // <= 4096 float4: at most 16 per thread
+    float4 r[16];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 16; ++u) {
       const int e = threadIdx.x + u * 256;
-      if (e < dg * 16) r[u] = __ldg(reinterpret_cast<const float4*>(M + (size_t)(e >> 4) * dg) + (e & 15));
+      if (e < n4) r[u] = __ldg(reinterpret_cast<const float4*>(M) + e);
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 16; ++u) {
       const int e = threadIdx.x + u * 256;
-      if (e < dg * 16) m4[e] = r[u];
+      if (e < n4) m4[e] = r[u];
     }
   }
   for (int e = threadIdx.x; e < kRep * dg; e += blockDim.x) {
     const int h = e / dg, j = e % dg;
-    const size_t at = (size_t)(grp * kRep + h) * D + off + j;
-    if constexpr (std::is_same<T, float>::value) qs[h][j] = q[at];
-    else qs[h][j] = __bfloat162float(q[at]);
+    const int rowq = grp * kRep + h;
+    float v = 0.f;
+    if (rowq < nrows) {
+      const size_t at = (size_t)rowq * ldq + off + j;
+      if constexpr (std::is_same<T, float>::value) v = q[at];
+      else v = __bfloat162float(q[at]);
+    }
+    qs[h][j] = v;
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp < kRep) {
-    float s = 0.f;
-    for (int j = lane; j < dg; j += 32) s = fmaf(qs[warp][j], qs[warp][j], s);
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) qn[warp] = sqrtf(s);
-  }
   const int h = threadIdx.x >> 6, oc = threadIdx.x & 63;
-  float a0 = 0.f, a1 = 0.f;
+  float o0 = 0.f, o1 = 0.f;
+  if (oc < dg) {
 #pragma unroll 8
-  for (int j = 0; j < dg; j += 2) {
-    a0 = fmaf(ms[j * 64 + oc], qs[h][j], a0);
-    a1 = fmaf(ms[(j + 1) * 64 + oc], qs[h][j + 1], a1);
+    for (int j = 0; j < dg; ++j) o0 = fmaf(ms[j * dg + oc], qs[h][j], o0);
   }
+  if (oc + 64 < dg) {
+#pragma unroll 8
+    for (int j = 0; j < dg; ++j) o1 = fmaf(ms[j * dg + oc + 64], qs[h][j], o1);
+  }
+  // per-row max |output|: the 64 threads of row h are warps 2h and 2h+1
+  float mx = fmaxf(fabsf(o0), fabsf(o1));
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[warp] = mx;
   __syncthreads();
-  const bool sq = o0 >= dg;
-  const float bound = sq ? qn[h] * s_rowmax : qn[h];
-  const float sc = bound > 0.f ? kFix / bound : 0.f;
+  mx = fmaxf(red[2 * h], red[2 * h + 1]);
+  const float sc = mx > 0.f ? kFix / mx : 0.f;
   const size_t row = (size_t)(grp * kRep + h) * G + gi;
-  qfix[row * 2 * D + (sq ? D + o0 - dg : o0) + oc] = (int16_t)__float2int_rn((a0 + a1) * sc);
-  if (oc == 0 && (o0 == 0 || o0 == dg)) qinv[row * 2 + (sq ? 1 : 0)] = bound / kFix;
+  int16_t* dst = qfix + row * 2 * D + part * D;
+  if (oc < dg) dst[oc] = (int16_t)__float2int_rn(o0 * sc);
+  if (oc + 64 < dg) dst[oc + 64] = (int16_t)__float2int_rn(o1 * sc);
+  if (oc == 0) qinv[row * 2 + part] = mx / kFix;
 }
 
 // Log-sum-exp merge of the context splits and the inverse rotation of the value groups:
@@ -737,6 +723,174 @@ __global__ void __launch_bounds__(256) decode_merge_mma_kernel(Merge2Args A) {
     A.out[(size_t)row * D + c] = (red[0][oc] + red[1][oc]) + (red[2][oc] + red[3][oc]);
 }
 
+// Prepared queries of nrows rows (blocks of kRep) for one group.
+int launch_prep(const void* q, int q_dtype, int ldq, int off, int dg, int nrows, const tq_ctx* kc, int16_t* qfix,
+                float* qinv, int D, int G, int gi, cudaStream_t st) {
+  const dim3 grid((nrows + kRep - 1) / kRep, 2);
+  const size_t smem = (size_t)dg * dg * sizeof(float);
+  cudaError_t e;
+  if (q_dtype == TQ_DTYPE_F32) {
+    e = cudaFuncSetAttribute(decode_prep_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_prep_kernel)");
+    decode_prep_kernel<float><<<grid, 256, smem, st>>>(static_cast<const float*>(q), ldq, off, dg, nrows, kc->PiT,
+                                                       kc->ST, qfix, qinv, D, G, gi);
+  } else {
+    e = cudaFuncSetAttribute(decode_prep_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_prep_kernel)");
+    decode_prep_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(q), ldq, off, dg,
+                                                               nrows, kc->PiT, kc->ST, qfix, qinv, D, G, gi);
+  }
+  count_launch();
+  return check_launch("decode_prep_kernel");
+}
+
+// Words of a record from global memory (same shapes as lds_words).
+template <int DG, int P>
+__device__ __forceinline__ void ldg_words(Words<DG, P>& r, const uint8_t* rec, int l) {
+  if constexpr (DG == 128 && P == 4) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(rec + 16 * l));
+    r.w[0] = v.x; r.w[1] = v.y; r.w[2] = v.z; r.w[3] = v.w;
+  } else if constexpr (DG == 64 && P == 4) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(rec + 8 * l));
+    r.w[0] = v.x; r.w[1] = v.y;
+  } else if constexpr (DG == 128) {
+    const uint32_t* p = reinterpret_cast<const uint32_t*>(rec + 4 * P * l);
+#pragma unroll
+    for (int i = 0; i < P; ++i) r.w[i] = __ldg(p + i);
+  } else {
+    const uint32_t* p = reinterpret_cast<const uint32_t*>(rec + 4 * P * (l >> 1));
+#pragma unroll
+    for (int i = 0; i < P; ++i) r.w[i] = __ldg(p + i);
+    const int odd = l & 1;
+    if constexpr (P == 3) {
+      r.w[0] >>= 2 * odd;
+      r.w[1] >>= 2 * odd;
+    } else {
+      r.w[0] >>= 2 * odd;
+    }
+    r.w[P - 1] <<= 4 * odd;
+  }
+}
+
+// Standalone attention logits on the tensor cores.  A logit is compared to the float64
+// definition at 1e-3 absolute, about 2^-17 of |q||k| for unit-scale d = 128 vectors, so
+// this kernel carries both operands at ~2^-22: centroids as fp16 hi + lo (two A
+// operands), the prepared query Pi q / S q as fp16 hi + lo in the 8 columns (4 queries x
+// hi/lo), products exact in the fp32 accumulator (m16n8k16).  CTA = (key range, block of
+// kRep queries), 4 warps; every warp scores 16 keys per step.
+struct LogitArgs {
+  const uint8_t* codes;
+  const uint16_t* norm;
+  const uint16_t* rnorm;
+  const float* qprep;     // [nq][2d]: (Pi q, S q) in fp32
+  int64_t n, keys_per_cta;
+  int nq, d;
+  float coef;
+  uint32_t ch[2][2], cl[2][2];   // fp16 centroid tables by code: [low byte, high byte] of c_hi, c_lo
+  float* out;
+};
+
+// fp16 pairs of coordinates (4h, 4h+1), (4h+2, 4h+3) of a half-slice from byte tables
+__device__ __forceinline__ void lookup16(const uint32_t (&t)[2][2], uint32_t sel, uint32_t& x01, uint32_t& x23) {
+  const uint32_t L = prmt(t[0][0], t[0][1], sel), H = prmt(t[1][0], t[1][1], sel);
+  x01 = prmt(L, H, 0x5140u);
+  x23 = prmt(L, H, 0x7362u);
+}
+// +-1.0 in fp16 for the same coordinates: msb of byte t of `top` set -> +1 (sign bit [S r >= 0])
+__device__ __forceinline__ void signs16(uint32_t top, uint32_t& x01, uint32_t& x23) {
+  const uint32_t H = (~top & 0x80808080u) | 0x3C3C3C3Cu;   // fp16 high bytes of +1 / -1
+  x01 = prmt(0u, H, 0x5040u);
+  x23 = prmt(0u, H, 0x7060u);
+}
+
+template <class GC>
+__global__ void __launch_bounds__(128) logits_mma_kernel(LogitArgs A) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, l = lane & 3;
+  const int qb = blockIdx.y;
+  // B fragments: column g = query qb*kRep + g/2, hi (g even) or lo part; k-slots of
+  // (slice u, half h) = this thread's coordinates CQ l + 8u + 4h + {0, 1 | 2, 3}
+  uint32_t bm[GC::NS][2][2], bs[GC::NS][2][2];
+  {
+    const int qrow = qb * kRep + (g >> 1);
+    const bool lo = (g & 1) != 0;
+    const float* src = A.qprep + (size_t)(qrow < A.nq ? qrow : 0) * 2 * A.d;
+    const bool ok = qrow < A.nq;
+    auto part = [&](float v) {
+      if (!ok) return 0.f;
+      const float h = __half2float(__float2half_rn(v));
+      return lo ? v - h : h;
+    };
+#pragma unroll
+    for (int u = 0; u < GC::NS; ++u)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c = GC::CQ * l + 8 * u + 4 * h;
+        bm[u][h][0] = pack_h2(part(src[c]), part(src[c + 1]));
+        bm[u][h][1] = pack_h2(part(src[c + 2]), part(src[c + 3]));
+        bs[u][h][0] = pack_h2(part(src[A.d + c]), part(src[A.d + c + 1]));
+        bs[u][h][1] = pack_h2(part(src[A.d + c + 2]), part(src[A.d + c + 3]));
+      }
+  }
+  const int64_t k0 = (int64_t)blockIdx.x * A.keys_per_cta;
+  const int64_t k1 = min(A.n, k0 + A.keys_per_cta);
+  const int qi = qb * kRep + l;
+  for (int64_t base = k0 + warp * 16; base < k1; base += 64) {
+    const int64_t ka = base + g, kb = base + g + 8;
+    const bool va = ka < k1, vb = kb < k1;
+    Words<GC::DG, GC::PK> wa, wb;
+#pragma unroll
+    for (int i = 0; i < Words<GC::DG, GC::PK>::N; ++i) wa.w[i] = wb.w[i] = 0u;
+    if (va) ldg_words(wa, A.codes + ka * GC::KB, l);
+    if (vb) ldg_words(wb, A.codes + kb * GC::KB, l);
+    float mse[4] = {0.f, 0.f, 0.f, 0.f}, sgn[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < GC::NS; ++u) {
+      const uint32_t sa = low_sel(wa, u), sb = low_sel(wb, u);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t xa = h ? sa >> 16 : sa, xb = h ? sb >> 16 : sb;
+        uint32_t a01, a23, b01, b23;
+        lookup16(A.ch, xa, a01, a23);
+        lookup16(A.ch, xb, b01, b23);
+        mma16816(mse, a01, b01, a23, b23, bm[u][h][0], bm[u][h][1]);
+        lookup16(A.cl, xa, a01, a23);
+        lookup16(A.cl, xb, b01, b23);
+        mma16816(mse, a01, b01, a23, b23, bm[u][h][0], bm[u][h][1]);
+        signs16(top_bits(wa, u, h), a01, a23);
+        signs16(top_bits(wb, u, h), b01, b23);
+        mma16816(sgn, a01, b01, a23, b23, bs[u][h][0], bs[u][h][1]);
+      }
+    }
+    const float na = va ? h2f(__ldg(A.norm + ka)) : 0.f, ra = va ? h2f(__ldg(A.rnorm + ka)) : 0.f;
+    const float nb = vb ? h2f(__ldg(A.norm + kb)) : 0.f, rb = vb ? h2f(__ldg(A.rnorm + kb)) : 0.f;
+    const float la = na * fmaf(A.coef * ra, sgn[0] + sgn[1], mse[0] + mse[1]);
+    const float lb = nb * fmaf(A.coef * rb, sgn[2] + sgn[3], mse[2] + mse[3]);
+    if (qi < A.nq) {
+      if (va) A.out[(size_t)qi * A.n + ka] = la;
+      if (vb) A.out[(size_t)qi * A.n + kb] = lb;
+    }
+  }
+}
+
+template <class GC>
+int launch_logits_t(LogitArgs A, cudaStream_t st) {
+  const int nqb = (A.nq + kRep - 1) / kRep;
+  // about 4 CTAs per SM in total (the query fragments are built once per CTA), whole
+  // 64-key steps per CTA
+  int64_t ctas = (int64_t)148 * 4 / nqb;
+  if (ctas < 1) ctas = 1;
+  int64_t per = (A.n + ctas - 1) / ctas;
+  per = ((per + 63) / 64) * 64;
+  if (per < 64) per = 64;
+  A.keys_per_cta = per;
+  const int64_t nblk = (A.n + per - 1) / per;
+  logits_mma_kernel<GC><<<dim3((unsigned)nblk, (unsigned)nqb), 128, 0, st>>>(A);
+  count_launch();
+  return check_launch("logits_mma_kernel");
+}
+
 template <class G0, class G1>
 int launch_mma_t(const MmaArgs& A, int nsplit, int BHkv, cudaStream_t st) {
   constexpr bool TWO = !std::is_same<G1, void>::value;
@@ -763,7 +917,7 @@ int launch_mma_t(const MmaArgs& A, int nsplit, int BHkv, cudaStream_t st) {
 }  // namespace
 
 // Tables of one (key context, value context) pair; returns the key-centroid scale inverse.
-float host_luts(const tq_ctx* kc, const tq_ctx* vc, Luts* t) {
+float mmaops::host_luts(const tq_ctx* kc, const tq_ctx* vc, Luts* t) {
   *t = Luts{};
   const Codebook& kb = kc->cb;
   float cmax = 0.f;
@@ -818,17 +972,7 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
   float* qinv = reinterpret_cast<float*>(base + W.qp + (((size_t)B * Hq * G * 2 * D * 2 + 255) / 256) * 256);
   float* part = reinterpret_cast<float*>(base + W.part);
   for (int g = 0; g < G; ++g) {
-    const int dg = kctx[g]->lay.d;
-    const dim3 pgrid(B * Hkv, 2 * dg / 64);
-    if (q_dtype == TQ_DTYPE_F32)
-      decode_prep_kernel<float><<<pgrid, 256, 0, st>>>(static_cast<const float*>(q), D, off[g], dg, kctx[g]->PiT,
-                                                       kctx[g]->ST, kctx[g]->s_rowmax, qfix, qinv, G, g);
-    else
-      decode_prep_kernel<__nv_bfloat16><<<pgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), D, off[g], dg,
-                                                               kctx[g]->PiT, kctx[g]->ST, kctx[g]->s_rowmax, qfix,
-                                                               qinv, G, g);
-    count_launch();
-    int r = check_launch("decode_prep_kernel");
+    int r = launch_prep(q, q_dtype, D, off[g], kctx[g]->lay.d, B * Hq, kctx[g], qfix, qinv, D, G, g, st);
     if (r != TQ_OK) return r;
   }
   MmaArgs A{};
@@ -869,6 +1013,40 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
   count_launch();
   if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(decode_merge_mma_kernel)");
   return check_launch("decode_merge_mma_kernel");
+}
+
+// Standalone logits for prod contexts with d in {64, 128} and 2..4 code bits: workspace
+// holds the prepared queries in fp32 ([nq][2d]); kNotHandled otherwise.
+size_t logits_mma_workspace(int64_t nq, int d) { return (size_t)nq * 2 * d * sizeof(float); }
+
+int launch_logits_mma(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* keys, int64_t n, float* out,
+                      void* ws, cudaStream_t st) {
+  const int d = ctx->lay.d, P = ctx->lay.planes;
+  if (ctx->mode != TQ_MODE_PROD || (d != 64 && d != 128) || P < 2 || P > 4) return kNotHandled;
+  if (nq > (int64_t)kRep * 65535) return kNotHandled;
+  if ((reinterpret_cast<uintptr_t>(keys->codes) & 15) != 0) return kNotHandled;
+  float* qprep = static_cast<float*>(ws);
+  int r = launch_prepare_queries(ctx, q, TQ_DTYPE_F32, nq, d, qprep, 2 * d, st);
+  if (r != TQ_OK) return r;
+  LogitArgs A{};
+  A.codes = keys->codes; A.norm = keys->norm; A.rnorm = keys->rnorm; A.qprep = qprep;
+  A.n = n; A.nq = (int)nq; A.d = d; A.coef = ctx->sqrt_pi_over_2_over_m; A.out = out;
+  const Codebook& cb = ctx->cb;
+  for (int code = 0; code < cb.K && code < 8; ++code) {
+    const __half h = __float2half_rn(cb.cc[code]);
+    const __half lo = __float2half_rn(cb.cc[code] - __half2float(h));
+    const uint16_t bh = *reinterpret_cast<const uint16_t*>(&h), bl = *reinterpret_cast<const uint16_t*>(&lo);
+    A.ch[0][code / 4] |= (uint32_t)(bh & 0xFF) << (8 * (code % 4));
+    A.ch[1][code / 4] |= (uint32_t)(bh >> 8) << (8 * (code % 4));
+    A.cl[0][code / 4] |= (uint32_t)(bl & 0xFF) << (8 * (code % 4));
+    A.cl[1][code / 4] |= (uint32_t)(bl >> 8) << (8 * (code % 4));
+  }
+  if (d == 128 && P == 4) return launch_logits_t<GroupCfg<128, 4, 4>>(A, st);
+  if (d == 128 && P == 3) return launch_logits_t<GroupCfg<128, 3, 3>>(A, st);
+  if (d == 128) return launch_logits_t<GroupCfg<128, 2, 2>>(A, st);
+  if (P == 4) return launch_logits_t<GroupCfg<64, 4, 4>>(A, st);
+  if (P == 3) return launch_logits_t<GroupCfg<64, 3, 3>>(A, st);
+  return launch_logits_t<GroupCfg<64, 2, 2>>(A, st);
 }
 
 }  // namespace tq

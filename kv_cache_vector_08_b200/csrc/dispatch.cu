@@ -26,8 +26,15 @@ int launch_quantize(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, in
   return launch_quantize_simt(ctx, x, x_dtype, n, ld, dst, slots, st);
 }
 
-int launch_logits(const tq_ctx* ctx, const float* qprep, int64_t nq, const tq_packed* keys, int64_t n,
-                  float* logits, cudaStream_t st) {
+int launch_logits(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* keys, int64_t n, float* logits,
+                  void* ws, cudaStream_t st) {
+  if (!force_simt()) {
+    int r = launch_logits_mma(ctx, q, nq, keys, n, logits, ws, st);
+    if (r != kNotHandled) return r;
+  }
+  float* qprep = static_cast<float*>(ws);
+  int r = launch_prepare_queries(ctx, q, TQ_DTYPE_F32, nq, ctx->lay.d, qprep, ctx->lay.d + ctx->m, st);
+  if (r != TQ_OK) return r;
   return launch_logits_simt(ctx, qprep, nq, keys, n, logits, st);
 }
 
@@ -41,6 +48,15 @@ int launch_decode(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const in
   }
   return launch_decode_simt(kctx, vctx, off, G, q, q_dtype, kc, vc, seq_lens, B, Hq, Hkv, D, max_len, scale, out, ws,
                             st);
+}
+
+int launch_search(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* db, int64_t N, int k,
+                  float* scores, int64_t* ids, void* ws, cudaStream_t st) {
+  if (!force_simt()) {
+    int r = launch_search_mma(ctx, q, nq, db, N, k, scores, ids, ws, st);
+    if (r != kNotHandled) return r;
+  }
+  return launch_search_simt(ctx, q, nq, db, N, k, scores, ids, ws, st);
 }
 
 }  // namespace tq

@@ -33,7 +33,15 @@ int launch_decode_merge(const tq_ctx* const* vctx, const int* off, int G, const 
 int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G, const void* q,
                       int q_dtype, const tq_packed* kc, const tq_packed* vc, const int32_t* seq_lens, int B, int Hq,
                       int Hkv, int D, int64_t max_len, float scale, float* out, void* ws, cudaStream_t st);
+size_t logits_mma_workspace(int64_t nq, int d);
+int launch_logits_mma(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* keys, int64_t n, float* out,
+                      void* ws, cudaStream_t st);
 size_t search_workspace_bytes(const tq_ctx* ctx, int64_t nq, int64_t N, int k);
+size_t search_mma_workspace(const tq_ctx* ctx, int64_t nq, int64_t N, int k);
+int launch_search_mma(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* db, int64_t N, int k,
+                      float* scores, int64_t* ids, void* ws, cudaStream_t st);
+int launch_search_merge(float* cand_s, int64_t* cand_i, int64_t nq, int64_t ncand, int k, float* scores, int64_t* ids,
+                        cudaStream_t st);
 int launch_search_simt(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* db, int64_t N, int k,
                        float* scores, int64_t* ids, void* ws, cudaStream_t st);
 
@@ -43,9 +51,11 @@ namespace tq {
 // Dispatchers: pick the fastest kernel family that supports the shape.
 int launch_quantize(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld, const tq_packed* dst,
                     const int64_t* slots, cudaStream_t st);
-int launch_logits(const tq_ctx* ctx, const float* qprep, int64_t nq, const tq_packed* keys, int64_t n,
-                  float* logits, cudaStream_t st);
+int launch_logits(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* keys, int64_t n, float* logits,
+                  void* ws, cudaStream_t st);
 int launch_decode(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G, const void* q,
                   int q_dtype, const tq_packed* kc, const tq_packed* vc, const int32_t* seq_lens, int B, int Hq,
                   int Hkv, int D, int64_t max_len, float scale, float* out, void* ws, cudaStream_t st);
+int launch_search(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* db, int64_t N, int k,
+                  float* scores, int64_t* ids, void* ws, cudaStream_t st);
 }  // namespace tq

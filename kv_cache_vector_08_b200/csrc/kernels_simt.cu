@@ -863,7 +863,12 @@ int launch_search_simt(const tq_ctx* ctx, const float* q, int64_t nq, const tq_p
   count_launch();
   r = check_launch("search_block_kernel");
   if (r != TQ_OK) return r;
-  search_merge_kernel<<<(unsigned)nq, 256, 0, st>>>(cs, ci, nblk * k, k, scores, ids);
+  return launch_search_merge(cs, ci, nq, nblk * k, k, scores, ids, st);
+}
+
+int launch_search_merge(float* cand_s, int64_t* cand_i, int64_t nq, int64_t ncand, int k, float* scores, int64_t* ids,
+                        cudaStream_t st) {
+  search_merge_kernel<<<(unsigned)nq, 256, 0, st>>>(cand_s, cand_i, ncand, k, scores, ids);
   count_launch();
   return check_launch("search_merge_kernel");
 }

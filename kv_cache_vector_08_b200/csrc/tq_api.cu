@@ -310,7 +310,11 @@ int tq_prepare_queries(const tq_ctx* ctx, const float* q, int64_t nq, int64_t ld
 
 size_t tq_attn_logits_workspace_size(const tq_ctx* ctx, int64_t nq) {
   if (!ctx || nq < 0) return 0;
-  return (size_t)nq * (ctx->lay.d + ctx->m) * sizeof(float);
+  // the larger of the two kernel families' needs (prepared queries in fp32, or in
+  // 16-bit fixed point with per-row scales)
+  const size_t simt = (size_t)nq * (ctx->lay.d + ctx->m) * sizeof(float);
+  const size_t mma = logits_mma_workspace(nq, ctx->lay.d);
+  return simt > mma ? simt : mma;
 }
 
 int tq_attn_logits(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* keys, int64_t n, float* logits,
@@ -325,10 +329,7 @@ int tq_attn_logits(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packe
   if (need > 0 && (!workspace || ws_bytes < need)) return fail(TQ_ERR_WORKSPACE, "workspace too small");
   if ((r = check_device(ctx)) != TQ_OK) return r;
   if (nq == 0 || n == 0) return TQ_OK;
-  float* qprep = static_cast<float*>(workspace);
-  r = launch_prepare_queries(ctx, q, TQ_DTYPE_F32, nq, ctx->lay.d, qprep, ctx->lay.d + ctx->m, (cudaStream_t)stream);
-  if (r != TQ_OK) return r;
-  return launch_logits(ctx, qprep, nq, keys, n, logits, (cudaStream_t)stream);
+  return launch_logits(ctx, q, nq, keys, n, logits, workspace, (cudaStream_t)stream);
 }
 
 size_t tq_decode_workspace_size(int B, int Hq, int Hkv, int D, int ngroups, int64_t max_len) {
@@ -372,7 +373,9 @@ int tq_decode_attention(const tq_ctx* const* kctx, const tq_ctx* const* vctx, co
 
 size_t tq_search_workspace_size(const tq_ctx* ctx, int64_t nq, int64_t N, int k) {
   if (!ctx || nq < 0 || N < 0 || k < 1) return 0;
-  return search_workspace_bytes(ctx, nq, N, k);
+  const size_t simt = search_workspace_bytes(ctx, nq, N, k);
+  const size_t mma = search_mma_workspace(ctx, nq, N, k);
+  return simt > mma ? simt : mma;
 }
 
 int tq_search_topk(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* db, int64_t N, int k,
@@ -388,7 +391,7 @@ int tq_search_topk(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packe
   size_t need = tq_search_workspace_size(ctx, nq, N, k);
   if (!workspace || ws_bytes < need) return fail(TQ_ERR_WORKSPACE, "workspace too small");
   if ((r = check_device(ctx)) != TQ_OK) return r;
-  return launch_search_simt(ctx, q, nq, db, N, k, scores, ids, workspace, (cudaStream_t)stream);
+  return launch_search(ctx, q, nq, db, N, k, scores, ids, workspace, (cudaStream_t)stream);
 }
 
 }  // extern "C"
