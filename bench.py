@@ -336,11 +336,11 @@ def run_gpu(args):
             "decode_frac_of_8tbs": dec_bytes / t_dec_alone / 1e9 / NOMINAL_HBM_GBS,
         },
         "timing": "device time of CUDA-graph replays of the library calls (captured once), L2 flushed before each step",
-        "roofline": dict(roof(dominant), traffic=None),
+        "roofline": dict(roof(dominant), traffic=recorded_traffic(dominant)),
         "roofline_quantize_values": roof("quantize_values"),
         "roofline_decode": {"bound": "hbm", "achieved": dec_bytes / t_dec_alone / 1e9, "peak": peaks["hbm"],
                             "unit": "GB/s", "frac": dec_bytes / t_dec_alone / 1e9 / peaks["hbm"],
-                            "bytes_per_launch": dec_bytes},
+                            "bytes_per_launch": dec_bytes, "traffic": recorded_traffic("decode_attention")},
         "e2e": e2e,
         "gpu_launches": int(launches),
         "clocks": clocks,
@@ -369,6 +369,22 @@ def _time_device(fn, flush, reps):
         b.synchronize()
         ts.append(a.elapsed_time(b) / 1e3)
     return float(np.median(ts))
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu record (profiles/), or None when the
+    kernel's source has changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "dram_traffic_llama_32k.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["sha256"]:
+        return None
+    return rec["bytes_per_launch"]
 
 
 def fp32_fma_peak_tflops():

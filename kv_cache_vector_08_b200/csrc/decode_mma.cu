@@ -637,25 +637,27 @@ struct Merge2Args {
   float* out;
 };
 
-__global__ void __launch_bounds__(256) decode_merge_mma_kernel(Merge2Args A) {
+constexpr int kMergeThreads = 512;   // 8 row parts of the rotation, up to 4 split partitions
+
+__global__ void __launch_bounds__(kMergeThreads) decode_merge_mma_kernel(Merge2Args A) {
   __shared__ float s_acc[4][256];
   __shared__ float s_ml[4][256][2];
-  __shared__ float red[4][64];
+  __shared__ float red[8][64];
   const int row = blockIdx.x, c0 = blockIdx.y * 64;
   const int D = A.D, ns = A.nsplit;
-  // rotation column of this thread's output, quarter qtr of its rows (before the wait)
+  // rotation column of this thread's output, eighth qtr of its rows (before the wait)
   const int oc = threadIdx.x & 63, qtr = threadIdx.x >> 6;
   const int c = c0 + oc;
-  float pv[32];
+  float pv[16];
   int gsel = 0, goff = 0, gd = 0;
   if (c < D) {
     gsel = (A.G > 1 && c >= A.off[1]) ? 1 : 0;
     goff = A.off[gsel];
     gd = A.off[gsel + 1] - goff;
     const float* Pi = A.PiV[gsel] + (c - goff);
-    const int i0 = qtr * (gd / 4), n = gd / 4;   // n <= 32
+    const int i0 = qtr * (gd / 8), n = gd / 8;   // n <= 16
 #pragma unroll
-    for (int u = 0; u < 32; ++u) pv[u] = (u < n) ? __ldg(Pi + (size_t)(i0 + u) * gd) : 0.f;
+    for (int u = 0; u < 16; ++u) pv[u] = (u < n) ? __ldg(Pi + (size_t)(i0 + u) * gd) : 0.f;
   }
   grid_dependency_wait();
   // merged rotated-basis accumulator: thread (coordinate i, half hs) runs over splits
@@ -712,15 +714,16 @@ __global__ void __launch_bounds__(256) decode_merge_mma_kernel(Merge2Args A) {
   __syncthreads();
   float o = 0.f;
   if (c < D) {
-    const int i0 = qtr * (gd / 4), n = gd / 4;
+    const int i0 = qtr * (gd / 8), n = gd / 8;
 #pragma unroll
-    for (int u = 0; u < 32; ++u)
+    for (int u = 0; u < 16; ++u)
       if (u < n) o = fmaf(pv[u], s_acc[0][goff + i0 + u], o);
   }
   red[qtr][oc] = o;
   __syncthreads();
   if (qtr == 0 && c < D)
-    A.out[(size_t)row * D + c] = (red[0][oc] + red[1][oc]) + (red[2][oc] + red[3][oc]);
+    A.out[(size_t)row * D + c] =
+        ((red[0][oc] + red[1][oc]) + (red[2][oc] + red[3][oc])) + ((red[4][oc] + red[5][oc]) + (red[6][oc] + red[7][oc]));
 }
 
 // Prepared queries of nrows rows (blocks of kRep) for one group.
@@ -1002,7 +1005,7 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
   M.off[G] = D;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(B * Hq, div_up(D, 64));
-  cfg.blockDim = dim3(256);
+  cfg.blockDim = dim3(kMergeThreads);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
