@@ -20,15 +20,20 @@
 // one prmt.  Keys: the two centroid digits are two lookups, the sign bytes one prmt.
 // Values: magnitude bytes are looked up (low and high byte of the fp16 magnitude), the
 // negative flag is XORed into the sign bit, two prmt interleave the bytes, movmatrix turns
-// the 8x8 blocks around.  Integer products are exact; the fixed-point scales (|q| bound
-// for the query, max |c| for the centroids) keep every digit in range, so the logits carry
-// only the 2^-15 rounding of the two fixed-point operands.
+// the 8x8 blocks around.  Integer products are exact; the fixed-point scales (max |v| of
+// each prepared query row, max |c| for the centroids) keep every digit in range, so the
+// logits carry only the 2^-15 rounding of the two fixed-point operands.
 //
-// One CTA (4 consumer warps + 1 producer warp) handles one (sequence, kv head, context
-// split).  The producer stages 64 tokens of K/V code bytes and norms per pipeline stage
-// with bulk copies; consumer warps take one 16-token tile of every stage, keep an online
-// softmax (log2 domain) per head, and merge their states in shared memory before writing
-// one partial (m, l, acc) per query head and split.
+// Three kernels, linked by programmatic dependent launch: the prep kernel rotates the
+// queries (fp32, one warp per 8 rows x 8 outputs, small enough to share an SM with the
+// decode CTAs, which start at once and stream their first stages meanwhile); the decode
+// kernel, where one CTA (4 consumer warps + 1 producer warp) handles one (sequence, kv
+// head, context split): the producer stages 64 tokens of K/V code bytes and norms per
+// pipeline stage with bulk copies, consumer warps form the query digits, take one 16-token
+// tile of every stage, keep an online softmax (log2 domain) per head, and merge their
+// states in shared memory before writing one partial (m, l, acc) per query head and split;
+// and the merge kernel (log-sum-exp over the splits, then the inverse value rotation).
+#include <algorithm>
 #include <cfloat>
 #include <type_traits>
 
@@ -149,10 +154,12 @@ struct MmaArgs {
   int64_t max_len;
   float scale_log2;        // softmax scale * log2(e)
   const int32_t* seq_lens;
-  const int16_t* qfix;     // [B*Hq][G][2][D]: round(Pi q * s_m), round(S q * s_s)
-  const float* qinv;       // [B*Hq][G][2]: 1/s_m, 1/s_s
-  float* part;             // [B*Hq][nsplit][D+2]: (m, l, acc) per split
+  const float* qprep;      // [B*Hq][G][2][D]: Pi q, S q of every group (fp32)
+  float* part;             // [B*Hq] rows of part_ld floats: [nsplit][D+2] (m, l, acc) per split
+  int64_t part_ld;
   int* err;                // device error word (a pipeline wait that timed out)
+  const float* piv[2];     // value-group rotations, read by the merge kernel: prefetched
+  uint32_t piv_bytes[2];   // into L2 at the start of this kernel
 };
 
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
@@ -172,8 +179,28 @@ __device__ __forceinline__ void load_qops(QOps<GC>& f, const MmaArgs& A, int gi,
   const int g = lane >> 2, l = lane & 3;
   const int head = hk * kRep + (g >> 1);
   const bool lo = (g & 1) != 0;
-  const int16_t* qm = A.qfix + ((size_t)(b * A.Hq + head) * A.G + gi) * 2 * A.D + GC::CQ * l;
-  const int16_t* qs = qm + A.D;
+  const float* pm = A.qprep + ((size_t)(b * A.Hq + head) * A.G + gi) * 2 * A.D + GC::CQ * l;
+  const float* ps = pm + A.D;
+  // fixed-point scale of each (head, part) row: 32000 / max |v| over the group's
+  // coordinates (the four threads of a quad hold the head's d_g coordinates); all of the
+  // thread's values are loaded in one round
+  float4 va[GC::CQ / 4], vc[GC::CQ / 4];
+#pragma unroll
+  for (int u = 0; u < GC::CQ / 4; ++u) {
+    va[u] = __ldg(reinterpret_cast<const float4*>(pm) + u);
+    vc[u] = __ldg(reinterpret_cast<const float4*>(ps) + u);
+  }
+  float mm = 0.f, ms = 0.f;
+#pragma unroll
+  for (int u = 0; u < GC::CQ / 4; ++u) {
+    mm = fmaxf(mm, fmaxf(fmaxf(fabsf(va[u].x), fabsf(va[u].y)), fmaxf(fabsf(va[u].z), fabsf(va[u].w))));
+    ms = fmaxf(ms, fmaxf(fmaxf(fabsf(vc[u].x), fabsf(vc[u].y)), fmaxf(fabsf(vc[u].z), fabsf(vc[u].w))));
+  }
+  mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, 1));
+  mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, 2));
+  ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, 1));
+  ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, 2));
+  const float scm = mm > 0.f ? kFix / mm : 0.f, scs = ms > 0.f ? kFix / ms : 0.f;
   auto digit = [&](int v) -> uint32_t {
     const int hi = (v + 128) >> 8;
     return (uint32_t)(uint8_t)(lo ? v - (hi << 8) : hi);
@@ -181,17 +208,15 @@ __device__ __forceinline__ void load_qops(QOps<GC>& f, const MmaArgs& A, int gi,
   int ssum = 0;
 #pragma unroll
   for (int u = 0; u < GC::NS; ++u) {
-    const uint4 vm = *reinterpret_cast<const uint4*>(qm + 8 * u);
-    const uint4 vs = *reinterpret_cast<const uint4*>(qs + 8 * u);
-    const uint32_t wm[4] = {vm.x, vm.y, vm.z, vm.w}, ws[4] = {vs.x, vs.y, vs.z, vs.w};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
+      const float4 a = va[2 * u + h], c = vc[2 * u + h];
+      const float xa[4] = {a.x, a.y, a.z, a.w}, xc[4] = {c.x, c.y, c.z, c.w};
       uint32_t dm = 0, ds = 0;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const int j = 4 * h + t;
-        const int vmj = (int)(int16_t)(wm[j >> 1] >> (16 * (j & 1)));
-        const int vsj = (int)(int16_t)(ws[j >> 1] >> (16 * (j & 1)));
+        const int vmj = __float2int_rn(xa[t] * scm);
+        const int vsj = __float2int_rn(xc[t] * scs);
         dm |= digit(vmj) << (8 * t);
         ds |= digit(vsj) << (8 * t);
         ssum += vsj;
@@ -205,9 +230,10 @@ __device__ __forceinline__ void load_qops(QOps<GC>& f, const MmaArgs& A, int gi,
   ssum += __shfl_xor_sync(0xffffffffu, ssum, 1);
   ssum += __shfl_xor_sync(0xffffffffu, ssum, 2);
   ssum = __shfl_sync(0xffffffffu, ssum, 8 * l);
-  const float* inv = A.qinv + ((size_t)(b * A.Hq + hk * kRep + l) * A.G + gi) * 2;
-  f.inv_m = inv[0];
-  f.inv_s = inv[1];
+  mm = __shfl_sync(0xffffffffu, mm, 8 * l);
+  ms = __shfl_sync(0xffffffffu, ms, 8 * l);
+  f.inv_m = mm / kFix;
+  f.inv_s = ms / kFix;
   f.sum_s = (float)ssum;
 }
 
@@ -347,6 +373,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
 
   if (warp == kWarps) {
     // ---------------------------------------------------------------- producer warp
+    if (split == 0 && bh == 0 && lane < (TWO ? 2 : 1)) bulk_prefetch_l2(A.piv[lane], A.piv_bytes[lane]);
     int it = 0;
     int pending[kNStage];
     for (int i = 0; i < kNStage; ++i) pending[i] = -1;
@@ -542,7 +569,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
       L += f * s_l[w][h];
       acc += f * s_acc[w][h][c];
     }
-    float* dst = A.part + ((size_t)(b * A.Hq + hk * kRep + h) * A.nsplit + split) * (A.D + 2);
+    float* dst = A.part + (size_t)(b * A.Hq + hk * kRep + h) * A.part_ld + (size_t)split * (A.D + 2);
     if (c == 0) {
       dst[0] = (M == -INFINITY) ? -INFINITY : M * ln2;
       dst[1] = L;
@@ -555,195 +582,202 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
   allow_dependent_launch();
 }
 
-// Prepared queries of the kRep query rows grp*kRep .. +kRep-1 for one group and one part
-// (blockIdx.y = 0: Pi q, 1: S q), as 16-bit fixed point round(v * 32000 / max_o |v_o|) per
-// row, so every digit pair stays in range and the rounding is 2^-15 of the row's largest
-// output.  The d_g columns of Pi^T or S^T are staged in shared memory with 16-byte loads,
-// all in flight at once; thread (row, o) computes outputs o and o + 64.  Rows >= nrows
-// (padding of the last block) read as zero.
+// Rotated queries Pi q and S q of one group in fp32 (the fixed-point digits are formed by
+// the consumer warps, which see a whole head row).  CTA = one warp for (8 query rows,
+// part, 8 output coordinates): small enough to share an SM sub-partition with the decode
+// kernel's warps, which may launch at once (their first bulk copies overlap these loads).
+// The 8 columns of Pi^T (blockIdx.y = 0) or S^T (1) and the 8 rows are staged in shared
+// memory with one round of loads; thread (row, pair) runs two d_g-term dot products.
+// Rows >= nrows (padding of the last block) are skipped.
+constexpr int kPrepRows = 8;
+
 template <typename T>
-__global__ void __launch_bounds__(256) decode_prep_kernel(const T* __restrict__ q, int ldq, int off, int dg,
-                                                          int nrows, const float* __restrict__ PiT,
-                                                          const float* __restrict__ ST, int16_t* __restrict__ qfix,
-                                                          float* __restrict__ qinv, int D, int G, int gi) {
-  extern __shared__ float4 prep_smem[];
-  float* ms = reinterpret_cast<float*>(prep_smem);   // [dg][dg]
-  __shared__ float qs[kRep][128];
-  __shared__ float red[8];
+__global__ void __launch_bounds__(32) decode_prep_kernel(const T* __restrict__ q, int ldq, int off, int dg,
+                                                         int nrows, const float* __restrict__ PiT,
+                                                         const float* __restrict__ ST, float* __restrict__ qp,
+                                                         int D, int G, int gi) {
+  __shared__ float4 ms4[128][2];                 // [j][o/4]: M^T[j][o0 + o]
+  __shared__ float qs[kPrepRows][130];           // padded rows: conflict-free column reads
   allow_dependent_launch();
-  const int grp = blockIdx.x, part = blockIdx.y;
+  const int r0 = blockIdx.x * kPrepRows, part = blockIdx.y, o0 = blockIdx.z * 8;
   const float* M = part == 0 ? PiT : ST;
-  float4* m4 = reinterpret_cast<float4*>(ms);
-  {
-    const int n4 = dg * dg / 4;                 // <= 4096 float4: at most 16 per thread
-    float4 r[16];
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const int e = threadIdx.x + u * 256;
-      if (e < n4) r[u] = __ldg(reinterpret_cast<const float4*>(M) + e);
+  const int t = threadIdx.x, lg = dg == 128 ? 6 : 5;   // log2 of the pairs per row
+  for (int e = t; e < 2 * dg; e += 32)
+    ms4[e >> 1][e & 1] = __ldg(reinterpret_cast<const float4*>(M + (size_t)(e >> 1) * dg + o0) + (e & 1));
+  for (int e = t; e < kPrepRows * dg / 2; e += 32) {
+    const int r = e >> lg, j = 2 * (e & (dg / 2 - 1));
+    float2 v = make_float2(0.f, 0.f);
+    if (r0 + r < nrows) {
+      const size_t at = (size_t)(r0 + r) * ldq + off + j;
+      if constexpr (std::is_same<T, float>::value) v = __ldg(reinterpret_cast<const float2*>(q + at));
+      else v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + at));
     }
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const int e = threadIdx.x + u * 256;
-      if (e < n4) m4[e] = r[u];
-    }
+    qs[r][j] = v.x;
+    qs[r][j + 1] = v.y;
   }
-  for (int e = threadIdx.x; e < kRep * dg; e += blockDim.x) {
-    const int h = e / dg, j = e % dg;
-    const int rowq = grp * kRep + h;
-    float v = 0.f;
-    if (rowq < nrows) {
-      const size_t at = (size_t)rowq * ldq + off + j;
-      if constexpr (std::is_same<T, float>::value) v = q[at];
-      else v = __bfloat162float(q[at]);
-    }
-    qs[h][j] = v;
-  }
-  __syncthreads();
-  const int h = threadIdx.x >> 6, oc = threadIdx.x & 63;
-  float o0 = 0.f, o1 = 0.f;
-  if (oc < dg) {
+  __syncwarp();
+  const int r = t >> 2, o = 2 * (t & 3);
+  const float2* mcol = reinterpret_cast<const float2*>(ms4) + (t & 3);
+  float a0 = 0.f, a1 = 0.f;
 #pragma unroll 8
-    for (int j = 0; j < dg; ++j) o0 = fmaf(ms[j * dg + oc], qs[h][j], o0);
+  for (int j = 0; j < dg; ++j) {
+    const float2 m = mcol[4 * j];
+    const float x = qs[r][j];
+    a0 = fmaf(m.x, x, a0);
+    a1 = fmaf(m.y, x, a1);
   }
-  if (oc + 64 < dg) {
-#pragma unroll 8
-    for (int j = 0; j < dg; ++j) o1 = fmaf(ms[j * dg + oc + 64], qs[h][j], o1);
+  if (r0 + r < nrows) {
+    float* dst = qp + ((size_t)(r0 + r) * G + gi) * 2 * D + part * D + o0 + o;
+    dst[0] = a0;
+    dst[1] = a1;
   }
-  // per-row max |output|: the 64 threads of row h are warps 2h and 2h+1
-  float mx = fmaxf(fabsf(o0), fabsf(o1));
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  const int warp = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) red[warp] = mx;
-  __syncthreads();
-  mx = fmaxf(red[2 * h], red[2 * h + 1]);
-  const float sc = mx > 0.f ? kFix / mx : 0.f;
-  const size_t row = (size_t)(grp * kRep + h) * G + gi;
-  int16_t* dst = qfix + row * 2 * D + part * D;
-  if (oc < dg) dst[oc] = (int16_t)__float2int_rn(o0 * sc);
-  if (oc + 64 < dg) dst[oc + 64] = (int16_t)__float2int_rn(o1 * sc);
-  if (oc == 0) qinv[row * 2 + part] = mx / kFix;
 }
 
 // Log-sum-exp merge of the context splits and the inverse rotation of the value groups:
-// one CTA per (query row, 64 output channels).  The rotation entries are fetched before
-// the dependency wait; after it, every split's (m, l, acc) is loaded at once and merged
-// with a running maximum, so the merge costs one dependent round trip.
+// one CTA per (query row, 64 output channels).  The rotation entries of the CTA's
+// channels are loaded before the dependency wait; after it, the row's partials (m, l, acc
+// per split, contiguous) come into shared memory by bulk copies of up to kMergeChunk
+// splits and are merged with a running maximum.
 struct Merge2Args {
   const float* part;
+  int64_t part_ld;
   int nsplit, D, G;
   int off[3];
   const float* PiV[2];
   float* out;
+  int* err;
 };
 
-constexpr int kMergeThreads = 512;   // 8 row parts of the rotation, up to 4 split partitions
+constexpr int kMergeThreads = 256;   // 4 row quarters of the rotation x 64 channels
+constexpr int kMergeChunk = 96;      // splits per bulk copy (a multiple of 4: 16-byte aligned starts)
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
 
 __global__ void __launch_bounds__(kMergeThreads) decode_merge_mma_kernel(Merge2Args A) {
-  __shared__ float s_acc[4][256];
-  __shared__ float s_ml[4][256][2];
-  __shared__ float red[8][64];
+  extern __shared__ float4 merge_smem[];
+  float* msm = reinterpret_cast<float*>(merge_smem);   // [chunk][D+2] staged partials
+  __shared__ float s_w[kMergeChunk];
+  __shared__ float s_acc[256], s_fin[256];
+  __shared__ float red[4][64];
+  __shared__ __align__(8) uint64_t bar;
   const int row = blockIdx.x, c0 = blockIdx.y * 64;
-  const int D = A.D, ns = A.nsplit;
-  // rotation column of this thread's output, eighth qtr of its rows (before the wait)
-  const int oc = threadIdx.x & 63, qtr = threadIdx.x >> 6;
+  const int D = A.D, ns = A.nsplit, W = D + 2;
+  const int oc = threadIdx.x & 63, qtr = threadIdx.x >> 6, lane = threadIdx.x & 31;
   const int c = c0 + oc;
-  float pv[16];
-  int gsel = 0, goff = 0, gd = 0;
+  float pv[32];
+  int goff = 0, gd = 0;
   if (c < D) {
-    gsel = (A.G > 1 && c >= A.off[1]) ? 1 : 0;
+    const int gsel = (A.G > 1 && c >= A.off[1]) ? 1 : 0;
     goff = A.off[gsel];
     gd = A.off[gsel + 1] - goff;
     const float* Pi = A.PiV[gsel] + (c - goff);
-    const int i0 = qtr * (gd / 8), n = gd / 8;   // n <= 16
+    const int n = gd / 4, i0 = qtr * n;   // n <= 32
 #pragma unroll
-    for (int u = 0; u < 16; ++u) pv[u] = (u < n) ? __ldg(Pi + (size_t)(i0 + u) * gd) : 0.f;
+    for (int u = 0; u < 32; ++u) pv[u] = (u < n) ? __ldg(Pi + (size_t)(i0 + u) * gd) : 0.f;
   }
-  grid_dependency_wait();
-  // merged rotated-basis accumulator: thread (coordinate i, half hs) runs over splits
-  // hs, hs + halves, ... with a running maximum
-  const float* P = A.part + (size_t)row * ns * (D + 2);
-  int halves = blockDim.x / D;
-  halves = halves < 1 ? 1 : (halves > 4 ? 4 : halves);
-  const int i = threadIdx.x % D, hs = threadIdx.x / D;
-  if (hs < halves) {
-    float M = -INFINITY, L = 0.f, acc = 0.f;
-    for (int s0 = hs; s0 < ns; s0 += 16 * halves) {
-      float m16[16], l16[16], a16[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int s = s0 + u * halves;
-        const float* ps = P + (size_t)s * (D + 2);
-        m16[u] = s < ns ? ps[0] : -INFINITY;
-        l16[u] = s < ns ? ps[1] : 0.f;
-        a16[u] = s < ns ? ps[2 + i] : 0.f;
-      }
-      float mx = M;
-#pragma unroll
-      for (int u = 0; u < 16; ++u) mx = fmaxf(mx, m16[u]);
-      if (mx > -INFINITY) {
-        const float f = M == -INFINITY ? 0.f : __expf(M - mx);
-        L *= f;
-        acc *= f;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const float w = m16[u] == -INFINITY ? 0.f : __expf(m16[u] - mx);
-          L = fmaf(w, l16[u], L);
-          acc = fmaf(w, a16[u], acc);
-        }
-        M = mx;
-      }
-    }
-    s_acc[hs][i] = acc;
-    s_ml[hs][i][0] = M;
-    s_ml[hs][i][1] = L;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
   }
   __syncthreads();
-  // thread i combines the partial states of coordinate i (only it touches index i)
-  if (threadIdx.x < D) {
-    float M = -INFINITY;
-    for (int h = 0; h < halves; ++h) M = fmaxf(M, s_ml[h][i][0]);
-    float L = 0.f, acc = 0.f;
-    for (int h = 0; h < halves; ++h) {
-      const float f = s_ml[h][i][0] == -INFINITY ? 0.f : __expf(s_ml[h][i][0] - M);
-      L = fmaf(f, s_ml[h][i][1], L);
-      acc = fmaf(f, s_acc[h][i], acc);
+  grid_dependency_wait();
+  const float* P = A.part + (size_t)row * A.part_ld;
+  // thread (coordinate i, part hs) accumulates the splits s = hs (mod halves)
+  int halves = kMergeThreads / D;
+  if (halves < 1) halves = 1;
+  const int i = threadIdx.x % D, hs = threadIdx.x / D;
+  float M = -INFINITY, L = 0.f, acc = 0.f;
+  uint32_t phase = 0;
+  bool inflight = false;
+  for (int s0 = 0; s0 < ns; s0 += kMergeChunk) {
+    const int n = min(kMergeChunk, ns - s0);
+    if (threadIdx.x == 0) {
+      const uint32_t bytes = (uint32_t)(((size_t)n * W * sizeof(float) + 15) & ~(size_t)15);
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&bar, bytes);
+      bulk_load(msm, P + (size_t)s0 * W, bytes, &bar);
     }
-    s_acc[0][i] = L > 0.f ? acc / L : 0.f;
+    inflight = true;
+    const bool ok = __syncthreads_and(mbar_wait(&bar, phase, nullptr, kDecWaitNs));
+    if (!ok) {
+      if (threadIdx.x == 0 && A.err) atomicCAS(A.err, 0, 203);
+      break;
+    }
+    inflight = false;
+    phase ^= 1;
+    // chunk maximum (every warp reduces the same values in the same order)
+    float mc = -INFINITY;
+    for (int s = lane; s < n; s += 32) mc = fmaxf(mc, msm[s * W]);
+    mc = warp_max(mc);
+    const float Mn = fmaxf(M, mc);
+    if (Mn != -INFINITY) {
+      const float alpha = (M == -INFINITY) ? 0.f : __expf(M - Mn);
+      for (int s = threadIdx.x; s < n; s += blockDim.x) {
+        const float m = msm[s * W];
+        s_w[s] = (m == -INFINITY) ? 0.f : __expf(m - Mn);
+      }
+      __syncthreads();
+      float lc = 0.f;
+      for (int s = lane; s < n; s += 32) lc = fmaf(s_w[s], msm[s * W + 1], lc);
+      L = fmaf(L, alpha, warp_sum(lc));
+      float a = 0.f;
+      if (hs < halves)
+        for (int s = hs; s < n; s += halves) a = fmaf(s_w[s], msm[s * W + 2 + i], a);
+      acc = fmaf(acc, alpha, a);
+      M = Mn;
+    }
+    __syncthreads();   // the staged chunk and its weights are consumed before the next copy
+  }
+  if (inflight) {      // a copy that did not complete in time still lands before the CTA exits
+    if (threadIdx.x == 0) mbar_wait(&bar, phase, nullptr, kDecWaitNs);
+    return;
+  }
+  if (hs < halves) s_acc[hs * D + i] = acc;
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float t = 0.f;
+    for (int h = 0; h < halves; ++h) t += s_acc[h * D + threadIdx.x];
+    s_fin[threadIdx.x] = L > 0.f ? t / L : 0.f;
   }
   __syncthreads();
   float o = 0.f;
   if (c < D) {
-    const int i0 = qtr * (gd / 8), n = gd / 8;
+    const int n = gd / 4, i0 = qtr * n;
 #pragma unroll
-    for (int u = 0; u < 16; ++u)
-      if (u < n) o = fmaf(pv[u], s_acc[0][goff + i0 + u], o);
+    for (int u = 0; u < 32; ++u)
+      if (u < n) o = fmaf(pv[u], s_fin[goff + i0 + u], o);
   }
   red[qtr][oc] = o;
   __syncthreads();
-  if (qtr == 0 && c < D)
-    A.out[(size_t)row * D + c] =
-        ((red[0][oc] + red[1][oc]) + (red[2][oc] + red[3][oc])) + ((red[4][oc] + red[5][oc]) + (red[6][oc] + red[7][oc]));
+  if (qtr == 0 && c < D) A.out[(size_t)row * D + c] = (red[0][oc] + red[1][oc]) + (red[2][oc] + red[3][oc]);
 }
 
-// Prepared queries of nrows rows (blocks of kRep) for one group.
-int launch_prep(const void* q, int q_dtype, int ldq, int off, int dg, int nrows, const tq_ctx* kc, int16_t* qfix,
-                float* qinv, int D, int G, int gi, cudaStream_t st) {
-  const dim3 grid((nrows + kRep - 1) / kRep, 2);
-  const size_t smem = (size_t)dg * dg * sizeof(float);
-  cudaError_t e;
-  if (q_dtype == TQ_DTYPE_F32) {
-    e = cudaFuncSetAttribute(decode_prep_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_prep_kernel)");
-    decode_prep_kernel<float><<<grid, 256, smem, st>>>(static_cast<const float*>(q), ldq, off, dg, nrows, kc->PiT,
-                                                       kc->ST, qfix, qinv, D, G, gi);
-  } else {
-    e = cudaFuncSetAttribute(decode_prep_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_prep_kernel)");
-    decode_prep_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(q), ldq, off, dg,
-                                                               nrows, kc->PiT, kc->ST, qfix, qinv, D, G, gi);
-  }
+// Rotated queries of nrows rows for one group.
+int launch_prep(const void* q, int q_dtype, int ldq, int off, int dg, int nrows, const tq_ctx* kc, float* qp, int D,
+                int G, int gi, cudaStream_t st) {
+  const dim3 grid((nrows + kPrepRows - 1) / kPrepRows, 2, dg / 8);
+  cudaError_t e = q_dtype == TQ_DTYPE_F32
+                      ? cudaFuncSetAttribute(decode_prep_kernel<float>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                             cudaSharedmemCarveoutMaxShared)
+                      : cudaFuncSetAttribute(decode_prep_kernel<__nv_bfloat16>,
+                                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                                             cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_prep_kernel carveout)");
+  if (q_dtype == TQ_DTYPE_F32)
+    decode_prep_kernel<float><<<grid, 32, 0, st>>>(static_cast<const float*>(q), ldq, off, dg, nrows, kc->PiT,
+                                                    kc->ST, qp, D, G, gi);
+  else
+    decode_prep_kernel<__nv_bfloat16><<<grid, 32, 0, st>>>(static_cast<const __nv_bfloat16*>(q), ldq, off, dg,
+                                                            nrows, kc->PiT, kc->ST, qp, D, G, gi);
   count_launch();
   return check_launch("decode_prep_kernel");
 }
@@ -901,6 +935,10 @@ int launch_mma_t(const MmaArgs& A, int nsplit, int BHkv, cudaStream_t st) {
   const int dyn = kNStage * Stage<G0, G1c, TWO>::BYTES;
   cudaError_t ea = cudaFuncSetAttribute(decode_mma_kernel<G0, G1>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
   if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncSetAttribute(decode_mma_kernel)");
+  // one shared-memory carveout for the prep, decode and merge kernels, so they can share SMs
+  ea = cudaFuncSetAttribute(decode_mma_kernel<G0, G1>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                            cudaSharedmemCarveoutMaxShared);
+  if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncSetAttribute(decode_mma_kernel carveout)");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nsplit, BHkv);
   cfg.blockDim = dim3((kWarps + 1) * 32);
@@ -971,17 +1009,16 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
   const DecodeWs W = decode_ws(B, Hq, Hkv, D, G, max_len);
   if (W.nsplit > 512) return kNotHandled;
   char* base = static_cast<char*>(ws);
-  int16_t* qfix = reinterpret_cast<int16_t*>(base + W.qp);
-  float* qinv = reinterpret_cast<float*>(base + W.qp + (((size_t)B * Hq * G * 2 * D * 2 + 255) / 256) * 256);
+  float* qp = reinterpret_cast<float*>(base + W.qp);
   float* part = reinterpret_cast<float*>(base + W.part);
   for (int g = 0; g < G; ++g) {
-    int r = launch_prep(q, q_dtype, D, off[g], kctx[g]->lay.d, B * Hq, kctx[g], qfix, qinv, D, G, g, st);
+    int r = launch_prep(q, q_dtype, D, off[g], kctx[g]->lay.d, B * Hq, kctx[g], qp, D, G, g, st);
     if (r != TQ_OK) return r;
   }
   MmaArgs A{};
   A.B = B; A.Hq = Hq; A.Hkv = Hkv; A.D = D; A.nsplit = W.nsplit; A.chunk = W.chunk; A.G = G;
   A.max_len = max_len; A.scale_log2 = scale * 1.4426950408889634f; A.seq_lens = seq_lens;
-  A.qfix = qfix; A.qinv = qinv; A.part = part;
+  A.qprep = qp; A.part = part; A.part_ld = W.part_ld;
   for (int g = 0; g < G; ++g) {
     MmaGroup& gr = A.g[g];
     gr.kcodes = kc[g].codes; gr.knorm = kc[g].norm; gr.krnorm = kc[g].rnorm;
@@ -993,6 +1030,10 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
     gr.vcap = vc[g].cap;
   }
   A.err = kctx[0]->dev_err;
+  for (int g = 0; g < G; ++g) {
+    A.piv[g] = vctx[g]->Pi;
+    A.piv_bytes[g] = (uint32_t)(vctx[g]->lay.d * vctx[g]->lay.d * sizeof(float));
+  }
   int r;
   if (G == 1 && sig[0] == 12844) r = launch_mma_t<C128_44, void>(A, W.nsplit, B * Hkv, st);
   else if (G == 1) r = launch_mma_t<C128_33, void>(A, W.nsplit, B * Hkv, st);
@@ -1000,12 +1041,19 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
   else r = launch_mma_t<C64_33, C64_22>(A, W.nsplit, B * Hkv, st);
   if (r != TQ_OK) return r;
   Merge2Args M{};
-  M.part = part; M.nsplit = W.nsplit; M.D = D; M.G = G; M.out = out;
+  M.part = part; M.part_ld = W.part_ld; M.nsplit = W.nsplit; M.D = D; M.G = G; M.out = out; M.err = A.err;
   for (int g = 0; g < G; ++g) { M.off[g] = off[g]; M.PiV[g] = vctx[g]->Pi; }
   M.off[G] = D;
+  const int mdyn = (int)((((size_t)std::min(W.nsplit, kMergeChunk) * (D + 2) * sizeof(float)) + 15) / 16 * 16);
+  cudaError_t em = cudaFuncSetAttribute(decode_merge_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mdyn);
+  if (em == cudaSuccess)
+    em = cudaFuncSetAttribute(decode_merge_mma_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              cudaSharedmemCarveoutMaxShared);
+  if (em != cudaSuccess) return cuda_fail(em, "cudaFuncSetAttribute(decode_merge_mma_kernel)");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(B * Hq, div_up(D, 64));
   cfg.blockDim = dim3(kMergeThreads);
+  cfg.dynamicSmemBytes = mdyn;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

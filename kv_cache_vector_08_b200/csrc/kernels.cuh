@@ -20,6 +20,7 @@ void decode_geometry(int B, int Hkv, int64_t max_len, int* nsplit, int* chunk);
 struct DecodeWs {
   size_t qp, part, cnt, total;  // byte offsets of the regions and total size
   int nsplit, chunk;
+  int64_t part_ld;              // floats per query row of the split partials (16-byte multiple)
 };
 DecodeWs decode_ws(int B, int Hq, int Hkv, int D, int G, int64_t max_len);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int ngroups, int64_t max_len, int qp_ld);

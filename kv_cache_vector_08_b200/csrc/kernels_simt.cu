@@ -764,7 +764,8 @@ DecodeWs decode_ws(int B, int Hq, int Hkv, int D, int G, int64_t max_len) {
   auto up = [](size_t x) { return ((x + 255) / 256) * 256; };
   w.qp = 0;
   w.part = up((size_t)B * Hq * G * 2 * D * sizeof(float));
-  w.cnt = w.part + up((size_t)B * Hq * w.nsplit * (D + 2) * sizeof(float));
+  w.part_ld = ((int64_t)w.nsplit * (D + 2) + 3) / 4 * 4;
+  w.cnt = w.part + up((size_t)B * Hq * w.part_ld * sizeof(float));
   w.total = w.cnt + up((size_t)B * Hkv * sizeof(int));
   return w;
 }
