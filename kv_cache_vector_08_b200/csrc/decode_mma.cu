@@ -356,6 +356,10 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
   const int t_begin = split * A.chunk;
   const int t_end = min(T, t_begin + A.chunk);
   const int64_t slot0 = (int64_t)bh * A.max_len;
+  // The merge kernel behind this one may launch at once: every CTA of this grid is
+  // resident from the start, so its CTAs only take slots that finished CTAs free, and its
+  // grid-dependency wait still sees every partial.
+  allow_dependent_launch();
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNStage; ++i) {
       mbar_init(full + i, 32);
@@ -371,57 +375,9 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
     if (A.err) atomicCAS(A.err, 0, code);
   };
 
-  if (warp == kWarps) {
-    // ---------------------------------------------------------------- producer warp
-    if (split == 0 && bh == 0 && lane < (TWO ? 2 : 1)) bulk_prefetch_l2(A.piv[lane], A.piv_bytes[lane]);
-    int it = 0;
-    int pending[kNStage];
-    for (int i = 0; i < kNStage; ++i) pending[i] = -1;
-    for (int ts = t_begin; ts < t_end; ts += kStageTok, ++it) {
-      const int s = it % kNStage;
-      const uint32_t ph = (it / kNStage) & 1;
-      if (!mbar_wait(empty + s, ph ^ 1, abort_v, kDecWaitNs)) { fail(201); break; }
-      const int ntok = min(kStageTok, t_end - ts);
-      uint8_t* st = dsm + s * ST::BYTES;
-      const int64_t first = slot0 + ts, last = slot0 + ts + ntok;
-      auto spans = [&](bool issue) {
-        uint32_t tx = 0;
-        const MmaGroup& g0 = A.g[0];
-        tx += stage_span(st + ST::OFF_K0, g0.kcodes, first * ST::KB0, last * ST::KB0, g0.kcap * ST::KB0, full + s, issue);
-        tx += stage_span(st + ST::OFF_V0, g0.vcodes, first * ST::VB0, last * ST::VB0, g0.vcap * ST::VB0, full + s, issue);
-        if constexpr (TWO) {
-          const MmaGroup& g1 = A.g[1];
-          tx += stage_span(st + ST::OFF_K1, g1.kcodes, first * ST::KB1, last * ST::KB1, g1.kcap * ST::KB1, full + s, issue);
-          tx += stage_span(st + ST::OFF_V1, g1.vcodes, first * ST::VB1, last * ST::VB1, g1.vcap * ST::VB1, full + s, issue);
-        }
-#pragma unroll
-        for (int gi = 0; gi < (TWO ? 2 : 1); ++gi) {
-          const MmaGroup& gr = A.g[gi];
-          uint8_t* nb = st + ST::OFF_N + gi * 3 * ST::NB;
-          const uint8_t* kn = reinterpret_cast<const uint8_t*>(gr.knorm);
-          const uint8_t* kr = reinterpret_cast<const uint8_t*>(gr.krnorm);
-          const uint8_t* vn = reinterpret_cast<const uint8_t*>(gr.vnorm);
-          tx += stage_span(nb, kn, first * 2, last * 2, gr.kcap * 2, full + s, issue);
-          tx += stage_span(nb + ST::NB, kr, first * 2, last * 2, gr.kcap * 2, full + s, issue);
-          tx += stage_span(nb + 2 * ST::NB, vn, first * 2, last * 2, gr.vcap * 2, full + s, issue);
-        }
-        return tx;
-      };
-      if (lane == 0) {
-        mbar_expect_tx(full + s, spans(false));
-        spans(true);
-      }
-      __syncwarp();
-      mbar_arrive(full + s);
-      if (lane == 0) pending[s] = (int)ph;
-    }
-    // bulk copies still in flight land before the CTA exits
-    if (lane == 0)
-      for (int i = 0; i < kNStage; ++i)
-        if (pending[i] >= 0) mbar_wait(full + i, (uint32_t)pending[i], nullptr, kDecWaitNs);
-  }
-
   // ------------------------------------------------------------------ consumer warps
+  // (their code comes first: the consumers' path from the kernel entry is straight-line,
+  // which shortens the cold instruction fetch before their first loads)
   float acc0[G0::NS][2][4];
   float acc1[G1c::NS][2][4];
   float m_run = -INFINITY, l_run = 0.f;
@@ -553,7 +509,55 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
     };
     store_acc(acc0, G0{}, A.g[0].off);
     if constexpr (TWO) store_acc(acc1, G1c{}, A.g[1].off);
-  }
+  } else {
+    // ---------------------------------------------------------------- producer warp
+    if (split == 0 && bh == 0 && lane < (TWO ? 2 : 1)) bulk_prefetch_l2(A.piv[lane], A.piv_bytes[lane]);
+    int it = 0;
+    int pending[kNStage];
+    for (int i = 0; i < kNStage; ++i) pending[i] = -1;
+    for (int ts = t_begin; ts < t_end; ts += kStageTok, ++it) {
+      const int s = it % kNStage;
+      const uint32_t ph = (it / kNStage) & 1;
+      if (!mbar_wait(empty + s, ph ^ 1, abort_v, kDecWaitNs)) { fail(201); break; }
+      const int ntok = min(kStageTok, t_end - ts);
+      uint8_t* st = dsm + s * ST::BYTES;
+      const int64_t first = slot0 + ts, last = slot0 + ts + ntok;
+      auto spans = [&](bool issue) {
+        uint32_t tx = 0;
+        const MmaGroup& g0 = A.g[0];
+        tx += stage_span(st + ST::OFF_K0, g0.kcodes, first * ST::KB0, last * ST::KB0, g0.kcap * ST::KB0, full + s, issue);
+        tx += stage_span(st + ST::OFF_V0, g0.vcodes, first * ST::VB0, last * ST::VB0, g0.vcap * ST::VB0, full + s, issue);
+        if constexpr (TWO) {
+          const MmaGroup& g1 = A.g[1];
+          tx += stage_span(st + ST::OFF_K1, g1.kcodes, first * ST::KB1, last * ST::KB1, g1.kcap * ST::KB1, full + s, issue);
+          tx += stage_span(st + ST::OFF_V1, g1.vcodes, first * ST::VB1, last * ST::VB1, g1.vcap * ST::VB1, full + s, issue);
+        }
+#pragma unroll
+        for (int gi = 0; gi < (TWO ? 2 : 1); ++gi) {
+          const MmaGroup& gr = A.g[gi];
+          uint8_t* nb = st + ST::OFF_N + gi * 3 * ST::NB;
+          const uint8_t* kn = reinterpret_cast<const uint8_t*>(gr.knorm);
+          const uint8_t* kr = reinterpret_cast<const uint8_t*>(gr.krnorm);
+          const uint8_t* vn = reinterpret_cast<const uint8_t*>(gr.vnorm);
+          tx += stage_span(nb, kn, first * 2, last * 2, gr.kcap * 2, full + s, issue);
+          tx += stage_span(nb + ST::NB, kr, first * 2, last * 2, gr.kcap * 2, full + s, issue);
+          tx += stage_span(nb + 2 * ST::NB, vn, first * 2, last * 2, gr.vcap * 2, full + s, issue);
+        }
+        return tx;
+      };
+      if (lane == 0) {
+        mbar_expect_tx(full + s, spans(false));
+        spans(true);
+      }
+      __syncwarp();
+      mbar_arrive(full + s);
+      if (lane == 0) pending[s] = (int)ph;
+    }
+    // bulk copies still in flight land before the CTA exits
+    if (lane == 0)
+      for (int i = 0; i < kNStage; ++i)
+        if (pending[i] >= 0) mbar_wait(full + i, (uint32_t)pending[i], nullptr, kDecWaitNs);
+    }
   __syncthreads();
   // ---- merge the warps: one partial per (query head, split); m in natural-log units
   const float ln2 = 0.69314718055994531f;
@@ -576,10 +580,6 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
     }
     dst[2 + c] = acc;
   }
-  // the merge kernel (launched programmatically behind this one) may start once every
-  // CTA has written its partial
-  __syncthreads();
-  allow_dependent_launch();
 }
 
 // Rotated queries Pi q and S q of one group in fp32 (the fixed-point digits are formed by
@@ -688,77 +688,90 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_mma_kernel(Merge2A
     mbar_init(&bar, 1);
     fence_barrier_init();
   }
+  for (int i = threadIdx.x; i < min(ns, kMergeChunk) * W; i += blockDim.x) msm[i] = 0.f;
   __syncthreads();
-  grid_dependency_wait();
   const float* P = A.part + (size_t)row * A.part_ld;
   // thread (coordinate i, part hs) accumulates the splits s = hs (mod halves)
   int halves = kMergeThreads / D;
   if (halves < 1) halves = 1;
   const int i = threadIdx.x % D, hs = threadIdx.x / D;
-  float M = -INFINITY, L = 0.f, acc = 0.f;
-  uint32_t phase = 0;
-  bool inflight = false;
-  for (int s0 = 0; s0 < ns; s0 += kMergeChunk) {
-    const int n = min(kMergeChunk, ns - s0);
-    if (threadIdx.x == 0) {
-      const uint32_t bytes = (uint32_t)(((size_t)n * W * sizeof(float) + 15) & ~(size_t)15);
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&bar, bytes);
-      bulk_load(msm, P + (size_t)s0 * W, bytes, &bar);
-    }
-    inflight = true;
-    const bool ok = __syncthreads_and(mbar_wait(&bar, phase, nullptr, kDecWaitNs));
-    if (!ok) {
-      if (threadIdx.x == 0 && A.err) atomicCAS(A.err, 0, 203);
-      break;
-    }
-    inflight = false;
-    phase ^= 1;
-    // chunk maximum (every warp reduces the same values in the same order)
-    float mc = -INFINITY;
-    for (int s = lane; s < n; s += 32) mc = fmaxf(mc, msm[s * W]);
-    mc = warp_max(mc);
-    const float Mn = fmaxf(M, mc);
-    if (Mn != -INFINITY) {
-      const float alpha = (M == -INFINITY) ? 0.f : __expf(M - Mn);
-      for (int s = threadIdx.x; s < n; s += blockDim.x) {
-        const float m = msm[s * W];
-        s_w[s] = (m == -INFINITY) ? 0.f : __expf(m - Mn);
+  // Pass 0 runs the whole merge on zeroed shared memory and discards it, before the
+  // grid-dependency wait: this kernel launches while the decode kernel still runs, so the
+  // instruction fetch of its code is hidden there instead of following the wait.  Pass 1
+  // is the merge.
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const bool real = pass == 1;
+    if (real) grid_dependency_wait();
+    float M = -INFINITY, L = 0.f, acc = 0.f;
+    uint32_t phase = 0;
+    bool inflight = false;
+    for (int s0 = 0; s0 < (real ? ns : 1); s0 += kMergeChunk) {
+      const int n = min(kMergeChunk, ns - s0);
+      if (real) {
+        if (threadIdx.x == 0) {
+          const uint32_t bytes = (uint32_t)(((size_t)n * W * sizeof(float) + 15) & ~(size_t)15);
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(&bar, bytes);
+          bulk_load(msm, P + (size_t)s0 * W, bytes, &bar);
+        }
+        inflight = true;
+        const bool ok = __syncthreads_and(mbar_wait(&bar, phase, nullptr, kDecWaitNs));
+        if (!ok) {
+          if (threadIdx.x == 0 && A.err) atomicCAS(A.err, 0, 203);
+          break;
+        }
+        inflight = false;
+        phase ^= 1;
       }
-      __syncthreads();
-      float lc = 0.f;
-      for (int s = lane; s < n; s += 32) lc = fmaf(s_w[s], msm[s * W + 1], lc);
-      L = fmaf(L, alpha, warp_sum(lc));
-      float a = 0.f;
-      if (hs < halves)
-        for (int s = hs; s < n; s += halves) a = fmaf(s_w[s], msm[s * W + 2 + i], a);
-      acc = fmaf(acc, alpha, a);
-      M = Mn;
+      // chunk maximum (every warp reduces the same values in the same order)
+      float mc = -INFINITY;
+      for (int s = lane; s < n; s += 32) mc = fmaxf(mc, msm[s * W]);
+      mc = warp_max(mc);
+      const float Mn = fmaxf(M, mc);
+      if (Mn != -INFINITY) {
+        const float alpha = (M == -INFINITY) ? 0.f : __expf(M - Mn);
+        for (int s = threadIdx.x; s < n; s += blockDim.x) {
+          const float m = msm[s * W];
+          s_w[s] = (m == -INFINITY) ? 0.f : __expf(m - Mn);
+        }
+        __syncthreads();
+        float lc = 0.f;
+        for (int s = lane; s < n; s += 32) lc = fmaf(s_w[s], msm[s * W + 1], lc);
+        L = fmaf(L, alpha, warp_sum(lc));
+        float a = 0.f;
+        if (hs < halves)
+          for (int s = hs; s < n; s += halves) a = fmaf(s_w[s], msm[s * W + 2 + i], a);
+        acc = fmaf(acc, alpha, a);
+        M = Mn;
+      }
+      __syncthreads();   // the staged chunk and its weights are consumed before the next copy
     }
-    __syncthreads();   // the staged chunk and its weights are consumed before the next copy
-  }
-  if (inflight) {      // a copy that did not complete in time still lands before the CTA exits
-    if (threadIdx.x == 0) mbar_wait(&bar, phase, nullptr, kDecWaitNs);
-    return;
-  }
-  if (hs < halves) s_acc[hs * D + i] = acc;
-  __syncthreads();
-  if (threadIdx.x < D) {
-    float t = 0.f;
-    for (int h = 0; h < halves; ++h) t += s_acc[h * D + threadIdx.x];
-    s_fin[threadIdx.x] = L > 0.f ? t / L : 0.f;
-  }
-  __syncthreads();
-  float o = 0.f;
-  if (c < D) {
-    const int n = gd / 4, i0 = qtr * n;
+    if (inflight) {      // a copy that did not complete in time still lands before the CTA exits
+      if (threadIdx.x == 0) mbar_wait(&bar, phase, nullptr, kDecWaitNs);
+      return;
+    }
+    if (hs < halves) s_acc[hs * D + i] = acc;
+    __syncthreads();
+    if (threadIdx.x < D) {
+      float t = 0.f;
+      for (int h = 0; h < halves; ++h) t += s_acc[h * D + threadIdx.x];
+      s_fin[threadIdx.x] = L > 0.f ? t / L : 0.f;
+    }
+    __syncthreads();
+    float o = 0.f;
+    if (c < D) {
+      const int n = gd / 4, i0 = qtr * n;
 #pragma unroll
-    for (int u = 0; u < 32; ++u)
-      if (u < n) o = fmaf(pv[u], s_fin[goff + i0 + u], o);
+      for (int u = 0; u < 32; ++u)
+        if (u < n) o = fmaf(pv[u], s_fin[goff + i0 + u], o);
+    }
+    red[qtr][oc] = o;
+    __syncthreads();
+    if (real && qtr == 0 && c < D)
+      A.out[(size_t)row * D + c] = (red[0][oc] + red[1][oc]) + (red[2][oc] + red[3][oc]);
+    __syncthreads();
   }
-  red[qtr][oc] = o;
-  __syncthreads();
-  if (qtr == 0 && c < D) A.out[(size_t)row * D + c] = (red[0][oc] + red[1][oc]) + (red[2][oc] + red[3][oc]);
 }
 
 // Rotated queries of nrows rows for one group.
