@@ -290,6 +290,13 @@ def test_search_topk_matches_oracle(d, N, k):
         assert row.index(7) < row.index(N // 2)        # equal scores: lower id first
 
 
+def test_decode_many_splits():
+    """One kv head over 7000 tokens: 110 context splits of 64 tokens, so the merge stages the
+    partials in two bulk-copy chunks (96 + 14 splits) and one query-prep block is ragged."""
+    out, ref, _ = _decode_case(1, 1, 4, 128, ((0, 128, 4, 4),), [7000], 7040, 11)
+    parity.assert_close(out, ref, "decode, 110 splits")
+
+
 @pytest.mark.parametrize("Hkv,Hq", [(2, 4), (1, 8), (3, 12)])
 def test_decode_other_gqa_ratios(Hkv, Hq):
     """GQA ratios 2, 8 (SIMT kernel) and 4 with three kv heads (tensor-core kernel)."""
