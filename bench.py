@@ -52,6 +52,23 @@ def _dist():
     return ws, rank, local
 
 
+def max_over_ranks(x, ws, device=None):
+    """The largest value of a per-rank float over all ranks (a job takes as long as its
+    slowest rank).  Every rank must call it, in the same order as the other collectives."""
+    if ws <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, ws, seconds):
+    """Units processed by all ranks per second of the slowest rank's time."""
+    return units_per_rank * ws / seconds
+
+
 # ------------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
@@ -261,11 +278,7 @@ def run_gpu(args):
     t_qk = np.array([a.elapsed_time(b) for a, b, c, d in recs]) / 1e3
     t_qv = np.array([b.elapsed_time(c) for a, b, c, d in recs]) / 1e3
     t_dec = np.array([c.elapsed_time(d) for a, b, c, d in recs]) / 1e3
-    ms_step = float(t_step.mean() * 1e3)
-    if ws > 1:
-        tt = torch.tensor([ms_step], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms_step = float(tt.item())
+    ms_step = max_over_ranks(float(t_step.mean() * 1e3), ws, dev)
 
     # decode alone, L2 flushed before every launch (the HBM GB/s figure)
     dec = []
@@ -279,8 +292,11 @@ def run_gpu(args):
     torch.cuda.synchronize()
     t_dec_alone = float(np.median([a.elapsed_time(b) for a, b in dec]) / 1e3)
 
-    # end to end through the public API from pinned host buffers
+    # end to end through the public API from pinned host buffers (whole job: all ranks'
+    # keys over the slowest rank's time)
     e2e = run_e2e(bench, st, args.steps, args.warmup)
+    e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], ws, dev)
+    e2e["value"] = whole_job_rate(bench.keys, ws, e2e["ms_per_step"] / 1e3)
 
     if rank != 0:
         if ws > 1:
@@ -289,8 +305,7 @@ def run_gpu(args):
     peaks = _peaks()
     qk_bytes, qv_bytes = bench.quantize_bytes()
     dec_bytes = bench.decode_bytes()
-    keys_total = bench.keys * ws
-    value = keys_total / (ms_step / 1e3)
+    value = whole_job_rate(bench.keys, ws, ms_step / 1e3)
     kernels = {"quantize_keys": float(t_qk.mean()), "quantize_values": float(t_qv.mean()),
                "decode_attention": float(t_dec.mean())}
     dominant = max(kernels, key=kernels.get)
