@@ -218,13 +218,17 @@ int tq_decode_attention(const tq_ctx* const* kctx, const tq_ctx* const* vctx, co
  * that loads the library holds until the process exits.  The call allocates nothing.
  * Arguments, layout and results are those of tq_decode_attention.
  * Set-up: the first call on each device (with that device current) looks up the array's
- * device address once; make that first call before any stream capture.
+ * device address once and caches it; make that first call before any stream capture.  The
+ * cached address does not survive a cudaDeviceReset of that device: do not call this
+ * function again in a process after resetting the device.
  * Shared state: every call uses the same array and leaves its contents behind; nothing in
  * it needs to start at zero.  Calls whose GPU work overlaps (on different streams, or
  * from different host threads) race on the array, so serialise them.
- * Errors: TQ_ERR_WORKSPACE when the shape needs more scratch than the array holds
- * (tq_decode_workspace_size > TQ_DECODE_STATIC_SCRATCH_BYTES; use tq_decode_attention
- * with a caller workspace instead), otherwise those of tq_decode_attention. */
+ * Errors: first every argument error of tq_decode_attention (TQ_ERR_INVALID_ARG,
+ * TQ_ERR_UNSUPPORTED), then TQ_ERR_WORKSPACE when the shape needs more scratch than the
+ * array holds (tq_decode_workspace_size > TQ_DECODE_STATIC_SCRATCH_BYTES; use
+ * tq_decode_attention with a caller workspace instead), then TQ_ERR_CUDA.  A rejected call
+ * launches nothing. */
 int tq_decode_attention_static(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off,
                                int ngroups, const void* q, int q_dtype, const tq_packed* kcache,
                                const tq_packed* vcache, const int32_t* seq_lens, int B, int Hq, int Hkv, int D,

@@ -356,9 +356,9 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
   const int t_begin = split * A.chunk;
   const int t_end = min(T, t_begin + A.chunk);
   const int64_t slot0 = (int64_t)bh * A.max_len;
-  // The merge kernel behind this one may launch at once: every CTA of this grid is
-  // resident from the start, so its CTAs only take slots that finished CTAs free, and its
-  // grid-dependency wait still sees every partial.
+  // The merge kernel behind this one may launch once every CTA of this grid has run this
+  // trigger (or exited), so its CTAs only take slots of the last wave; its grid-dependency
+  // wait still waits for the whole grid, so it sees every partial.
   allow_dependent_launch();
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNStage; ++i) {

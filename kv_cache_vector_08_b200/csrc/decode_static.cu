@@ -20,7 +20,8 @@ std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device; looked up on the first call
-// for each device (with that device current) and cached.
+// for each device (with that device current) and cached for the life of the process.  A
+// cudaDeviceReset of that device invalidates the cached address.
 int static_scratch(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -45,6 +46,12 @@ extern "C" int tq_decode_attention_static(const tq_ctx* const* kctx, const tq_ct
                                           const tq_packed* kcache, const tq_packed* vcache,
                                           const int32_t* seq_lens, int B, int Hq, int Hkv, int D,
                                           int64_t max_len, float scale, float* out, tq_stream_t stream) {
+  // the arguments first (an invalid shape is TQ_ERR_INVALID_ARG whatever its size), then the
+  // scratch size, then the array's address; nothing is launched before all three pass
+  int r = tq::check_decode_args(kctx, vctx, group_off, ngroups, q, q_dtype, kcache, vcache, seq_lens, B, Hq, Hkv, D,
+                                max_len, out);
+  if (r != TQ_OK) return r;
+  if (B == 0) return TQ_OK;
   size_t need = tq_decode_workspace_size(B, Hq, Hkv, D, ngroups, max_len);
   if (need > (size_t)TQ_DECODE_STATIC_SCRATCH_BYTES)
     return tq::fail(TQ_ERR_WORKSPACE,
@@ -53,7 +60,7 @@ extern "C" int tq_decode_attention_static(const tq_ctx* const* kctx, const tq_ct
                         std::to_string((size_t)TQ_DECODE_STATIC_SCRATCH_BYTES) +
                         " bytes; use tq_decode_attention with a caller workspace");
   void* scratch = nullptr;
-  int r = tq::static_scratch(&scratch);
+  r = tq::static_scratch(&scratch);
   if (r != TQ_OK) return r;
   // Nothing in the scratch has to start at zero: the query-preparation kernel writes every
   // prepared query and the split kernel writes every partial state before the merge reads it.

@@ -59,4 +59,7 @@ int launch_decode(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const in
                   int Hkv, int D, int64_t max_len, float scale, float* out, void* ws, cudaStream_t st);
 int launch_search(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* db, int64_t N, int k,
                   float* scores, int64_t* ids, void* ws, cudaStream_t st);
+int check_decode_args(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off, int ngroups,
+                      const void* q, int q_dtype, const tq_packed* kcache, const tq_packed* vcache,
+                      const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len, const float* out);
 }  // namespace tq

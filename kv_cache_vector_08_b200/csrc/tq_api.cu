@@ -138,6 +138,39 @@ int check_args_common(int d, int bits, int mode) {
 }
 
 }  // namespace
+
+// Every argument check of tq_decode_attention except the workspace size (shared with
+// tq_decode_attention_static, which checks its own scratch size after these).
+int check_decode_args(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off, int ngroups,
+                      const void* q, int q_dtype, const tq_packed* kcache, const tq_packed* vcache,
+                      const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len, const float* out) {
+  if (!kctx || !vctx || !group_off || !kcache || !vcache) return fail(TQ_ERR_INVALID_ARG, "NULL argument");
+  if (ngroups < 1 || ngroups > 4) return fail(TQ_ERR_UNSUPPORTED, "ngroups must be in [1, 4]");
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_len < 0) return fail(TQ_ERR_INVALID_ARG, "bad sizes");
+  if (Hq % Hkv != 0) return fail(TQ_ERR_INVALID_ARG, "Hq must be a multiple of Hkv");
+  if (q_dtype != TQ_DTYPE_F32 && q_dtype != TQ_DTYPE_BF16) return fail(TQ_ERR_INVALID_ARG, "q_dtype must be F32 or BF16");
+  if (group_off[0] != 0 || group_off[ngroups] != D) return fail(TQ_ERR_INVALID_ARG, "group_off must span [0, D]");
+  if (B == 0) return TQ_OK;
+  if (!q || !seq_lens || !out) return fail(TQ_ERR_INVALID_ARG, "NULL q, seq_lens or out");
+  for (int g = 0; g < ngroups; ++g) {
+    const tq_ctx* kc = kctx[g];
+    const tq_ctx* vc = vctx[g];
+    if (!kc || !vc) return fail(TQ_ERR_INVALID_ARG, "NULL context");
+    int w = group_off[g + 1] - group_off[g];
+    if (w <= 0) return fail(TQ_ERR_INVALID_ARG, "group_off must be increasing");
+    if (kc->mode != TQ_MODE_PROD || vc->mode != TQ_MODE_MSE)
+      return fail(TQ_ERR_INVALID_ARG, "key contexts must be prod mode, value contexts MSE mode");
+    if (kc->lay.d != w || vc->lay.d != w) return fail(TQ_ERR_INVALID_ARG, "context dimension differs from its group width");
+    int r = check_packed(kc, &kcache[g], "kcache");
+    if (r != TQ_OK) return r;
+    if ((r = check_packed(vc, &vcache[g], "vcache")) != TQ_OK) return r;
+    int64_t need = (int64_t)B * Hkv * max_len;
+    if (kcache[g].cap < need || vcache[g].cap < need) return fail(TQ_ERR_INVALID_ARG, "cache capacity below B*Hkv*max_len");
+    if ((r = check_device(kc)) != TQ_OK) return r;
+  }
+  return TQ_OK;
+}
+
 }  // namespace tq
 
 using namespace tq;
@@ -341,30 +374,10 @@ int tq_decode_attention(const tq_ctx* const* kctx, const tq_ctx* const* vctx, co
                         const void* q, int q_dtype, const tq_packed* kcache, const tq_packed* vcache,
                         const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len, float scale,
                         float* out, void* workspace, size_t ws_bytes, tq_stream_t stream) {
-  if (!kctx || !vctx || !group_off || !kcache || !vcache) return fail(TQ_ERR_INVALID_ARG, "NULL argument");
-  if (ngroups < 1 || ngroups > 4) return fail(TQ_ERR_UNSUPPORTED, "ngroups must be in [1, 4]");
-  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_len < 0) return fail(TQ_ERR_INVALID_ARG, "bad sizes");
-  if (Hq % Hkv != 0) return fail(TQ_ERR_INVALID_ARG, "Hq must be a multiple of Hkv");
-  if (q_dtype != TQ_DTYPE_F32 && q_dtype != TQ_DTYPE_BF16) return fail(TQ_ERR_INVALID_ARG, "q_dtype must be F32 or BF16");
-  if (group_off[0] != 0 || group_off[ngroups] != D) return fail(TQ_ERR_INVALID_ARG, "group_off must span [0, D]");
+  int r = check_decode_args(kctx, vctx, group_off, ngroups, q, q_dtype, kcache, vcache, seq_lens, B, Hq, Hkv, D,
+                            max_len, out);
+  if (r != TQ_OK) return r;
   if (B == 0) return TQ_OK;
-  if (!q || !seq_lens || !out) return fail(TQ_ERR_INVALID_ARG, "NULL q, seq_lens or out");
-  for (int g = 0; g < ngroups; ++g) {
-    const tq_ctx* kc = kctx[g];
-    const tq_ctx* vc = vctx[g];
-    if (!kc || !vc) return fail(TQ_ERR_INVALID_ARG, "NULL context");
-    int w = group_off[g + 1] - group_off[g];
-    if (w <= 0) return fail(TQ_ERR_INVALID_ARG, "group_off must be increasing");
-    if (kc->mode != TQ_MODE_PROD || vc->mode != TQ_MODE_MSE)
-      return fail(TQ_ERR_INVALID_ARG, "key contexts must be prod mode, value contexts MSE mode");
-    if (kc->lay.d != w || vc->lay.d != w) return fail(TQ_ERR_INVALID_ARG, "context dimension differs from its group width");
-    int r = check_packed(kc, &kcache[g], "kcache");
-    if (r != TQ_OK) return r;
-    if ((r = check_packed(vc, &vcache[g], "vcache")) != TQ_OK) return r;
-    int64_t need = (int64_t)B * Hkv * max_len;
-    if (kcache[g].cap < need || vcache[g].cap < need) return fail(TQ_ERR_INVALID_ARG, "cache capacity below B*Hkv*max_len");
-    if ((r = check_device(kc)) != TQ_OK) return r;
-  }
   size_t need = tq_decode_workspace_size(B, Hq, Hkv, D, ngroups, max_len);
   if (!workspace || ws_bytes < need) return fail(TQ_ERR_WORKSPACE, "workspace too small");
   return launch_decode(kctx, vctx, group_off, ngroups, q, q_dtype, kcache, vcache, seq_lens, B, Hq, Hkv, D, max_len,

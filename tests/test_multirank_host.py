@@ -59,12 +59,42 @@ def test_single_rank_needs_no_process_group():
     assert bench.whole_job_rate(10, 1, 2.0) == 5.0
 
 
+class _FakeSample:
+    """Stands in for the oracle sample: counts steps, scores 1000 keys per step."""
+    made = []
+
+    def __init__(self, w, kind, heads, seed=0):
+        self.heads = heads
+        _FakeSample.made.append(self)
+
+    def step(self):
+        return 1000
+
+    def describe(self, dt):
+        return "fake sample"
+
+
 def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     import bench
-    called = []
-    monkeypatch.setattr(bench, "oracle_sample_step", lambda *a, **k: called.append(1) or 1)
+    _FakeSample.made = []
+    monkeypatch.setattr(bench, "OracleSample", _FakeSample)
     monkeypatch.setenv("WORLD_SIZE", "2")
     monkeypatch.setenv("RANK", "1")
-    args = types.SimpleNamespace(steps=2, warmup=3, cpu_sample_heads=1)
+    args = types.SimpleNamespace(steps=2, warmup=3, config="serving")
     bench.run_reference(args)
-    assert called == [] and capsys.readouterr().out == ""
+    assert _FakeSample.made == [] and capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_on_rank_zero(monkeypatch, capsys):
+    import json
+    import bench
+    _FakeSample.made = []
+    monkeypatch.setattr(bench, "OracleSample", _FakeSample)
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "0")
+    args = types.SimpleNamespace(steps=2, warmup=3, config="serving")
+    bench.run_reference(args)
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["impl"] == "reference" and line["unit"] == "keys/s" and line["n_gpus"] == 2
+    assert line["config"]["workload"] == "serving-decode-3.5bit"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"

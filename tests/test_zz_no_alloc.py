@@ -80,14 +80,39 @@ def test_static_scratch_decode_matches_workspace_decode(groups, B, seq_lens, max
         parity.assert_close(out.cpu().numpy(), ref.cpu().numpy(), "static call %d" % call)
 
 
+def test_static_scratch_call_allocates_nothing():
+    """After a first call (which looks up the array and lets the driver load the kernels),
+    a call leaves the device's free memory unchanged."""
+    groups = ((0, 128, 4, 4),)
+    B, Hkv, Hq, D, max_len = 2, 8, 32, 128, 2048
+    kctx, vctx, offs, q, kc, vc, seq = _case(B, Hkv, Hq, D, groups, [2048, 1500], max_len, 7)
+    plan = tq.DecodePlan(kctx, vctx, offs, kc, vc, B, Hq, Hkv, D, max_len)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=DEV)
+    assert _call_static(plan, q, seq, 0.1, out) == 0, tq.lib().tq_last_error()
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    n0 = tq.launch_count()
+    assert _call_static(plan, q, seq, 0.1, out) == 0, tq.lib().tq_last_error()
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert tq.launch_count() > n0
+    assert free1 == free0, "free device memory changed by %d bytes" % (free0 - free1)
+
+
 def test_static_scratch_rejects_shapes_above_its_size():
     groups = ((0, 128, 4, 4),)
-    kctx, vctx, offs, q, kc, vc, seq = _case(1, 8, 32, 128, groups, [16], 16, 6)
     B, Hq, Hkv, D, max_len = 512, 64, 8, 128, 16    # prepared queries alone need 32 MiB
+    kctx, vctx, offs, q, kc, vc, seq = _case(B, Hkv, Hq, D, groups, [16] * B, max_len, 6)
     assert tq.decode_workspace_size(B, Hq, Hkv, D, 1, max_len) > STATIC_BYTES
-    plan = tq.DecodePlan(kctx, vctx, offs, kc, vc, 1, 32, 8, 128, 16)
-    plan.B, plan.Hq, plan.Hkv = B, Hq, Hkv
-    out = torch.empty(1, dtype=torch.float32, device=DEV)
+    plan = tq.DecodePlan(kctx, vctx, offs, kc, vc, B, Hq, Hkv, D, max_len)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=DEV)
+    torch.cuda.synchronize()
+    n0 = tq.launch_count()
     status = _call_static(plan, q, seq, 1.0, out)
-    assert status == 5                              # TQ_ERR_WORKSPACE, before any launch
+    assert status == 5                              # TQ_ERR_WORKSPACE
     assert b"static scratch" in tq.lib().tq_last_error()
+    assert tq.launch_count() == n0                  # nothing was launched
+    # an invalid shape is reported as such even when it is also too large
+    plan.Hq = 63
+    assert _call_static(plan, q, seq, 1.0, out) == 1    # TQ_ERR_INVALID_ARG
+    assert tq.launch_count() == n0
