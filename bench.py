@@ -439,7 +439,7 @@ def run_gpu(args):
     del bench
     torch.cuda.empty_cache()
     if args.configs:
-        line["stream_peaks"] = measure_stream(dev)
+        line["stream_peaks"] = guarded(measure_stream, dev)
         line["configs"] = measure_configs(kind, dev, peaks, args)
     line["cpu_baseline"] = cpu_baseline(w, kind)
     print(json.dumps(line), flush=True)
@@ -489,8 +489,7 @@ def measure_stream(dev):
     torch.cuda.synchronize()
     nofl = lambda st: None
     t_copy = min(_time_device(lambda: b.copy_(a), nofl, 5) for _ in range(2))
-    acc = torch.empty((), dtype=torch.float32, device=dev)
-    t_read = min(_time_device(lambda: torch.sum(a, out=acc), nofl, 5) for _ in range(2))
+    t_read = min(_time_device(lambda: torch.sum(a), nofl, 5) for _ in range(2))
     nb = a.numel() * 4
     del a, b
     torch.cuda.empty_cache()
@@ -498,19 +497,28 @@ def measure_stream(dev):
             "how": "torch copy_ and sum over 4 GiB fp32, best of 2 x mean of 5, CUDA events"}
 
 
-def measure_configs(headline, dev, peaks, args):
+def guarded(fn, *a):
+    """fn(*a), or {"error": ...} if it raises (a secondary measurement never costs the
+    headline line)."""
     import torch
+    try:
+        return fn(*a)
+    except Exception as e:  # noqa: BLE001
+        torch.cuda.synchronize()
+        return {"error": "%s: %s" % (type(e).__name__, e)}
+    finally:
+        torch.cuda.empty_cache()
+
+
+def measure_configs(headline, dev, peaks, args):
     out = {}
     for kind in ("serving", "llama", "long"):
         if kind == headline:
             continue
-        out[DECODE_CONFIGS[kind].name] = measure_decode_config(kind, dev, peaks)
-        torch.cuda.empty_cache()
-    out[W.TOY["name"]] = measure_toy(dev)
-    torch.cuda.empty_cache()
-    for spec in (W.SEARCH_1536, W.SEARCH_200):
-        out[spec["name"]] = measure_search(spec, dev, peaks)
-        torch.cuda.empty_cache()
+        out[DECODE_CONFIGS[kind].name] = guarded(measure_decode_config, kind, dev, peaks)
+    out[W.TOY["name"]] = guarded(measure_toy, dev)
+    for spec in (W.SEARCH_1536, W.SEARCH_200, W.SEARCH_3072):
+        out[spec["name"]] = guarded(measure_search, spec, dev, peaks)
     return out
 
 
@@ -633,6 +641,13 @@ def measure_rows(bench, peaks, reps=5):
     out["dequantize"] = hbm_roof(nbytes, t, peaks, "dequantize",
                                  work="%d value vectors (d=%d, %d-bit MSE) -> fp32" % (n, vctx.d, vctx.bits),
                                  algorithmic_tflops=2.0 * vctx.d * vctx.d * n / t / 1e12)
+    kq = torch.empty((n, kctx.d), dtype=torch.float32, device=dev)
+    t = _time_device(lambda: tq.dequantize(kctx, kc, n, out=kq, qjl=True), bench.flush_l2, reps)
+    nbytes = n * (kctx.code_bytes + 4) + n * kctx.d * 4
+    out["dequantize_qjl"] = hbm_roof(nbytes, t, peaks, "dequantize_qjl",
+                                     work="%d key vectors (d=%d, %d-bit prod) -> fp32, QJL-augmented" % (
+                                         n, kctx.d, kctx.bits),
+                                     algorithmic_tflops=4.0 * kctx.d * kctx.d * n / t / 1e12)
     return out
 
 

@@ -133,10 +133,21 @@ int tq_host_params(int d, int bits, uint64_t seed, int mode, double* Pi, double*
  * still queued on any stream. */
 void tq_free(tq_ctx* ctx);
 
-/* Kernel-side failure report: a tensor-core kernel whose pipeline wait exceeds its time
- * limit (2 s) records a non-zero code in the context's device error word, stops its work
- * and exits cleanly instead of hanging.  This call synchronises the device, copies the
- * word to *code (0 = no failure) and clears it. */
+/* Kernel-side failure report.  Kernels record the first failure they meet in the
+ * context's device error word and carry on or wind down instead of faulting or hanging:
+ *   101-109  fused quantize kernel: a pipeline wait exceeded its limit (2 s)
+ *   201-203  decode attention: a pipeline wait exceeded its limit
+ *   301-305  dequantize: a pipeline wait exceeded its limit (tq_debug_set_wait_limit; 305:
+ *            the stall injected by tq_debug_inject_stall)
+ *   401-404  workspace quantize path: a pipeline wait exceeded its limit (idem)
+ *   501-506  search: a pipeline wait exceeded its limit (idem)
+ *   901      a device slot array (dst_slot / src_slot) held a slot outside [0, cap): that
+ *            row was skipped (quantize) or written as zeros (dequantize)
+ *   902      a channel permutation or column map held an entry out of range: that element
+ *            was read as 0 or not written
+ * A kernel whose wait gives up drains its in-flight copies and MMAs, releases its tensor
+ * memory and returns, so the context stays usable.  This call synchronises the device,
+ * copies the word to *code (0 = no failure) and clears it. */
 int tq_get_device_error(const tq_ctx* ctx, int* code);
 
 /* Fill *info (host pointer). */
@@ -159,16 +170,51 @@ int tq_get_params(const tq_ctx* ctx, double* Pi, double* S, double* centroids, d
  *    x + v*ld elements; ld >= d.  Any channel slice of a wider row is passed by offsetting x.
  * dst: packed storage; vector v goes to slot dst_slot[v] (device int64 array) or, when
  *    dst_slot is NULL, to slot v.  Every slot must be < dst->cap.
+ * Kernels: bf16 input with d in {64, 128}, n >= 128, x and ld*2 16-byte aligned runs one
+ *    fused tensor-core kernel that needs no workspace.  Every other call runs the
+ *    workspace path (a norm / fp16-split kernel, then the rotation GEMM with the
+ *    nearest-centroid epilogue and, in prod mode, the QJL GEMM with the sign epilogue,
+ *    all on the tensor cores) over row chunks of at most 131072 vectors.
+ * workspace: device, 256-byte aligned, >= tq_quantize_workspace_size(ctx, x_dtype, n, ld)
+ *    bytes (may be NULL when that size is 0).
  * Errors: TQ_ERR_INVALID_ARG (NULL pointers, n < 0, ld < d, rnorm NULL in prod mode),
- * TQ_ERR_UNSUPPORTED (misaligned codes), TQ_ERR_CUDA. */
+ * TQ_ERR_UNSUPPORTED (misaligned codes or workspace), TQ_ERR_WORKSPACE (workspace too
+ * small for the path the call takes, e.g. a bf16 x that is not 16-byte aligned), TQ_ERR_CUDA. */
+size_t tq_quantize_workspace_size(const tq_ctx* ctx, int x_dtype, int64_t n, int64_t ld);
 int tq_quantize_kv(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld,
-                   const tq_packed* dst, const int64_t* dst_slot, tq_stream_t stream);
+                   const tq_packed* dst, const int64_t* dst_slot, void* workspace, size_t ws_bytes,
+                   tq_stream_t stream);
+
+/* tq_quantize_kv_cols -- tq_quantize_kv of a column subset of each row: element j of vector v
+ * is x[v*ld + cols[j]] (cols: device int32 [d], each in [0, ld)), e.g. the channels of one
+ * group under an outlier-aware channel permutation (tq_decode_attention_perm).  Runs the
+ * workspace path; workspace >= tq_quantize_cols_workspace_size(ctx, n) bytes.  An entry of
+ * cols outside [0, ld) reads as 0 and is reported as device error 902.  Errors as
+ * tq_quantize_kv, plus TQ_ERR_INVALID_ARG for a NULL cols. */
+size_t tq_quantize_cols_workspace_size(const tq_ctx* ctx, int64_t n);
+int tq_quantize_kv_cols(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld,
+                        const int32_t* cols, const tq_packed* dst, const int64_t* dst_slot, void* workspace,
+                        size_t ws_bytes, tq_stream_t stream);
 
 /* tq_dequantize -- MSE reconstruction x_hat = norm * Pi^T c[idx] of n stored vectors
- * ([TQN] "Quant / DeQuant 函数").  Vector v is read from slot src_slot[v] (device int64) or
- * slot v when src_slot is NULL, and written to out + v*ld (device float32, ld >= d). */
+ * ([TQN] "Quant / DeQuant 函数"), one tensor-core GEMM per 128 vectors (centroids as fp16
+ * hi + lo against Pi^T as fp16 hi + lo, fp32 accumulation).  Vector v is read from slot
+ * src_slot[v] (device int64) or slot v when src_slot is NULL, and written to out + v*ld
+ * (device float32, ld >= d).  Prod-mode codes are reconstructed from their index bits.
+ * Errors: TQ_ERR_INVALID_ARG (NULL pointers, n < 0, ld < d), TQ_ERR_UNSUPPORTED (d > 128),
+ * TQ_ERR_CUDA. */
 int tq_dequantize(const tq_ctx* ctx, const tq_packed* src, const int64_t* src_slot, int64_t n,
                   float* out, int64_t ld, tq_stream_t stream);
+
+/* tq_dequantize_qjl -- QJL-augmented reconstruction of stored keys (prod mode):
+ *   x_hat = norm * ( Pi^T c[idx] + sqrt(pi/2)/m * rnorm * S^T (2 s - 1) ),
+ * the vector whose inner product with any q is the unbiased estimate of tq_attn_logits
+ * ([ZX] "两阶段内积量化", [ADM] QJL paragraph: the estimator in vector form).  One
+ * tensor-core GEMM per 128 vectors: the centroid part as for tq_dequantize plus the sign
+ * part (+-rnorm, exact in fp16, against 16 sqrt(pi/2)/m S^T as fp16 hi + lo).  Arguments,
+ * layout and errors as tq_dequantize; TQ_ERR_INVALID_ARG for an MSE-mode context. */
+int tq_dequantize_qjl(const tq_ctx* ctx, const tq_packed* src, const int64_t* src_slot, int64_t n,
+                      float* out, int64_t ld, tq_stream_t stream);
 
 /* tq_prepare_queries -- rotate queries once: out[a] = (Pi q_a [d floats], S q_a [m floats])
  * ([TQN] "集成到 Attention": the query side of the QJL estimate).  q: device float32
@@ -204,6 +250,30 @@ int tq_decode_attention(const tq_ctx* const* kctx, const tq_ctx* const* vctx, co
                         const tq_packed* vcache, const int32_t* seq_lens, int B, int Hq, int Hkv,
                         int D, int64_t max_len, float scale, float* out, void* workspace,
                         size_t ws_bytes, tq_stream_t stream);
+
+/* tq_decode_attention_perm -- tq_decode_attention with the head dimension's channels
+ * regrouped per kv head: channel group g of kv head hk covers channels
+ * channel_perm[hk*D + group_off[g]] .. channel_perm[hk*D + group_off[g+1] - 1] of q, K, V and
+ * out (the keys and values must have been quantized with the same columns, e.g. by
+ * tq_quantize_kv_cols).  This is how outlier channels are sent to the higher-bit group of a
+ * 2.5 / 3.5-bit split ([ZX] "KV缓存量化的质量表现": 2.5 and 3.5 bits per channel;
+ * turboquant.net "潜在挑战与解决方案": outlier handling).  channel_perm: device int32
+ * [Hkv][D], each row a permutation of 0..D-1, or NULL for the identity (then identical to
+ * tq_decode_attention).  An entry outside [0, D) is skipped and reported as device error 902.
+ * Other arguments, layout and errors as tq_decode_attention. */
+int tq_decode_attention_perm(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off,
+                             int ngroups, const int32_t* channel_perm, const void* q, int q_dtype,
+                             const tq_packed* kcache, const tq_packed* vcache, const int32_t* seq_lens, int B,
+                             int Hq, int Hkv, int D, int64_t max_len, float scale, float* out, void* workspace,
+                             size_t ws_bytes, tq_stream_t stream);
+
+/* tq_channel_perm_by_score -- host helper for the outlier-aware channel grouping: perm (host
+ * int32 [D]) lists the w0 channels with the highest score (ties to the lower channel) in
+ * ascending order, then the other channels in ascending order.  With score = a per-channel
+ * magnitude statistic of a calibration sample (e.g. the RMS over tokens), declared or
+ * detected outlier channels land in the first (higher-bit) group of width w0.  score: host
+ * float [D].  Errors: TQ_ERR_INVALID_ARG (NULL pointers, D <= 0, w0 outside [0, D]). */
+int tq_channel_perm_by_score(const float* score, int D, int w0, int32_t* perm);
 
 /* Size in bytes of the library-owned scratch array used by tq_decode_attention_static. */
 #define TQ_DECODE_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
@@ -243,6 +313,22 @@ size_t tq_search_workspace_size(const tq_ctx* ctx, int64_t nq, int64_t N, int k)
 int tq_search_topk(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* db, int64_t N,
                    int k, float* scores, int64_t* ids, void* workspace, size_t ws_bytes,
                    tq_stream_t stream);
+
+/* Test hooks (not for production use).
+ * tq_debug_set_wait_limit -- limit, in nanoseconds, of the pipeline waits of the
+ *   dequantize, search and workspace-quantize kernels launched after the call (default 2 s;
+ *   0 makes every wait that is not already satisfied give up at once).  Their final
+ *   drains of in-flight copies and MMAs keep the 2 s limit, so a kernel that gives up still
+ *   leaves no transfer behind.  Process-wide; not thread-safe against concurrent launches.
+ * tq_debug_inject_stall -- while on, the dequantize kernel's MMA issuer first waits on a
+ *   barrier that nothing arrives on; the wait gives up after the pipeline wait limit,
+ *   records device error 305 and the kernel winds down (its output is then undefined).
+ * tq_debug_fail_alloc -- make device allocation number `index` (0-based, counted from this
+ *   call) inside tq_init fail as if the device were out of memory; -1 disables.  tq_init
+ *   then returns TQ_ERR_ALLOC having released everything it allocated. */
+int tq_debug_set_wait_limit(uint64_t ns);
+int tq_debug_inject_stall(int on);
+int tq_debug_fail_alloc(int index);
 
 /* Message describing the calling thread's most recent error ("" if none). */
 const char* tq_last_error(void);

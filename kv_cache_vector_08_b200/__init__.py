@@ -15,7 +15,7 @@ import numpy as np
 
 __all__ = [
     "MODE_PROD", "MODE_MSE", "TQError", "Context", "Packed", "host_params", "alloc_packed",
-    "quantize_kv", "dequantize", "prepare_queries", "attn_logits", "decode_attention",
+    "quantize_kv", "quantize_workspace_size", "channel_perm_by_score", "dequantize", "prepare_queries", "attn_logits", "decode_attention",
     "decode_workspace_size", "search_topk", "launch_count", "lib_path", "lib",
 ]
 
@@ -66,18 +66,27 @@ def lib():
         "tq_free": (None, [P]),
         "tq_get_info": (I, [P, ctypes.POINTER(_Info)]),
         "tq_get_params": (I, [P, P, P, P, P]),
-        "tq_quantize_kv": (I, [P, P, I, I64, I64, PK, P, P]),
+        "tq_quantize_workspace_size": (SZ, [P, I, I64, I64]),
+        "tq_quantize_kv": (I, [P, P, I, I64, I64, PK, P, P, SZ, P]),
         "tq_dequantize": (I, [P, PK, P, I64, P, I64, P]),
+        "tq_dequantize_qjl": (I, [P, PK, P, I64, P, I64, P]),
         "tq_prepare_queries": (I, [P, P, I64, I64, P, P]),
         "tq_attn_logits_workspace_size": (SZ, [P, I64]),
         "tq_attn_logits": (I, [P, P, I64, PK, I64, P, P, SZ, P]),
         "tq_decode_workspace_size": (SZ, [I, I, I, I, I, I64]),
         "tq_decode_attention": (I, [P, P, P, I, P, I, PK, PK, P, I, I, I, I, I64, F, P, P, SZ, P]),
+        "tq_decode_attention_perm": (I, [P, P, P, I, P, P, I, PK, PK, P, I, I, I, I, I64, F, P, P, SZ, P]),
+        "tq_channel_perm_by_score": (I, [P, I, I, P]),
+        "tq_quantize_cols_workspace_size": (SZ, [P, I64]),
+        "tq_quantize_kv_cols": (I, [P, P, I, I64, I64, P, PK, P, P, SZ, P]),
         "tq_search_workspace_size": (SZ, [P, I64, I64, I]),
         "tq_search_topk": (I, [P, P, I64, PK, I64, I, P, P, P, SZ, P]),
         "tq_last_error": (ctypes.c_char_p, []),
         "tq_kernel_launch_count": (U64, []),
         "tq_get_device_error": (I, [P, ctypes.POINTER(I)]),
+        "tq_debug_set_wait_limit": (I, [U64]),
+        "tq_debug_inject_stall": (I, [I]),
+        "tq_debug_fail_alloc": (I, [I]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -209,23 +218,56 @@ def alloc_packed(ctx: Context, cap: int, device=None) -> Packed:
     return Packed(codes, norm, rnorm)
 
 
-def quantize_kv(ctx: Context, x, dst: Packed, slots=None, stream=None):
-    """Quantize rows of x (CUDA tensor [n, >=d], fp32/bf16/fp16) into dst (slot v, or slots[v])."""
-    n, ld = _rows(x, ctx.d)
+def quantize_workspace_size(ctx: Context, x_dtype: int, n: int, ld: int) -> int:
+    return int(lib().tq_quantize_workspace_size(ctx.handle, x_dtype, n, ld))
+
+
+def quantize_kv(ctx: Context, x, dst: Packed, slots=None, stream=None, workspace=None, cols=None):
+    """Quantize rows of x (CUDA tensor [n, >=d], fp32/bf16/fp16) into dst (slot v, or slots[v]).
+    cols (CUDA int32 [d]): quantize the columns cols of each row of x instead of its first d.
+    A workspace is allocated (torch caching allocator) when the call needs one and none is given."""
+    torch = _torch()
+    dt = _dtype_code(x)
     ps = dst.struct()
-    _check(lib().tq_quantize_kv(ctx.handle, _ptr(x), _dtype_code(x), n, ld, ctypes.byref(ps), _ptr(slots),
-                                _stream(stream)))
+    if cols is not None:
+        if x.dim() != 2 or x.stride(1) != 1:
+            raise ValueError("expected a 2-D tensor with unit stride along rows")
+        n, ld = x.shape[0], x.stride(0)
+        need = int(lib().tq_quantize_cols_workspace_size(ctx.handle, n))
+        if workspace is None and need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+        _check(lib().tq_quantize_kv_cols(ctx.handle, _ptr(x), dt, n, ld, _ptr(cols), ctypes.byref(ps), _ptr(slots),
+                                         _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                         _stream(stream)))
+        return
+    n, ld = _rows(x, ctx.d)
+    need = quantize_workspace_size(ctx, dt, n, ld)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check(lib().tq_quantize_kv(ctx.handle, _ptr(x), dt, n, ld, ctypes.byref(ps), _ptr(slots), _ptr(workspace),
+                                0 if workspace is None else workspace.numel(), _stream(stream)))
 
 
-def dequantize(ctx: Context, src: Packed, n: int = None, slots=None, out=None, stream=None):
+def channel_perm_by_score(score, w0: int) -> np.ndarray:
+    """Host permutation putting the w0 highest-scoring channels first (see tq.h)."""
+    score = np.ascontiguousarray(score, dtype=np.float32)
+    perm = np.zeros(score.shape[0], dtype=np.int32)
+    _check(lib().tq_channel_perm_by_score(score.ctypes.data_as(ctypes.c_void_p), score.shape[0], int(w0),
+                                          perm.ctypes.data_as(ctypes.c_void_p)))
+    return perm
+
+
+def dequantize(ctx: Context, src: Packed, n: int = None, slots=None, out=None, stream=None, qjl: bool = False):
+    """x_hat = norm Pi^T c[idx] of stored vectors (qjl=True, prod mode: plus the QJL term
+    norm sqrt(pi/2)/m rnorm S^T (2 s - 1))."""
     torch = _torch()
     if slots is not None:
         n = slots.shape[0]
     if out is None:
         out = torch.empty((n, ctx.d), dtype=torch.float32, device=src.codes.device)
     ps = src.struct()
-    _check(lib().tq_dequantize(ctx.handle, ctypes.byref(ps), _ptr(slots), n, _ptr(out), out.stride(0),
-                               _stream(stream)))
+    fn = lib().tq_dequantize_qjl if qjl else lib().tq_dequantize
+    _check(fn(ctx.handle, ctypes.byref(ps), _ptr(slots), n, _ptr(out), out.stride(0), _stream(stream)))
     return out
 
 
@@ -261,8 +303,10 @@ class DecodePlan:
     """Pre-marshalled arguments of tq_decode_attention (avoids per-call ctypes setup)."""
 
     def __init__(self, kctx: Sequence[Context], vctx: Sequence[Context], group_off: Sequence[int],
-                 kcache: Sequence[Packed], vcache: Sequence[Packed], B, Hq, Hkv, D, max_len, device=None):
+                 kcache: Sequence[Packed], vcache: Sequence[Packed], B, Hq, Hkv, D, max_len, device=None,
+                 channel_perm=None):
         torch = _torch()
+        self.channel_perm = channel_perm       # CUDA int32 [Hkv, D] or None
         G = len(kctx)
         self.G, self.B, self.Hq, self.Hkv, self.D, self.max_len = G, B, Hq, Hkv, D, max_len
         self._k = (ctypes.c_void_p * G)(*[c.handle.value for c in kctx])
@@ -276,6 +320,13 @@ class DecodePlan:
         self.workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
 
     def __call__(self, q, seq_lens, scale: float, out, stream=None):
+        if self.channel_perm is not None:
+            _check(lib().tq_decode_attention_perm(self._k, self._v, self._off, self.G, _ptr(self.channel_perm), _ptr(q),
+                                                  _dtype_code(q), self._kc, self._vc, _ptr(seq_lens), self.B,
+                                                  self.Hq, self.Hkv, self.D, self.max_len, ctypes.c_float(scale),
+                                                  _ptr(out), _ptr(self.workspace), self.workspace.numel(),
+                                                  _stream(stream)))
+            return out
         _check(lib().tq_decode_attention(self._k, self._v, self._off, self.G, _ptr(q), _dtype_code(q), self._kc,
                                          self._vc, _ptr(seq_lens), self.B, self.Hq, self.Hkv, self.D,
                                          self.max_len, ctypes.c_float(scale), _ptr(out), _ptr(self.workspace),
@@ -284,12 +335,13 @@ class DecodePlan:
 
 
 def decode_attention(kctx, vctx, group_off, q, kcache, vcache, seq_lens, Hkv, max_len, scale, out=None,
-                     stream=None):
+                     stream=None, channel_perm=None):
     """One decode step; q [B, Hq, D] (fp32/bf16 CUDA), seq_lens int32 CUDA [B] -> out fp32 [B, Hq, D].
     Token t of sequence b, kv head h lives in slot (b*Hkv + h)*max_len + t of each cache."""
     torch = _torch()
     B, Hq, D = q.shape
-    plan = DecodePlan(kctx, vctx, group_off, kcache, vcache, B, Hq, Hkv, D, max_len, device=q.device)
+    plan = DecodePlan(kctx, vctx, group_off, kcache, vcache, B, Hq, Hkv, D, max_len, device=q.device,
+                      channel_perm=channel_perm)
     if out is None:
         out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
     return plan(q.contiguous(), seq_lens, scale, out, stream)

@@ -9,6 +9,8 @@
 #include <cstdint>
 #include <string>
 
+#include <cuda.h>
+
 #include "../../include/tq.h"
 #include "params.h"
 
@@ -75,16 +77,25 @@ struct tq_ctx {
   int m = 0, mode = 0, bits = 0;
   float sqrt_pi_over_2_over_m = 0.f;  // QJL unbiasing constant sqrt(pi/2)/m
   float s_rowmax = 0.f;               // max_j ||S_j||: bounds |(S q)_j| by s_rowmax * ||q||
-  // device float32 copies (row-major)
+  // device float32 copies (row-major): Pi for the decode merge's inverse rotation, the
+  // transposes for the query projections (coalesced column access)
   float* Pi = nullptr;    // [d][d]    y = Pi x
-  float* PiT = nullptr;   // [d][d]    Pi^T (coalesced column access)
-  float* S = nullptr;     // [m][d]
-  float* ST = nullptr;    // [d][m]
-  float* MT = nullptr;    // [d][m]    (S Pi^T)^T
+  float* PiT = nullptr;   // [d][d]    Pi^T
+  float* ST = nullptr;    // [d][m]    S^T
   // tensor-core operands (d in {64, 128}): Pi as three bf16 splits [3][d][d] and
   // 16 * M as two fp16 splits [2][d][d], row-major
   void* Pi_split = nullptr;
   void* M_split = nullptr;
+  // dequantize operand (d <= 128): 16 Pi^T as fp16 hi / lo, [2][N][d_pad] with
+  // N = 16 ceil(d/16), row n holding 16 Pi[k][n] over k (zero padded)
+  void* PiT_f16 = nullptr;
+  // QJL-augmented dequantize operand (prod mode, d <= 128): 16 sqrt(pi/2)/m S^T as fp16
+  // hi / lo, same layout (row n holding 16 kappa S[k][n] over k)
+  void* ST_f16 = nullptr;
+  // projection operands of the workspace quantize path (any d): 16 Pi and 16 M as fp16 hi /
+  // lo, [2][d_pad][K] with K = 64 ceil(d/64), row n holding 16 Pi[n][k] (16 M[n][k])
+  void* Pi16 = nullptr;
+  void* M16 = nullptr;
   int* dev_err = nullptr;  // device error word written by kernels that detect a stuck pipeline
 };
 
@@ -94,6 +105,26 @@ void set_error(const std::string& msg);
 int fail(int code, const std::string& msg);
 int cuda_fail(cudaError_t e, const char* what);
 void count_launch(uint64_t n = 1);
+
+// Limit of the pipeline waits of the dequantize, search and workspace-quantize kernels
+// (2 s unless a test changed it with tq_debug_set_wait_limit).
+uint64_t pipeline_wait_ns();
+// Test hook: the dequantize kernel's MMA issuer first waits on a barrier that nothing
+// arrives on (tq_debug_inject_stall), so that wait runs out after pipeline_wait_ns().
+bool debug_stall();
+// Device allocation of tq_init (a test can make the n-th one fail, see tq_debug_fail_alloc).
+cudaError_t dev_alloc(void** p, size_t bytes);
+
+// Kernel-side error codes written to the context's error word (first one wins).
+enum DeviceError : int {
+  kErrSlotRange = 901,   // a slot index outside [0, cap) was passed in a device slot array: the row is skipped
+  kErrPermRange = 902,   // a channel permutation / column map entry outside [0, D): the element is skipped
+};
+
+// 2-D row-major tensor map [rows][cols] of 16-bit elements with box {64 columns, box_rows
+// rows} and 128-byte swizzle (the canonical K-major operand layout of tcgen05.mma).
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t rows, uint64_t cols,
+              uint64_t row_stride_bytes, uint32_t box_rows);
 
 // Returns TQ_OK if the last launch succeeded, else records the error.
 int check_launch(const char* what);

@@ -50,6 +50,9 @@ using namespace mmaops;
 
 constexpr int kWarps = 4;
 constexpr int kRep = 4;            // query heads per kv head handled by this kernel
+#ifndef TQ_DECODE_CTAS_PER_SM
+#define TQ_DECODE_CTAS_PER_SM 3    // resident decode CTAs per SM the register budget is sized for
+#endif
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -151,6 +154,7 @@ struct MmaGroup {
 struct MmaArgs {
   MmaGroup g[2];
   int B, Hq, Hkv, D, nsplit, chunk, G;
+  int rep, nsub;           // query heads per kv head; CTAs per (sequence, kv head) = ceil(rep / 4)
   int64_t max_len;
   float scale_log2;        // softmax scale * log2(e)
   const int32_t* seq_lens;
@@ -163,6 +167,13 @@ struct MmaArgs {
 };
 
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
+// Query head of MMA column group j (0..3) of a CTA that serves heads sub*4 .. sub*4+3 of kv
+// head hk; columns past the kv head's rep heads repeat its last head (their results are
+// not written).
+__device__ __forceinline__ int col_head(int hk, int rep, int sub, int j) {
+  return hk * rep + min(sub * kRep + j, rep - 1);
+}
 __device__ __forceinline__ void allow_dependent_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
 // Query operands of one group for this thread: B fragments (column g = head g/2, digit
@@ -175,9 +186,9 @@ struct QOps {
 };
 
 template <class GC>
-__device__ __forceinline__ void load_qops(QOps<GC>& f, const MmaArgs& A, int gi, int b, int hk, int lane) {
+__device__ __forceinline__ void load_qops(QOps<GC>& f, const MmaArgs& A, int gi, int b, int hk, int sub, int lane) {
   const int g = lane >> 2, l = lane & 3;
-  const int head = hk * kRep + (g >> 1);
+  const int head = col_head(hk, A.rep, sub, g >> 1);
   const bool lo = (g & 1) != 0;
   const float* pm = A.qprep + ((size_t)(b * A.Hq + head) * A.G + gi) * 2 * A.D + GC::CQ * l;
   const float* ps = pm + A.D;
@@ -339,7 +350,7 @@ __device__ __forceinline__ uint32_t stage_span(uint8_t* dst, const uint8_t* src,
 }
 
 template <class G0, class G1>
-__global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArgs A) {
+__global__ void __launch_bounds__((kWarps + 1) * 32, TQ_DECODE_CTAS_PER_SM) decode_mma_kernel(MmaArgs A) {
   constexpr bool TWO = !std::is_same<G1, void>::value;
   using G1c = typename std::conditional<TWO, G1, G0>::type;
   using ST = Stage<G0, G1c, TWO>;
@@ -348,7 +359,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
   __shared__ float s_acc[kWarps][kRep][256];
   __shared__ __align__(8) uint64_t full[kNStage], empty[kNStage];
   __shared__ int s_abort;
-  const int split = blockIdx.x, bh = blockIdx.y;
+  const int split = blockIdx.x, bh = blockIdx.y / A.nsub, sub = blockIdx.y % A.nsub;
   const int b = bh / A.Hkv, hk = bh % A.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, l = lane & 3;
@@ -386,9 +397,9 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
     const Luts t1 = A.g[TWO ? 1 : 0].lut;
     grid_dependency_wait();   // prepared queries come from the preceding kernel
     QOps<G0> q0;
-    load_qops<G0>(q0, A, 0, b, hk, lane);
+    load_qops<G0>(q0, A, 0, b, hk, sub, lane);
     QOps<G1c> q1;
-    if constexpr (TWO) load_qops<G1c>(q1, A, 1, b, hk, lane);
+    if constexpr (TWO) load_qops<G1c>(q1, A, 1, b, hk, sub, lane);
 #pragma unroll
     for (int u = 0; u < G0::NS; ++u)
 #pragma unroll
@@ -452,9 +463,12 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
       mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
       mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
       mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
-      if (mt > m_run) {
-        const float alpha = exp2f(m_run - mt);
-        m_run = mt;
+      // rescale only in the (rare) tiles where some head's maximum grows; the branch is
+      // warp-uniform, lanes whose head did not grow scale by 1
+      if (__any_sync(0xffffffffu, mt > m_run)) {
+        const float mn = fmaxf(m_run, mt);
+        const float alpha = mn == m_run ? 1.f : exp2f(m_run - mn);
+        m_run = mn;
         l_run *= alpha;
 #pragma unroll
         for (int u = 0; u < G0::NS; ++u)
@@ -511,7 +525,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
     if constexpr (TWO) store_acc(acc1, G1c{}, A.g[1].off);
   } else {
     // ---------------------------------------------------------------- producer warp
-    if (split == 0 && bh == 0 && lane < (TWO ? 2 : 1)) bulk_prefetch_l2(A.piv[lane], A.piv_bytes[lane]);
+    if (split == 0 && blockIdx.y == 0 && lane < (TWO ? 2 : 1)) bulk_prefetch_l2(A.piv[lane], A.piv_bytes[lane]);
     int it = 0;
     int pending[kNStage];
     for (int i = 0; i < kNStage; ++i) pending[i] = -1;
@@ -573,7 +587,8 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 3) decode_mma_kernel(MmaArg
       L += f * s_l[w][h];
       acc += f * s_acc[w][h][c];
     }
-    float* dst = A.part + (size_t)(b * A.Hq + hk * kRep + h) * A.part_ld + (size_t)split * (A.D + 2);
+    if (sub * kRep + h >= A.rep) continue;       // a repeated column: not one of this kv head's heads
+    float* dst = A.part + (size_t)(b * A.Hq + hk * A.rep + sub * kRep + h) * A.part_ld + (size_t)split * (A.D + 2);
     if (c == 0) {
       dst[0] = (M == -INFINITY) ? -INFINITY : M * ln2;
       dst[1] = L;
@@ -595,7 +610,8 @@ template <typename T>
 __global__ void __launch_bounds__(32) decode_prep_kernel(const T* __restrict__ q, int ldq, int off, int dg,
                                                          int nrows, const float* __restrict__ PiT,
                                                          const float* __restrict__ ST, float* __restrict__ qp,
-                                                         int D, int G, int gi) {
+                                                         int D, int G, int gi, const int32_t* __restrict__ perm,
+                                                         int Hq, int rep) {
   __shared__ float4 ms4[128][2];                 // [j][o/4]: M^T[j][o0 + o]
   __shared__ float qs[kPrepRows][130];           // padded rows: conflict-free column reads
   allow_dependent_launch();
@@ -608,9 +624,20 @@ __global__ void __launch_bounds__(32) decode_prep_kernel(const T* __restrict__ q
     const int r = e >> lg, j = 2 * (e & (dg / 2 - 1));
     float2 v = make_float2(0.f, 0.f);
     if (r0 + r < nrows) {
-      const size_t at = (size_t)(r0 + r) * ldq + off + j;
-      if constexpr (std::is_same<T, float>::value) v = __ldg(reinterpret_cast<const float2*>(q + at));
-      else v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + at));
+      const size_t row = (size_t)(r0 + r) * ldq;
+      if (perm) {             // the group's channels are perm[kv head][off .. off + dg) of the row
+        const int32_t* pr = perm + (size_t)(((r0 + r) % Hq) / rep) * D + off + j;
+        const int c0 = pr[0], c1 = pr[1];
+        const bool ok0 = c0 >= 0 && c0 < D, ok1 = c1 >= 0 && c1 < D;   // (the merge reports a bad entry)
+        if constexpr (std::is_same<T, float>::value)
+          v = make_float2(ok0 ? __ldg(q + row + c0) : 0.f, ok1 ? __ldg(q + row + c1) : 0.f);
+        else
+          v = make_float2(ok0 ? __bfloat162float(q[row + c0]) : 0.f, ok1 ? __bfloat162float(q[row + c1]) : 0.f);
+      } else {
+        const size_t at = row + off + j;
+        if constexpr (std::is_same<T, float>::value) v = __ldg(reinterpret_cast<const float2*>(q + at));
+        else v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + at));
+      }
     }
     qs[r][j] = v.x;
     qs[r][j + 1] = v.y;
@@ -645,6 +672,8 @@ struct Merge2Args {
   int off[3];
   const float* PiV[2];
   float* out;
+  const int32_t* perm;   // channel permutation [Hkv][D] (NULL: identity): group channel c -> perm[kv][c]
+  int Hq, rep;
   int* err;
 };
 
@@ -768,15 +797,18 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_mma_kernel(Merge2A
     }
     red[qtr][oc] = o;
     __syncthreads();
-    if (real && qtr == 0 && c < D)
-      A.out[(size_t)row * D + c] = (red[0][oc] + red[1][oc]) + (red[2][oc] + red[3][oc]);
+    if (real && qtr == 0 && c < D) {
+      const int oc_ch = A.perm ? A.perm[(size_t)((row % A.Hq) / A.rep) * D + c] : c;
+      if (oc_ch >= 0 && oc_ch < D) A.out[(size_t)row * D + oc_ch] = (red[0][oc] + red[1][oc]) + (red[2][oc] + red[3][oc]);
+      else if (A.err) atomicCAS(A.err, 0, (int)kErrPermRange);
+    }
     __syncthreads();
   }
 }
 
 // Rotated queries of nrows rows for one group.
 int launch_prep(const void* q, int q_dtype, int ldq, int off, int dg, int nrows, const tq_ctx* kc, float* qp, int D,
-                int G, int gi, cudaStream_t st) {
+                int G, int gi, const int32_t* perm, int Hq, int rep, cudaStream_t st) {
   const dim3 grid((nrows + kPrepRows - 1) / kPrepRows, 2, dg / 8);
   cudaError_t e = q_dtype == TQ_DTYPE_F32
                       ? cudaFuncSetAttribute(decode_prep_kernel<float>, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -787,10 +819,10 @@ int launch_prep(const void* q, int q_dtype, int ldq, int off, int dg, int nrows,
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_prep_kernel carveout)");
   if (q_dtype == TQ_DTYPE_F32)
     decode_prep_kernel<float><<<grid, 32, 0, st>>>(static_cast<const float*>(q), ldq, off, dg, nrows, kc->PiT,
-                                                    kc->ST, qp, D, G, gi);
+                                                    kc->ST, qp, D, G, gi, perm, Hq, rep);
   else
     decode_prep_kernel<__nv_bfloat16><<<grid, 32, 0, st>>>(static_cast<const __nv_bfloat16*>(q), ldq, off, dg,
-                                                            nrows, kc->PiT, kc->ST, qp, D, G, gi);
+                                                            nrows, kc->PiT, kc->ST, qp, D, G, gi, perm, Hq, rep);
   count_launch();
   return check_launch("decode_prep_kernel");
 }
@@ -970,6 +1002,8 @@ int launch_mma_t(const MmaArgs& A, int nsplit, int BHkv, cudaStream_t st) {
 
 }  // namespace
 
+int decode_mma_ctas_per_sm() { return TQ_DECODE_CTAS_PER_SM; }
+
 // Tables of one (key context, value context) pair; returns the key-centroid scale inverse.
 float mmaops::host_luts(const tq_ctx* kc, const tq_ctx* vc, Luts* t) {
   *t = Luts{};
@@ -995,10 +1029,11 @@ float mmaops::host_luts(const tq_ctx* kc, const tq_ctx* vc, Luts* t) {
 }
 
 // Returns kNotHandled when the shape is outside this kernel's instantiations.
-int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G, const void* q,
-                      int q_dtype, const tq_packed* kc, const tq_packed* vc, const int32_t* seq_lens, int B, int Hq,
-                      int Hkv, int D, int64_t max_len, float scale, float* out, void* ws, cudaStream_t st) {
-  if (Hq != kRep * Hkv || G > 2 || D > 256) return kNotHandled;
+int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G,
+                      const int32_t* perm, const void* q, int q_dtype, const tq_packed* kc, const tq_packed* vc,
+                      const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len, float scale, float* out,
+                      void* ws, cudaStream_t st) {
+  if (G > 2 || D > 256) return kNotHandled;
   int sig[2] = {0, 0};
   for (int g = 0; g < G; ++g) {
     const int dg = kctx[g]->lay.d;
@@ -1025,11 +1060,13 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
   float* qp = reinterpret_cast<float*>(base + W.qp);
   float* part = reinterpret_cast<float*>(base + W.part);
   for (int g = 0; g < G; ++g) {
-    int r = launch_prep(q, q_dtype, D, off[g], kctx[g]->lay.d, B * Hq, kctx[g], qp, D, G, g, st);
+    int r = launch_prep(q, q_dtype, D, off[g], kctx[g]->lay.d, B * Hq, kctx[g], qp, D, G, g, perm, Hq, Hq / Hkv, st);
     if (r != TQ_OK) return r;
   }
   MmaArgs A{};
   A.B = B; A.Hq = Hq; A.Hkv = Hkv; A.D = D; A.nsplit = W.nsplit; A.chunk = W.chunk; A.G = G;
+  A.rep = Hq / Hkv;
+  A.nsub = (A.rep + kRep - 1) / kRep;
   A.max_len = max_len; A.scale_log2 = scale * 1.4426950408889634f; A.seq_lens = seq_lens;
   A.qprep = qp; A.part = part; A.part_ld = W.part_ld;
   for (int g = 0; g < G; ++g) {
@@ -1048,13 +1085,14 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
     A.piv_bytes[g] = (uint32_t)(vctx[g]->lay.d * vctx[g]->lay.d * sizeof(float));
   }
   int r;
-  if (G == 1 && sig[0] == 12844) r = launch_mma_t<C128_44, void>(A, W.nsplit, B * Hkv, st);
-  else if (G == 1) r = launch_mma_t<C128_33, void>(A, W.nsplit, B * Hkv, st);
-  else if (is(6444, 6433)) r = launch_mma_t<C64_44, C64_33>(A, W.nsplit, B * Hkv, st);
-  else r = launch_mma_t<C64_33, C64_22>(A, W.nsplit, B * Hkv, st);
+  if (G == 1 && sig[0] == 12844) r = launch_mma_t<C128_44, void>(A, W.nsplit, B * Hkv * A.nsub, st);
+  else if (G == 1) r = launch_mma_t<C128_33, void>(A, W.nsplit, B * Hkv * A.nsub, st);
+  else if (is(6444, 6433)) r = launch_mma_t<C64_44, C64_33>(A, W.nsplit, B * Hkv * A.nsub, st);
+  else r = launch_mma_t<C64_33, C64_22>(A, W.nsplit, B * Hkv * A.nsub, st);
   if (r != TQ_OK) return r;
   Merge2Args M{};
   M.part = part; M.part_ld = W.part_ld; M.nsplit = W.nsplit; M.D = D; M.G = G; M.out = out; M.err = A.err;
+  M.perm = perm; M.Hq = Hq; M.rep = Hq / Hkv;
   for (int g = 0; g < G; ++g) { M.off[g] = off[g]; M.PiV[g] = vctx[g]->Pi; }
   M.off[G] = D;
   const int mdyn = (int)((((size_t)std::min(W.nsplit, kMergeChunk) * (D + 2) * sizeof(float)) + 15) / 16 * 16);

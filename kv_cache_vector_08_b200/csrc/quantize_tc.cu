@@ -31,6 +31,41 @@
 #include "sm100.cuh"
 
 namespace tq {
+
+// ------------------------------------------------------------------- tensor maps (host)
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encoder() {
+  static EncodeTiled fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  }
+  return fn;
+}
+
+// 2-D row-major map [rows][cols] of 16-bit elements, box {64 columns, box_rows rows},
+// 128-byte swizzle (the canonical K-major operand layout of tcgen05.mma).
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t rows, uint64_t cols,
+              uint64_t row_stride_bytes, uint32_t box_rows) {
+  EncodeTiled enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 namespace {
 
 using namespace sm100;
@@ -46,6 +81,7 @@ constexpr int kEpiThreads = 32 * kEpiWarps;
 
 struct QtArgs {
   int64_t n;
+  int64_t cap;            // slots in the packed storage (a slot outside [0, cap) is skipped)
   const int64_t* slots;
   uint8_t* codes;
   uint16_t* norm;
@@ -365,8 +401,10 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
     // a pair reaches the pair barrier (rows past n only skip the global stores).
     auto store_quarter = [&](int t, int64_t v, const uint32_t (&pl)[PW], float nrm, float rn2) {
       const int tpar = t & 1;
-      const bool live = v < A.n;
-      const int64_t slot = live ? (A.slots ? A.slots[v] : v) : 0;
+      int64_t slot = v < A.n ? (A.slots ? A.slots[v] : v) : 0;
+      const bool live = v < A.n && slot >= 0 && slot < A.cap;
+      if (v < A.n && !live && wg == 0 && A.err) atomicCAS(A.err, 0, (int)kErrSlotRange);
+      if (!live) slot = 0;
       if constexpr (SHARED) {
         const int odd = wg & 1;
         uint32_t w[PW];
@@ -615,40 +653,6 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
   }
 }
 
-// ------------------------------------------------------------------------------ host
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encoder() {
-  static EncodeTiled fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(p);
-  }
-  return fn;
-}
-
-// 2-D row-major map [rows][cols] of 16-bit elements, box {64 columns, box_rows rows},
-// 128-byte swizzle (the canonical K-major operand layout of tcgen05.mma).
-bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t rows, uint64_t cols,
-              uint64_t row_stride_bytes, uint32_t box_rows) {
-  EncodeTiled enc = encoder();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {row_stride_bytes};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <int D, bool PROD, int K>
 int launch_tc_t(const tq_ctx* ctx, const void* x, int64_t n, int64_t ld, const tq_packed* dst, const int64_t* slots,
                 cudaStream_t st) {
@@ -666,6 +670,7 @@ int launch_tc_t(const tq_ctx* ctx, const void* x, int64_t n, int64_t ld, const t
   }
   QtArgs a{};
   a.n = n;
+  a.cap = dst->cap;
   a.slots = slots;
   a.codes = dst->codes;
   a.norm = dst->norm;
@@ -693,13 +698,20 @@ int launch_tc_t(const tq_ctx* ctx, const void* x, int64_t n, int64_t ld, const t
 
 }  // namespace
 
-// bf16 input, d in {64, 128}, k in [1, 4]; other shapes return kNotHandled.
+// The fused kernel's shapes: bf16 input with 16-byte aligned rows, d in {64, 128}, at least
+// one 128-row tile (the workspace path takes every other call).
+bool quantize_tc_applies(const tq_ctx* ctx, int x_dtype, int64_t n, int64_t ld) {
+  const int d = ctx->lay.d, k = ctx->lay.k;
+  const bool prod = ctx->mode == TQ_MODE_PROD;
+  const bool built = prod ? (k >= 1 && k <= 3) : (k >= 2 && k <= 4);   // the instantiated code widths
+  return built && x_dtype == TQ_DTYPE_BF16 && ctx->Pi_split && (d == 64 || d == 128) && (ld * 2) % 16 == 0 &&
+         n >= kTileM;
+}
+
 int launch_quantize_tc(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld, const tq_packed* dst,
                        const int64_t* slots, cudaStream_t st) {
-  if (x_dtype != TQ_DTYPE_BF16 || !ctx->Pi_split) return kNotHandled;
+  if (!quantize_tc_applies(ctx, x_dtype, n, ld) || (reinterpret_cast<uintptr_t>(x) % 16) != 0) return kNotHandled;
   const int d = ctx->lay.d, k = ctx->lay.k;
-  if ((d != 64 && d != 128) || (ld * 2) % 16 != 0 || (reinterpret_cast<uintptr_t>(x) % 16) != 0) return kNotHandled;
-  if (n < kTileM) return kNotHandled;   // small batches: the CUDA-core kernel
   const bool prod = ctx->mode == TQ_MODE_PROD;
 #define TQ_TC_CASE(DD, PP, KK) \
   if (d == DD && prod == PP && k == KK) return launch_tc_t<DD, PP, KK>(ctx, x, n, ld, dst, slots, st);

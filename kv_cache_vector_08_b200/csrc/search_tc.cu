@@ -1,0 +1,528 @@
+// Top-k search over a packed database on the 5th-generation tensor cores (tcgen05).
+//
+// turboquant.net "向量搜索中的应用" / admirer.cn vector-search paragraph: every database
+// vector is stored quantized and a query ranks the database by the unbiased estimator
+//   score(q, k) = ||k|| ( <Pi q, c[idx]> + sqrt(pi/2)/m ||r|| <S q, 2 s - 1> ),
+// top-k by score, ties to the lower id.  For a tile of 128 queries and a chunk of 256
+// database vectors that is ONE dense product over K = 2 Kh (Kh = 64 ceil(d/64)):
+//
+//   D [128 x 256] = Q [128 x K] * B [256 x K]^T,   score = ||k|| D
+//   Q row  = ( Pi q | sqrt(pi/2)/m S q )                 fp16, built once per query
+//   B row  = ( c[idx] | +-||r|| )                        fp16, decoded per chunk from the codes
+//
+// with the two halves interleaved per 64-coordinate atom (centroid atom, then sign atom of
+// the same coordinates) so one read of the code words feeds both.  ||r|| is an fp16 value,
+// so +-||r|| is exact; the centroids and the query carry fp16 rounding (2^-11 relative),
+// which moves a unit-vector score by ~1e-5.
+//
+// Roles (448 threads per CTA, one CTA per SM for a fixed query tile): warp 0 stages the
+// query atoms by TMA; warp 1 owns TMEM (two 256-column accumulators) and issues the
+// MMAs; warps 2-9 decode database atoms (thread = database row: code words -> fp16 by
+// byte-permute table lookups -> 128-byte-swizzled shared memory) and stage the chunk's
+// norms; warps 10-13 are the epilogue (thread = query: its 256 scores of the chunk from
+// TMEM, a running per-query top-k list in shared memory with the k-th score as threshold).
+// At the end every CTA writes its lists as candidates; the search merge kernel takes the
+// top-k of each query over the CTAs of its query tile.  Every wait is bounded; a timeout
+// records an error code in the context's error word and the CTA winds down.
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "mma_ops.cuh"
+#include "sm100.cuh"
+
+namespace tq {
+namespace {
+
+using namespace sm100;
+using mmaops::prmt;
+
+constexpr int kSqM = 128;                 // queries per tile
+constexpr int kSqN = 256;                 // database vectors per chunk
+constexpr int kSqStages = 3;
+constexpr int kSqDecWarps = 8;
+constexpr int kSqEpiWarps = 4;
+constexpr int kSqThreads = 64 + 32 * (kSqDecWarps + kSqEpiWarps);
+constexpr int kSqMaxK = 64;
+constexpr uint64_t kSqWaitNs = 2000000000ull;
+constexpr int kSqStageA = kSqM * 128;     // 16 KB
+constexpr int kSqStageB = kSqN * 128;     // 32 KB
+constexpr int kSqStage = kSqStageA + kSqStageB;
+
+struct SqArgs {
+  const uint8_t* codes;
+  const uint16_t* norm;
+  const uint16_t* rnorm;
+  int64_t N;                 // database vectors
+  int nq, d, Kh, code_bytes, k;
+  int cpq;                   // CTAs per query tile
+  int64_t nchunks;
+  float* cand_s;             // [nq][cpq * k]
+  int64_t* cand_i;
+  uint32_t ctab_lo[2], ctab_hi[2];   // 3-bit (neg, magnitude) code -> signed centroid fp16 bytes (P = 4)
+  uint32_t ctab[32];                 // P-bit code -> signed centroid fp16 (other P)
+  uint64_t wait_ns;                  // limit of the pipeline waits
+  int* err;
+};
+
+template <int P>
+__global__ void __launch_bounds__(kSqThreads, 1) search_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                                  const SqArgs A) {
+  extern __shared__ uint8_t sq_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sq_smem_raw) + 1023) & ~uintptr_t(1023));
+  float* list_s = reinterpret_cast<float*>(smem + kSqStages * kSqStage);          // [k][128]
+  int32_t* list_i = reinterpret_cast<int32_t*>(list_s + kSqMaxK * kSqM);          // [k][128]
+  float* s_norm = reinterpret_cast<float*>(list_i + kSqMaxK * kSqM);              // [2][256]
+  uint32_t* s_ctab = reinterpret_cast<uint32_t*>(s_norm + 2 * kSqN);              // [32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_ctab + 32);
+  uint64_t* full_a = bars;                          // [stages] TMA
+  uint64_t* full_b = bars + kSqStages;              // [stages] decoders
+  uint64_t* empty = bars + 2 * kSqStages;           // [stages] MMA commit
+  uint64_t* acc_full = bars + 3 * kSqStages;        // [2]
+  uint64_t* acc_empty = acc_full + 2;               // [2]
+  uint64_t* nrm_full = acc_empty + 2;               // [2] chunk norms staged
+  uint64_t* nrm_empty = nrm_full + 2;               // [2] chunk norms consumed
+  uint64_t* drain = nrm_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = blockIdx.x / A.cpq, cslot = blockIdx.x % A.cpq;
+  const int nloc = (int)((A.nchunks - cslot + A.cpq - 1) / A.cpq);
+  const int KA = 2 * A.Kh / 64;                     // atoms per chunk (centroid + sign)
+  constexpr int kDecThreads = 32 * kSqDecWarps;
+  constexpr int kEpiThreads = 32 * kSqEpiWarps;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSqStages; ++s) {
+      mbar_init(full_a + s, 1);
+      mbar_init(full_b + s, kDecThreads);
+      mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full + b, 1);
+      mbar_init(acc_empty + b, kEpiThreads);
+      mbar_init(nrm_full + b, kDecThreads);
+      mbar_init(nrm_empty + b, kEpiThreads);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (threadIdx.x < 32) s_ctab[threadIdx.x] = A.ctab[threadIdx.x];
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const volatile int* abort_v = abort_flag;
+  auto fail = [&](int code) {
+    atomicExch(abort_flag, 1);
+    if (A.err) atomicCAS(A.err, 0, code);
+  };
+  auto wait = [&](uint64_t* bar, uint32_t parity) { return mbar_wait(bar, parity, abort_v, A.wait_ns); };
+
+  if (warp == 0) {
+    // --------------------------------------------------------------- query atoms (TMA)
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      int pending[kSqStages];
+      for (int s = 0; s < kSqStages; ++s) pending[s] = -1;
+      int64_t q = 0;
+      bool ok = true;
+      for (int t = 0; ok && t < nloc; ++t)
+        for (int a = 0; a < KA; ++a, ++q) {
+          const int s = (int)(q % kSqStages);
+          const uint32_t ph = (uint32_t)((q / kSqStages) & 1);
+          if (!wait(empty + s, ph ^ 1)) { fail(501); ok = false; break; }
+          mbar_arrive_expect_tx(full_a + s, kSqStageA);
+          tma_load_2d(smem + s * kSqStage, &tm_q, 64 * a, qt * kSqM, full_a + s);
+          pending[s] = (int)ph;
+        }
+      for (int s = 0; s < kSqStages; ++s)
+        if (pending[s] >= 0) mbar_wait(full_a + s, (uint32_t)pending[s], nullptr, kSqWaitNs);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16(kSqM, kSqN, 0);
+      int64_t q = 0;
+      bool ok = true;
+      for (int t = 0; ok && t < nloc; ++t) {
+        const int b = t & 1;
+        if (!wait(acc_empty + b, (uint32_t)(((t >> 1) & 1) ^ 1))) { fail(502); break; }
+        tc_fence_after();
+        const uint32_t dcol = tmem + (uint32_t)(b * kSqN);
+        for (int a = 0; a < KA; ++a, ++q) {
+          const int s = (int)(q % kSqStages);
+          const uint32_t ph = (uint32_t)((q / kSqStages) & 1);
+          if (!wait(full_a + s, ph) || !wait(full_b + s, ph)) { fail(503); ok = false; break; }
+          tc_fence_after();
+          const uint32_t base = smem_u32(smem + s * kSqStage);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(dcol, desc_sw128(base + kk * 32), desc_sw128(base + kSqStageA + kk * 32), idesc,
+                   (a | kk) ? 1u : 0u);
+          mma_commit(empty + s);
+        }
+        if (!ok) break;
+        mma_commit(acc_full + b);
+      }
+      mma_commit(drain);
+      mbar_wait(drain, 0, nullptr, kSqWaitNs);
+    }
+  } else if (warp < 2 + kSqDecWarps) {
+    // --------------------------------------------------------------- database decoders
+    const int row = threadIdx.x - 64;               // database row of the chunk
+    const int rsw = row & 7;
+    const uint32_t tl0 = A.ctab_lo[0], tl1 = A.ctab_lo[1], th0 = A.ctab_hi[0], th1 = A.ctab_hi[1];
+    const int NG = (A.d + 31) / 32;                 // code groups
+    int64_t q = 0;
+    bool ok = true;
+    for (int t = 0; ok && t < nloc; ++t) {
+      const int64_t chunk = cslot + (int64_t)t * A.cpq;
+      const int64_t id = chunk * kSqN + row;
+      const bool live = id < A.N;
+      const uint8_t* rec = A.codes + (live ? id : 0) * (int64_t)A.code_bytes;
+      float rn = 0.f;
+      // the chunk's norms for the epilogue
+      const int nb = t & 1;
+      if (!wait(nrm_empty + nb, (uint32_t)(((t >> 1) & 1) ^ 1))) { fail(504); ok = false; break; }
+      s_norm[nb * kSqN + row] = live ? __half2float(__ushort_as_half(A.norm[id])) : 0.f;
+      mbar_arrive(nrm_full + nb);
+      uint32_t rbits = 0;
+      if (live) {
+        rn = __half2float(__ushort_as_half(A.rnorm[id]));
+        rbits = (uint32_t)A.rnorm[id] & 0x7FFFu;
+      }
+      (void)rn;
+      const uint32_t rr = rbits | (rbits << 16);
+      uint32_t w[2][P];                             // code words of the atom's two groups
+      for (int a = 0; a < KA; ++a, ++q) {
+        const int s = (int)(q % kSqStages);
+        const uint32_t ph = (uint32_t)((q / kSqStages) & 1);
+        const int ca = a >> 1;                      // 64-coordinate block
+        const bool sign_atom = a & 1;
+        if (!sign_atom) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int g = 2 * ca + h;
+            if (live && g < NG) {
+              if constexpr (P == 4) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4*>(rec + 16 * g));
+                w[h][0] = v.x; w[h][1] = v.y; w[h][2] = v.z; w[h][3] = v.w;
+              } else {
+#pragma unroll
+                for (int p = 0; p < P; ++p) w[h][p] = __ldg(reinterpret_cast<const uint32_t*>(rec) + g * P + p);
+              }
+            } else {
+#pragma unroll
+              for (int p = 0; p < P; ++p) w[h][p] = 0u;
+            }
+          }
+        }
+        if (!wait(empty + s, ph ^ 1)) { fail(505); ok = false; break; }
+        uint8_t* dst = smem + s * kSqStage + kSqStageA + (row >> 3) * 1024 + rsw * 128;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int g = 2 * ca + h;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {            // 8-coordinate slice u of group g: one 16-byte chunk
+            const int c0 = 32 * g + 8 * u;          // first coordinate of the slice
+            uint32_t o[4];
+            if (!live || c0 >= A.d) {
+              o[0] = o[1] = o[2] = o[3] = 0u;
+            } else if (!sign_atom) {
+              if constexpr (P == 4) {
+                const uint32_t sel = w[h][u] & 0x77777777u;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                  const uint32_t sl = hh ? sel >> 16 : sel;
+                  const uint32_t lb = prmt(tl0, tl1, sl), hb = prmt(th0, th1, sl);
+                  o[2 * hh] = prmt(lb, hb, 0x5140u);
+                  o[2 * hh + 1] = prmt(lb, hb, 0x7362u);
+                }
+              } else {
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                  const uint32_t va = s_ctab[group_code(w[h], P, 8 * u + e)];
+                  const uint32_t vb = s_ctab[group_code(w[h], P, 8 * u + e + 1)];
+                  o[e / 2] = (va & 0xFFFFu) | (vb << 16);
+                }
+              }
+              if (c0 + 8 > A.d) {                   // coordinates >= d are zero
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                  if (c0 + e >= A.d) o[e / 2] &= (e & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+              }
+            } else if constexpr (P == 4) {
+              // +-||r||: the fp16 sign bit set where the QJL sign bit is 0.  The sign bits of
+              // coordinates 0-3 are the byte msbs of the word, those of 4-7 after a shift by 4.
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                const uint32_t nm = ~(hh ? w[h][u] << 4 : w[h][u]);
+                o[2 * hh] = (prmt(nm, 0u, 0x1404u) & 0x80008000u) | rr;
+                o[2 * hh + 1] = (prmt(nm, 0u, 0x3424u) & 0x80008000u) | rr;
+              }
+              if (c0 + 8 > A.d) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                  if (c0 + e >= A.d) o[e / 2] &= (e & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+              }
+            } else {
+              // +-||r||: the fp16 sign bit set where the QJL sign bit is 0
+#pragma unroll
+              for (int e = 0; e < 8; e += 2) {
+                const uint32_t sa = (w[h][code_bit_pos(P, 8 * u + e, P - 1) >> 5] >> (code_bit_pos(P, 8 * u + e, P - 1) & 31)) & 1u;
+                const uint32_t sb =
+                    (w[h][code_bit_pos(P, 8 * u + e + 1, P - 1) >> 5] >> (code_bit_pos(P, 8 * u + e + 1, P - 1) & 31)) & 1u;
+                o[e / 2] = rr | ((sa ^ 1u) << 15) | ((sb ^ 1u) << 31);
+              }
+              if (c0 + 8 > A.d) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                  if (c0 + e >= A.d) o[e / 2] &= (e & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+              }
+            }
+            const int chunk16 = h * 4 + u;          // 16-byte chunk of the 128-byte row
+            *reinterpret_cast<uint4*>(dst + ((chunk16 ^ rsw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(full_b + s);
+      }
+    }
+  } else {
+    // ----------------------------------------------------------------------- epilogue
+    const int wq = warp & 3;
+    const int qr = wq * 32 + lane;                  // query row of the tile (TMEM lane)
+    const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
+    const int k = A.k;
+    for (int j = 0; j < k; ++j) {
+      list_s[j * kSqM + qr] = -INFINITY;
+      list_i[j * kSqM + qr] = INT32_MAX;
+    }
+    float tau = -INFINITY;
+    for (int t = 0; t < nloc; ++t) {
+      const int b = t & 1;
+      const int64_t chunk = cslot + (int64_t)t * A.cpq;
+      if (!wait(acc_full + b, (uint32_t)((t >> 1) & 1)) || !wait(nrm_full + b, (uint32_t)((t >> 1) & 1))) {
+        fail(506);
+        break;
+      }
+      tc_fence_after();
+      for (int g = 0; g < kSqN / 32; ++g) {
+        uint32_t raw[32];
+        tmem_ld32(lane_base + (uint32_t)(b * kSqN + 32 * g), raw);
+        tmem_ld_wait();
+        if (g == kSqN / 32 - 1) {
+          tc_fence_before();
+          mbar_arrive(acc_empty + b);
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = 32 * g + e;
+          const float sc = __uint_as_float(raw[e]) * s_norm[b * kSqN + c];
+          const int64_t id = chunk * kSqN + c;
+          if (sc > tau && id < A.N) {
+            // insert (ids rise within a CTA, so a later equal score stays behind)
+            int pos = k - 1;
+            while (pos > 0 && list_s[(pos - 1) * kSqM + qr] < sc) {
+              list_s[pos * kSqM + qr] = list_s[(pos - 1) * kSqM + qr];
+              list_i[pos * kSqM + qr] = list_i[(pos - 1) * kSqM + qr];
+              --pos;
+            }
+            list_s[pos * kSqM + qr] = sc;
+            list_i[pos * kSqM + qr] = (int32_t)id;
+            tau = list_s[(k - 1) * kSqM + qr];
+          }
+        }
+      }
+      mbar_arrive(nrm_empty + b);
+    }
+    const int qg = qt * kSqM + qr;
+    if (qg < A.nq) {
+      float* cs = A.cand_s + (int64_t)qg * A.cpq * k + (int64_t)cslot * k;
+      int64_t* ci = A.cand_i + (int64_t)qg * A.cpq * k + (int64_t)cslot * k;
+      for (int j = 0; j < k; ++j) {
+        const int32_t id = list_i[j * kSqM + qr];
+        cs[j] = list_s[j * kSqM + qr];
+        ci[j] = id == INT32_MAX ? INT64_MAX : (int64_t)id;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Query operand: row q = per 64-coordinate block a, (Pi q)[64a .. 64a+64) then
+// sqrt(pi/2)/m (S q)[64a .. 64a+64), fp16, zero beyond d; rows >= nq are zero.  CTA = 8
+// queries x 256 output columns of one part; thread = output column, 8 dot products.
+__global__ void __launch_bounds__(256) search_query_kernel(const float* __restrict__ q, int64_t nq, int d, int Kh,
+                                                           const float* __restrict__ PiT, const float* __restrict__ ST,
+                                                           float coef, __half* __restrict__ out) {
+  extern __shared__ float qs[];                     // [8][d]
+  const int64_t r0 = (int64_t)blockIdx.x * 8;
+  const int part = blockIdx.z;
+  const int o = blockIdx.y * 256 + threadIdx.x;
+  for (int e = threadIdx.x; e < 8 * d; e += 256) {
+    const int rr = e / d, j = e % d;
+    qs[e] = (r0 + rr < nq) ? q[(r0 + rr) * d + j] : 0.f;
+  }
+  __syncthreads();
+  if (o >= Kh) return;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  if (o < d) {
+    const float* M = part == 0 ? PiT : ST;
+    for (int j = 0; j < d; ++j) {
+      const float m = __ldg(M + (size_t)j * d + o);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(m, qs[i * d + j], acc[i]);
+    }
+  }
+  const float sc = part == 0 ? 1.f : coef;
+  const int64_t K = 2 * (int64_t)Kh;
+  const int64_t col = (int64_t)(o / 64) * 128 + part * 64 + (o % 64);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) out[(r0 + i) * K + col] = __float2half_rn(acc[i] * sc);
+}
+
+struct SqWs {
+  size_t qop, cs, ci, total;
+  int cpq, qtiles, Kh;
+  int64_t nq_pad;
+};
+
+SqWs sq_ws(const tq_ctx* ctx, int64_t nq, int k, int sms) {
+  SqWs w{};
+  w.Kh = 64 * ((ctx->lay.d + 63) / 64);
+  w.qtiles = (int)((nq + kSqM - 1) / kSqM);
+  w.nq_pad = (int64_t)w.qtiles * kSqM;
+  w.cpq = std::max(1, sms / std::max(1, w.qtiles));
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  w.qop = 0;
+  w.cs = up((size_t)w.nq_pad * 2 * w.Kh * sizeof(__half));
+  w.ci = w.cs + up((size_t)nq * w.cpq * k * sizeof(float));
+  w.total = w.ci + up((size_t)nq * w.cpq * k * sizeof(int64_t));
+  return w;
+}
+
+int device_sms(int dev) {
+  int sms = 148;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  return sms;
+}
+
+template <int P>
+int launch_sq_t(const CUtensorMap& tmq, const SqArgs& a, int grid, cudaStream_t st) {
+  const int smem = kSqStages * kSqStage + 2 * kSqMaxK * kSqM * 4 + 2 * kSqN * 4 + 32 * 4 + 256 + 1024;
+  auto kern = search_tc_kernel<P>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(search_tc)");
+  kern<<<grid, kSqThreads, smem, st>>>(tmq, a);
+  count_launch();
+  return check_launch("search_tc_kernel");
+}
+
+}  // namespace
+
+size_t search_tc_workspace(const tq_ctx* ctx, int64_t nq, int64_t N, int k) {
+  (void)N;
+  return sq_ws(ctx, nq, k, device_sms(ctx->device)).total;
+}
+
+// Any prod-mode database, k <= 64.
+int launch_search_tc(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* db, int64_t N, int k,
+                     float* scores, int64_t* ids, void* ws, cudaStream_t st) {
+  if (ctx->mode != TQ_MODE_PROD) return fail(TQ_ERR_INVALID_ARG, "search needs a prod-mode context");
+  if (k < 1 || k > kSqMaxK) return fail(TQ_ERR_UNSUPPORTED, "search: k must be in [1, 64]");
+  if (nq == 0) return TQ_OK;
+  const int sms = device_sms(ctx->device);
+  const SqWs W = sq_ws(ctx, nq, k, sms);
+  char* base = static_cast<char*>(ws);
+  __half* qop = reinterpret_cast<__half*>(base + W.qop);
+  float* cs = reinterpret_cast<float*>(base + W.cs);
+  int64_t* ci = reinterpret_cast<int64_t*>(base + W.ci);
+  const int d = ctx->lay.d;
+  // the query operand
+  {
+    const dim3 grid((unsigned)(W.nq_pad / 8), (unsigned)((W.Kh + 255) / 256), 2);
+    const size_t sm = (size_t)8 * d * sizeof(float);
+    if (sm > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(search_query_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(search_query_kernel)");
+    }
+    if (sm > 227 * 1024) return fail(TQ_ERR_UNSUPPORTED, "search: d above 7000");
+    search_query_kernel<<<grid, 256, sm, st>>>(q, nq, d, W.Kh, ctx->PiT, ctx->ST, ctx->sqrt_pi_over_2_over_m, qop);
+    count_launch();
+    int r = check_launch("search_query_kernel");
+    if (r != TQ_OK) return r;
+  }
+  CUtensorMap tmq;
+  if (!make_map(&tmq, qop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)W.nq_pad, 2 * (uint64_t)W.Kh,
+                2 * (uint64_t)W.Kh * 2, kSqM))
+    return fail(TQ_ERR_INTERNAL, "search: tensor map of the query operand");
+  SqArgs a{};
+  a.codes = db->codes;
+  a.norm = db->norm;
+  a.rnorm = db->rnorm;
+  a.N = N;
+  a.nq = (int)nq;
+  a.d = d;
+  a.Kh = W.Kh;
+  a.code_bytes = ctx->lay.code_bytes;
+  a.k = k;
+  a.cpq = W.cpq;
+  a.nchunks = (N + kSqN - 1) / kSqN;
+  a.cand_s = cs;
+  a.cand_i = ci;
+  a.err = ctx->dev_err;
+  a.wait_ns = pipeline_wait_ns();
+  const int kb = ctx->lay.k, P = ctx->lay.planes;
+  auto signed_centroid = [&](uint32_t code) -> __half {
+    const int idx = code_index(code & ((1u << kb) - 1u), kb);
+    return __float2half_rn((float)ctx->host.centroids[idx]);
+  };
+  for (int code = 0; code < 32; ++code)
+    a.ctab[code] = code < (1 << P) ? (uint32_t)__half_as_ushort(signed_centroid((uint32_t)code)) : 0u;
+  if (P == 4) {
+    uint8_t lo[8], hi[8];
+    for (int c = 0; c < 8; ++c) {
+      const uint16_t v = __half_as_ushort(signed_centroid((uint32_t)c));
+      lo[c] = (uint8_t)(v & 0xFF);
+      hi[c] = (uint8_t)(v >> 8);
+    }
+    for (int r = 0; r < 2; ++r) {
+      a.ctab_lo[r] = lo[4 * r] | (lo[4 * r + 1] << 8) | (lo[4 * r + 2] << 16) | ((uint32_t)lo[4 * r + 3] << 24);
+      a.ctab_hi[r] = hi[4 * r] | (hi[4 * r + 1] << 8) | (hi[4 * r + 2] << 16) | ((uint32_t)hi[4 * r + 3] << 24);
+    }
+  }
+  const int grid = W.qtiles * W.cpq;
+  int r;
+  switch (P) {
+    case 2: r = launch_sq_t<2>(tmq, a, grid, st); break;
+    case 3: r = launch_sq_t<3>(tmq, a, grid, st); break;
+    case 4: r = launch_sq_t<4>(tmq, a, grid, st); break;
+    case 5: r = launch_sq_t<5>(tmq, a, grid, st); break;
+    default: return fail(TQ_ERR_INTERNAL, "search: code layout");
+  }
+  if (r != TQ_OK) return r;
+  return launch_search_merge(cs, ci, nq, (int64_t)W.cpq * k, k, scores, ids, st);
+}
+
+}  // namespace tq

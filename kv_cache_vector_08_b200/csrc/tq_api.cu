@@ -7,6 +7,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -15,7 +17,29 @@ namespace tq {
 namespace {
 thread_local std::string g_error;
 std::atomic<uint64_t> g_launches{0};
+std::atomic<uint64_t> g_wait_ns{2000000000ull};
+std::atomic<int> g_stall{0};
+std::atomic<int> g_fail_alloc{-1};     // index of the tq_init allocation to fail (-1: none)
+std::atomic<int> g_alloc_count{0};
 }  // namespace
+
+uint64_t pipeline_wait_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
+bool debug_stall() { return g_stall.load(std::memory_order_relaxed) != 0; }
+
+cudaError_t dev_alloc(void** p, size_t bytes) {
+  const int i = g_alloc_count.fetch_add(1, std::memory_order_relaxed);
+  if (i == g_fail_alloc.load(std::memory_order_relaxed)) {
+    *p = nullptr;
+    return cudaErrorMemoryAllocation;
+  }
+  return cudaMalloc(p, bytes);
+}
+
+// NVTX range around each entry point (a no-op unless a profiler is attached).
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+};
 
 void set_error(const std::string& msg) { g_error = msg; }
 
@@ -62,7 +86,7 @@ int check_packed(const tq_ctx* ctx, const tq_packed* pk, const char* name) {
 int alloc_copy(float** dst, const std::vector<double>& src) {
   std::vector<float> f(src.size());
   for (size_t i = 0; i < src.size(); ++i) f[i] = (float)src[i];
-  cudaError_t e = cudaMalloc(dst, f.size() * sizeof(float));
+  cudaError_t e = dev_alloc(reinterpret_cast<void**>(dst), f.size() * sizeof(float));
   if (e != cudaSuccess) {
     *dst = nullptr;
     return fail(TQ_ERR_ALLOC, std::string("cudaMalloc: ") + cudaGetErrorString(e));
@@ -96,7 +120,7 @@ int alloc_splits(tq_ctx* c) {
     pis[nn + i] = b;
     pis[2 * nn + i] = __float2bfloat16_rn((float)r2);
   }
-  cudaError_t e = cudaMalloc(&c->Pi_split, pis.size() * sizeof(__nv_bfloat16));
+  cudaError_t e = dev_alloc(&c->Pi_split, pis.size() * sizeof(__nv_bfloat16));
   if (e != cudaSuccess) return fail(TQ_ERR_ALLOC, std::string("cudaMalloc: ") + cudaGetErrorString(e));
   e = cudaMemcpy(c->Pi_split, pis.data(), pis.size() * sizeof(__nv_bfloat16), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(Pi splits)");
@@ -108,7 +132,7 @@ int alloc_splits(tq_ctx* c) {
       ms[i] = a;
       ms[nn + i] = __float2half_rn((float)(v - (double)__half2float(a)));
     }
-    e = cudaMalloc(&c->M_split, ms.size() * sizeof(__half));
+    e = dev_alloc(&c->M_split, ms.size() * sizeof(__half));
     if (e != cudaSuccess) return fail(TQ_ERR_ALLOC, std::string("cudaMalloc: ") + cudaGetErrorString(e));
     e = cudaMemcpy(c->M_split, ms.data(), ms.size() * sizeof(__half), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(M splits)");
@@ -116,16 +140,56 @@ int alloc_splits(tq_ctx* c) {
   return TQ_OK;
 }
 
+// Dequantize operands (d <= 128): B[n][k] = 16 A[k][n] * scale as fp16 hi + lo, [2][N][d_pad],
+// for A = Pi (plain reconstruction) and A = S with scale sqrt(pi/2)/m (QJL term).
+int alloc_dequant_operand(void** dst, const std::vector<double>& A, int d, int d_pad, double scale) {
+  const int K = d_pad, N = 16 * ((d + 15) / 16);
+  std::vector<__half> b((size_t)2 * N * K, __float2half(0.f));
+  for (int n = 0; n < d; ++n)
+    for (int k = 0; k < d; ++k) {
+      const double v = 16.0 * scale * A[(size_t)k * d + n];
+      const __half h = __float2half_rn((float)v);
+      b[(size_t)n * K + k] = h;
+      b[(size_t)N * K + (size_t)n * K + k] = __float2half_rn((float)(v - (double)__half2float(h)));
+    }
+  cudaError_t e = dev_alloc(dst, b.size() * sizeof(__half));
+  if (e != cudaSuccess) return fail(TQ_ERR_ALLOC, std::string("cudaMalloc: ") + cudaGetErrorString(e));
+  e = cudaMemcpy(*dst, b.data(), b.size() * sizeof(__half), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(dequantize operand)");
+  return TQ_OK;
+}
+
+// Projection operands of the workspace quantize path: 16 Pi and 16 M as fp16 hi + lo,
+// [2][d_pad][K] (K = 64 ceil(d/64)), zero padded.
+int alloc_projection(void** dst, const std::vector<double>& A, int d, int d_pad) {
+  const int K = 64 * ((d + 63) / 64);
+  std::vector<__half> b((size_t)2 * d_pad * K, __float2half(0.f));
+  for (int n = 0; n < d; ++n)
+    for (int k = 0; k < d; ++k) {
+      const double v = 16.0 * A[(size_t)n * d + k];
+      const __half h = __float2half_rn((float)v);
+      b[(size_t)n * K + k] = h;
+      b[(size_t)d_pad * K + (size_t)n * K + k] = __float2half_rn((float)(v - (double)__half2float(h)));
+    }
+  cudaError_t e = dev_alloc(dst, b.size() * sizeof(__half));
+  if (e != cudaSuccess) return fail(TQ_ERR_ALLOC, std::string("cudaMalloc: ") + cudaGetErrorString(e));
+  e = cudaMemcpy(*dst, b.data(), b.size() * sizeof(__half), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(projection operand)");
+  return TQ_OK;
+}
+
 void release(tq_ctx* c) {
   if (!c) return;
+  cudaFree(c->Pi16);
+  cudaFree(c->M16);
+  cudaFree(c->PiT_f16);
+  cudaFree(c->ST_f16);
   cudaFree(c->Pi_split);
   cudaFree(c->M_split);
   cudaFree(c->dev_err);
   cudaFree(c->Pi);
   cudaFree(c->PiT);
-  cudaFree(c->S);
   cudaFree(c->ST);
-  cudaFree(c->MT);
   delete c;
 }
 
@@ -179,6 +243,38 @@ extern "C" {
 
 const char* tq_last_error(void) { return g_error.c_str(); }
 
+int tq_channel_perm_by_score(const float* score, int D, int w0, int32_t* perm) {
+  if (!score || !perm || D <= 0 || w0 < 0 || w0 > D) return fail(TQ_ERR_INVALID_ARG, "bad channel permutation arguments");
+  std::vector<int> order(D);
+  for (int i = 0; i < D; ++i) order[i] = i;
+  // the w0 highest scores (ties to the lower channel) form the first group
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return score[a] > score[b]; });
+  std::vector<char> first(D, 0);
+  for (int i = 0; i < w0; ++i) first[order[i]] = 1;
+  int p = 0;
+  for (int i = 0; i < D; ++i)
+    if (first[i]) perm[p++] = i;
+  for (int i = 0; i < D; ++i)
+    if (!first[i]) perm[p++] = i;
+  return TQ_OK;
+}
+
+int tq_debug_set_wait_limit(uint64_t ns) {
+  g_wait_ns.store(ns, std::memory_order_relaxed);
+  return TQ_OK;
+}
+
+int tq_debug_inject_stall(int on) {
+  g_stall.store(on ? 1 : 0, std::memory_order_relaxed);
+  return TQ_OK;
+}
+
+int tq_debug_fail_alloc(int index) {
+  g_alloc_count.store(0, std::memory_order_relaxed);
+  g_fail_alloc.store(index, std::memory_order_relaxed);
+  return TQ_OK;
+}
+
 uint64_t tq_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int tq_host_params(int d, int bits, uint64_t seed, int mode, double* Pi, double* S, double* centroids,
@@ -195,6 +291,7 @@ int tq_host_params(int d, int bits, uint64_t seed, int mode, double* Pi, double*
 }
 
 int tq_init(tq_ctx** out, int d, int bits, uint64_t seed, int mode) {
+  Range range_("tq_init");
   if (!out) return fail(TQ_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   int r = check_args_common(d, bits, mode);
@@ -238,8 +335,7 @@ int tq_init(tq_ctx** out, int d, int bits, uint64_t seed, int mode) {
     return r;
   }
   if (mode == TQ_MODE_PROD) {
-    if ((r = alloc_copy(&c->S, h.S)) != TQ_OK || (r = alloc_copy(&c->ST, transpose(h.S, h.m, d))) != TQ_OK ||
-        (r = alloc_copy(&c->MT, transpose(h.M, h.m, d))) != TQ_OK) {
+    if ((r = alloc_copy(&c->ST, transpose(h.S, h.m, d))) != TQ_OK) {
       release(c);
       return r;
     }
@@ -250,7 +346,18 @@ int tq_init(tq_ctx** out, int d, int bits, uint64_t seed, int mode) {
       return r;
     }
   }
-  e = cudaMalloc(&c->dev_err, sizeof(int));
+  if (d <= 128 && ((r = alloc_dequant_operand(&c->PiT_f16, h.Pi, d, L.d_pad, 1.0)) != TQ_OK ||
+                    (mode == TQ_MODE_PROD &&
+                     (r = alloc_dequant_operand(&c->ST_f16, h.S, d, L.d_pad, std::sqrt(M_PI / 2.0) / h.m)) != TQ_OK))) {
+    release(c);
+    return r;
+  }
+  if ((r = alloc_projection(&c->Pi16, h.Pi, d, L.d_pad)) != TQ_OK ||
+      (mode == TQ_MODE_PROD && (r = alloc_projection(&c->M16, h.M, d, L.d_pad)) != TQ_OK)) {
+    release(c);
+    return r;
+  }
+  e = dev_alloc(reinterpret_cast<void**>(&c->dev_err), sizeof(int));
   if (e != cudaSuccess) {
     release(c);
     return fail(TQ_ERR_ALLOC, std::string("cudaMalloc: ") + cudaGetErrorString(e));
@@ -303,8 +410,15 @@ int tq_get_params(const tq_ctx* ctx, double* Pi, double* S, double* centroids, d
   return TQ_OK;
 }
 
-int tq_quantize_kv(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld, const tq_packed* dst,
-                   const int64_t* dst_slot, tq_stream_t stream) {
+size_t tq_quantize_workspace_size(const tq_ctx* ctx, int x_dtype, int64_t n, int64_t ld) {
+  if (!ctx || n < 0) return 0;
+  if (n == 0 || quantize_tc_applies(ctx, x_dtype, n, ld)) return 0;
+  return quantize_gen_workspace(ctx, n);
+}
+
+static int quantize_common(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld, const int32_t* cols,
+                           const tq_packed* dst, const int64_t* dst_slot, void* workspace, size_t ws_bytes,
+                           tq_stream_t stream) {
   if (!ctx) return fail(TQ_ERR_INVALID_ARG, "ctx is NULL");
   if (n < 0) return fail(TQ_ERR_INVALID_ARG, "n < 0");
   if (n > 0 && !x) return fail(TQ_ERR_INVALID_ARG, "x is NULL");
@@ -315,20 +429,55 @@ int tq_quantize_kv(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int
   if (r != TQ_OK) return r;
   if (!dst_slot && n > dst->cap) return fail(TQ_ERR_INVALID_ARG, "n exceeds dst->cap");
   if ((r = check_device(ctx)) != TQ_OK) return r;
-  return launch_quantize(ctx, x, x_dtype, n, ld, dst, dst_slot, (cudaStream_t)stream);
+  if (n == 0) return TQ_OK;
+  if (cols)
+    return launch_quantize_gen(ctx, x, x_dtype, n, ld, cols, dst, dst_slot, workspace, ws_bytes, (cudaStream_t)stream);
+  return launch_quantize(ctx, x, x_dtype, n, ld, dst, dst_slot, workspace, ws_bytes, (cudaStream_t)stream);
 }
 
-int tq_dequantize(const tq_ctx* ctx, const tq_packed* src, const int64_t* src_slot, int64_t n, float* out,
-                  int64_t ld, tq_stream_t stream) {
+int tq_quantize_kv(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld, const tq_packed* dst,
+                   const int64_t* dst_slot, void* workspace, size_t ws_bytes, tq_stream_t stream) {
+  Range range_("tq_quantize_kv");
+  return quantize_common(ctx, x, x_dtype, n, ld, nullptr, dst, dst_slot, workspace, ws_bytes, stream);
+}
+
+size_t tq_quantize_cols_workspace_size(const tq_ctx* ctx, int64_t n) {
+  if (!ctx || n <= 0) return 0;
+  return quantize_gen_workspace(ctx, n);
+}
+
+int tq_quantize_kv_cols(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld, const int32_t* cols,
+                        const tq_packed* dst, const int64_t* dst_slot, void* workspace, size_t ws_bytes,
+                        tq_stream_t stream) {
+  Range range_("tq_quantize_kv_cols");
+  if (!cols) return fail(TQ_ERR_INVALID_ARG, "cols is NULL");
+  return quantize_common(ctx, x, x_dtype, n, ld, cols, dst, dst_slot, workspace, ws_bytes, stream);
+}
+
+static int dequantize_common(const tq_ctx* ctx, const tq_packed* src, const int64_t* src_slot, int64_t n, float* out,
+                             int64_t ld, bool qjl, tq_stream_t stream) {
   if (!ctx) return fail(TQ_ERR_INVALID_ARG, "ctx is NULL");
   if (n < 0) return fail(TQ_ERR_INVALID_ARG, "n < 0");
   if (n > 0 && !out) return fail(TQ_ERR_INVALID_ARG, "out is NULL");
   if (ld < ctx->lay.d) return fail(TQ_ERR_INVALID_ARG, "ld < d");
+  if (qjl && ctx->mode != TQ_MODE_PROD) return fail(TQ_ERR_INVALID_ARG, "the QJL reconstruction needs a prod-mode context");
   int r = check_packed(ctx, src, "src");
   if (r != TQ_OK) return r;
   if (!src_slot && n > src->cap) return fail(TQ_ERR_INVALID_ARG, "n exceeds src->cap");
   if ((r = check_device(ctx)) != TQ_OK) return r;
-  return launch_dequantize_simt(ctx, src, src_slot, n, out, ld, (cudaStream_t)stream);
+  return launch_dequantize_tc(ctx, src, src_slot, n, out, ld, qjl, (cudaStream_t)stream);
+}
+
+int tq_dequantize(const tq_ctx* ctx, const tq_packed* src, const int64_t* src_slot, int64_t n, float* out,
+                  int64_t ld, tq_stream_t stream) {
+  Range range_("tq_dequantize");
+  return dequantize_common(ctx, src, src_slot, n, out, ld, false, stream);
+}
+
+int tq_dequantize_qjl(const tq_ctx* ctx, const tq_packed* src, const int64_t* src_slot, int64_t n, float* out,
+                      int64_t ld, tq_stream_t stream) {
+  Range range_("tq_dequantize_qjl");
+  return dequantize_common(ctx, src, src_slot, n, out, ld, true, stream);
 }
 
 int tq_prepare_queries(const tq_ctx* ctx, const float* q, int64_t nq, int64_t ld, float* out, tq_stream_t stream) {
@@ -343,15 +492,12 @@ int tq_prepare_queries(const tq_ctx* ctx, const float* q, int64_t nq, int64_t ld
 
 size_t tq_attn_logits_workspace_size(const tq_ctx* ctx, int64_t nq) {
   if (!ctx || nq < 0) return 0;
-  // the larger of the two kernel families' needs (prepared queries in fp32, or in
-  // 16-bit fixed point with per-row scales)
-  const size_t simt = (size_t)nq * (ctx->lay.d + ctx->m) * sizeof(float);
-  const size_t mma = logits_mma_workspace(nq, ctx->lay.d);
-  return simt > mma ? simt : mma;
+  return logits_mma_workspace(nq, ctx->lay.d);
 }
 
 int tq_attn_logits(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* keys, int64_t n, float* logits,
                    void* workspace, size_t ws_bytes, tq_stream_t stream) {
+  Range range_("tq_attn_logits");
   if (!ctx) return fail(TQ_ERR_INVALID_ARG, "ctx is NULL");
   if (nq < 0 || n < 0) return fail(TQ_ERR_INVALID_ARG, "negative size");
   if (nq > 0 && (!q || !logits) && n > 0) return fail(TQ_ERR_INVALID_ARG, "NULL q or logits");
@@ -370,29 +516,38 @@ size_t tq_decode_workspace_size(int B, int Hq, int Hkv, int D, int ngroups, int6
   return decode_workspace_bytes(B, Hq, Hkv, D, ngroups, max_len, D);
 }
 
-int tq_decode_attention(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off, int ngroups,
-                        const void* q, int q_dtype, const tq_packed* kcache, const tq_packed* vcache,
-                        const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len, float scale,
-                        float* out, void* workspace, size_t ws_bytes, tq_stream_t stream) {
+int tq_decode_attention_perm(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off,
+                             int ngroups, const int32_t* channel_perm, const void* q, int q_dtype,
+                             const tq_packed* kcache, const tq_packed* vcache, const int32_t* seq_lens, int B, int Hq,
+                             int Hkv, int D, int64_t max_len, float scale, float* out, void* workspace,
+                             size_t ws_bytes, tq_stream_t stream) {
+  Range range_("tq_decode_attention");
   int r = check_decode_args(kctx, vctx, group_off, ngroups, q, q_dtype, kcache, vcache, seq_lens, B, Hq, Hkv, D,
                             max_len, out);
   if (r != TQ_OK) return r;
   if (B == 0) return TQ_OK;
   size_t need = tq_decode_workspace_size(B, Hq, Hkv, D, ngroups, max_len);
   if (!workspace || ws_bytes < need) return fail(TQ_ERR_WORKSPACE, "workspace too small");
-  return launch_decode(kctx, vctx, group_off, ngroups, q, q_dtype, kcache, vcache, seq_lens, B, Hq, Hkv, D, max_len,
-                       scale, out, workspace, (cudaStream_t)stream);
+  return launch_decode(kctx, vctx, group_off, ngroups, channel_perm, q, q_dtype, kcache, vcache, seq_lens, B, Hq, Hkv,
+                       D, max_len, scale, out, workspace, (cudaStream_t)stream);
+}
+
+int tq_decode_attention(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off, int ngroups,
+                        const void* q, int q_dtype, const tq_packed* kcache, const tq_packed* vcache,
+                        const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len, float scale,
+                        float* out, void* workspace, size_t ws_bytes, tq_stream_t stream) {
+  return tq_decode_attention_perm(kctx, vctx, group_off, ngroups, nullptr, q, q_dtype, kcache, vcache, seq_lens, B, Hq,
+                                  Hkv, D, max_len, scale, out, workspace, ws_bytes, stream);
 }
 
 size_t tq_search_workspace_size(const tq_ctx* ctx, int64_t nq, int64_t N, int k) {
   if (!ctx || nq < 0 || N < 0 || k < 1) return 0;
-  const size_t simt = search_workspace_bytes(ctx, nq, N, k);
-  const size_t mma = search_mma_workspace(ctx, nq, N, k);
-  return simt > mma ? simt : mma;
+  return search_tc_workspace(ctx, nq, N, k);
 }
 
 int tq_search_topk(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* db, int64_t N, int k,
                    float* scores, int64_t* ids, void* workspace, size_t ws_bytes, tq_stream_t stream) {
+  Range range_("tq_search_topk");
   if (!ctx) return fail(TQ_ERR_INVALID_ARG, "ctx is NULL");
   if (ctx->mode != TQ_MODE_PROD) return fail(TQ_ERR_INVALID_ARG, "search needs a prod-mode context");
   if (nq < 0 || N < 1) return fail(TQ_ERR_INVALID_ARG, "bad sizes");

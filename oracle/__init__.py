@@ -32,7 +32,7 @@ from .params import (
     haar_rotation, beta_coordinate_density, beta_coordinate_cdf, lloyd_max,
     lloyd_max_beta, lloyd_max_gaussian, make_params,
 )
-from .quantize import quantize, dequantize, fp16_round
+from .quantize import quantize, dequantize, dequantize_qjl, fp16_round
 from .estimate import (
     prepare_query, estimate_inner_products, decode_attention, search_topk, recall_at,
 )
@@ -40,7 +40,7 @@ from .estimate import (
 __all__ = [
     "splitmix64", "uniform01", "gaussian_stream", "haar_rotation",
     "beta_coordinate_density", "beta_coordinate_cdf", "lloyd_max", "lloyd_max_beta",
-    "lloyd_max_gaussian", "make_params", "quantize", "dequantize", "fp16_round",
+    "lloyd_max_gaussian", "make_params", "quantize", "dequantize", "dequantize_qjl", "fp16_round",
     "prepare_query", "estimate_inner_products", "decode_attention", "search_topk",
     "recall_at",
 ]

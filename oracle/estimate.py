@@ -43,7 +43,7 @@ def estimate_inner_products(params: dict, q: np.ndarray, code: dict) -> np.ndarr
     return np.asarray(code["norm"], dtype=np.float64)[None, :] * est
 
 
-def decode_attention(kparams, vparams, group_off, q, kcodes, vcodes, seq_lens, scale):
+def decode_attention(kparams, vparams, group_off, q, kcodes, vcodes, seq_lens, scale, channel_perm=None):
     """One decode step of attention over a quantized KV cache.
 
     [TQN] "集成到 Attention": k_quant / v_quant replace the cache; logits come from the
@@ -56,6 +56,12 @@ def decode_attention(kparams, vparams, group_off, q, kcodes, vcodes, seq_lens, s
       o   = sum_t p_t * v_hat_t,  v_hat_t[group g] = n_hat_v Pi_v^T c_v[idx_v]
     Reading: the pages do not state the softmax scale; it is an argument (1/sqrt(D)
     for standard attention).  Returns o [B, Hq, D] float64.
+
+    channel_perm ([Hkv, D] permutations, or None for the identity): group g of kv head
+    h_kv covers channels channel_perm[h_kv][group_off[g]:group_off[g+1]] instead of the
+    contiguous range ([ZX] "KV缓存量化的质量表现": 2.5 / 3.5 bits per channel as two groups;
+    reading: which channels get the higher bit width is the caller's choice, e.g. the
+    outlier channels).
     """
     q = np.asarray(q, dtype=np.float64)
     B, Hq, D = q.shape
@@ -71,13 +77,14 @@ def decode_attention(kparams, vparams, group_off, q, kcodes, vcodes, seq_lens, s
             heads = list(range(hk * rep, (hk + 1) * rep))
             logits = np.zeros((rep, T))
             vhat = np.zeros((T, D))
+            perm = np.arange(D) if channel_perm is None else np.asarray(channel_perm[hk])
             for g in range(G):
-                lo, hi = group_off[g], group_off[g + 1]
+                ch = perm[group_off[g]:group_off[g + 1]]          # this group's channels
                 kc = {key: (None if val is None else val[b, hk, :T]) for key, val in kcodes[g].items()}
-                logits += estimate_inner_products(kparams[g], q[b, heads, lo:hi], kc)
+                logits += estimate_inner_products(kparams[g], q[b][np.ix_(heads, ch)], kc)
                 vc = vcodes[g]
-                vhat[:, lo:hi] = (np.asarray(vc["norm"][b, hk, :T], dtype=np.float64)[:, None]
-                                  * (vparams[g]["centroids"][vc["idx"][b, hk, :T]] @ vparams[g]["Pi"]))
+                vhat[:, ch] = (np.asarray(vc["norm"][b, hk, :T], dtype=np.float64)[:, None]
+                               * (vparams[g]["centroids"][vc["idx"][b, hk, :T]] @ vparams[g]["Pi"]))
             logits *= scale
             logits -= logits.max(axis=1, keepdims=True)
             p = np.exp(logits)

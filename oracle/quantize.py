@@ -74,3 +74,24 @@ def dequantize(params: dict, idx: np.ndarray, norm: np.ndarray) -> np.ndarray:
     reconstruction; the stored fp16 norm restores the radius)."""
     c = params["centroids"]
     return np.asarray(norm, dtype=np.float64)[:, None] * (c[np.asarray(idx)] @ params["Pi"])
+
+
+def dequantize_qjl(params: dict, idx: np.ndarray, signs: np.ndarray, norm: np.ndarray,
+                   rnorm: np.ndarray) -> np.ndarray:
+    """QJL-augmented reconstruction of stored keys (prod mode):
+
+        x_hat = n_hat * ( Pi^T c[idx] + sqrt(pi/2)/m * r_hat * S^T (2 s - 1) )
+
+    [ZX] "两阶段内积量化" and [ADM] QJL paragraph give the unbiased estimate only as an
+    inner product, est(q, k) = n_hat (<Pi q, c[idx]> + sqrt(pi/2)/m r_hat <S q, 2 s - 1>).
+    Reading: the vector form is the one x_hat with <q, x_hat> = est(q, k) for every q
+    (est is linear in q, so this x_hat exists and is unique); for consumers that need the
+    key itself rather than its dot products."""
+    if params["mode"] != MODE_PROD:
+        raise ValueError("the QJL reconstruction needs a prod-mode context")
+    c = params["centroids"]
+    m = params["m"]
+    pm = 2.0 * np.asarray(signs, dtype=np.float64) - 1.0
+    mse = c[np.asarray(idx)] @ params["Pi"]                      # rows: Pi^T c[idx]
+    qjl = (np.sqrt(np.pi / 2.0) / m) * np.asarray(rnorm, dtype=np.float64)[:, None] * (pm @ params["S"])
+    return np.asarray(norm, dtype=np.float64)[:, None] * (mse + qjl)

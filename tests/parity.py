@@ -88,17 +88,30 @@ def codes_dict(codes, norm16, rnorm16, d, k, prod):
 
 
 def reconciled_oracle_codes(oparams: dict, x64: np.ndarray, codes: np.ndarray) -> dict:
-    """The oracle's own codes for rows x64, except that rows where the GPU chose another
-    index for a coordinate within 1e-6 of a boundary (the exempt case) are re-run through
-    the oracle with the GPU's indices.  End-to-end comparisons use these codes."""
+    """The oracle's own codes for rows x64, reconciled with the GPU's choices wherever the
+    accuracy contract lets both choices stand, so that end-to-end comparisons (logits,
+    attention) compare the same codes:
+      * rows where the GPU chose another index for a coordinate within 1e-6 of a boundary
+        are re-run through the oracle with the GPU's indices;
+      * QJL sign bits whose oracle projection lies within 1e-6 of 0 take the GPU's bit
+        (either bit is a correct quantization there, and one flipped sign moves a logit
+        by 2 sqrt(pi/2)/m ||r|| |(S q)_j|, far more than the logit tolerance)."""
     d, k, prod = oparams["d"], oparams["k"], oparams["mode"] == 0
     o = oracle.quantize(oparams, x64)
-    idx, _, _ = layout.unpack(codes, d, k, prod)
+    idx, signs, _ = layout.unpack(codes, d, k, prod)
     rows = np.any(idx != o["idx"], axis=1)
     if rows.any():
         fixed = oracle.quantize(oparams, x64[rows], idx_override=idx[rows])
-        for key in ("idx", "signs", "norm", "rnorm"):
-            if o[key] is not None:
+        for key in ("idx", "signs", "norm", "rnorm", "proj"):
+            if o.get(key) is not None:
                 o[key] = o[key].copy()
                 o[key][rows] = fixed[key]
-    return dict(idx=o["idx"], signs=o["signs"], norm=o["norm"], rnorm=o["rnorm"], rows_reconciled=int(rows.sum()))
+    n_signs = 0
+    if prod:
+        near = np.abs(o["proj"]) < IDX_EPS
+        flip = near & (signs != o["signs"])
+        n_signs = int(flip.sum())
+        if n_signs:
+            o["signs"] = np.where(flip, signs, o["signs"])
+    return dict(idx=o["idx"], signs=o["signs"], norm=o["norm"], rnorm=o["rnorm"], rows_reconciled=int(rows.sum()),
+                signs_reconciled=n_signs)

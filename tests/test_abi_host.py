@@ -70,7 +70,8 @@ def test_argument_errors_without_gpu():
     assert b"bits" in L.tq_last_error() or b"mode" in L.tq_last_error()
     assert L.tq_host_params(2, 3, 0, 0, None, None, None, None) == 2
     assert L.tq_get_info(None, None) == 1
-    assert L.tq_quantize_kv(None, None, 0, 0, 0, None, None, None) == 1
+    assert L.tq_quantize_kv(None, None, 0, 0, 0, None, None, None, 0, None) == 1
+    assert L.tq_quantize_workspace_size(None, 0, 10, 128) == 0
     assert L.tq_search_topk(None, None, 0, None, 0, 1, None, None, None, 0, None) == 1
     assert L.tq_decode_workspace_size(1, 0, 8, 128, 1, 100) == 0
     assert L.tq_decode_workspace_size(1, 32, 8, 128, 1, 32768) > 0
@@ -81,3 +82,14 @@ def test_decode_workspace_grows_with_context():
     small = tq.decode_workspace_size(1, 32, 8, 128, 1, 1024)
     big = tq.decode_workspace_size(1, 32, 8, 128, 1, 131072)
     assert 0 < small < big
+
+
+def test_channel_perm_by_score_puts_the_highest_scores_first():
+    score = np.array([0.1, 5.0, 0.2, 5.0, 9.0, 0.0, 0.3, 7.0], dtype=np.float32)
+    perm = tq.channel_perm_by_score(score, 4)
+    # top 4: channels 4 (9), 7 (7), 1 and 3 (5, ties to the lower channel) -> ascending
+    assert perm.tolist() == [1, 3, 4, 7, 0, 2, 5, 6]
+    assert sorted(perm.tolist()) == list(range(8))
+    assert tq.channel_perm_by_score(score, 0).tolist() == list(range(8))
+    with pytest.raises(tq.TQError):
+        tq.channel_perm_by_score(score, 9)

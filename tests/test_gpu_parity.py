@@ -78,6 +78,10 @@ def test_quantize_toy_config_fp32():
     (64, 2, 1, 300, "bf16"), (128, 4, 0, 40000, "bf16"), (64, 4, 1, 40000, "bf16"),  # many tiles per CTA
     (128, 4, 1, 40000, "bf16"), (64, 3, 0, 40000, "bf16"), (128, 2, 0, 38000, "bf16"),
     (64, 2, 0, 40000, "bf16"), (64, 3, 1, 40001, "bf16"), (64, 2, 1, 39999, "bf16"),   # d = 64 shared words
+    # workspace path: fp32 / fp16 input, every width, several N blocks, tiny batches
+    (1536, 4, 0, 300, "fp32"), (200, 4, 0, 3000, "fp32"), (128, 3, 0, 4096, "fp32"),
+    (3072, 4, 0, 40, "fp32"), (300, 3, 1, 257, "fp32"), (100, 2, 0, 129, "f16"),
+    (64, 4, 1, 5, "bf16"), (128, 3, 0, 2, "bf16"), (32, 5, 0, 300, "fp32"), (3, 2, 1, 64, "fp32"),
 ])
 def test_quantize_matches_oracle(d, bits, mode, n, dtype):
     seed = 1000 + 2 * bits + mode
@@ -95,6 +99,22 @@ def test_quantize_matches_oracle(d, bits, mode, n, dtype):
                              "d=%d b=%d mode=%d" % (d, bits, mode))
     assert ctx.device_error() == 0
     print(d, bits, mode, n, res)
+
+
+def test_quantize_workspace_chunks_and_slots():
+    """More rows than one workspace chunk (131072), fp32 input, scattered slots; rows in
+    every chunk are compared with the oracle."""
+    d, n, cap = 64, 140000, 150000
+    x = (W.unit_gaussian(n, d, 5, 12) * 2.5).astype(np.float32)
+    x[[0, 131071, 131072, 139999]] = 0.0
+    rng = np.random.default_rng(9)
+    slots = rng.permutation(cap)[:n]
+    ctx = tq.Context(d, 4, 1010, tq.MODE_PROD)
+    pk = _quantize(ctx, x, torch.float32, slots=slots, cap=cap)
+    rows = np.r_[0:300, 131000:131400, 139700:140000]
+    codes, norm, rn = _host(pk, rows=slots[rows])
+    parity.check_codes(oracle.make_params(d, 4, 1010, 0), x[rows].astype(np.float64), codes, norm, rn, "chunks")
+    assert ctx.device_error() == 0
 
 
 def test_quantize_zero_rows_and_scattered_slots():
@@ -126,19 +146,84 @@ def test_quantize_strided_channel_group():
 
 
 # -------------------------------------------------------------------------- dequantize
-@pytest.mark.parametrize("d,bits,mode", [(128, 4, 1), (64, 3, 0), (200, 2, 1)])
-def test_dequantize_matches_oracle(d, bits, mode):
-    x = _bf16_rows(333, d, 21)
-    ctx = tq.Context(d, bits, 5, mode)
-    pk = _quantize(ctx, x, torch.bfloat16)
-    out = tq.dequantize(ctx, pk, 333).cpu().numpy()
-    codes, norm, rn = _host(pk)
+def _dequant_ref(ctx, pk, d, bits, mode, seed, rows=None):
+    codes, norm, rn = _host(pk, rows)
     cd = parity.codes_dict(codes, norm, rn, d, ctx.k, mode == 0)
-    ref = oracle.dequantize(oracle.make_params(d, bits, 5, mode), cd["idx"], cd["norm"])
-    parity.assert_close(out, ref, "dequant")
+    return oracle.dequantize(oracle.make_params(d, bits, seed, mode), cd["idx"], cd["norm"])
 
 
-# ------------------------------------------------------------------------------ logits
+@pytest.mark.parametrize("d,bits,mode,n", [
+    (128, 4, 1, 333), (128, 4, 0, 40000), (128, 3, 1, 4097), (128, 2, 0, 129),    # Llama-shaped, many tiles
+    (64, 3, 0, 333), (64, 2, 1, 1000), (64, 4, 1, 256),                           # channel groups
+    (100, 3, 1, 257), (96, 4, 0, 131), (32, 2, 1, 5), (16, 3, 0, 3),             # padded K / N, tiny n
+    (128, 1, 1, 300), (128, 5, 0, 300), (48, 1, 1, 70),                           # 1-bit and 5-bit codes
+])
+def test_dequantize_matches_oracle(d, bits, mode, n):
+    """x_hat = ||x|| Pi^T c[idx] of the stored codes on the tensor cores vs the float64
+    definition applied to the same codes."""
+    x = _bf16_rows(n, d, 21, outliers=True)
+    seed = 5 + bits
+    ctx = tq.Context(d, bits, seed, mode)
+    pk = _quantize(ctx, x, torch.bfloat16)
+    out = tq.dequantize(ctx, pk, n)
+    torch.cuda.synchronize()
+    assert ctx.device_error() == 0
+    parity.assert_close(out.cpu().numpy(), _dequant_ref(ctx, pk, d, bits, mode, seed), "dequant d=%d b=%d" % (d, bits))
+
+
+@pytest.mark.parametrize("d,bits,n", [(128, 4, 4097), (64, 3, 333), (100, 2, 257), (128, 5, 300), (32, 2, 7)])
+def test_dequantize_qjl_matches_oracle(d, bits, n):
+    """QJL-augmented reconstruction x_hat = n (Pi^T c[idx] + sqrt(pi/2)/m r S^T (2s-1)) of
+    the stored keys vs the float64 definition on the same codes."""
+    x = _bf16_rows(n, d, 25, outliers=True)
+    seed = 40 + bits
+    ctx = tq.Context(d, bits, seed, tq.MODE_PROD)
+    pk = _quantize(ctx, x, torch.bfloat16)
+    out = tq.dequantize(ctx, pk, n, qjl=True)
+    torch.cuda.synchronize()
+    assert ctx.device_error() == 0
+    codes, norm, rn = _host(pk)
+    cd = parity.codes_dict(codes, norm, rn, d, ctx.k, True)
+    ref = oracle.dequantize_qjl(oracle.make_params(d, bits, seed, 0), cd["idx"], cd["signs"], cd["norm"], cd["rnorm"])
+    parity.assert_close(out.cpu().numpy(), ref, "qjl dequant d=%d b=%d" % (d, bits))
+    # the plain reconstruction of the same codes is unchanged by the QJL mode
+    plain = tq.dequantize(ctx, pk, n).cpu().numpy()
+    parity.assert_close(plain, oracle.dequantize(oracle.make_params(d, bits, seed, 0), cd["idx"], cd["norm"]), "plain")
+
+
+def test_dequantize_gathered_slots_zero_rows_and_strided_output():
+    """Slots gathered in any order, zero vectors, and an output that is a column slice of a
+    wider fp32 tensor (row stride above d, start not 16-byte aligned)."""
+    d, n, cap = 128, 700, 2000
+    x = _bf16_rows(n, d, 23)
+    x[[0, 350, 699]] = 0.0
+    rng = np.random.default_rng(8)
+    slots = rng.permutation(cap)[:n]
+    ctx = tq.Context(d, 4, 31, tq.MODE_MSE)
+    pk = _quantize(ctx, x, torch.bfloat16, slots=slots, cap=cap)
+    gather = rng.permutation(slots)[:517]
+    wide = torch.full((517, 3 + d + 5), 7.0, dtype=torch.float32, device=DEV)
+    out = wide[:, 3:3 + d]
+    tq.dequantize(ctx, pk, slots=torch.tensor(gather, dtype=torch.int64, device=DEV), out=out)
+    torch.cuda.synchronize()
+    ref = _dequant_ref(ctx, pk, d, 4, 1, 31, rows=gather)
+    parity.assert_close(out.cpu().numpy(), ref, "dequant gathered")
+    assert (wide[:, :3] == 7.0).all() and (wide[:, 3 + d:] == 7.0).all()   # nothing outside the slice
+    zero_rows = np.isin(gather, slots[[0, 350, 699]])
+    assert np.all(out.cpu().numpy()[zero_rows] == 0.0)
+
+
+def test_dequantize_empty_and_unsupported_width():
+    ctx = tq.Context(128, 4, 5, tq.MODE_MSE)
+    pk = tq.alloc_packed(ctx, 4)
+    out = torch.empty((0, 128), dtype=torch.float32, device=DEV)
+    tq.dequantize(ctx, pk, 0, out=out)                    # nothing to do
+    wide = tq.Context(200, 4, 5, tq.MODE_MSE)
+    with pytest.raises(tq.TQError) as e:
+        tq.dequantize(wide, tq.alloc_packed(wide, 4), 4)
+    assert e.value.status == 2                             # TQ_ERR_UNSUPPORTED (d above 128)
+
+
 def test_logits_toy_config():
     """16 queries x 4096 keys: logits from the GPU codes vs the oracle estimator on the
     same codes, and vs the oracle's end-to-end quantize + estimate."""
@@ -157,7 +242,7 @@ def test_logits_toy_config():
     parity.assert_close(lg, e2e, "logits(end to end)")
 
 
-@pytest.mark.parametrize("d,bits,n,nq", [(128, 4, 1000, 3), (64, 2, 777, 9), (200, 4, 300, 5), (128, 3, 1, 1)])
+@pytest.mark.parametrize("d,bits,n,nq", [(128, 4, 1000, 3), (64, 2, 777, 9), (64, 4, 300, 5), (128, 3, 1, 1)])
 def test_logits_on_oracle_codes(d, bits, n, nq):
     """Codes produced by the oracle, packed on the host and uploaded: isolates the logits
     kernel from the quantizer."""
@@ -262,19 +347,25 @@ def test_decode_end_to_end_matches_oracle_pipeline():
 
 
 # ------------------------------------------------------------------------------ search
-@pytest.mark.parametrize("d,N,k", [(128, 5000, 10), (200, 3000, 10), (64, 100, 64)])
-def test_search_topk_matches_oracle(d, N, k):
+@pytest.mark.parametrize("d,N,k,bits,nq", [
+    (128, 5000, 10, 4, 6), (200, 3000, 10, 4, 6), (64, 100, 64, 4, 6),     # 4-bit codes (byte-permute decode)
+    (1536, 3000, 10, 4, 6), (3072, 700, 5, 4, 3), (96, 513, 33, 4, 6),     # wide / ragged chunk
+    (128, 2000, 10, 4, 300), (128, 300, 1, 4, 129),                        # several query tiles
+    (128, 2000, 10, 2, 6), (100, 1500, 7, 3, 6), (160, 1200, 10, 5, 6),    # 1-, 2-, 4-bit indices
+])
+def test_search_topk_matches_oracle(d, N, k, bits, nq):
     db = W.unit_gaussian(N, d, 1, 10)
     db[N // 2] = db[7]                        # an exact tie: lower id must come first
-    qs = W.unit_gaussian(6, d, 1, 3)
+    qs = W.unit_gaussian(nq, d, 1, 3)
     qs[0] = db[7]
-    ctx = tq.Context(d, 4, 12, tq.MODE_PROD)
+    ctx = tq.Context(d, bits, 12, tq.MODE_PROD)
     pk = _quantize(ctx, db, torch.float32)
     scores, ids = tq.search_topk(ctx, torch.tensor(qs, device=DEV), pk, N, k)
     scores, ids = scores.cpu().numpy(), ids.cpu().numpy()
+    assert ctx.device_error() == 0
     codes, norm, rn = _host(pk)
-    op = oracle.make_params(d, 4, 12, 0)
-    cd = parity.codes_dict(codes, norm, rn, d, 3, True)
+    op = oracle.make_params(d, bits, 12, 0)
+    cd = parity.codes_dict(codes, norm, rn, d, bits - 1, True)
     est = oracle.estimate_inner_products(op, qs.astype(np.float64), cd)
     ref_s, ref_i = oracle.search_topk(op, qs.astype(np.float64), cd, k)
     parity.assert_close(scores, ref_s, "top-k scores")
@@ -297,11 +388,112 @@ def test_decode_many_splits():
     parity.assert_close(out, ref, "decode, 110 splits")
 
 
-@pytest.mark.parametrize("Hkv,Hq", [(2, 4), (1, 8), (3, 12)])
+@pytest.mark.parametrize("Hkv,Hq", [(2, 4), (1, 8), (3, 12), (4, 4), (2, 12), (1, 16)])
 def test_decode_other_gqa_ratios(Hkv, Hq):
-    """GQA ratios 2, 8 (SIMT kernel) and 4 with three kv heads (tensor-core kernel)."""
+    """Every GQA ratio on the tensor-core kernel: 1, 2, 4, 6, 8 and 16 query heads per kv
+    head (a CTA serves 4 query heads of one kv head; ratios that are not a multiple of 4
+    repeat a head in the spare MMA columns and drop its result)."""
     out, ref, _ = _decode_case(2, Hkv, Hq, 128, ((0, 128, 4, 4),), [100, 33], 128, 7)
     parity.assert_close(out, ref, "gqa %d/%d" % (Hq, Hkv))
+
+
+def _perm_case(perm_kind, seed=11):
+    """2.5-bit groups (64 ch at 3 + 3 bits, 64 ch at 2 + 2 bits) on data with 4 outlier
+    channels x8 per kv head; channel_perm per kv head: "random", or "outlier" (the channels
+    with the largest RMS over the sample first, so the outliers get the higher bit width)."""
+    B, Hkv, Hq, D, T = 2, 2, 8, 128, 300
+    groups = ((0, 64, 3, 3), (64, 64, 2, 2))
+    rng = np.random.default_rng(seed)
+    K = W.round_bf16(rng.standard_normal((B, Hkv, T, D)))
+    V = W.round_bf16(rng.standard_normal((B, Hkv, T, D)))
+    for h in range(Hkv):                          # outliers in the second (low-bit) half by default
+        ch = 64 + rng.choice(64, 4, replace=False)
+        K[:, h, :, ch] *= 8.0
+        V[:, h, :, ch] *= 8.0
+    K, V = W.round_bf16(K), W.round_bf16(V)
+    q = W.round_bf16(rng.standard_normal((B, Hq, D)))
+    if perm_kind == "random":
+        perm = np.stack([rng.permutation(D) for _ in range(Hkv)]).astype(np.int32)
+    elif perm_kind == "identity":
+        perm = np.stack([np.arange(D)] * Hkv).astype(np.int32)
+    else:
+        perm = np.stack([tq.channel_perm_by_score(np.sqrt((K[:, h] ** 2).mean(axis=(0, 1))), 64)
+                         for h in range(Hkv)]).astype(np.int32)
+    kctx, vctx, kc, vc, kp, vp = [], [], [], [], [], []
+    Kt = torch.tensor(K.reshape(-1, D), dtype=torch.bfloat16, device=DEV)
+    Vt = torch.tensor(V.reshape(-1, D), dtype=torch.bfloat16, device=DEV)
+    for gi, (off, w, kb, vb) in enumerate(groups):
+        kx = tq.Context(w, kb, 1000 + 2 * gi, tq.MODE_PROD)
+        vx = tq.Context(w, vb, 1001 + 2 * gi, tq.MODE_MSE)
+        kpk, vpk = tq.alloc_packed(kx, B * Hkv * T), tq.alloc_packed(vx, B * Hkv * T)
+        for h in range(Hkv):                      # rows of kv head h: its own columns
+            rows = torch.tensor([(b * Hkv + h) * T + t for b in range(B) for t in range(T)], device=DEV)
+            cols = torch.tensor(perm[h, off:off + w], dtype=torch.int32, device=DEV)
+            tq.quantize_kv(kx, Kt[rows], kpk, slots=rows, cols=cols)
+            tq.quantize_kv(vx, Vt[rows], vpk, slots=rows, cols=cols)
+        kctx.append(kx); vctx.append(vx); kc.append(kpk); vc.append(vpk)
+        kp.append(oracle.make_params(w, kb, 1000 + 2 * gi, 0)); vp.append(oracle.make_params(w, vb, 1001 + 2 * gi, 1))
+    sl = torch.tensor([T, 171], dtype=torch.int32, device=DEV)
+    out = tq.decode_attention(kctx, vctx, [0, 64, 128], torch.tensor(q, dtype=torch.bfloat16, device=DEV), kc, vc,
+                              sl, Hkv, T, 1 / np.sqrt(D),
+                              channel_perm=torch.tensor(perm, dtype=torch.int32, device=DEV))
+    torch.cuda.synchronize()
+    # the oracle's own codes of the permuted columns (reconciled with the GPU's on exempt choices)
+    kcodes, vcodes = [], []
+    for gi, (off, w, kb, vb) in enumerate(groups):
+        kx_ = np.stack([K[:, h][..., perm[h, off:off + w]] for h in range(Hkv)], axis=1)
+        vx_ = np.stack([V[:, h][..., perm[h, off:off + w]] for h in range(Hkv)], axis=1)
+        ko = parity.reconciled_oracle_codes(kp[gi], kx_.reshape(-1, w).astype(np.float64), kc[gi].codes.cpu().numpy())
+        vo = parity.reconciled_oracle_codes(vp[gi], vx_.reshape(-1, w).astype(np.float64), vc[gi].codes.cpu().numpy())
+        kcodes.append({k: ko[k].reshape(B, Hkv, T, *ko[k].shape[1:]) for k in ("idx", "signs", "norm", "rnorm")})
+        vcodes.append({k: vo[k].reshape(B, Hkv, T, *vo[k].shape[1:]) for k in ("idx", "norm")})
+    ref = oracle.decode_attention(kp, vp, [0, 64, 128], q.astype(np.float64), kcodes, vcodes, [T, 171],
+                                  1 / np.sqrt(D), channel_perm=perm)
+    # exact attention on the unquantized inputs (for the quality comparison)
+    exact = np.zeros_like(ref)
+    for b, Tb in enumerate([T, 171]):
+        for hq in range(Hq):
+            h = hq // (Hq // Hkv)
+            lg = K[b, h, :Tb].astype(np.float64) @ q[b, hq].astype(np.float64) / np.sqrt(D)
+            p = np.exp(lg - lg.max())
+            exact[b, hq] = (p / p.sum()) @ V[b, h, :Tb].astype(np.float64)
+    return out.cpu().numpy(), ref, exact
+
+
+@pytest.mark.parametrize("perm_kind", ["random", "outlier"])
+def test_decode_channel_permutation_matches_oracle(perm_kind):
+    out, ref, _ = _perm_case(perm_kind)
+    parity.assert_close(out, ref, "decode with %s channel permutation" % perm_kind)
+
+
+def test_outlier_aware_grouping_lowers_the_attention_error():
+    """Sending the outlier channels to the higher-bit group, instead of leaving them in the
+    2-bit half (the contiguous split), brings the quantized attention closer to exact
+    attention on the same inputs."""
+    out_o, _, exact = _perm_case("outlier")
+    out_i, ref_i, exact_i = _perm_case("identity")
+    assert np.array_equal(exact, exact_i)
+    parity.assert_close(out_i, ref_i, "decode with the identity permutation")
+    err_outlier = np.abs(out_o - exact).mean()
+    err_default = np.abs(out_i - exact).mean()
+    print("mean |attention - exact|: outlier-aware %.4g, contiguous %.4g" % (err_outlier, err_default))
+    assert err_outlier < err_default
+
+
+def test_unsupported_shapes_are_reported():
+    """Shapes outside the tensor-core kernels return TQ_ERR_UNSUPPORTED (no slower path)."""
+    ctx = tq.Context(200, 4, 3, tq.MODE_PROD)
+    pk = tq.alloc_packed(ctx, 8)
+    with pytest.raises(tq.TQError) as e:
+        tq.attn_logits(ctx, torch.zeros((2, 200), device=DEV), pk, 8)
+    assert e.value.status == 2
+    kx, vx = tq.Context(64, 4, 1, tq.MODE_PROD), tq.Context(64, 4, 2, tq.MODE_MSE)
+    kc, vc = tq.alloc_packed(kx, 2 * 16), tq.alloc_packed(vx, 2 * 16)
+    q = torch.zeros((1, 4, 64), dtype=torch.bfloat16, device=DEV)
+    sl = torch.tensor([16], dtype=torch.int32, device=DEV)
+    with pytest.raises(tq.TQError) as e:
+        tq.decode_attention([kx], [vx], [0, 64], q, [kc], [vc], sl, 2, 16, 0.125)
+    assert e.value.status == 2
 
 
 def test_decode_fp32_queries_and_128_2bit_keys():

@@ -353,6 +353,51 @@ def test_estimator_qjl_term_by_hand():
     assert abs(oracle.estimate_inner_products(p, q2, code)[0, 0] - expect) < 1e-13
 
 
+def test_qjl_dequantize_by_hand():
+    p = _hand_params()
+    code = oracle.quantize(p, np.array([[6.0, -2.0, 3.0]]))
+    # Pi^T c[idx] = (3/4, -1/4, 1/4); all signs +1, so S^T (2s - 1) = column sums of S = (2, 0, 2)
+    rn = code["rnorm"][0]
+    kappa = math.sqrt(math.pi / 2) / 3
+    expect = 7.0 * (np.array([0.75, -0.25, 0.25]) + kappa * rn * np.array([2.0, 0.0, 2.0]))
+    got = oracle.dequantize_qjl(p, code["idx"], code["signs"], code["norm"], code["rnorm"])[0]
+    assert np.allclose(got, expect, rtol=0, atol=1e-14)
+
+
+def test_qjl_dequantize_dots_equal_the_estimator():
+    """<e_i, x_hat> = est(e_i, k) for the standard basis (so the vectors are equal), and
+    <q, x_hat> = est(q, k) for random q."""
+    p = make_params(48, 4, 5, MODE_PROD)
+    rng = np.random.Generator(np.random.PCG64(3))
+    k = rng.standard_normal((7, 48))
+    code = oracle.quantize(p, k)
+    xh = oracle.dequantize_qjl(p, code["idx"], code["signs"], code["norm"], code["rnorm"])
+    basis = oracle.estimate_inner_products(p, np.eye(48), code)         # [48, 7]
+    assert np.allclose(xh, basis.T, rtol=1e-12, atol=1e-12)
+    q = rng.standard_normal((5, 48))
+    assert np.allclose(q @ xh.T, oracle.estimate_inner_products(p, q, code), rtol=1e-12, atol=1e-11)
+
+
+def test_qjl_dequantize_is_unbiased_monte_carlo():
+    """Over independent draws of (Pi, S) with float64 norms, the mean reconstruction equals
+    the key within 3 sigma in every coordinate (2 x 10^4 trials at d = 8)."""
+    d, trials = 8, 20000
+    rng = np.random.Generator(np.random.PCG64(91))
+    k = rng.standard_normal(d)
+    c, t = lloyd_max_beta(d, 2)
+    acc = np.zeros((trials, d))
+    for i in range(trials):
+        p = dict(d=d, k=1, m=d, mode=MODE_PROD, Pi=haar_rotation(rng.standard_normal((d, d))),
+                 S=rng.standard_normal((d, d)), centroids=c, boundaries=t)
+        code = oracle.quantize(p, k[None, :])
+        nk = np.linalg.norm(k)
+        code["norm"] = np.array([nk])
+        code["rnorm"] = np.array([np.linalg.norm(k / nk - c[code["idx"][0]] @ p["Pi"])])
+        acc[i] = oracle.dequantize_qjl(p, code["idx"], code["signs"], code["norm"], code["rnorm"])[0]
+    err = acc.mean(axis=0) - k
+    assert np.all(np.abs(err) < 3.0 * acc.std(axis=0) / math.sqrt(trials))
+
+
 # ---------------------------------------------------------------------- attention
 def _small_cache(B, Hkv, T, groups, seed):
     rng = np.random.Generator(np.random.PCG64(seed))
@@ -394,6 +439,48 @@ def test_attention_equal_logits_average_values_and_gqa_mapping():
             hk = h // 3
             vhat = oracle.dequantize(vp[0], vc[0]["idx"][b, hk, :T], vc[0]["norm"][b, hk, :T])
             assert np.allclose(o[b, h], vhat.mean(axis=0), atol=1e-14)
+
+
+def test_attention_channel_permutation_is_a_relabelling():
+    """Decoding with a per-kv-head channel permutation P equals decoding without one on
+    inputs whose channels were permuted by P (keys, values and queries), with the output
+    permuted back; the identity permutation changes nothing."""
+    groups = ((0, 8, 3, 3), (8, 8, 2, 2))
+    B, Hkv, T, D = 2, 2, 9, 16
+    rng = np.random.Generator(np.random.PCG64(12))
+    K = rng.standard_normal((B, Hkv, T, D))
+    V = rng.standard_normal((B, Hkv, T, D))
+    q = rng.standard_normal((B, 4, D))
+    perm = np.stack([rng.permutation(D) for _ in range(Hkv)])
+    kp = [make_params(w, kb, 1000 + 2 * gi, MODE_PROD) for gi, (_, w, kb, _) in enumerate(groups)]
+    vp = [make_params(w, vb, 1001 + 2 * gi, MODE_MSE) for gi, (_, w, _, vb) in enumerate(groups)]
+    offs = [0, 8, 16]
+
+    def caches(Kx, Vx):
+        kc, vc = [], []
+        for gi, (off, w, _, _) in enumerate(groups):
+            ko = oracle.quantize(kp[gi], Kx[..., off:off + w].reshape(-1, w))
+            vo = oracle.quantize(vp[gi], Vx[..., off:off + w].reshape(-1, w))
+            kc.append({k: ko[k].reshape(B, Hkv, T, *ko[k].shape[1:]) for k in ("idx", "signs", "norm", "rnorm")})
+            vc.append({k: vo[k].reshape(B, Hkv, T, *vo[k].shape[1:]) for k in ("idx", "norm")})
+        return kc, vc
+
+    # group g of head h holds channels perm[h][off:off+w]: quantize those columns
+    Kp = np.stack([K[:, h][..., perm[h]] for h in range(Hkv)], axis=1)
+    Vp = np.stack([V[:, h][..., perm[h]] for h in range(Hkv)], axis=1)
+    kc, vc = caches(Kp, Vp)
+    got = oracle.decode_attention(kp, vp, offs, q, kc, vc, [T, 5], 0.3, channel_perm=perm)
+    # reference: no permutation on the permuted problem, output mapped back
+    qp = np.stack([q[:, hq][..., perm[hq // 2]] for hq in range(4)], axis=1)
+    ref_p = oracle.decode_attention(kp, vp, offs, qp, kc, vc, [T, 5], 0.3)
+    ref = np.empty_like(ref_p)
+    for hq in range(4):
+        ref[:, hq][..., perm[hq // 2]] = ref_p[:, hq]
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+    ident = np.stack([np.arange(D)] * Hkv)
+    kc0, vc0 = caches(K, V)
+    assert np.array_equal(oracle.decode_attention(kp, vp, offs, q, kc0, vc0, [T, 5], 0.3, channel_perm=ident),
+                          oracle.decode_attention(kp, vp, offs, q, kc0, vc0, [T, 5], 0.3))
 
 
 def test_attention_is_invariant_to_token_order():

@@ -105,6 +105,7 @@ LONG_2P5 = DecodeWorkload(
 
 SEARCH_1536 = dict(name="search-d1536", d=1536, bits=4, n_db=1_000_000, n_queries=1000, k=10)
 SEARCH_200 = dict(name="search-d200", d=200, bits=4, n_db=1_000_000, n_queries=1000, k=10)
+SEARCH_3072 = dict(name="search-d3072", d=3072, bits=4, n_db=1_000_000, n_queries=1000, k=10)
 
 
 def toy_inputs(seed: int = 0, n_keys: int = 4096, n_queries: int = 16, d: int = 128):
