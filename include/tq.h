@@ -251,21 +251,38 @@ int tq_decode_attention(const tq_ctx* const* kctx, const tq_ctx* const* vctx, co
                         int D, int64_t max_len, float scale, float* out, void* workspace,
                         size_t ws_bytes, tq_stream_t stream);
 
-/* tq_decode_attention_perm -- tq_decode_attention with the head dimension's channels
- * regrouped per kv head: channel group g of kv head hk covers channels
- * channel_perm[hk*D + group_off[g]] .. channel_perm[hk*D + group_off[g+1] - 1] of q, K, V and
- * out (the keys and values must have been quantized with the same columns, e.g. by
- * tq_quantize_kv_cols).  This is how outlier channels are sent to the higher-bit group of a
- * 2.5 / 3.5-bit split ([ZX] "KV缓存量化的质量表现": 2.5 and 3.5 bits per channel;
- * turboquant.net "潜在挑战与解决方案": outlier handling).  channel_perm: device int32
- * [Hkv][D], each row a permutation of 0..D-1, or NULL for the identity (then identical to
- * tq_decode_attention).  An entry outside [0, D) is skipped and reported as device error 902.
- * Other arguments, layout and errors as tq_decode_attention. */
-int tq_decode_attention_perm(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off,
-                             int ngroups, const int32_t* channel_perm, const void* q, int q_dtype,
-                             const tq_packed* kcache, const tq_packed* vcache, const int32_t* seq_lens, int B,
-                             int Hq, int Hkv, int D, int64_t max_len, float scale, float* out, void* workspace,
-                             size_t ws_bytes, tq_stream_t stream);
+/* Options of tq_decode_attention_ex (zero / NULL fields keep the defaults).
+ * channel_perm -- device int32 [Hkv][D], each row a permutation of 0..D-1: channel group g
+ *   of kv head hk covers channels channel_perm[hk*D + group_off[g]] ..
+ *   channel_perm[hk*D + group_off[g+1] - 1] of q, K, V and out (the keys and values must
+ *   have been quantized with the same columns, e.g. by tq_quantize_kv_cols).  This is how
+ *   outlier channels are sent to the higher-bit group of a 2.5 / 3.5-bit split ([ZX]
+ *   "KV缓存量化的质量表现": 2.5 and 3.5 bits per channel; turboquant.net "潜在挑战与解决方案":
+ *   outlier handling).  NULL: the identity.  An entry outside [0, D) is skipped and
+ *   reported as device error 902.
+ * block_table, page_tokens -- paged caches ([TQN] "集成到 Attention": the quantized cache
+ *   replaces the KV storage of a serving engine; the paging itself is not on the pages):
+ *   block_table is device int32 [B][max_len / page_tokens]; token t of sequence b lives in
+ *   physical page p = block_table[b][t / page_tokens], and page p of a cache holds kv head
+ *   hk's tokens in slots (p*Hkv + hk)*page_tokens .. + page_tokens - 1 (so every cache's
+ *   capacity is a whole number of pages of Hkv*page_tokens slots).  page_tokens must be a
+ *   positive multiple of 64 dividing max_len.  A page index outside the caches reads page 0
+ *   and is reported as device error 901.  NULL: the contiguous layout of
+ *   tq_decode_attention. */
+typedef struct tq_decode_opts {
+  const int32_t* channel_perm;
+  const int32_t* block_table;
+  int page_tokens;
+} tq_decode_opts;
+
+/* tq_decode_attention_ex -- tq_decode_attention with options (opts may be NULL).  Other
+ * arguments, layout and errors as tq_decode_attention, except that a paged call only needs
+ * caches of at least one page; TQ_ERR_INVALID_ARG for a bad page_tokens. */
+int tq_decode_attention_ex(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off,
+                           int ngroups, const void* q, int q_dtype, const tq_packed* kcache,
+                           const tq_packed* vcache, const int32_t* seq_lens, int B, int Hq, int Hkv, int D,
+                           int64_t max_len, float scale, float* out, const tq_decode_opts* opts,
+                           void* workspace, size_t ws_bytes, tq_stream_t stream);
 
 /* tq_channel_perm_by_score -- host helper for the outlier-aware channel grouping: perm (host
  * int32 [D]) lists the w0 channels with the highest score (ties to the lower channel) in

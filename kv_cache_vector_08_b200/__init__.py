@@ -39,6 +39,10 @@ class _Packed(ctypes.Structure):
                 ("cap", ctypes.c_int64)]
 
 
+class _DecodeOpts(ctypes.Structure):
+    _fields_ = [("channel_perm", ctypes.c_void_p), ("block_table", ctypes.c_void_p), ("page_tokens", ctypes.c_int)]
+
+
 class _Info(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int), ("bits", ctypes.c_int), ("k", ctypes.c_int), ("m", ctypes.c_int),
                 ("mode", ctypes.c_int), ("planes", ctypes.c_int), ("d_pad", ctypes.c_int),
@@ -75,7 +79,8 @@ def lib():
         "tq_attn_logits": (I, [P, P, I64, PK, I64, P, P, SZ, P]),
         "tq_decode_workspace_size": (SZ, [I, I, I, I, I, I64]),
         "tq_decode_attention": (I, [P, P, P, I, P, I, PK, PK, P, I, I, I, I, I64, F, P, P, SZ, P]),
-        "tq_decode_attention_perm": (I, [P, P, P, I, P, P, I, PK, PK, P, I, I, I, I, I64, F, P, P, SZ, P]),
+        "tq_decode_attention_ex": (I, [P, P, P, I, P, I, PK, PK, P, I, I, I, I, I64, F, P, ctypes.POINTER(_DecodeOpts),
+                                       P, SZ, P]),
         "tq_channel_perm_by_score": (I, [P, I, I, P]),
         "tq_quantize_cols_workspace_size": (SZ, [P, I64]),
         "tq_quantize_kv_cols": (I, [P, P, I, I64, I64, P, PK, P, P, SZ, P]),
@@ -304,9 +309,14 @@ class DecodePlan:
 
     def __init__(self, kctx: Sequence[Context], vctx: Sequence[Context], group_off: Sequence[int],
                  kcache: Sequence[Packed], vcache: Sequence[Packed], B, Hq, Hkv, D, max_len, device=None,
-                 channel_perm=None):
+                 channel_perm=None, block_table=None, page_tokens: int = 0):
         torch = _torch()
-        self.channel_perm = channel_perm       # CUDA int32 [Hkv, D] or None
+        # options: channel_perm CUDA int32 [Hkv, D]; block_table CUDA int32 [B, max_len / page_tokens]
+        self._opts = None
+        if channel_perm is not None or block_table is not None:
+            self._opts = _DecodeOpts(0 if channel_perm is None else channel_perm.data_ptr(),
+                                     0 if block_table is None else block_table.data_ptr(), int(page_tokens))
+            self._keep_opts = (channel_perm, block_table)
         G = len(kctx)
         self.G, self.B, self.Hq, self.Hkv, self.D, self.max_len = G, B, Hq, Hkv, D, max_len
         self._k = (ctypes.c_void_p * G)(*[c.handle.value for c in kctx])
@@ -320,12 +330,11 @@ class DecodePlan:
         self.workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
 
     def __call__(self, q, seq_lens, scale: float, out, stream=None):
-        if self.channel_perm is not None:
-            _check(lib().tq_decode_attention_perm(self._k, self._v, self._off, self.G, _ptr(self.channel_perm), _ptr(q),
-                                                  _dtype_code(q), self._kc, self._vc, _ptr(seq_lens), self.B,
-                                                  self.Hq, self.Hkv, self.D, self.max_len, ctypes.c_float(scale),
-                                                  _ptr(out), _ptr(self.workspace), self.workspace.numel(),
-                                                  _stream(stream)))
+        if self._opts is not None:
+            _check(lib().tq_decode_attention_ex(self._k, self._v, self._off, self.G, _ptr(q), _dtype_code(q), self._kc,
+                                                self._vc, _ptr(seq_lens), self.B, self.Hq, self.Hkv, self.D,
+                                                self.max_len, ctypes.c_float(scale), _ptr(out), ctypes.byref(self._opts),
+                                                _ptr(self.workspace), self.workspace.numel(), _stream(stream)))
             return out
         _check(lib().tq_decode_attention(self._k, self._v, self._off, self.G, _ptr(q), _dtype_code(q), self._kc,
                                          self._vc, _ptr(seq_lens), self.B, self.Hq, self.Hkv, self.D,
@@ -335,13 +344,13 @@ class DecodePlan:
 
 
 def decode_attention(kctx, vctx, group_off, q, kcache, vcache, seq_lens, Hkv, max_len, scale, out=None,
-                     stream=None, channel_perm=None):
+                     stream=None, channel_perm=None, block_table=None, page_tokens=0):
     """One decode step; q [B, Hq, D] (fp32/bf16 CUDA), seq_lens int32 CUDA [B] -> out fp32 [B, Hq, D].
     Token t of sequence b, kv head h lives in slot (b*Hkv + h)*max_len + t of each cache."""
     torch = _torch()
     B, Hq, D = q.shape
     plan = DecodePlan(kctx, vctx, group_off, kcache, vcache, B, Hq, Hkv, D, max_len, device=q.device,
-                      channel_perm=channel_perm)
+                      channel_perm=channel_perm, block_table=block_table, page_tokens=page_tokens)
     if out is None:
         out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
     return plan(q.contiguous(), seq_lens, scale, out, stream)

@@ -125,6 +125,9 @@ enum DeviceError : int {
 // rows} and 128-byte swizzle (the canonical K-major operand layout of tcgen05.mma).
 bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t rows, uint64_t cols,
               uint64_t row_stride_bytes, uint32_t box_rows);
+// 2-D row-major tensor map with box {box_cols, box_rows} and no swizzle.
+bool make_map_plain(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t rows, uint64_t cols,
+                    uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows);
 
 // Returns TQ_OK if the last launch succeeded, else records the error.
 int check_launch(const char* what);

@@ -164,7 +164,24 @@ struct MmaArgs {
   int* err;                // device error word (a pipeline wait that timed out)
   const float* piv[2];     // value-group rotations, read by the merge kernel: prefetched
   uint32_t piv_bytes[2];   // into L2 at the start of this kernel
+  const int32_t* table;    // paged cache: physical page of (sequence, logical page), or NULL
+  int page, max_pages;     // tokens per page (a multiple of the 64-token stage), pages per sequence
+  int64_t npages;          // physical pages the caches hold (min over the groups' caches)
 };
+
+// First cache slot of the 64-token stage starting at token ts of (sequence b, kv head hk).
+// Contiguous caches: slot0 + ts.  Paged caches: page p of the pool holds kv head hk's
+// tokens in slots (p Hkv + hk) page .. + page - 1; a stage never crosses a page.  A page
+// index outside the pool reads page 0 and is reported as device error 901.
+__device__ __forceinline__ int64_t stage_slot(const MmaArgs& A, int b, int hk, int ts, int64_t slot0) {
+  if (!A.table) return slot0 + ts;
+  int pg = __ldg(A.table + (size_t)b * A.max_pages + ts / A.page);
+  if (pg < 0 || pg >= A.npages) {
+    if (A.err) atomicCAS(A.err, 0, (int)kErrSlotRange);
+    pg = 0;
+  }
+  return ((int64_t)pg * A.Hkv + hk) * A.page + ts % A.page;
+}
 
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 
@@ -415,7 +432,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, TQ_DECODE_CTAS_PER_SM) deco
       const int tt = ts + warp * 16;           // this warp's 16-token tile
       const bool live = tt < t_end;
       const uint8_t* st = dsm + s * ST::BYTES;
-      const int64_t first = slot0 + ts;
+      const int64_t first = stage_slot(A, b, hk, ts, slot0);
       const int ja = warp * 16 + g, jb = ja + 8;   // stage-local token rows of this lane
       KeyTile<G0> k0;
       ValTile<G0> v0;
@@ -463,12 +480,9 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, TQ_DECODE_CTAS_PER_SM) deco
       mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
       mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
       mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
-      // rescale only in the (rare) tiles where some head's maximum grows; the branch is
-      // warp-uniform, lanes whose head did not grow scale by 1
-      if (__any_sync(0xffffffffu, mt > m_run)) {
-        const float mn = fmaxf(m_run, mt);
-        const float alpha = mn == m_run ? 1.f : exp2f(m_run - mn);
-        m_run = mn;
+      if (mt > m_run) {
+        const float alpha = exp2f(m_run - mt);
+        m_run = mt;
         l_run *= alpha;
 #pragma unroll
         for (int u = 0; u < G0::NS; ++u)
@@ -535,7 +549,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, TQ_DECODE_CTAS_PER_SM) deco
       if (!mbar_wait(empty + s, ph ^ 1, abort_v, kDecWaitNs)) { fail(201); break; }
       const int ntok = min(kStageTok, t_end - ts);
       uint8_t* st = dsm + s * ST::BYTES;
-      const int64_t first = slot0 + ts, last = slot0 + ts + ntok;
+      const int64_t first = stage_slot(A, b, hk, ts, slot0), last = first + ntok;
       auto spans = [&](bool issue) {
         uint32_t tx = 0;
         const MmaGroup& g0 = A.g[0];
@@ -660,11 +674,7 @@ __global__ void __launch_bounds__(32) decode_prep_kernel(const T* __restrict__ q
   }
 }
 
-// Log-sum-exp merge of the context splits and the inverse rotation of the value groups:
-// one CTA per (query row, 64 output channels).  The rotation entries of the CTA's
-// channels are loaded before the dependency wait; after it, the row's partials (m, l, acc
-// per split, contiguous) come into shared memory by bulk copies of up to kMergeChunk
-// splits and are merged with a running maximum.
+// Arguments of the merge kernel (below).
 struct Merge2Args {
   const float* part;
   int64_t part_ld;
@@ -673,136 +683,75 @@ struct Merge2Args {
   const float* PiV[2];
   float* out;
   const int32_t* perm;   // channel permutation [Hkv][D] (NULL: identity): group channel c -> perm[kv][c]
-  int Hq, rep;
+  int Hq, rep, Hkv, nsub;
   int* err;
 };
 
-constexpr int kMergeThreads = 256;   // 4 row quarters of the rotation x 64 channels
-constexpr int kMergeChunk = 96;      // splits per bulk copy (a multiple of 4: 16-byte aligned starts)
+// Log-sum-exp merge of the context splits and the inverse value rotation, one CTA per
+// (sequence, kv head, group of 4 query heads): thread (head, coordinate) folds the splits'
+// (m, l, acc) against the maximum taken in a first pass, the merged rotated values go
+// to shared memory, and thread (output channel) applies the group's Pi_v^T to all 4 heads
+// with one read of every rotation entry (the rotation is read once per CTA, not once per
+// query row and channel block).
+constexpr int kMergeHThreads = 256;
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
-__global__ void __launch_bounds__(kMergeThreads) decode_merge_mma_kernel(Merge2Args A) {
-  extern __shared__ float4 merge_smem[];
-  float* msm = reinterpret_cast<float*>(merge_smem);   // [chunk][D+2] staged partials
-  __shared__ float s_w[kMergeChunk];
-  __shared__ float s_acc[256], s_fin[256];
-  __shared__ float red[4][64];
-  __shared__ __align__(8) uint64_t bar;
-  const int row = blockIdx.x, c0 = blockIdx.y * 64;
+__global__ void __launch_bounds__(kMergeHThreads) decode_merge_heads_kernel(Merge2Args A) {
+  __shared__ float s_v[kRep][256];           // merged rotated values (<= 256 channels)
+  __shared__ float s_Mw[kRep][2];            // per head: the split maxima of its two warps
   const int D = A.D, ns = A.nsplit, W = D + 2;
-  const int oc = threadIdx.x & 63, qtr = threadIdx.x >> 6, lane = threadIdx.x & 31;
-  const int c = c0 + oc;
-  float pv[32];
-  int goff = 0, gd = 0;
-  if (c < D) {
-    const int gsel = (A.G > 1 && c >= A.off[1]) ? 1 : 0;
-    goff = A.off[gsel];
-    gd = A.off[gsel + 1] - goff;
-    const float* Pi = A.PiV[gsel] + (c - goff);
-    const int n = gd / 4, i0 = qtr * n;   // n <= 32
+  const int bh = blockIdx.x / A.nsub, sub = blockIdx.x % A.nsub;
+  const int b = bh / A.Hkv, hk = bh % A.Hkv;
+  const int nh = min(kRep, A.rep - sub * kRep);      // query heads of this CTA
+  const int row0 = b * A.Hq + hk * A.rep + sub * kRep;
+  const int h = threadIdx.x >> 6, t64 = threadIdx.x & 63;   // head, coordinate lane of the head
+  // pass 1 (after the decode grid is complete): the maximum of the head's split maxima
+  grid_dependency_wait();
+  if (h < nh) {
+    const float* P = A.part + (size_t)(row0 + h) * A.part_ld;
+    float M = -INFINITY;
+    for (int s2 = t64; s2 < ns; s2 += 64) M = fmaxf(M, P[(size_t)s2 * W]);
 #pragma unroll
-    for (int u = 0; u < 32; ++u) pv[u] = (u < n) ? __ldg(Pi + (size_t)(i0 + u) * gd) : 0.f;
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if ((threadIdx.x & 31) == 0) s_Mw[h][(threadIdx.x >> 5) & 1] = M;
   }
-  if (threadIdx.x == 0) {
-    mbar_init(&bar, 1);
-    fence_barrier_init();
-  }
-  for (int i = threadIdx.x; i < min(ns, kMergeChunk) * W; i += blockDim.x) msm[i] = 0.f;
   __syncthreads();
-  const float* P = A.part + (size_t)row * A.part_ld;
-  // thread (coordinate i, part hs) accumulates the splits s = hs (mod halves)
-  int halves = kMergeThreads / D;
-  if (halves < 1) halves = 1;
-  const int i = threadIdx.x % D, hs = threadIdx.x / D;
-  // Pass 0 runs the whole merge on zeroed shared memory and discards it, before the
-  // grid-dependency wait: this kernel launches while the decode kernel still runs, so the
-  // instruction fetch of its code is hidden there instead of following the wait.  Pass 1
-  // is the merge.
-#pragma unroll 1
-  for (int pass = 0; pass < 2; ++pass) {
-    const bool real = pass == 1;
-    if (real) grid_dependency_wait();
-    float M = -INFINITY, L = 0.f, acc = 0.f;
-    uint32_t phase = 0;
-    bool inflight = false;
-    for (int s0 = 0; s0 < (real ? ns : 1); s0 += kMergeChunk) {
-      const int n = min(kMergeChunk, ns - s0);
-      if (real) {
-        if (threadIdx.x == 0) {
-          const uint32_t bytes = (uint32_t)(((size_t)n * W * sizeof(float) + 15) & ~(size_t)15);
-          fence_proxy_async_smem();
-          mbar_arrive_expect_tx(&bar, bytes);
-          bulk_load(msm, P + (size_t)s0 * W, bytes, &bar);
-        }
-        inflight = true;
-        const bool ok = __syncthreads_and(mbar_wait(&bar, phase, nullptr, kDecWaitNs));
-        if (!ok) {
-          if (threadIdx.x == 0 && A.err) atomicCAS(A.err, 0, 203);
-          break;
-        }
-        inflight = false;
-        phase ^= 1;
-      }
-      // chunk maximum (every warp reduces the same values in the same order)
-      float mc = -INFINITY;
-      for (int s = lane; s < n; s += 32) mc = fmaxf(mc, msm[s * W]);
-      mc = warp_max(mc);
-      const float Mn = fmaxf(M, mc);
-      if (Mn != -INFINITY) {
-        const float alpha = (M == -INFINITY) ? 0.f : __expf(M - Mn);
-        for (int s = threadIdx.x; s < n; s += blockDim.x) {
-          const float m = msm[s * W];
-          s_w[s] = (m == -INFINITY) ? 0.f : __expf(m - Mn);
-        }
-        __syncthreads();
-        float lc = 0.f;
-        for (int s = lane; s < n; s += 32) lc = fmaf(s_w[s], msm[s * W + 1], lc);
-        L = fmaf(L, alpha, warp_sum(lc));
-        float a = 0.f;
-        if (hs < halves)
-          for (int s = hs; s < n; s += halves) a = fmaf(s_w[s], msm[s * W + 2 + i], a);
-        acc = fmaf(acc, alpha, a);
-        M = Mn;
-      }
-      __syncthreads();   // the staged chunk and its weights are consumed before the next copy
-    }
-    if (inflight) {      // a copy that did not complete in time still lands before the CTA exits
-      if (threadIdx.x == 0) mbar_wait(&bar, phase, nullptr, kDecWaitNs);
-      return;
-    }
-    if (hs < halves) s_acc[hs * D + i] = acc;
-    __syncthreads();
-    if (threadIdx.x < D) {
-      float t = 0.f;
-      for (int h = 0; h < halves; ++h) t += s_acc[h * D + threadIdx.x];
-      s_fin[threadIdx.x] = L > 0.f ? t / L : 0.f;
-    }
-    __syncthreads();
-    float o = 0.f;
-    if (c < D) {
-      const int n = gd / 4, i0 = qtr * n;
+  // pass 2: weights e^(m_s - M), the sum L and the merged accumulators of the head
+  if (h < nh) {
+    const float* P = A.part + (size_t)(row0 + h) * A.part_ld;
+    const float M = fmaxf(s_Mw[h][0], s_Mw[h][1]);
+    float L = 0.f;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};           // coordinates t64 + 64 j
+    for (int s2 = 0; s2 < ns; ++s2) {
+      const float* ps = P + (size_t)s2 * W;
+      const float m = ps[0];
+      const float w = (m == -INFINITY) ? 0.f : __expf(m - M);
+      L = fmaf(w, ps[1], L);
 #pragma unroll
-      for (int u = 0; u < 32; ++u)
-        if (u < n) o = fmaf(pv[u], s_fin[goff + i0 + u], o);
+      for (int j = 0; j < 4; ++j)
+        if (t64 + 64 * j < D) acc[j] = fmaf(w, ps[2 + t64 + 64 * j], acc[j]);
     }
-    red[qtr][oc] = o;
-    __syncthreads();
-    if (real && qtr == 0 && c < D) {
-      const int oc_ch = A.perm ? A.perm[(size_t)((row % A.Hq) / A.rep) * D + c] : c;
-      if (oc_ch >= 0 && oc_ch < D) A.out[(size_t)row * D + oc_ch] = (red[0][oc] + red[1][oc]) + (red[2][oc] + red[3][oc]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (t64 + 64 * j < D) s_v[h][t64 + 64 * j] = L > 0.f ? acc[j] / L : 0.f;
+  }
+  __syncthreads();
+  // inverse rotation of each group: out[ch] = sum_i Pi_g[i][ch - off] v[off + i]
+  for (int c = threadIdx.x; c < D; c += blockDim.x) {
+    const int gsel = (A.G > 1 && c >= A.off[1]) ? 1 : 0;
+    const int goff = A.off[gsel], gd = A.off[gsel + 1] - goff;
+    const float* Pi = A.PiV[gsel] + (c - goff);
+    float o[kRep] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < gd; ++i) {
+      const float pv = __ldg(Pi + (size_t)i * gd);
+#pragma unroll
+      for (int hh = 0; hh < kRep; ++hh) o[hh] = fmaf(pv, s_v[hh][goff + i], o[hh]);
+    }
+    for (int hh = 0; hh < nh; ++hh) {
+      const int row = row0 + hh;
+      const int oc_ch = A.perm ? A.perm[(size_t)hk * D + c] : c;
+      if (oc_ch >= 0 && oc_ch < D) A.out[(size_t)row * D + oc_ch] = o[hh];
       else if (A.err) atomicCAS(A.err, 0, (int)kErrPermRange);
     }
-    __syncthreads();
   }
 }
 
@@ -1030,9 +979,9 @@ float mmaops::host_luts(const tq_ctx* kc, const tq_ctx* vc, Luts* t) {
 
 // Returns kNotHandled when the shape is outside this kernel's instantiations.
 int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G,
-                      const int32_t* perm, const void* q, int q_dtype, const tq_packed* kc, const tq_packed* vc,
-                      const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len, float scale, float* out,
-                      void* ws, cudaStream_t st) {
+                      const int32_t* perm, const int32_t* table, int page, const void* q, int q_dtype,
+                      const tq_packed* kc, const tq_packed* vc, const int32_t* seq_lens, int B, int Hq, int Hkv, int D,
+                      int64_t max_len, float scale, float* out, void* ws, cudaStream_t st) {
   if (G > 2 || D > 256) return kNotHandled;
   int sig[2] = {0, 0};
   for (int g = 0; g < G; ++g) {
@@ -1080,6 +1029,14 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
     gr.vcap = vc[g].cap;
   }
   A.err = kctx[0]->dev_err;
+  A.table = table;
+  if (table) {
+    A.page = page;
+    A.max_pages = (int)(max_len / page);
+    int64_t pool = INT64_MAX;
+    for (int g = 0; g < G; ++g) pool = std::min(pool, std::min(kc[g].cap, vc[g].cap));
+    A.npages = pool / ((int64_t)Hkv * page);
+  }
   for (int g = 0; g < G; ++g) {
     A.piv[g] = vctx[g]->Pi;
     A.piv_bytes[g] = (uint32_t)(vctx[g]->lay.d * vctx[g]->lay.d * sizeof(float));
@@ -1095,26 +1052,25 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
   M.perm = perm; M.Hq = Hq; M.rep = Hq / Hkv;
   for (int g = 0; g < G; ++g) { M.off[g] = off[g]; M.PiV[g] = vctx[g]->Pi; }
   M.off[G] = D;
-  const int mdyn = (int)((((size_t)std::min(W.nsplit, kMergeChunk) * (D + 2) * sizeof(float)) + 15) / 16 * 16);
-  cudaError_t em = cudaFuncSetAttribute(decode_merge_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mdyn);
-  if (em == cudaSuccess)
-    em = cudaFuncSetAttribute(decode_merge_mma_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                              cudaSharedmemCarveoutMaxShared);
-  if (em != cudaSuccess) return cuda_fail(em, "cudaFuncSetAttribute(decode_merge_mma_kernel)");
+  M.Hkv = Hkv;
+  M.nsub = A.nsub;
+  cudaError_t em = cudaFuncSetAttribute(decode_merge_heads_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                        cudaSharedmemCarveoutMaxShared);
+  if (em != cudaSuccess) return cuda_fail(em, "cudaFuncSetAttribute(decode_merge_heads_kernel)");
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(B * Hq, div_up(D, 64));
-  cfg.blockDim = dim3(kMergeThreads);
-  cfg.dynamicSmemBytes = mdyn;
+  cfg.gridDim = dim3(B * Hkv * A.nsub);
+  cfg.blockDim = dim3(kMergeHThreads);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_merge_mma_kernel, M);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_merge_heads_kernel, M);
   count_launch();
-  if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(decode_merge_mma_kernel)");
-  return check_launch("decode_merge_mma_kernel");
+  if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(decode_merge_heads_kernel)");
+  return check_launch("decode_merge_heads_kernel");
 }
 
 // Standalone logits for prod contexts with d in {64, 128} and 2..4 code bits: workspace

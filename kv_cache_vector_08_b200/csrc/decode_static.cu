@@ -49,7 +49,7 @@ extern "C" int tq_decode_attention_static(const tq_ctx* const* kctx, const tq_ct
   // the arguments first (an invalid shape is TQ_ERR_INVALID_ARG whatever its size), then the
   // scratch size, then the array's address; nothing is launched before all three pass
   int r = tq::check_decode_args(kctx, vctx, group_off, ngroups, q, q_dtype, kcache, vcache, seq_lens, B, Hq, Hkv, D,
-                                max_len, out);
+                                max_len, out, 0);
   if (r != TQ_OK) return r;
   if (B == 0) return TQ_OK;
   size_t need = tq_decode_workspace_size(B, Hq, Hkv, D, ngroups, max_len);

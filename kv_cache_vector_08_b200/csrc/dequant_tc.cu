@@ -28,12 +28,14 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "mma_ops.cuh"
 #include "sm100.cuh"
 
 namespace tq {
 namespace {
 
 using namespace sm100;
+using mmaops::prmt;
 
 constexpr int kDqTile = 128;
 constexpr int kDqWorkerWarps = 8;
@@ -56,6 +58,11 @@ struct DqArgs {
   uint64_t wait_ns;     // limit of the pipeline waits
   int stall;            // test hook: the MMA issuer first waits on a barrier nothing arrives on
   uint32_t tbl[32];     // P-bit code -> fp16 hi (bits 0-15) | fp16 lo (bits 16-31) of its centroid
+  // 4-bit codes: byte tables indexed by the low 3 code bits (8 entries = 2 registers each):
+  // low / high bytes of the fp16 hi and lo parts; in MSE mode the entries are the
+  // magnitudes and the top (sign) bit is applied separately, in prod mode they are signed
+  uint32_t bt[4][2];
+  int mse_sign;         // 1: MSE mode (apply the top bit as the sign)
   int* err;
 };
 
@@ -253,6 +260,50 @@ __global__ void __launch_bounds__(kDqThreads, 1) dequant_tc_kernel(const __grid_
       load_row(t + 1, nxt, nxt_n, nxt_v, nxt_r);       // one tile ahead: its loads fly during this tile
       // codes -> fp16 (hi, lo) pairs of the centroids, two coordinates per 32-bit column
       uint32_t hi[G0][16], lo[G0][16], sg[QJL ? G0 : 1][16];
+      if constexpr (P == 4) {
+        // 4-bit codes: slice u of a group is word u, coordinate j of the slice has its low
+        // three code bits in nibble j and its top bit at the msb of byte j (j < 4) or, after
+        // a shift by 4, of byte j - 4; one byte permute looks up four bytes
+#pragma unroll
+        for (int g = 0; g < G0; ++g) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t w = cur[g * P + u];
+            const uint32_t sel = w & 0x77777777u;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const uint32_t sl = hh ? sel >> 16 : sel;
+              const uint32_t top = hh ? w << 4 : w;        // top bits at byte msbs
+              const uint32_t sgn = A.mse_sign ? (top & 0x80808080u) : 0u;
+              const uint32_t hl = prmt(A.bt[0][0], A.bt[0][1], sl), hh8 = prmt(A.bt[1][0], A.bt[1][1], sl) ^ sgn;
+              const uint32_t ll = prmt(A.bt[2][0], A.bt[2][1], sl), lh8 = prmt(A.bt[3][0], A.bt[3][1], sl) ^ sgn;
+              const int i = 4 * u + 2 * hh;                // pair index of coordinates 8u + 4hh, +1
+              hi[g][i] = prmt(hl, hh8, 0x5140u);
+              hi[g][i + 1] = prmt(hl, hh8, 0x7362u);
+              lo[g][i] = prmt(ll, lh8, 0x5140u);
+              lo[g][i + 1] = prmt(ll, lh8, 0x7362u);
+              if constexpr (QJL) {
+                const uint32_t nm = ~top;                  // fp16 sign set where the QJL bit is 0
+                sg[g][i] = (prmt(nm, 0u, 0x1404u) & 0x80008000u) | (cur_r | (cur_r << 16));
+                sg[g][i + 1] = (prmt(nm, 0u, 0x3424u) & 0x80008000u) | (cur_r | (cur_r << 16));
+              }
+            }
+          }
+          // coordinates >= d are zero
+          const int j0 = 32 * (g_lo + g);
+          if (j0 + 32 > A.d) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (j0 + e >= A.d) {
+                const uint32_t keep = (e & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+                hi[g][e / 2] &= keep;
+                lo[g][e / 2] &= keep;
+                if constexpr (QJL) sg[g][e / 2] &= keep;
+              }
+            }
+          }
+        }
+      } else {
 #pragma unroll
       for (int g = 0; g < G0; ++g) {
 #pragma unroll
@@ -270,6 +321,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) dequant_tc_kernel(const __grid_
             sg[g][e / 2] = sa | (sb << 16);
           }
         }
+      }
       }
       if (!wait(a_empty + ab, (uint32_t)(((t / NA) & 1) ^ 1))) { fail(304); ok = false; break; }
       tc_fence_after();
@@ -367,6 +419,26 @@ int launch_dequantize_tc(const tq_ctx* ctx, const tq_packed* src, const int64_t*
       v = (uint32_t)__half_as_ushort(h) | ((uint32_t)__half_as_ushort(l) << 16);
     }
     a.tbl[code] = v;
+  }
+  if (P == 4) {
+    // 8-entry byte tables over the low three code bits (MSE: magnitude rank; prod: sign flag
+    // and magnitude rank), for the fp16 hi and lo parts of the centroid
+    const bool mse = ctx->mode == TQ_MODE_MSE;
+    a.mse_sign = mse ? 1 : 0;
+    uint8_t b[4][8];
+    for (int c3 = 0; c3 < 8; ++c3) {
+      const double c = mse ? ctx->host.centroids[(1 << (k - 1)) + c3] : ctx->host.centroids[code_index((uint32_t)c3, k)];
+      const __half h = __float2half_rn((float)c);
+      const __half l = __float2half_rn((float)(c - (double)__half2float(h)));
+      const uint16_t hb = __half_as_ushort(h), lb = __half_as_ushort(l);
+      b[0][c3] = (uint8_t)(hb & 0xFF);
+      b[1][c3] = (uint8_t)(hb >> 8);
+      b[2][c3] = (uint8_t)(lb & 0xFF);
+      b[3][c3] = (uint8_t)(lb >> 8);
+    }
+    for (int t = 0; t < 4; ++t)
+      for (int r = 0; r < 2; ++r)
+        a.bt[t][r] = b[t][4 * r] | (b[t][4 * r + 1] << 8) | (b[t][4 * r + 2] << 16) | ((uint32_t)b[t][4 * r + 3] << 24);
   }
   const int dev = ctx->device;
 #define TQ_DQ_CASE(GG, PP) \

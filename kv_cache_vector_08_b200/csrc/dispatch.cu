@@ -23,10 +23,11 @@ int launch_logits(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed
 }
 
 int launch_decode(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G, const int32_t* perm,
-                  const void* q, int q_dtype, const tq_packed* kc, const tq_packed* vc, const int32_t* seq_lens, int B,
-                  int Hq, int Hkv, int D, int64_t max_len, float scale, float* out, void* ws, cudaStream_t st) {
-  int r = launch_decode_mma(kctx, vctx, off, G, perm, q, q_dtype, kc, vc, seq_lens, B, Hq, Hkv, D, max_len, scale,
-                            out, ws, st);
+                  const int32_t* table, int page, const void* q, int q_dtype, const tq_packed* kc,
+                  const tq_packed* vc, const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len,
+                  float scale, float* out, void* ws, cudaStream_t st) {
+  int r = launch_decode_mma(kctx, vctx, off, G, perm, table, page, q, q_dtype, kc, vc, seq_lens, B, Hq, Hkv, D,
+                            max_len, scale, out, ws, st);
   if (r != kNotHandled) return r;
   return fail(TQ_ERR_UNSUPPORTED,
               "tq_decode_attention: supported channel groups are one group of d = 128 with 4 + 4 or 3 + 3 key / value "

@@ -28,9 +28,9 @@ bool quantize_tc_applies(const tq_ctx* ctx, int x_dtype, int64_t n, int64_t ld);
 int launch_quantize_tc(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, int64_t ld, const tq_packed* dst,
                        const int64_t* slots, cudaStream_t st);
 int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G,
-                      const int32_t* perm, const void* q, int q_dtype, const tq_packed* kc, const tq_packed* vc,
-                      const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len, float scale, float* out,
-                      void* ws, cudaStream_t st);
+                      const int32_t* perm, const int32_t* table, int page, const void* q, int q_dtype,
+                      const tq_packed* kc, const tq_packed* vc, const int32_t* seq_lens, int B, int Hq, int Hkv, int D,
+                      int64_t max_len, float scale, float* out, void* ws, cudaStream_t st);
 size_t logits_mma_workspace(int64_t nq, int d);
 int launch_logits_mma(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* keys, int64_t n, float* out,
                       void* ws, cudaStream_t st);
@@ -49,11 +49,13 @@ int launch_quantize(const tq_ctx* ctx, const void* x, int x_dtype, int64_t n, in
 int launch_logits(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* keys, int64_t n, float* logits,
                   void* ws, cudaStream_t st);
 int launch_decode(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* off, int G, const int32_t* perm,
-                  const void* q, int q_dtype, const tq_packed* kc, const tq_packed* vc, const int32_t* seq_lens, int B,
-                  int Hq, int Hkv, int D, int64_t max_len, float scale, float* out, void* ws, cudaStream_t st);
-int launch_search(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* db, int64_t N, int k,
-                  float* scores, int64_t* ids, void* ws, cudaStream_t st);
+                  const int32_t* table, int page, const void* q, int q_dtype, const tq_packed* kc,
+                  const tq_packed* vc, const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len,
+                  float scale, float* out, void* ws, cudaStream_t st);
 int check_decode_args(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off, int ngroups,
                       const void* q, int q_dtype, const tq_packed* kcache, const tq_packed* vcache,
-                      const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len, const float* out);
+                      const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len, const float* out,
+                      int page);
+int launch_search(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* db, int64_t N, int k,
+                  float* scores, int64_t* ids, void* ws, cudaStream_t st);
 }  // namespace tq

@@ -43,7 +43,9 @@ using mmaops::prmt;
 
 constexpr int kSqM = 128;                 // queries per tile
 constexpr int kSqN = 256;                 // database vectors per chunk
-constexpr int kSqStages = 3;
+constexpr int kSqStages = 2;
+constexpr int kSqCStages = 4;             // ring of code tiles (4-bit codes): 256 rows x 32 bytes each
+constexpr int kSqCStage = kSqN * 32;
 constexpr int kSqDecWarps = 8;
 constexpr int kSqEpiWarps = 4;
 constexpr int kSqThreads = 64 + 32 * (kSqDecWarps + kSqEpiWarps);
@@ -71,10 +73,16 @@ struct SqArgs {
 
 template <int P>
 __global__ void __launch_bounds__(kSqThreads, 1) search_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                                  const __grid_constant__ CUtensorMap tm_c,
                                                                   const SqArgs A) {
+  // 4-bit codes: the code words of each 64-coordinate block of the chunk (256 rows x 32
+  // bytes) are staged by TMA into a ring a few blocks ahead of the decoders; other widths
+  // are read by the decoders straight from global memory
+  constexpr bool RING = P == 4;
   extern __shared__ uint8_t sq_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sq_smem_raw) + 1023) & ~uintptr_t(1023));
-  float* list_s = reinterpret_cast<float*>(smem + kSqStages * kSqStage);          // [k][128]
+  uint8_t* cring = smem + kSqStages * kSqStage;                                  // [cstages][256][32]
+  float* list_s = reinterpret_cast<float*>(cring + (RING ? kSqCStages * kSqCStage : 0));   // [k][128]
   int32_t* list_i = reinterpret_cast<int32_t*>(list_s + kSqMaxK * kSqM);          // [k][128]
   float* s_norm = reinterpret_cast<float*>(list_i + kSqMaxK * kSqM);              // [2][256]
   uint32_t* s_ctab = reinterpret_cast<uint32_t*>(s_norm + 2 * kSqN);              // [32]
@@ -87,7 +95,9 @@ __global__ void __launch_bounds__(kSqThreads, 1) search_tc_kernel(const __grid_c
   uint64_t* nrm_full = acc_empty + 2;               // [2] chunk norms staged
   uint64_t* nrm_empty = nrm_full + 2;               // [2] chunk norms consumed
   uint64_t* drain = nrm_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* cfull = drain + 1;                      // [cstages] code tile landed
+  uint64_t* cempty = cfull + kSqCStages;            // [cstages] code tile decoded
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cempty + kSqCStages);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -110,6 +120,10 @@ __global__ void __launch_bounds__(kSqThreads, 1) search_tc_kernel(const __grid_c
       mbar_init(nrm_empty + b, kEpiThreads);
     }
     mbar_init(drain, 1);
+    for (int c = 0; c < kSqCStages; ++c) {
+      mbar_init(cfull + c, 1);
+      mbar_init(cempty + c, kDecThreads);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -148,6 +162,26 @@ __global__ void __launch_bounds__(kSqThreads, 1) search_tc_kernel(const __grid_c
         }
       for (int s = 0; s < kSqStages; ++s)
         if (pending[s] >= 0) mbar_wait(full_a + s, (uint32_t)pending[s], nullptr, kSqWaitNs);
+    } else if (RING && lane == 1) {
+      // code tiles of every 64-coordinate block of every chunk, kSqCStages ahead
+      prefetch_tensormap(&tm_c);
+      int pending[kSqCStages];
+      for (int c = 0; c < kSqCStages; ++c) pending[c] = -1;
+      int64_t cq = 0;
+      bool ok = true;
+      for (int t = 0; ok && t < nloc; ++t) {
+        const int64_t chunk = cslot + (int64_t)t * A.cpq;
+        for (int pr = 0; pr < KA / 2; ++pr, ++cq) {
+          const int c = (int)(cq % kSqCStages);
+          const uint32_t ph = (uint32_t)((cq / kSqCStages) & 1);
+          if (!wait(cempty + c, ph ^ 1)) { fail(507); ok = false; break; }
+          mbar_arrive_expect_tx(cfull + c, kSqCStage);
+          tma_load_2d(cring + c * kSqCStage, &tm_c, 32 * pr, (int)(chunk * kSqN), cfull + c);
+          pending[c] = (int)ph;
+        }
+      }
+      for (int c = 0; c < kSqCStages; ++c)
+        if (pending[c] >= 0) mbar_wait(cfull + c, (uint32_t)pending[c], nullptr, kSqWaitNs);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------- MMA issuer
@@ -209,7 +243,16 @@ __global__ void __launch_bounds__(kSqThreads, 1) search_tc_kernel(const __grid_c
         const uint32_t ph = (uint32_t)((q / kSqStages) & 1);
         const int ca = a >> 1;                      // 64-coordinate block
         const bool sign_atom = a & 1;
-        if (!sign_atom) {
+        const int64_t cq = (int64_t)t * (KA / 2) + ca;   // code tile of this block
+        if (RING && !sign_atom) {
+          const int c = (int)(cq % kSqCStages);
+          if (!wait(cfull + c, (uint32_t)((cq / kSqCStages) & 1))) { fail(508); ok = false; break; }
+          const uint4* src = reinterpret_cast<const uint4*>(cring + c * kSqCStage + row * 32);
+          const uint4 v0 = src[0], v1 = src[1];
+          w[0][0] = v0.x; w[0][1] = v0.y; w[0][2] = v0.z; w[0][3] = v0.w;
+          w[1][0 % P] = v1.x; w[1][1 % P] = v1.y; w[1][2 % P] = v1.z; w[1][3 % P] = v1.w;
+          mbar_arrive(cempty + c);                  // the words are in registers
+        } else if (!RING && !sign_atom) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int g = 2 * ca + h;
@@ -366,37 +409,57 @@ __global__ void __launch_bounds__(kSqThreads, 1) search_tc_kernel(const __grid_c
 }
 
 // Query operand: row q = per 64-coordinate block a, (Pi q)[64a .. 64a+64) then
-// sqrt(pi/2)/m (S q)[64a .. 64a+64), fp16, zero beyond d; rows >= nq are zero.  CTA = 8
-// queries x 256 output columns of one part; thread = output column, 8 dot products.
+// sqrt(pi/2)/m (S q)[64a .. 64a+64), fp16, zero beyond d; rows >= nq are zero.  A tiled fp32
+// product [nq x d] x [d x d] per part: CTA = 64 queries x 64 outputs, K in steps of 16
+// through shared memory, thread = 4 queries x 4 outputs.
 __global__ void __launch_bounds__(256) search_query_kernel(const float* __restrict__ q, int64_t nq, int d, int Kh,
                                                            const float* __restrict__ PiT, const float* __restrict__ ST,
                                                            float coef, __half* __restrict__ out) {
-  extern __shared__ float qs[];                     // [8][d]
-  const int64_t r0 = (int64_t)blockIdx.x * 8;
-  const int part = blockIdx.z;
-  const int o = blockIdx.y * 256 + threadIdx.x;
-  for (int e = threadIdx.x; e < 8 * d; e += 256) {
-    const int rr = e / d, j = e % d;
-    qs[e] = (r0 + rr < nq) ? q[(r0 + rr) * d + j] : 0.f;
-  }
-  __syncthreads();
-  if (o >= Kh) return;
-  float acc[8];
+  __shared__ float Qs[16][68];                       // [k][query]
+  __shared__ float Ms[16][68];                       // [k][output]
+  const int64_t r0 = (int64_t)blockIdx.x * 64;
+  const int o0 = blockIdx.y * 64, part = blockIdx.z;
+  const float* M = part == 0 ? PiT : ST;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  if (o < d) {
-    const float* M = part == 0 ? PiT : ST;
-    for (int j = 0; j < d; ++j) {
-      const float m = __ldg(M + (size_t)j * d + o);
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = fmaf(m, qs[i * d + j], acc[i]);
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  for (int k0 = 0; k0 < d; k0 += 16) {
+    for (int e = threadIdx.x; e < 1024; e += 256) {
+      const int qq = e >> 4, kk = e & 15;
+      Qs[kk][qq] = (r0 + qq < nq && k0 + kk < d) ? __ldg(q + (r0 + qq) * d + k0 + kk) : 0.f;
+      const int kr = e >> 6, oo = e & 63;
+      Ms[kr][oo] = (k0 + kr < d && o0 + oo < d) ? __ldg(M + (size_t)(k0 + kr) * d + o0 + oo) : 0.f;
     }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        av[i] = Qs[kk][ty * 4 + i];
+        bv[i] = Ms[kk][tx * 4 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
   }
   const float sc = part == 0 ? 1.f : coef;
   const int64_t K = 2 * (int64_t)Kh;
-  const int64_t col = (int64_t)(o / 64) * 128 + part * 64 + (o % 64);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) out[(r0 + i) * K + col] = __float2half_rn(acc[i] * sc);
+  for (int i = 0; i < 4; ++i) {
+    const int64_t row = r0 + ty * 4 + i;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int o = o0 + tx * 4 + j;
+      if (o < Kh) out[row * K + (int64_t)(o / 64) * 128 + part * 64 + (o % 64)] = __float2half_rn(acc[i][j] * sc);
+    }
+  }
 }
 
 struct SqWs {
@@ -429,12 +492,13 @@ int device_sms(int dev) {
 }
 
 template <int P>
-int launch_sq_t(const CUtensorMap& tmq, const SqArgs& a, int grid, cudaStream_t st) {
-  const int smem = kSqStages * kSqStage + 2 * kSqMaxK * kSqM * 4 + 2 * kSqN * 4 + 32 * 4 + 256 + 1024;
+int launch_sq_t(const CUtensorMap& tmq, const CUtensorMap& tmc, const SqArgs& a, int grid, cudaStream_t st) {
+  const int smem = kSqStages * kSqStage + (P == 4 ? kSqCStages * kSqCStage : 0) + 2 * kSqMaxK * kSqM * 4 +
+                   2 * kSqN * 4 + 32 * 4 + 256 + 1024;
   auto kern = search_tc_kernel<P>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(search_tc)");
-  kern<<<grid, kSqThreads, smem, st>>>(tmq, a);
+  kern<<<grid, kSqThreads, smem, st>>>(tmq, tmc, a);
   count_launch();
   return check_launch("search_tc_kernel");
 }
@@ -461,14 +525,8 @@ int launch_search_tc(const tq_ctx* ctx, const float* q, int64_t nq, const tq_pac
   const int d = ctx->lay.d;
   // the query operand
   {
-    const dim3 grid((unsigned)(W.nq_pad / 8), (unsigned)((W.Kh + 255) / 256), 2);
-    const size_t sm = (size_t)8 * d * sizeof(float);
-    if (sm > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(search_query_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(search_query_kernel)");
-    }
-    if (sm > 227 * 1024) return fail(TQ_ERR_UNSUPPORTED, "search: d above 7000");
-    search_query_kernel<<<grid, 256, sm, st>>>(q, nq, d, W.Kh, ctx->PiT, ctx->ST, ctx->sqrt_pi_over_2_over_m, qop);
+    const dim3 grid((unsigned)(W.nq_pad / 64), (unsigned)((W.Kh + 63) / 64), 2);
+    search_query_kernel<<<grid, 256, 0, st>>>(q, nq, d, W.Kh, ctx->PiT, ctx->ST, ctx->sqrt_pi_over_2_over_m, qop);
     count_launch();
     int r = check_launch("search_query_kernel");
     if (r != TQ_OK) return r;
@@ -477,6 +535,11 @@ int launch_search_tc(const tq_ctx* ctx, const float* q, int64_t nq, const tq_pac
   if (!make_map(&tmq, qop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)W.nq_pad, 2 * (uint64_t)W.Kh,
                 2 * (uint64_t)W.Kh * 2, kSqM))
     return fail(TQ_ERR_INTERNAL, "search: tensor map of the query operand");
+  CUtensorMap tmc = tmq;
+  if (ctx->lay.planes == 4 &&
+      !make_map_plain(&tmc, db->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)N, (uint64_t)ctx->lay.code_bytes,
+                      (uint64_t)ctx->lay.code_bytes, 32, kSqN))
+    return fail(TQ_ERR_INTERNAL, "search: tensor map of the database codes");
   SqArgs a{};
   a.codes = db->codes;
   a.norm = db->norm;
@@ -515,10 +578,10 @@ int launch_search_tc(const tq_ctx* ctx, const float* q, int64_t nq, const tq_pac
   const int grid = W.qtiles * W.cpq;
   int r;
   switch (P) {
-    case 2: r = launch_sq_t<2>(tmq, a, grid, st); break;
-    case 3: r = launch_sq_t<3>(tmq, a, grid, st); break;
-    case 4: r = launch_sq_t<4>(tmq, a, grid, st); break;
-    case 5: r = launch_sq_t<5>(tmq, a, grid, st); break;
+    case 2: r = launch_sq_t<2>(tmq, tmc, a, grid, st); break;
+    case 3: r = launch_sq_t<3>(tmq, tmc, a, grid, st); break;
+    case 4: r = launch_sq_t<4>(tmq, tmc, a, grid, st); break;
+    case 5: r = launch_sq_t<5>(tmq, tmc, a, grid, st); break;
     default: return fail(TQ_ERR_INTERNAL, "search: code layout");
   }
   if (r != TQ_OK) return r;

@@ -207,7 +207,8 @@ int check_args_common(int d, int bits, int mode) {
 // tq_decode_attention_static, which checks its own scratch size after these).
 int check_decode_args(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off, int ngroups,
                       const void* q, int q_dtype, const tq_packed* kcache, const tq_packed* vcache,
-                      const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len, const float* out) {
+                      const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len, const float* out,
+                      int page) {
   if (!kctx || !vctx || !group_off || !kcache || !vcache) return fail(TQ_ERR_INVALID_ARG, "NULL argument");
   if (ngroups < 1 || ngroups > 4) return fail(TQ_ERR_UNSUPPORTED, "ngroups must be in [1, 4]");
   if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_len < 0) return fail(TQ_ERR_INVALID_ARG, "bad sizes");
@@ -228,8 +229,11 @@ int check_decode_args(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
     int r = check_packed(kc, &kcache[g], "kcache");
     if (r != TQ_OK) return r;
     if ((r = check_packed(vc, &vcache[g], "vcache")) != TQ_OK) return r;
-    int64_t need = (int64_t)B * Hkv * max_len;
-    if (kcache[g].cap < need || vcache[g].cap < need) return fail(TQ_ERR_INVALID_ARG, "cache capacity below B*Hkv*max_len");
+    // contiguous caches hold every (sequence, kv head, token) slot; paged ones at least one page
+    int64_t need = page > 0 ? (int64_t)Hkv * page : (int64_t)B * Hkv * max_len;
+    if (kcache[g].cap < need || vcache[g].cap < need)
+      return fail(TQ_ERR_INVALID_ARG, page > 0 ? "cache capacity below one page (Hkv*page_tokens)"
+                                               : "cache capacity below B*Hkv*max_len");
     if ((r = check_device(kc)) != TQ_OK) return r;
   }
   return TQ_OK;
@@ -516,28 +520,33 @@ size_t tq_decode_workspace_size(int B, int Hq, int Hkv, int D, int ngroups, int6
   return decode_workspace_bytes(B, Hq, Hkv, D, ngroups, max_len, D);
 }
 
-int tq_decode_attention_perm(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off,
-                             int ngroups, const int32_t* channel_perm, const void* q, int q_dtype,
-                             const tq_packed* kcache, const tq_packed* vcache, const int32_t* seq_lens, int B, int Hq,
-                             int Hkv, int D, int64_t max_len, float scale, float* out, void* workspace,
-                             size_t ws_bytes, tq_stream_t stream) {
+int tq_decode_attention_ex(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off, int ngroups,
+                           const void* q, int q_dtype, const tq_packed* kcache, const tq_packed* vcache,
+                           const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len, float scale,
+                           float* out, const tq_decode_opts* opts, void* workspace, size_t ws_bytes,
+                           tq_stream_t stream) {
   Range range_("tq_decode_attention");
+  const int32_t* perm = opts ? opts->channel_perm : nullptr;
+  const int32_t* table = opts ? opts->block_table : nullptr;
+  const int page = table ? opts->page_tokens : 0;
+  if (table && (page <= 0 || page % 64 != 0 || max_len % page != 0))
+    return fail(TQ_ERR_INVALID_ARG, "page_tokens must be a positive multiple of 64 that divides max_len");
   int r = check_decode_args(kctx, vctx, group_off, ngroups, q, q_dtype, kcache, vcache, seq_lens, B, Hq, Hkv, D,
-                            max_len, out);
+                            max_len, out, page);
   if (r != TQ_OK) return r;
   if (B == 0) return TQ_OK;
   size_t need = tq_decode_workspace_size(B, Hq, Hkv, D, ngroups, max_len);
   if (!workspace || ws_bytes < need) return fail(TQ_ERR_WORKSPACE, "workspace too small");
-  return launch_decode(kctx, vctx, group_off, ngroups, channel_perm, q, q_dtype, kcache, vcache, seq_lens, B, Hq, Hkv,
-                       D, max_len, scale, out, workspace, (cudaStream_t)stream);
+  return launch_decode(kctx, vctx, group_off, ngroups, perm, table, page, q, q_dtype, kcache, vcache, seq_lens, B, Hq,
+                       Hkv, D, max_len, scale, out, workspace, (cudaStream_t)stream);
 }
 
 int tq_decode_attention(const tq_ctx* const* kctx, const tq_ctx* const* vctx, const int* group_off, int ngroups,
                         const void* q, int q_dtype, const tq_packed* kcache, const tq_packed* vcache,
                         const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int64_t max_len, float scale,
                         float* out, void* workspace, size_t ws_bytes, tq_stream_t stream) {
-  return tq_decode_attention_perm(kctx, vctx, group_off, ngroups, nullptr, q, q_dtype, kcache, vcache, seq_lens, B, Hq,
-                                  Hkv, D, max_len, scale, out, workspace, ws_bytes, stream);
+  return tq_decode_attention_ex(kctx, vctx, group_off, ngroups, q, q_dtype, kcache, vcache, seq_lens, B, Hq, Hkv, D,
+                                max_len, scale, out, nullptr, workspace, ws_bytes, stream);
 }
 
 size_t tq_search_workspace_size(const tq_ctx* ctx, int64_t nq, int64_t N, int k) {

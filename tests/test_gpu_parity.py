@@ -499,3 +499,135 @@ def test_unsupported_shapes_are_reported():
 def test_decode_fp32_queries_and_128_2bit_keys():
     out, ref, _ = _decode_case(1, 2, 8, 128, ((0, 128, 3, 3),), [513], 600, 8, q_dtype=torch.float32)
     parity.assert_close(out, ref, "fp32 q, 3-bit keys / values")
+
+
+# ------------------------------------------------------------- paged caches, one-graph steps
+def _oracle_decode(groups, K, V, q, lens, D, kc_gpu, vc_gpu, max_len):
+    """Oracle decode of K/V [B, Hkv, T, D] over the oracle's codes, reconciled with the GPU's
+    exempt choices (codes of token t of (b, h) in slot (b*Hkv + h)*max_len + t of the given
+    contiguous GPU caches)."""
+    B, Hkv, T, _ = K.shape
+    kp = [oracle.make_params(w, kb, 1000 + 2 * gi, 0) for gi, (_, w, kb, _) in enumerate(groups)]
+    vp = [oracle.make_params(w, vb, 1001 + 2 * gi, 1) for gi, (_, w, _, vb) in enumerate(groups)]
+    rows = torch.tensor([(b * Hkv + h) * max_len + t for b in range(B) for h in range(Hkv) for t in range(T)],
+                        device=DEV)
+    kc, vc = [], []
+    for gi, (off, w, _, _) in enumerate(groups):
+        ko = parity.reconciled_oracle_codes(kp[gi], K[..., off:off + w].reshape(-1, w).astype(np.float64),
+                                            kc_gpu[gi].codes[rows].cpu().numpy())
+        vo = parity.reconciled_oracle_codes(vp[gi], V[..., off:off + w].reshape(-1, w).astype(np.float64),
+                                            vc_gpu[gi].codes[rows].cpu().numpy())
+        kc.append({k: ko[k].reshape(B, Hkv, T, *ko[k].shape[1:]) for k in ("idx", "signs", "norm", "rnorm")})
+        vc.append({k: vo[k].reshape(B, Hkv, T, *vo[k].shape[1:]) for k in ("idx", "norm")})
+    offs = [g[0] for g in groups] + [D]
+    return oracle.decode_attention(kp, vp, offs, q.astype(np.float64), kc, vc, lens, 1 / math.sqrt(D))
+
+
+def test_paged_cache_decode_matches_contiguous_and_oracle():
+    """A pool of 64-token pages in shuffled physical order (block table per sequence) gives
+    the same attention as the contiguous cache, and both match the oracle."""
+    groups = ((0, 64, 4, 4), (64, 64, 3, 3))
+    B, Hkv, Hq, D, page, max_pages = 3, 2, 8, 128, 64, 5
+    max_len = page * max_pages
+    lens = [300, 129, 64]
+    rng = np.random.default_rng(21)
+    K = W.round_bf16(rng.standard_normal((B, Hkv, max_len, D)))
+    V = W.round_bf16(rng.standard_normal((B, Hkv, max_len, D)))
+    q = W.round_bf16(rng.standard_normal((B, Hq, D)))
+    npool = B * max_pages + 2
+    table = rng.permutation(npool)[:B * max_pages].reshape(B, max_pages).astype(np.int32)
+    Kt = torch.tensor(K.reshape(-1, D), dtype=torch.bfloat16, device=DEV)
+    Vt = torch.tensor(V.reshape(-1, D), dtype=torch.bfloat16, device=DEV)
+    # slot of row (b, h, t) in the contiguous and in the paged cache
+    b_, h_, t_ = np.meshgrid(np.arange(B), np.arange(Hkv), np.arange(max_len), indexing="ij")
+    paged = (table[b_, t_ // page].astype(np.int64) * Hkv + h_) * page + t_ % page
+    paged = torch.tensor(paged.reshape(-1), device=DEV)
+    kx, vx, kc, vc, kpg, vpg = [], [], [], [], [], []
+    for gi, (off, w, kb, vb) in enumerate(groups):
+        a, b = tq.Context(w, kb, 1000 + 2 * gi, tq.MODE_PROD), tq.Context(w, vb, 1001 + 2 * gi, tq.MODE_MSE)
+        kx.append(a); vx.append(b)
+        kc.append(tq.alloc_packed(a, B * Hkv * max_len)); vc.append(tq.alloc_packed(b, B * Hkv * max_len))
+        kpg.append(tq.alloc_packed(a, npool * Hkv * page)); vpg.append(tq.alloc_packed(b, npool * Hkv * page))
+        tq.quantize_kv(a, Kt[:, off:off + w], kc[gi]); tq.quantize_kv(b, Vt[:, off:off + w], vc[gi])
+        tq.quantize_kv(a, Kt[:, off:off + w], kpg[gi], slots=paged)
+        tq.quantize_kv(b, Vt[:, off:off + w], vpg[gi], slots=paged)
+    qt = torch.tensor(q, dtype=torch.bfloat16, device=DEV)
+    sl = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    out_c = tq.decode_attention(kx, vx, [0, 64, 128], qt, kc, vc, sl, Hkv, max_len, 1 / math.sqrt(D))
+    out_p = tq.decode_attention(kx, vx, [0, 64, 128], qt, kpg, vpg, sl, Hkv, max_len, 1 / math.sqrt(D),
+                                block_table=torch.tensor(table, device=DEV), page_tokens=page)
+    torch.cuda.synchronize()
+    assert kx[0].device_error() == 0
+    assert torch.equal(out_c, out_p)
+    ref = _oracle_decode(groups, K, V, q, lens, D, kc, vc, max_len)
+    parity.assert_close(out_p.cpu().numpy(), ref, "paged decode")
+
+
+def test_append_and_decode_replayed_as_one_cuda_graph():
+    """One CUDA graph holds a step's append-quantize (one new token per sequence and kv head,
+    scattered slots) and its decode; the host only refreshes the graph's input buffers
+    (new rows, slots, sequence lengths, query) between replays."""
+    groups = ((0, 64, 4, 4), (64, 64, 3, 3))
+    B, Hkv, Hq, D, T0, steps = 4, 2, 8, 128, 200, 3
+    max_len = T0 + steps
+    rng = np.random.default_rng(33)
+    K = W.round_bf16(rng.standard_normal((B, Hkv, max_len, D)))
+    V = W.round_bf16(rng.standard_normal((B, Hkv, max_len, D)))
+    qs = W.round_bf16(rng.standard_normal((steps, B, Hq, D)))
+    kx, vx, kc, vc = [], [], [], []
+    for gi, (off, w, kb, vb) in enumerate(groups):
+        a, b = tq.Context(w, kb, 1000 + 2 * gi, tq.MODE_PROD), tq.Context(w, vb, 1001 + 2 * gi, tq.MODE_MSE)
+        kx.append(a); vx.append(b)
+        kc.append(tq.alloc_packed(a, B * Hkv * max_len)); vc.append(tq.alloc_packed(b, B * Hkv * max_len))
+    # prefill T0 tokens
+    rows = torch.tensor([(bb * Hkv + h) * max_len + t for bb in range(B) for h in range(Hkv) for t in range(T0)],
+                        device=DEV)
+    Kt = torch.tensor(K.reshape(-1, D), dtype=torch.bfloat16, device=DEV)
+    Vt = torch.tensor(V.reshape(-1, D), dtype=torch.bfloat16, device=DEV)
+    for gi, (off, w, _, _) in enumerate(groups):
+        tq.quantize_kv(kx[gi], Kt[rows, off:off + w], kc[gi], slots=rows)
+        tq.quantize_kv(vx[gi], Vt[rows, off:off + w], vc[gi], slots=rows)
+    # static graph inputs
+    new_k = torch.zeros((B * Hkv, D), dtype=torch.bfloat16, device=DEV)
+    new_v = torch.zeros_like(new_k)
+    slots = torch.zeros(B * Hkv, dtype=torch.int64, device=DEV)
+    seq = torch.zeros(B, dtype=torch.int32, device=DEV)
+    qb = torch.zeros((B, Hq, D), dtype=torch.bfloat16, device=DEV)
+    out = torch.zeros((B, Hq, D), dtype=torch.float32, device=DEV)
+    plan = tq.DecodePlan(kx, vx, [0, 64, 128], kc, vc, B, Hq, Hkv, D, max_len)
+    # quantize workspaces sized once (the bf16 d = 64 rows of 8 tokens take the workspace path)
+    wks = [torch.empty(max(tq.quantize_workspace_size(c, 1, B * Hkv, D), 1), dtype=torch.uint8, device=DEV)
+           for c in kx + vx]
+
+    def step():
+        for gi, (off, w, _, _) in enumerate(groups):
+            tq.quantize_kv(kx[gi], new_k[:, off:off + w], kc[gi], slots=slots, workspace=wks[gi])
+            tq.quantize_kv(vx[gi], new_v[:, off:off + w], vc[gi], slots=slots, workspace=wks[len(groups) + gi])
+        plan(qb, seq, 1 / math.sqrt(D), out)
+
+    def load(s):
+        t = T0 + s
+        new_k.copy_(torch.tensor(K[:, :, t].reshape(-1, D), dtype=torch.bfloat16))
+        new_v.copy_(torch.tensor(V[:, :, t].reshape(-1, D), dtype=torch.bfloat16))
+        slots.copy_(torch.tensor([(bb * Hkv + h) * max_len + t for bb in range(B) for h in range(Hkv)]))
+        seq.fill_(t + 1)
+        qb.copy_(torch.tensor(qs[s], dtype=torch.bfloat16))
+
+    load(0)
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cs):
+        step()                                   # warm-up outside capture (first-use set-up)
+    torch.cuda.current_stream().wait_stream(cs)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for s in range(steps):
+        load(s)
+        graph.replay()
+        torch.cuda.synchronize()
+        T = T0 + s + 1
+        ref = _oracle_decode(groups, K[:, :, :T], V[:, :, :T], qs[s], [T] * B, D, kc, vc, max_len)
+        parity.assert_close(out.cpu().numpy(), ref, "graph step %d" % s)
+    assert kx[0].device_error() == 0
