@@ -330,7 +330,11 @@ __device__ __forceinline__ void group_values(const Luts& t, const ValTile<GC>& v
 }
 
 constexpr int kStageTok = kWarps * 16;  // tokens per pipeline stage: one 16-token tile per consumer warp
-constexpr int kNStage = 4;
+#ifndef TQ_DECODE_STAGES
+#define TQ_DECODE_STAGES 4
+#endif
+constexpr int kNStage = TQ_DECODE_STAGES;
+constexpr int kAccBytes = kWarps * kRep * 256 * 4;   // the warps' value accumulators at the end (aliases the ring)
 constexpr uint64_t kDecWaitNs = 2000000000ull;
 
 // Shared-memory layout of one pipeline stage: per group the K and V code bytes and the
@@ -369,11 +373,12 @@ __device__ __forceinline__ uint32_t stage_span(uint8_t* dst, const uint8_t* src,
 template <class G0, class G1>
 __global__ void __launch_bounds__((kWarps + 1) * 32, TQ_DECODE_CTAS_PER_SM) decode_mma_kernel(MmaArgs A) {
   constexpr bool TWO = !std::is_same<G1, void>::value;
+  constexpr int NG = TWO ? 2 : 1;
   using G1c = typename std::conditional<TWO, G1, G0>::type;
   using ST = Stage<G0, G1c, TWO>;
   extern __shared__ __align__(128) uint8_t dsm[];
   __shared__ float s_m[kWarps][kRep], s_l[kWarps][kRep];
-  __shared__ float s_acc[kWarps][kRep][256];
+  float(*s_acc)[kRep][256] = reinterpret_cast<float(*)[kRep][256]>(dsm);   // used once the ring is drained
   __shared__ __align__(8) uint64_t full[kNStage], empty[kNStage];
   __shared__ int s_abort;
   const int split = blockIdx.x, bh = blockIdx.y / A.nsub, sub = blockIdx.y % A.nsub;
@@ -523,6 +528,63 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, TQ_DECODE_CTAS_PER_SM) deco
       s_m[warp][l] = m_run;
       s_l[warp][l] = l_run;
     }
+  } else {
+    // ---------------------------------------------------------------- producer warp
+    if (split == 0 && blockIdx.y == 0 && lane < (TWO ? 2 : 1)) bulk_prefetch_l2(A.piv[lane], A.piv_bytes[lane]);
+    int it = 0;
+    uint32_t issued = 0, phases = 0;           // stages with copies issued, parity of their last phase
+    for (int ts = t_begin; ts < t_end; ts += kStageTok, ++it) {
+      const int s = it % kNStage;
+      const uint32_t ph = (it / kNStage) & 1;
+      if (!mbar_wait(empty + s, ph ^ 1, abort_v, kDecWaitNs)) { fail(201); break; }
+      const int ntok = min(kStageTok, t_end - ts);
+      uint8_t* st = dsm + s * ST::BYTES;
+      const int64_t first = stage_slot(A, b, hk, ts, slot0), last = first + ntok;
+      // one array per lane: lanes 0..2NG-1 the code arrays (K0, V0[, K1, V1]), the next 3NG
+      // lanes the norm arrays (key norm, residual norm, value norm of each group); each lane
+      // adds its own bytes to the stage's transaction count before its copy
+      if (lane < 5 * NG) {
+        const bool nrm = lane >= 2 * NG;
+        const int j = nrm ? lane - 2 * NG : lane;
+        const int gi = TWO ? (nrm ? j / 3 : j >> 1) : 0;
+        const int kind = nrm ? j % 3 : (j & 1);            // codes: 0 K, 1 V; norms: 0 kn, 1 kr, 2 vn
+        const MmaGroup& gr = A.g[0];
+        const MmaGroup& gq = A.g[TWO ? 1 : 0];
+        const bool second = gi != 0;
+        const uint8_t* src;
+        int64_t eb, cap;
+        int doff;
+        if (!nrm) {
+          const bool v = kind != 0;
+          src = v ? (second ? gq.vcodes : gr.vcodes) : (second ? gq.kcodes : gr.kcodes);
+          eb = v ? (second ? ST::VB1 : ST::VB0) : (second ? ST::KB1 : ST::KB0);
+          cap = v ? (second ? gq.vcap : gr.vcap) : (second ? gq.kcap : gr.kcap);
+          doff = v ? (second ? ST::OFF_V1 : ST::OFF_V0) : (second ? ST::OFF_K1 : ST::OFF_K0);
+        } else {
+          const uint16_t* p = kind == 0 ? (second ? gq.knorm : gr.knorm)
+                                        : kind == 1 ? (second ? gq.krnorm : gr.krnorm) : (second ? gq.vnorm : gr.vnorm);
+          src = reinterpret_cast<const uint8_t*>(p);
+          eb = 2;
+          cap = kind < 2 ? (second ? gq.kcap : gr.kcap) : (second ? gq.vcap : gr.vcap);
+          doff = ST::OFF_N + (gi * 3 + kind) * ST::NB;
+        }
+        const uint32_t bytes = stage_span(st + doff, src, first * eb, last * eb, cap * eb, full + s, false);
+        if (bytes) mbar_expect_tx(full + s, bytes);
+        stage_span(st + doff, src, first * eb, last * eb, cap * eb, full + s, true);
+      }
+      __syncwarp();
+      mbar_arrive(full + s);
+      issued |= 1u << s;
+      phases = (phases & ~(1u << s)) | (ph << s);
+    }
+    // bulk copies still in flight land before the CTA exits
+    if (lane == 0)
+      for (int i = 0; i < kNStage; ++i)
+        if ((issued >> i) & 1u) mbar_wait(full + i, (phases >> i) & 1u, nullptr, kDecWaitNs);
+    __syncwarp();
+  }
+  __syncthreads();   // the ring is drained: its memory now holds the warps' accumulators
+  if (warp < kWarps) {
     // row g of block (u, h) is coordinate CQ (g>>1) + 8u + 4h + (g&1), row g+8 adds 2
     auto store_acc = [&](auto& acc, auto gc_tag, int off) {
       using GC = decltype(gc_tag);
@@ -537,55 +599,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, TQ_DECODE_CTAS_PER_SM) deco
     };
     store_acc(acc0, G0{}, A.g[0].off);
     if constexpr (TWO) store_acc(acc1, G1c{}, A.g[1].off);
-  } else {
-    // ---------------------------------------------------------------- producer warp
-    if (split == 0 && blockIdx.y == 0 && lane < (TWO ? 2 : 1)) bulk_prefetch_l2(A.piv[lane], A.piv_bytes[lane]);
-    int it = 0;
-    int pending[kNStage];
-    for (int i = 0; i < kNStage; ++i) pending[i] = -1;
-    for (int ts = t_begin; ts < t_end; ts += kStageTok, ++it) {
-      const int s = it % kNStage;
-      const uint32_t ph = (it / kNStage) & 1;
-      if (!mbar_wait(empty + s, ph ^ 1, abort_v, kDecWaitNs)) { fail(201); break; }
-      const int ntok = min(kStageTok, t_end - ts);
-      uint8_t* st = dsm + s * ST::BYTES;
-      const int64_t first = stage_slot(A, b, hk, ts, slot0), last = first + ntok;
-      auto spans = [&](bool issue) {
-        uint32_t tx = 0;
-        const MmaGroup& g0 = A.g[0];
-        tx += stage_span(st + ST::OFF_K0, g0.kcodes, first * ST::KB0, last * ST::KB0, g0.kcap * ST::KB0, full + s, issue);
-        tx += stage_span(st + ST::OFF_V0, g0.vcodes, first * ST::VB0, last * ST::VB0, g0.vcap * ST::VB0, full + s, issue);
-        if constexpr (TWO) {
-          const MmaGroup& g1 = A.g[1];
-          tx += stage_span(st + ST::OFF_K1, g1.kcodes, first * ST::KB1, last * ST::KB1, g1.kcap * ST::KB1, full + s, issue);
-          tx += stage_span(st + ST::OFF_V1, g1.vcodes, first * ST::VB1, last * ST::VB1, g1.vcap * ST::VB1, full + s, issue);
-        }
-#pragma unroll
-        for (int gi = 0; gi < (TWO ? 2 : 1); ++gi) {
-          const MmaGroup& gr = A.g[gi];
-          uint8_t* nb = st + ST::OFF_N + gi * 3 * ST::NB;
-          const uint8_t* kn = reinterpret_cast<const uint8_t*>(gr.knorm);
-          const uint8_t* kr = reinterpret_cast<const uint8_t*>(gr.krnorm);
-          const uint8_t* vn = reinterpret_cast<const uint8_t*>(gr.vnorm);
-          tx += stage_span(nb, kn, first * 2, last * 2, gr.kcap * 2, full + s, issue);
-          tx += stage_span(nb + ST::NB, kr, first * 2, last * 2, gr.kcap * 2, full + s, issue);
-          tx += stage_span(nb + 2 * ST::NB, vn, first * 2, last * 2, gr.vcap * 2, full + s, issue);
-        }
-        return tx;
-      };
-      if (lane == 0) {
-        mbar_expect_tx(full + s, spans(false));
-        spans(true);
-      }
-      __syncwarp();
-      mbar_arrive(full + s);
-      if (lane == 0) pending[s] = (int)ph;
-    }
-    // bulk copies still in flight land before the CTA exits
-    if (lane == 0)
-      for (int i = 0; i < kNStage; ++i)
-        if (pending[i] >= 0) mbar_wait(full + i, (uint32_t)pending[i], nullptr, kDecWaitNs);
-    }
+  }
   __syncthreads();
   // ---- merge the warps: one partial per (query head, split); m in natural-log units
   const float ln2 = 0.69314718055994531f;
@@ -926,7 +940,7 @@ template <class G0, class G1>
 int launch_mma_t(const MmaArgs& A, int nsplit, int BHkv, cudaStream_t st) {
   constexpr bool TWO = !std::is_same<G1, void>::value;
   using G1c = typename std::conditional<TWO, G1, G0>::type;
-  const int dyn = kNStage * Stage<G0, G1c, TWO>::BYTES;
+  const int dyn = std::max(kNStage * Stage<G0, G1c, TWO>::BYTES, kAccBytes);
   cudaError_t ea = cudaFuncSetAttribute(decode_mma_kernel<G0, G1>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
   if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncSetAttribute(decode_mma_kernel)");
   // one shared-memory carveout for the prep, decode and merge kernels, so they can share SMs
