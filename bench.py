@@ -264,14 +264,26 @@ class DecodeBench:
             self.tq.quantize_kv(self.vctx[gi], self.Vf[:, off:off + wd], self.vc[gi], stream=stream)
 
     def append(self, t, stream=None, k=None, v=None):
-        """Quantize token t of every (sequence, kv head) into its cache slot."""
+        """Quantize token t of every (sequence, kv head) into its cache slot.  The key and
+        value calls of every group are independent, so they run on parallel streams (forked
+        from and joined back into the calling stream; parallel branches inside a graph)."""
+        torch = self.torch
         k = self.app_k[t] if k is None else k
         v = self.app_v[t] if v is None else v
+        jobs = []
         for gi, (off, wd, _, _) in enumerate(self.w.groups):
-            self.tq.quantize_kv(self.kctx[gi], k[:, off:off + wd], self.kc[gi], slots=self.app_slots[t],
-                                stream=stream)
-            self.tq.quantize_kv(self.vctx[gi], v[:, off:off + wd], self.vc[gi], slots=self.app_slots[t],
-                                stream=stream)
+            jobs.append((self.kctx[gi], k[:, off:off + wd], self.kc[gi]))
+            jobs.append((self.vctx[gi], v[:, off:off + wd], self.vc[gi]))
+        cur = torch.cuda.current_stream(self.dev) if stream is None else stream
+        if not hasattr(self, "side"):
+            self.side = [torch.cuda.Stream(device=self.dev) for _ in range(3)]
+        streams = [cur] + self.side[:len(jobs) - 1]
+        for s in streams[1:]:
+            s.wait_stream(cur)
+        for s, (ctx, x, dst) in zip(streams, jobs):
+            self.tq.quantize_kv(ctx, x, dst, slots=self.app_slots[t], stream=s)
+        for s in streams[1:]:
+            cur.wait_stream(s)
 
     def decode(self, seq, stream=None):
         self.plan(self.q, seq, self.scale, self.out, stream=stream)
@@ -766,7 +778,7 @@ def run_e2e(bench, kind, st, steps, warmup):
     keys = bench.B * bench.Hkv * bench.T
     return {"value": keys / t, "unit": "keys/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(oh.numel() * oh.element_size()), "ms_per_step": t * 1e3,
-            "how": "eager library calls (no graph) on the current stream, pinned host buffers"}
+            "how": "eager library calls (no graph; the append's key and value calls on parallel streams), pinned host buffers"}
 
 
 # -------------------------------------------------------------------- CPU oracle
@@ -869,6 +881,72 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------- small cases for profilers
+KERNEL_CASES = ("decode-serving-b16", "search-d1536-200k", "dequant-d128", "quantize-fp32-d1536")
+
+
+def run_kernel_case(args):
+    """One small case of a kernel family, run `reps` times, for ncu captures (inputs larger
+    than L2, a few GB on the device at most).  Prints the median device time of the call;
+    this is a profiling aid, not a bench line."""
+    import dataclasses
+    import torch
+    import kv_cache_vector_08_b200 as tq
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    case = args.kernel_case
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        return sorted(a.elapsed_time(b) for a, b in ts)[len(ts) // 2] * 1e3
+
+    if case == "decode-serving-b16":
+        w = dataclasses.replace(W.SERVING_3P5, batch=16, name="serving-decode-3.5bit-b16")
+        bench = DecodeBench(w, dev)
+        bench.prefill(bench.max_len)
+        seq = torch.full((bench.B,), bench.T, dtype=torch.int32, device=dev)
+        us = timed(lambda: bench.decode(seq))
+        note = "%d token-heads" % (bench.B * bench.Hkv * bench.T)
+    elif case == "search-d1536-200k":
+        d, N, nq = 1536, 200000, 1000
+        db = torch.nn.functional.normalize(torch.randn((N, d), generator=g, device=dev), dim=1)
+        qs = torch.nn.functional.normalize(torch.randn((nq, d), generator=g, device=dev), dim=1)
+        ctx = tq.Context(d, 4, 12, tq.MODE_PROD)
+        pk = tq.alloc_packed(ctx, N)
+        tq.quantize_kv(ctx, db, pk)
+        del db
+        us = timed(lambda: tq.search_topk(ctx, qs, pk, N, 10))
+        note = "%.0f TFLOP/s (4 d flops per pair)" % (4.0 * d * N * nq / us / 1e6)
+    elif case == "dequant-d128":
+        d, n = 128, 262144
+        x = torch.randn((n, d), generator=g, device=dev).to(torch.bfloat16)
+        ctx = tq.Context(d, 4, 5, tq.MODE_MSE)
+        pk = tq.alloc_packed(ctx, n)
+        tq.quantize_kv(ctx, x, pk)
+        out = torch.empty((n, d), device=dev)
+        us = timed(lambda: tq.dequantize(ctx, pk, n, out=out))
+        note = "%.0f GB/s (66 + 512 B per vector)" % (n * (66 + 512) / us / 1e3)
+    else:   # quantize-fp32-d1536
+        d, n = 1536, 32768
+        x = torch.nn.functional.normalize(torch.randn((n, d), generator=g, device=dev), dim=1)
+        ctx = tq.Context(d, 4, 12, tq.MODE_PROD)
+        pk = tq.alloc_packed(ctx, n)
+        ws = torch.empty(tq.quantize_workspace_size(ctx, 0, n, d), dtype=torch.uint8, device=dev)
+        us = timed(lambda: tq.quantize_kv(ctx, x, pk, workspace=ws))
+        note = "%.0f TFLOP/s algorithmic (4 d^2 per vector)" % (4.0 * d * d * n / us / 1e6)
+    print("%s: %.1f us per call (median of %d), %s" % (case, us, args.reps, note), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -879,10 +957,15 @@ def main():
                     help="headline decode workload")
     ap.add_argument("--no-configs", dest="configs", action="store_false",
                     help="skip the measurements of the other workloads")
+    ap.add_argument("--kernel-case", choices=KERNEL_CASES,
+                    help="run one small case of a kernel family for a profiler instead of the bench")
+    ap.add_argument("--reps", type=int, default=3, help="calls of --kernel-case")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.kernel_case:
+        run_kernel_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

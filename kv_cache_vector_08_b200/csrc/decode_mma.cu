@@ -336,6 +336,12 @@ constexpr int kStageTok = kWarps * 16;  // tokens per pipeline stage: one 16-tok
 constexpr int kNStage = TQ_DECODE_STAGES;
 constexpr int kAccBytes = kWarps * kRep * 256 * 4;   // the warps' value accumulators at the end (aliases the ring)
 constexpr uint64_t kDecWaitNs = 2000000000ull;
+// The producer waits most of the time (the ring is full while the consumers work): its
+// retries sleep instead of spinning, which leaves the issue slots to the consumer warps.
+constexpr uint32_t kDecSleepNs = 2000;
+#ifndef TQ_DECODE_CONSUMER_SLEEP
+#define TQ_DECODE_CONSUMER_SLEEP 1
+#endif
 
 // Shared-memory layout of one pipeline stage: per group the K and V code bytes and the
 // three fp16 norm arrays (key norm, residual norm, value norm) of 64 consecutive slots,
@@ -431,45 +437,50 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, TQ_DECODE_CTAS_PER_SM) deco
 #pragma unroll
       for (int h = 0; h < 2; ++h) acc1[u][h][0] = acc1[u][h][1] = acc1[u][h][2] = acc1[u][h][3] = 0.f;
     int it = 0;
+    // Where a staged array's first slot lands inside its stage buffer: the bulk copies keep
+    // the source's offset within 16 bytes.  Stages start at multiples of 64 tokens (and
+    // pages hold multiples of 64 slots), so the offset is the same for every stage.
+    const int64_t sbase = A.table ? 0 : slot0;
+    const int ja = warp * 16 + g, jb = ja + 8;   // stage-local token rows of this lane
+    const int ok0 = (int)((sbase * ST::KB0) & 15) + ST::OFF_K0, ov0 = (int)((sbase * ST::VB0) & 15) + ST::OFF_V0;
+    const int ok1 = (int)((sbase * ST::KB1) & 15) + ST::OFF_K1, ov1 = (int)((sbase * ST::VB1) & 15) + ST::OFF_V1;
+    const int nof = (int)((sbase * 2) & 15) + ST::OFF_N;
     for (int ts = t_begin; ts < t_end; ts += kStageTok, ++it) {
       const int s = it % kNStage;
+#if TQ_DECODE_CONSUMER_SLEEP
+      if (!mbar_wait_sleep(full + s, (it / kNStage) & 1, abort_v, kDecWaitNs, kDecSleepNs)) { fail(202); break; }
+#else
       if (!mbar_wait(full + s, (it / kNStage) & 1, abort_v, kDecWaitNs)) { fail(202); break; }
+#endif
       const int tt = ts + warp * 16;           // this warp's 16-token tile
       const bool live = tt < t_end;
       const uint8_t* st = dsm + s * ST::BYTES;
-      const int64_t first = stage_slot(A, b, hk, ts, slot0);
-      const int ja = warp * 16 + g, jb = ja + 8;   // stage-local token rows of this lane
       KeyTile<G0> k0;
       ValTile<G0> v0;
       KeyTile<G1c> k1;
       ValTile<G1c> v1;
       if (live) {
-        const uint8_t* kp = st + ST::OFF_K0 + ((first * ST::KB0) & 15);
-        const uint8_t* vp = st + ST::OFF_V0 + ((first * ST::VB0) & 15);
-        lds_words(k0.a, kp + ja * ST::KB0, l);
-        lds_words(k0.b, kp + jb * ST::KB0, l);
-        lds_words(v0.a, vp + ja * ST::VB0, l);
-        lds_words(v0.b, vp + jb * ST::VB0, l);
-        // norms of slots past the context (staged bytes of other slots) read as 0
+        lds_words(k0.a, st + ok0 + ja * ST::KB0, l);
+        lds_words(k0.b, st + ok0 + jb * ST::KB0, l);
+        lds_words(v0.a, st + ov0 + ja * ST::VB0, l);
+        lds_words(v0.b, st + ov0 + jb * ST::VB0, l);
+        // value norms of slots past the context (staged bytes of other slots, or bytes never
+        // written) read as 0; key norms need no guard, those tokens' logits become -inf
         const bool va = tt + g < t_end, vb = tt + g + 8 < t_end;
-        const int nof = (int)((first * 2) & 15);
-        auto nrm = [&](int gi, int a, int j, bool ok) {
-          const uint16_t* p = reinterpret_cast<const uint16_t*>(st + ST::OFF_N + (gi * 3 + a) * ST::NB + nof);
-          return ok ? h2f(p[j]) : 0.f;
+        auto nrm = [&](int gi, int a, int j) {
+          return h2f(reinterpret_cast<const uint16_t*>(st + nof + (gi * 3 + a) * ST::NB)[j]);
         };
-        k0.na = nrm(0, 0, ja, va); k0.nb = nrm(0, 0, jb, vb);
-        k0.ra = nrm(0, 1, ja, va); k0.rb = nrm(0, 1, jb, vb);
-        v0.na = nrm(0, 2, ja, va); v0.nb = nrm(0, 2, jb, vb);
+        k0.na = nrm(0, 0, ja); k0.nb = nrm(0, 0, jb);
+        k0.ra = nrm(0, 1, ja); k0.rb = nrm(0, 1, jb);
+        v0.na = va ? nrm(0, 2, ja) : 0.f; v0.nb = vb ? nrm(0, 2, jb) : 0.f;
         if constexpr (TWO) {
-          const uint8_t* kq = st + ST::OFF_K1 + ((first * ST::KB1) & 15);
-          const uint8_t* vq = st + ST::OFF_V1 + ((first * ST::VB1) & 15);
-          lds_words(k1.a, kq + ja * ST::KB1, l);
-          lds_words(k1.b, kq + jb * ST::KB1, l);
-          lds_words(v1.a, vq + ja * ST::VB1, l);
-          lds_words(v1.b, vq + jb * ST::VB1, l);
-          k1.na = nrm(1, 0, ja, va); k1.nb = nrm(1, 0, jb, vb);
-          k1.ra = nrm(1, 1, ja, va); k1.rb = nrm(1, 1, jb, vb);
-          v1.na = nrm(1, 2, ja, va); v1.nb = nrm(1, 2, jb, vb);
+          lds_words(k1.a, st + ok1 + ja * ST::KB1, l);
+          lds_words(k1.b, st + ok1 + jb * ST::KB1, l);
+          lds_words(v1.a, st + ov1 + ja * ST::VB1, l);
+          lds_words(v1.b, st + ov1 + jb * ST::VB1, l);
+          k1.na = nrm(1, 0, ja); k1.nb = nrm(1, 0, jb);
+          k1.ra = nrm(1, 1, ja); k1.rb = nrm(1, 1, jb);
+          v1.na = va ? nrm(1, 2, ja) : 0.f; v1.nb = vb ? nrm(1, 2, jb) : 0.f;
         }
       }
       __syncwarp();
@@ -536,7 +547,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, TQ_DECODE_CTAS_PER_SM) deco
     for (int ts = t_begin; ts < t_end; ts += kStageTok, ++it) {
       const int s = it % kNStage;
       const uint32_t ph = (it / kNStage) & 1;
-      if (!mbar_wait(empty + s, ph ^ 1, abort_v, kDecWaitNs)) { fail(201); break; }
+      if (!mbar_wait_sleep(empty + s, ph ^ 1, abort_v, kDecWaitNs, kDecSleepNs)) { fail(201); break; }
       const int ntok = min(kStageTok, t_end - ts);
       uint8_t* st = dsm + s * ST::BYTES;
       const int64_t first = stage_slot(A, b, hk, ts, slot0), last = first + ntok;
@@ -625,67 +636,69 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, TQ_DECODE_CTAS_PER_SM) deco
   }
 }
 
-// Rotated queries Pi q and S q of one group in fp32 (the fixed-point digits are formed by
-// the consumer warps, which see a whole head row).  CTA = one warp for (8 query rows,
-// part, 8 output coordinates): small enough to share an SM sub-partition with the decode
-// kernel's warps, which may launch at once (their first bulk copies overlap these loads).
-// The 8 columns of Pi^T (blockIdx.y = 0) or S^T (1) and the 8 rows are staged in shared
-// memory with one round of loads; thread (row, pair) runs two d_g-term dot products.
-// Rows >= nrows (padding of the last block) are skipped.
-constexpr int kPrepRows = 8;
+// Rotated queries Pi q and S q of every group in fp32 (the fixed-point digits are formed by
+// the consumer warps of the decode kernel, which see a whole head row), one launch for all
+// groups.  CTA = 16 query rows x 64 outputs of one (group, part): the 64 columns of Pi^T
+// (part 0) or S^T (part 1) and the 16 rows (channels gathered through the permutation) are
+// staged in shared memory with one round of loads; thread (row, 4 outputs) runs 4 dot
+// products of d_g terms.  The decode kernel is launched behind it and starts streaming the
+// cache at once; its consumer warps wait for this grid before reading the projections.
+constexpr int kPrepRows = 16;
 
-template <typename T>
-__global__ void __launch_bounds__(32) decode_prep_kernel(const T* __restrict__ q, int ldq, int off, int dg,
-                                                         int nrows, const float* __restrict__ PiT,
-                                                         const float* __restrict__ ST, float* __restrict__ qp,
-                                                         int D, int G, int gi, const int32_t* __restrict__ perm,
-                                                         int Hq, int rep) {
-  __shared__ float4 ms4[128][2];                 // [j][o/4]: M^T[j][o0 + o]
-  __shared__ float qs[kPrepRows][130];           // padded rows: conflict-free column reads
+struct PrepArgs {
+  const void* q;
+  int q_f32;
+  int nrows, D, G, Hq, rep, dg, obs;   // obs: 64-output blocks per group
+  const int32_t* perm;                 // [Hkv][D] channel permutation or NULL
+  int off[2];
+  const float* pit[2];
+  const float* stt[2];
+  float* qp;                           // [nrows][G][2][D]
+};
+
+__global__ void __launch_bounds__(256) decode_prep_kernel(PrepArgs A) {
+  __shared__ __align__(16) float ms[128][64];        // [j][o]: M^T[j][64 ob + o]
+  __shared__ float xs[kPrepRows][129];               // padded rows: conflict-free reads
   allow_dependent_launch();
-  const int r0 = blockIdx.x * kPrepRows, part = blockIdx.y, o0 = blockIdx.z * 8;
-  const float* M = part == 0 ? PiT : ST;
-  const int t = threadIdx.x, lg = dg == 128 ? 6 : 5;   // log2 of the pairs per row
-  for (int e = t; e < 2 * dg; e += 32)
-    ms4[e >> 1][e & 1] = __ldg(reinterpret_cast<const float4*>(M + (size_t)(e >> 1) * dg + o0) + (e & 1));
-  for (int e = t; e < kPrepRows * dg / 2; e += 32) {
-    const int r = e >> lg, j = 2 * (e & (dg / 2 - 1));
-    float2 v = make_float2(0.f, 0.f);
-    if (r0 + r < nrows) {
-      const size_t row = (size_t)(r0 + r) * ldq;
-      if (perm) {             // the group's channels are perm[kv head][off .. off + dg) of the row
-        const int32_t* pr = perm + (size_t)(((r0 + r) % Hq) / rep) * D + off + j;
-        const int c0 = pr[0], c1 = pr[1];
-        const bool ok0 = c0 >= 0 && c0 < D, ok1 = c1 >= 0 && c1 < D;   // (the merge reports a bad entry)
-        if constexpr (std::is_same<T, float>::value)
-          v = make_float2(ok0 ? __ldg(q + row + c0) : 0.f, ok1 ? __ldg(q + row + c1) : 0.f);
-        else
-          v = make_float2(ok0 ? __bfloat162float(q[row + c0]) : 0.f, ok1 ? __bfloat162float(q[row + c1]) : 0.f);
-      } else {
-        const size_t at = row + off + j;
-        if constexpr (std::is_same<T, float>::value) v = __ldg(reinterpret_cast<const float2*>(q + at));
-        else v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + at));
-      }
-    }
-    qs[r][j] = v.x;
-    qs[r][j + 1] = v.y;
+  const int r0 = blockIdx.x * kPrepRows;
+  const int y = blockIdx.y;                          // (group, part, output block)
+  const int ob = y % A.obs, part = (y / A.obs) & 1, gi = y / (2 * A.obs);
+  const int dg = A.dg, t = threadIdx.x;
+  const float* M = gi ? (part ? A.stt[1] : A.pit[1]) : (part ? A.stt[0] : A.pit[0]);
+  const int off = gi ? A.off[1] : A.off[0];
+  for (int e = t; e < dg * 16; e += 256) {
+    const int j = e >> 4, c4 = e & 15;
+    *reinterpret_cast<float4*>(&ms[j][4 * c4]) =
+        __ldg(reinterpret_cast<const float4*>(M + (size_t)j * dg + 64 * ob) + c4);
   }
-  __syncwarp();
-  const int r = t >> 2, o = 2 * (t & 3);
-  const float2* mcol = reinterpret_cast<const float2*>(ms4) + (t & 3);
-  float a0 = 0.f, a1 = 0.f;
+  for (int e = t; e < kPrepRows * dg; e += 256) {
+    const int r = e / dg, j = e % dg;
+    float v = 0.f;
+    if (r0 + r < A.nrows) {
+      const size_t row = (size_t)(r0 + r) * A.D;
+      int ch = off + j;
+      if (A.perm) ch = __ldg(A.perm + (size_t)(((r0 + r) % A.Hq) / A.rep) * A.D + off + j);
+      if (ch >= 0 && ch < A.D)   // (the merge kernel reports an out-of-range entry)
+        v = A.q_f32 ? __ldg(static_cast<const float*>(A.q) + row + ch)
+                    : __bfloat162float(static_cast<const __nv_bfloat16*>(A.q)[row + ch]);
+    }
+    xs[r][j] = v;
+  }
+  __syncthreads();
+  const int r = t % kPrepRows, og = t / kPrepRows;   // row, output group (4 outputs)
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
   for (int j = 0; j < dg; ++j) {
-    const float2 m = mcol[4 * j];
-    const float x = qs[r][j];
-    a0 = fmaf(m.x, x, a0);
-    a1 = fmaf(m.y, x, a1);
+    const float4 m = *reinterpret_cast<const float4*>(&ms[j][4 * og]);
+    const float x = xs[r][j];
+    a[0] = fmaf(m.x, x, a[0]);
+    a[1] = fmaf(m.y, x, a[1]);
+    a[2] = fmaf(m.z, x, a[2]);
+    a[3] = fmaf(m.w, x, a[3]);
   }
-  if (r0 + r < nrows) {
-    float* dst = qp + ((size_t)(r0 + r) * G + gi) * 2 * D + part * D + o0 + o;
-    dst[0] = a0;
-    dst[1] = a1;
-  }
+  if (r0 + r < A.nrows)
+    *reinterpret_cast<float4*>(A.qp + ((size_t)(r0 + r) * A.G + gi) * 2 * A.D + part * A.D + 64 * ob + 4 * og) =
+        make_float4(a[0], a[1], a[2], a[3]);
 }
 
 // Arguments of the merge kernel (below).
@@ -708,41 +721,69 @@ struct Merge2Args {
 // with one read of every rotation entry (the rotation is read once per CTA, not once per
 // query row and channel block).
 constexpr int kMergeHThreads = 256;
+constexpr int kMergeMaxSplit = 512;       // the split count is at most this (checked at launch)
 
-__global__ void __launch_bounds__(kMergeHThreads) decode_merge_heads_kernel(Merge2Args A) {
-  __shared__ float s_v[kRep][256];           // merged rotated values (<= 256 channels)
-  __shared__ float s_Mw[kRep][2];            // per head: the split maxima of its two warps
+__global__ void __launch_bounds__(kMergeHThreads, 4) decode_merge_heads_kernel(Merge2Args A) {
+  extern __shared__ __align__(16) float s_pi[];   // the value groups' Pi, [dg0^2 | dg1^2] (row-major)
+  __shared__ float s_v[kRep][256];                // merged rotated values (<= 256 channels)
+  __shared__ float s_w[kRep][kMergeMaxSplit];     // per head and split: e^(m_s - M)
+  __shared__ float s_red[kRep][2][2];             // per head: the two warps' maxima, then their sums
   const int D = A.D, ns = A.nsplit, W = D + 2;
   const int bh = blockIdx.x / A.nsub, sub = blockIdx.x % A.nsub;
   const int b = bh / A.Hkv, hk = bh % A.Hkv;
   const int nh = min(kRep, A.rep - sub * kRep);      // query heads of this CTA
   const int row0 = b * A.Hq + hk * A.rep + sub * kRep;
-  const int h = threadIdx.x >> 6, t64 = threadIdx.x & 63;   // head, coordinate lane of the head
-  // pass 1 (after the decode grid is complete): the maximum of the head's split maxima
-  grid_dependency_wait();
-  if (h < nh) {
-    const float* P = A.part + (size_t)(row0 + h) * A.part_ld;
-    float M = -INFINITY;
-    for (int s2 = t64; s2 < ns; s2 += 64) M = fmaxf(M, P[(size_t)s2 * W]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if ((threadIdx.x & 31) == 0) s_Mw[h][(threadIdx.x >> 5) & 1] = M;
+  const int h = threadIdx.x >> 6, t64 = threadIdx.x & 63;   // head, lane of the head
+  const int wh = (threadIdx.x >> 5) & 1;                     // warp of the head
+  // the rotations are constant: staged while the decode grid still runs
+  {
+    const int n0 = (A.off[1] - A.off[0]) * (A.off[1] - A.off[0]);
+    const int n1 = A.G > 1 ? (A.off[2] - A.off[1]) * (A.off[2] - A.off[1]) : 0;
+    for (int e = 4 * threadIdx.x; e < n0 + n1; e += 4 * kMergeHThreads) {
+      const float* src = e < n0 ? A.PiV[0] + e : A.PiV[1] + (e - n0);
+      *reinterpret_cast<float4*>(s_pi + e) = __ldg(reinterpret_cast<const float4*>(src));
+    }
   }
+  grid_dependency_wait();    // every partial of the decode grid is written
+  // pass 1: the head's maximum over the splits, the weights e^(m_s - M) and L = sum_s w_s l_s
+  const float* P = A.part + (size_t)(row0 + min(h, nh - 1)) * A.part_ld;
+  float mloc[kMergeMaxSplit / 64], lloc[kMergeMaxSplit / 64];
+  float M = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kMergeMaxSplit / 64; ++i) {
+    const int s2 = t64 + 64 * i;
+    mloc[i] = s2 < ns ? P[(size_t)s2 * W] : -INFINITY;
+    lloc[i] = s2 < ns ? P[(size_t)s2 * W + 1] : 0.f;
+    M = fmaxf(M, mloc[i]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if ((threadIdx.x & 31) == 0) s_red[h][wh][0] = M;
   __syncthreads();
-  // pass 2: weights e^(m_s - M), the sum L and the merged accumulators of the head
-  if (h < nh) {
-    const float* P = A.part + (size_t)(row0 + h) * A.part_ld;
-    const float M = fmaxf(s_Mw[h][0], s_Mw[h][1]);
-    float L = 0.f;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};           // coordinates t64 + 64 j
+  M = fmaxf(s_red[h][0][0], s_red[h][1][0]);
+  float L = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMergeMaxSplit / 64; ++i) {
+    const int s2 = t64 + 64 * i;
+    const float w = (mloc[i] == -INFINITY) ? 0.f : __expf(mloc[i] - M);
+    if (s2 < ns) s_w[h][s2] = w;
+    L = fmaf(w, lloc[i], L);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  if ((threadIdx.x & 31) == 0) s_red[h][wh][1] = L;
+  __syncthreads();
+  L = s_red[h][0][1] + s_red[h][1][1];
+  // pass 2: the merged accumulators of the head (coordinates t64 + 64 j)
+  {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
     for (int s2 = 0; s2 < ns; ++s2) {
-      const float* ps = P + (size_t)s2 * W;
-      const float m = ps[0];
-      const float w = (m == -INFINITY) ? 0.f : __expf(m - M);
-      L = fmaf(w, ps[1], L);
+      const float* ps = P + (size_t)s2 * W + 2;
+      const float w = s_w[h][s2];
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        if (t64 + 64 * j < D) acc[j] = fmaf(w, ps[2 + t64 + 64 * j], acc[j]);
+        if (t64 + 64 * j < D) acc[j] = fmaf(w, ps[t64 + 64 * j], acc[j]);
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j)
@@ -751,41 +792,36 @@ __global__ void __launch_bounds__(kMergeHThreads) decode_merge_heads_kernel(Merg
   __syncthreads();
   // inverse rotation of each group: out[ch] = sum_i Pi_g[i][ch - off] v[off + i]
   for (int c = threadIdx.x; c < D; c += blockDim.x) {
-    const int gsel = (A.G > 1 && c >= A.off[1]) ? 1 : 0;
-    const int goff = A.off[gsel], gd = A.off[gsel + 1] - goff;
-    const float* Pi = A.PiV[gsel] + (c - goff);
+    const bool second = A.G > 1 && c >= A.off[1];
+    const int goff = second ? A.off[1] : A.off[0], gd = (second ? A.off[2] : A.off[1]) - goff;
+    const float* Pi = s_pi + (second ? (A.off[1] - A.off[0]) * (A.off[1] - A.off[0]) : 0) + (c - goff);
     float o[kRep] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
     for (int i = 0; i < gd; ++i) {
-      const float pv = __ldg(Pi + (size_t)i * gd);
+      const float pv = Pi[i * gd];
 #pragma unroll
       for (int hh = 0; hh < kRep; ++hh) o[hh] = fmaf(pv, s_v[hh][goff + i], o[hh]);
     }
-    for (int hh = 0; hh < nh; ++hh) {
-      const int row = row0 + hh;
-      const int oc_ch = A.perm ? A.perm[(size_t)hk * D + c] : c;
-      if (oc_ch >= 0 && oc_ch < D) A.out[(size_t)row * D + oc_ch] = o[hh];
-      else if (A.err) atomicCAS(A.err, 0, (int)kErrPermRange);
+    const int oc_ch = A.perm ? A.perm[(size_t)hk * D + c] : c;
+    if (oc_ch < 0 || oc_ch >= D) {
+      if (A.err) atomicCAS(A.err, 0, (int)kErrPermRange);
+      continue;
     }
+#pragma unroll
+    for (int hh = 0; hh < kRep; ++hh)
+      if (hh < nh) A.out[(size_t)(row0 + hh) * D + oc_ch] = o[hh];
   }
 }
 
-// Rotated queries of nrows rows for one group.
-int launch_prep(const void* q, int q_dtype, int ldq, int off, int dg, int nrows, const tq_ctx* kc, float* qp, int D,
-                int G, int gi, const int32_t* perm, int Hq, int rep, cudaStream_t st) {
-  const dim3 grid((nrows + kPrepRows - 1) / kPrepRows, 2, dg / 8);
-  cudaError_t e = q_dtype == TQ_DTYPE_F32
-                      ? cudaFuncSetAttribute(decode_prep_kernel<float>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                             cudaSharedmemCarveoutMaxShared)
-                      : cudaFuncSetAttribute(decode_prep_kernel<__nv_bfloat16>,
-                                             cudaFuncAttributePreferredSharedMemoryCarveout,
-                                             cudaSharedmemCarveoutMaxShared);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_prep_kernel carveout)");
-  if (q_dtype == TQ_DTYPE_F32)
-    decode_prep_kernel<float><<<grid, 32, 0, st>>>(static_cast<const float*>(q), ldq, off, dg, nrows, kc->PiT,
-                                                    kc->ST, qp, D, G, gi, perm, Hq, rep);
-  else
-    decode_prep_kernel<__nv_bfloat16><<<grid, 32, 0, st>>>(static_cast<const __nv_bfloat16*>(q), ldq, off, dg,
-                                                            nrows, kc->PiT, kc->ST, qp, D, G, gi, perm, Hq, rep);
+// Rotated queries of all groups (one launch).
+int launch_prep(const void* q, int q_dtype, int nrows, const tq_ctx* const* kctx, const int* off, int G, float* qp,
+                int D, const int32_t* perm, int Hq, int rep, cudaStream_t st) {
+  PrepArgs P{};
+  P.q = q; P.q_f32 = q_dtype == TQ_DTYPE_F32; P.nrows = nrows; P.D = D; P.G = G; P.Hq = Hq; P.rep = rep;
+  P.dg = kctx[0]->lay.d; P.obs = P.dg / 64; P.perm = perm; P.qp = qp;
+  for (int g = 0; g < G; ++g) { P.off[g] = off[g]; P.pit[g] = kctx[g]->PiT; P.stt[g] = kctx[g]->ST; }
+  const dim3 grid((nrows + kPrepRows - 1) / kPrepRows, G * 2 * P.obs);
+  decode_prep_kernel<<<grid, 256, 0, st>>>(P);
   count_launch();
   return check_launch("decode_prep_kernel");
 }
@@ -1018,12 +1054,12 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
       return kNotHandled;
 
   const DecodeWs W = decode_ws(B, Hq, Hkv, D, G, max_len);
-  if (W.nsplit > 512) return kNotHandled;
+  if (W.nsplit > kMergeMaxSplit) return kNotHandled;
   char* base = static_cast<char*>(ws);
   float* qp = reinterpret_cast<float*>(base + W.qp);
   float* part = reinterpret_cast<float*>(base + W.part);
-  for (int g = 0; g < G; ++g) {
-    int r = launch_prep(q, q_dtype, D, off[g], kctx[g]->lay.d, B * Hq, kctx[g], qp, D, G, g, perm, Hq, Hq / Hkv, st);
+  {   // every group of an instantiated kernel has the same width (64 or 128)
+    int r = launch_prep(q, q_dtype, B * Hq, kctx, off, G, qp, D, perm, Hq, Hq / Hkv, st);
     if (r != TQ_OK) return r;
   }
   MmaArgs A{};
@@ -1068,13 +1104,18 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
   M.off[G] = D;
   M.Hkv = Hkv;
   M.nsub = A.nsub;
-  cudaError_t em = cudaFuncSetAttribute(decode_merge_heads_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                        cudaSharedmemCarveoutMaxShared);
+  int pi_floats = 0;
+  for (int g = 0; g < G; ++g) pi_floats += (M.off[g + 1] - M.off[g]) * (M.off[g + 1] - M.off[g]);
+  const int mdyn = pi_floats * (int)sizeof(float);
+  cudaError_t em = cudaFuncSetAttribute(decode_merge_heads_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mdyn);
+  if (em == cudaSuccess)
+    em = cudaFuncSetAttribute(decode_merge_heads_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              cudaSharedmemCarveoutMaxShared);
   if (em != cudaSuccess) return cuda_fail(em, "cudaFuncSetAttribute(decode_merge_heads_kernel)");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(B * Hkv * A.nsub);
   cfg.blockDim = dim3(kMergeHThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = mdyn;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -42,6 +42,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// try_wait with a suspend-time hint: a thread whose phase is not complete sleeps up to
+// hint_ns nanoseconds (or until the phase completes) instead of returning at once, so a
+// waiting warp does not take issue slots from the warps that are working.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
@@ -50,6 +62,17 @@ __device__ __forceinline__ uint64_t global_ns() {
 // Wait for the phase with the given parity to complete.  Gives up (returns false) after
 // limit_ns nanoseconds, or as soon as *abort becomes non-zero when abort is given, so a
 // stuck pipeline always winds down instead of spinning forever.
+// mbar_wait for waits that are often long: every retry sleeps (hint_ns) instead of spinning.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                                uint64_t limit_ns, uint32_t hint_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, hint_ns)) return true;
+    if (abort && *abort) return false;
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+}
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
                                           uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
