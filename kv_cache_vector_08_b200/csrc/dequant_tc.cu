@@ -221,17 +221,17 @@ __global__ void __launch_bounds__(kDqThreads, 1) dequant_tc_kernel(const __grid_
       const int b = t & 1;
       if (!wait(d_full + b, (uint32_t)((t >> 1) & 1))) { fail(303); return false; }
       tc_fence_after();
+      // all of the row's column chunks are requested before one wait (one TMEM round trip)
+      uint32_t r[4][16];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (ch_lo + c < ch_hi) tmem_ld16(lane_base + (uint32_t)(b * 128 + 16 * (ch_lo + c)), r[c]);
+      tmem_ld_wait();
       float acc[4][16];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (ch_lo + c < ch_hi) {
-          uint32_t r[16];
-          tmem_ld16(lane_base + (uint32_t)(b * 128 + 16 * (ch_lo + c)), r);
-          tmem_ld_wait();
+      for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int i = 0; i < 16; ++i) acc[c][i] = __uint_as_float(r[i]);
-        }
-      }
+        for (int i = 0; i < 16; ++i) acc[c][i] = __uint_as_float(r[c][i]);
       tc_fence_before();
       mbar_arrive(d_empty + b);
       if (v < A.n) {
