@@ -472,19 +472,33 @@ def workload_config(w, kind, ws):
 
 
 # ---------------------------------------------------------------- other workloads
-def _time_device(fn, flush, reps, warm=1):
-    """Mean device time (s) of fn() over reps, L2 flushed before every rep."""
+def _time_device(fn, flush, reps, warm=1, graph=False):
+    """Mean device time (s) of fn() over reps, L2 flushed before every rep.  graph=True
+    captures fn once in a CUDA graph and times its replays, so that the host's launch
+    latency (Python, ctypes) of a short call is not counted as device time."""
     import torch
     st = torch.cuda.current_stream()
     for _ in range(warm):
         fn()
     torch.cuda.synchronize()
+    run = fn
+    if graph:
+        side = torch.cuda.Stream()
+        side.wait_stream(st)
+        with torch.cuda.stream(side):
+            fn()
+        st.wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        run = g.replay
     ts = []
     for _ in range(reps):
         flush(st)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(st)
-        fn()
+        run()
         b.record(st)
         ts.append((a, b))
     torch.cuda.synchronize()
@@ -632,7 +646,8 @@ def measure_decode_config(kind, dev, peaks, steps=10):
 
 def measure_rows(bench, peaks, reps=5):
     """Standalone logits (4 queries x every cached key of group 0) and dequantize (every
-    cached value vector of group 0) on a decode workload's caches."""
+    cached value vector of group 0) on a decode workload's caches; device time of CUDA-graph
+    replays of the library call."""
     import torch
     tq, dev = bench.tq, bench.dev
     out = {}
@@ -642,19 +657,19 @@ def measure_rows(bench, peaks, reps=5):
     lg = torch.empty((4, n), dtype=torch.float32, device=dev)
     ws = torch.empty(max(int(tq.lib().tq_attn_logits_workspace_size(kctx.handle, 4)), 1), dtype=torch.uint8,
                      device=dev)
-    t = _time_device(lambda: tq.attn_logits(kctx, q4, kc, n, out=lg, workspace=ws), bench.flush_l2, reps)
+    t = _time_device(lambda: tq.attn_logits(kctx, q4, kc, n, out=lg, workspace=ws), bench.flush_l2, reps, graph=True)
     nbytes = n * (kctx.code_bytes + 4) + 4 * n * 4
     out["logits"] = hbm_roof(nbytes, t, peaks, "attn_logits",
                              work="4 queries x %d keys (d=%d, %d-bit prod)" % (n, kctx.d, kctx.bits))
     vctx, vc = bench.vctx[0], bench.vc[0]
     xo = torch.empty((n, vctx.d), dtype=torch.float32, device=dev)
-    t = _time_device(lambda: tq.dequantize(vctx, vc, n, out=xo), bench.flush_l2, reps)
+    t = _time_device(lambda: tq.dequantize(vctx, vc, n, out=xo), bench.flush_l2, reps, graph=True)
     nbytes = n * (vctx.code_bytes + 2) + n * vctx.d * 4
     out["dequantize"] = hbm_roof(nbytes, t, peaks, "dequantize",
                                  work="%d value vectors (d=%d, %d-bit MSE) -> fp32" % (n, vctx.d, vctx.bits),
                                  algorithmic_tflops=2.0 * vctx.d * vctx.d * n / t / 1e12)
     kq = torch.empty((n, kctx.d), dtype=torch.float32, device=dev)
-    t = _time_device(lambda: tq.dequantize(kctx, kc, n, out=kq, qjl=True), bench.flush_l2, reps)
+    t = _time_device(lambda: tq.dequantize(kctx, kc, n, out=kq, qjl=True), bench.flush_l2, reps, graph=True)
     nbytes = n * (kctx.code_bytes + 4) + n * kctx.d * 4
     out["dequantize_qjl"] = hbm_roof(nbytes, t, peaks, "dequantize_qjl",
                                      work="%d key vectors (d=%d, %d-bit prod) -> fp32, QJL-augmented" % (
@@ -882,7 +897,7 @@ def run_reference(args):
 
 
 # ------------------------------------------------------- small cases for profilers
-KERNEL_CASES = ("decode-serving-b16", "search-d1536-200k", "dequant-d128", "quantize-fp32-d1536")
+KERNEL_CASES = ("decode-serving-b16", "search-d1536-200k", "dequant-d128", "quantize-fp32-d1536", "logits-d128")
 
 
 def run_kernel_case(args):
@@ -936,6 +951,18 @@ def run_kernel_case(args):
         out = torch.empty((n, d), device=dev)
         us = timed(lambda: tq.dequantize(ctx, pk, n, out=out))
         note = "%.0f GB/s (66 + 512 B per vector)" % (n * (66 + 512) / us / 1e3)
+    elif case == "logits-d128":
+        d, n, nq = 128, 262144, 4
+        x = torch.randn((n, d), generator=g, device=dev).to(torch.bfloat16)
+        ctx = tq.Context(d, 4, 1000, tq.MODE_PROD)
+        pk = tq.alloc_packed(ctx, n)
+        tq.quantize_kv(ctx, x, pk)
+        q4 = torch.randn((nq, d), generator=g, device=dev)
+        lg = torch.empty((nq, n), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(int(tq.lib().tq_attn_logits_workspace_size(ctx.handle, nq)), 1), dtype=torch.uint8,
+                         device=dev)
+        us = timed(lambda: tq.attn_logits(ctx, q4, pk, n, out=lg, workspace=ws))
+        note = "%.0f GB/s (68 B of codes and norms + 16 B of logits per key)" % (n * 84 / us / 1e3)
     else:   # quantize-fp32-d1536
         d, n = 1536, 32768
         x = torch.nn.functional.normalize(torch.randn((n, d), generator=g, device=dev), dim=1)

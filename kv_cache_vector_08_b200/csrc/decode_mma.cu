@@ -917,18 +917,35 @@ __global__ void __launch_bounds__(128) logits_mma_kernel(LogitArgs A) {
   const int64_t k0 = (int64_t)blockIdx.x * A.keys_per_cta;
   const int64_t k1 = min(A.n, k0 + A.keys_per_cta);
   const int qi = qb * kRep + l;
-  for (int64_t base = k0 + warp * 16; base < k1; base += 64) {
+  // the next tile's code words and norms are loaded before this tile is computed, so the
+  // global-memory latency overlaps the tensor-core work
+  struct Tile {
+    Words<GC::DG, GC::PK> wa, wb;
+    float na, ra, nb, rb;
+  };
+  auto load = [&](int64_t base, Tile& T) {
     const int64_t ka = base + g, kb = base + g + 8;
     const bool va = ka < k1, vb = kb < k1;
-    Words<GC::DG, GC::PK> wa, wb;
 #pragma unroll
-    for (int i = 0; i < Words<GC::DG, GC::PK>::N; ++i) wa.w[i] = wb.w[i] = 0u;
-    if (va) ldg_words(wa, A.codes + ka * GC::KB, l);
-    if (vb) ldg_words(wb, A.codes + kb * GC::KB, l);
+    for (int i = 0; i < Words<GC::DG, GC::PK>::N; ++i) T.wa.w[i] = T.wb.w[i] = 0u;
+    if (va) ldg_words(T.wa, A.codes + ka * GC::KB, l);
+    if (vb) ldg_words(T.wb, A.codes + kb * GC::KB, l);
+    T.na = va ? h2f(__ldg(A.norm + ka)) : 0.f;
+    T.ra = va ? h2f(__ldg(A.rnorm + ka)) : 0.f;
+    T.nb = vb ? h2f(__ldg(A.norm + kb)) : 0.f;
+    T.rb = vb ? h2f(__ldg(A.rnorm + kb)) : 0.f;
+  };
+  Tile cur, nxt;
+  int64_t base = k0 + warp * 16;
+  if (base < k1) load(base, cur);
+  for (; base < k1; base += 64) {
+    if (base + 64 < k1) load(base + 64, nxt);
+    const int64_t ka = base + g, kb = base + g + 8;
+    const bool va = ka < k1, vb = kb < k1;
     float mse[4] = {0.f, 0.f, 0.f, 0.f}, sgn[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int u = 0; u < GC::NS; ++u) {
-      const uint32_t sa = low_sel(wa, u), sb = low_sel(wb, u);
+      const uint32_t sa = low_sel(cur.wa, u), sb = low_sel(cur.wb, u);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const uint32_t xa = h ? sa >> 16 : sa, xb = h ? sb >> 16 : sb;
@@ -939,28 +956,27 @@ __global__ void __launch_bounds__(128) logits_mma_kernel(LogitArgs A) {
         lookup16(A.cl, xa, a01, a23);
         lookup16(A.cl, xb, b01, b23);
         mma16816(mse, a01, b01, a23, b23, bm[u][h][0], bm[u][h][1]);
-        signs16(top_bits(wa, u, h), a01, a23);
-        signs16(top_bits(wb, u, h), b01, b23);
+        signs16(top_bits(cur.wa, u, h), a01, a23);
+        signs16(top_bits(cur.wb, u, h), b01, b23);
         mma16816(sgn, a01, b01, a23, b23, bs[u][h][0], bs[u][h][1]);
       }
     }
-    const float na = va ? h2f(__ldg(A.norm + ka)) : 0.f, ra = va ? h2f(__ldg(A.rnorm + ka)) : 0.f;
-    const float nb = vb ? h2f(__ldg(A.norm + kb)) : 0.f, rb = vb ? h2f(__ldg(A.rnorm + kb)) : 0.f;
-    const float la = na * fmaf(A.coef * ra, sgn[0] + sgn[1], mse[0] + mse[1]);
-    const float lb = nb * fmaf(A.coef * rb, sgn[2] + sgn[3], mse[2] + mse[3]);
+    const float la = cur.na * fmaf(A.coef * cur.ra, sgn[0] + sgn[1], mse[0] + mse[1]);
+    const float lb = cur.nb * fmaf(A.coef * cur.rb, sgn[2] + sgn[3], mse[2] + mse[3]);
     if (qi < A.nq) {
       if (va) A.out[(size_t)qi * A.n + ka] = la;
       if (vb) A.out[(size_t)qi * A.n + kb] = lb;
     }
+    cur = nxt;
   }
 }
 
 template <class GC>
 int launch_logits_t(LogitArgs A, cudaStream_t st) {
   const int nqb = (A.nq + kRep - 1) / kRep;
-  // about 4 CTAs per SM in total (the query fragments are built once per CTA), whole
+  // about 8 CTAs per SM in total (the query fragments are built once per CTA), whole
   // 64-key steps per CTA
-  int64_t ctas = (int64_t)148 * 4 / nqb;
+  int64_t ctas = (int64_t)148 * 8 / nqb;
   if (ctas < 1) ctas = 1;
   int64_t per = (A.n + ctas - 1) / ctas;
   per = ((per + 63) / 64) * 64;
