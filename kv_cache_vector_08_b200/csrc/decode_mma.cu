@@ -777,8 +777,8 @@ __global__ void __launch_bounds__(kMergeHThreads, 4) decode_merge_heads_kernel(M
   // pass 2: the merged accumulators of the head (coordinates t64 + 64 j)
   {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int s2 = 0; s2 < ns; ++s2) {
+#pragma unroll 8
+    for (int s2 = 0; s2 < ns; ++s2) {   // (8 splits' loads in flight: long split lists are latency-bound)
       const float* ps = P + (size_t)s2 * W + 2;
       const float w = s_w[h][s2];
 #pragma unroll

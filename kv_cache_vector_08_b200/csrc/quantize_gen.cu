@@ -331,6 +331,26 @@ __global__ void __launch_bounds__(kGenThreads, 1) quantize_gemm_kernel(const __g
       int nb, width;
       unit_of(t, mt, nb, width);
       const bool g0 = 64 * part < width, g1 = 64 * part + 32 < width;   // this thread's code groups
+      // the row's slot and scale (and, for the sign pass, its code words and the parts of
+      // ||r||^2) are loaded before the accumulation, so their latency hides under it
+      const int64_t r = mt * kGenTile + row;              // row within the chunk
+      int64_t slot = r < A.n ? (A.slots ? A.slots[A.row0 + r] : A.row0 + r) : 0;
+      const bool live = r < A.n && slot >= 0 && slot < A.cap;   // (the prep kernel reported a bad slot)
+      if (!live) slot = 0;
+      const RowInfo ri = live ? A.info[r] : RowInfo{0.f, 0.f};
+      uint32_t* rec = reinterpret_cast<uint32_t*>(A.codes + slot * (int64_t)A.code_bytes);
+      uint32_t old[2][P];
+      float rn2_all = 0.f;
+      if constexpr (SIGN) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int grp = (nb * kGenNb) / 32 + 2 * part + h;
+#pragma unroll
+          for (int p = 0; p < P; ++p) old[h][p] = (live && (h ? g1 : g0)) ? rec[grp * P + p] : 0u;
+        }
+        if (live && nb == 0 && part == 0)
+          for (int j = 0; j < 4 * A.NB; ++j) rn2_all += A.rn2[r * A.NB * 4 + j];
+      }
       float acc[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) acc[i] = 0.f;
@@ -352,12 +372,6 @@ __global__ void __launch_bounds__(kGenThreads, 1) quantize_gemm_kernel(const __g
         mbar_arrive(acc_empty + b);
       }
       if (!ok) break;
-      const int64_t r = mt * kGenTile + row;              // row within the chunk
-      int64_t slot = r < A.n ? (A.slots ? A.slots[A.row0 + r] : A.row0 + r) : 0;
-      const bool live = r < A.n && slot >= 0 && slot < A.cap;   // (the prep kernel reported a bad slot)
-      if (!live) slot = 0;
-      const RowInfo ri = live ? A.info[r] : RowInfo{0.f, 0.f};
-      uint32_t* rec = reinterpret_cast<uint32_t*>(A.codes + slot * (int64_t)A.code_bytes);
       float rn2 = 0.f;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -424,18 +438,15 @@ __global__ void __launch_bounds__(kGenThreads, 1) quantize_gemm_kernel(const __g
           }
           if (live)
 #pragma unroll
-            for (int p = 0; p < P; ++p) rec[grp * P + p] |= w[p];
+            for (int p = 0; p < P; ++p) rec[grp * P + p] = old[h][p] | w[p];
         }
       }
       if constexpr (!SIGN) {
         // partial ||r||^2 of this thread's columns: 4 parts per N block
         if (PROD && live) A.rn2[(r * A.NB + nb) * 4 + part] = rn2;
       } else {
-        if (live && nb == 0 && part == 0) {
-          float sum = 0.f;
-          for (int j = 0; j < 4 * A.NB; ++j) sum += A.rn2[r * A.NB * 4 + j];
-          A.rnorm[slot] = ri.nrm > 0.f ? __half_as_ushort(__float2half_rn(sqrtf(sum))) : (uint16_t)0;
-        }
+        if (live && nb == 0 && part == 0)
+          A.rnorm[slot] = ri.nrm > 0.f ? __half_as_ushort(__float2half_rn(sqrtf(rn2_all))) : (uint16_t)0;
       }
     }
   }
