@@ -638,17 +638,17 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, TQ_DECODE_CTAS_PER_SM) deco
 
 // Rotated queries Pi q and S q of every group in fp32 (the fixed-point digits are formed by
 // the consumer warps of the decode kernel, which see a whole head row), one launch for all
-// groups.  CTA = 16 query rows x 64 outputs of one (group, part): the 64 columns of Pi^T
+// groups.  CTA = 16 query rows x 16 outputs of one (group, part): the 16 columns of Pi^T
 // (part 0) or S^T (part 1) and the 16 rows (channels gathered through the permutation) are
-// staged in shared memory with one round of loads; thread (row, 4 outputs) runs 4 dot
-// products of d_g terms.  The decode kernel is launched behind it and starts streaming the
+// staged in shared memory with one round of loads; thread (row, 4 outputs, K quarter) runs
+// 4 dot products over a quarter of the d_g terms and the quarters are summed by shuffles.  The decode kernel is launched behind it and starts streaming the
 // cache at once; its consumer warps wait for this grid before reading the projections.
 constexpr int kPrepRows = 16;
 
 struct PrepArgs {
   const void* q;
   int q_f32;
-  int nrows, D, G, Hq, rep, dg, obs;   // obs: 64-output blocks per group
+  int nrows, D, G, Hq, rep, dg, obs;   // obs: output blocks (16 or 64 outputs) per group
   const int32_t* perm;                 // [Hkv][D] channel permutation or NULL
   int off[2];
   const float* pit[2];
@@ -657,6 +657,61 @@ struct PrepArgs {
 };
 
 __global__ void __launch_bounds__(256) decode_prep_kernel(PrepArgs A) {
+  __shared__ __align__(16) float ms[128][16];        // [j][o]: M^T[j][16 ob + o]
+  __shared__ float xs[kPrepRows][129];               // padded rows
+  allow_dependent_launch();
+  const int r0 = blockIdx.x * kPrepRows;
+  const int y = blockIdx.y;                          // (group, part, 16-output block)
+  const int ob = y % A.obs, part = (y / A.obs) & 1, gi = y / (2 * A.obs);
+  const int dg = A.dg, t = threadIdx.x;
+  const float* M = gi ? (part ? A.stt[1] : A.pit[1]) : (part ? A.stt[0] : A.pit[0]);
+  const int off = gi ? A.off[1] : A.off[0];
+  for (int e = t; e < dg * 4; e += 256) {
+    const int jj = e >> 2, c4 = e & 3;
+    *reinterpret_cast<float4*>(&ms[jj][4 * c4]) =
+        __ldg(reinterpret_cast<const float4*>(M + (size_t)jj * dg + 16 * ob) + c4);
+  }
+  for (int e = t; e < kPrepRows * dg; e += 256) {
+    const int r = e / dg, jj = e % dg;
+    float v = 0.f;
+    if (r0 + r < A.nrows) {
+      const size_t row = (size_t)(r0 + r) * A.D;
+      int ch = off + jj;
+      if (A.perm) ch = __ldg(A.perm + (size_t)(((r0 + r) % A.Hq) / A.rep) * A.D + off + jj);
+      if (ch >= 0 && ch < A.D)   // (the merge kernel reports an out-of-range entry)
+        v = A.q_f32 ? __ldg(static_cast<const float*>(A.q) + row + ch)
+                    : __bfloat162float(static_cast<const __nv_bfloat16*>(A.q)[row + ch]);
+    }
+    xs[r][jj] = v;
+  }
+  __syncthreads();
+  // thread = (row, 4-output group, K quarter): terms j = 4 i + kq, then the four quarters
+  // (adjacent lanes) are summed by shuffles
+  const int kq = t & 3, og = (t >> 2) & 3, r = t >> 4;
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+  for (int jj = kq; jj < dg; jj += 4) {
+    const float4 m = *reinterpret_cast<const float4*>(&ms[jj][4 * og]);
+    const float x = xs[r][jj];
+    a[0] = fmaf(m.x, x, a[0]);
+    a[1] = fmaf(m.y, x, a[1]);
+    a[2] = fmaf(m.z, x, a[2]);
+    a[3] = fmaf(m.w, x, a[3]);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    a[k] += __shfl_xor_sync(0xffffffffu, a[k], 1);
+    a[k] += __shfl_xor_sync(0xffffffffu, a[k], 2);
+  }
+  if (kq == 0 && r0 + r < A.nrows)
+    *reinterpret_cast<float4*>(A.qp + ((size_t)(r0 + r) * A.G + gi) * 2 * A.D + part * A.D + 16 * ob + 4 * og) =
+        make_float4(a[0], a[1], a[2], a[3]);
+}
+
+// The same projection for many query rows: CTA = 16 rows x 64 outputs, thread = (row, 4
+// outputs) over all d_g terms; four times fewer CTAs than the 16-output form, so that a
+// large batch's prep leaves the SMs to the decode kernel sooner.
+__global__ void __launch_bounds__(256) decode_prep_wide_kernel(PrepArgs A) {
   __shared__ __align__(16) float ms[128][64];        // [j][o]: M^T[j][64 ob + o]
   __shared__ float xs[kPrepRows][129];               // padded rows: conflict-free reads
   allow_dependent_launch();
@@ -711,6 +766,8 @@ struct Merge2Args {
   float* out;
   const int32_t* perm;   // channel permutation [Hkv][D] (NULL: identity): group channel c -> perm[kv][c]
   int Hq, rep, Hkv, nsub;
+  int pi_floats;         // floats of the staged rotations (a multiple of 4)
+  int stage_parts;       // copy the CTA's split partials into shared memory first (they fit)
   int* err;
 };
 
@@ -735,6 +792,13 @@ __global__ void __launch_bounds__(kMergeHThreads, 4) decode_merge_heads_kernel(M
   const int row0 = b * A.Hq + hk * A.rep + sub * kRep;
   const int h = threadIdx.x >> 6, t64 = threadIdx.x & 63;   // head, lane of the head
   const int wh = (threadIdx.x >> 5) & 1;                     // warp of the head
+  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ int s_ok;
+  if (threadIdx.x == 0) {
+    mbar_init(&s_bar, 1);
+    s_ok = 1;
+    fence_barrier_init();
+  }
   // the rotations are constant: staged while the decode grid still runs
   {
     const int n0 = (A.off[1] - A.off[0]) * (A.off[1] - A.off[0]);
@@ -744,9 +808,29 @@ __global__ void __launch_bounds__(kMergeHThreads, 4) decode_merge_heads_kernel(M
       *reinterpret_cast<float4*>(s_pi + e) = __ldg(reinterpret_cast<const float4*>(src));
     }
   }
+  __syncthreads();
   grid_dependency_wait();    // every partial of the decode grid is written
+  // With few splits the CTA's partial rows (nh rows of part_ld floats, 16-byte multiples)
+  // come into shared memory by bulk copies in one round trip; the passes below then read
+  // shared memory instead of making a dependent global round trip per split.
+  float* s_parts = s_pi + A.pi_floats;
+  if (A.stage_parts) {
+    if (threadIdx.x == 0) {
+      const uint32_t bytes = (uint32_t)(A.part_ld * sizeof(float));
+      mbar_arrive_expect_tx(&s_bar, bytes * (uint32_t)nh);
+      for (int hh = 0; hh < nh; ++hh)
+        bulk_load(s_parts + (size_t)hh * A.part_ld, A.part + (size_t)(row0 + hh) * A.part_ld, bytes, &s_bar);
+      if (!mbar_wait(&s_bar, 0, nullptr, kDecWaitNs)) {
+        s_ok = 0;
+        if (A.err) atomicCAS(A.err, 0, 203);
+      }
+    }
+    __syncthreads();
+    if (!s_ok) return;   // (every thread of the CTA leaves here)
+  }
   // pass 1: the head's maximum over the splits, the weights e^(m_s - M) and L = sum_s w_s l_s
-  const float* P = A.part + (size_t)(row0 + min(h, nh - 1)) * A.part_ld;
+  const float* P = A.stage_parts ? s_parts + (size_t)min(h, nh - 1) * A.part_ld
+                                 : A.part + (size_t)(row0 + min(h, nh - 1)) * A.part_ld;
   float mloc[kMergeMaxSplit / 64], lloc[kMergeMaxSplit / 64];
   float M = -INFINITY;
 #pragma unroll
@@ -818,10 +902,16 @@ int launch_prep(const void* q, int q_dtype, int nrows, const tq_ctx* const* kctx
                 int D, const int32_t* perm, int Hq, int rep, cudaStream_t st) {
   PrepArgs P{};
   P.q = q; P.q_f32 = q_dtype == TQ_DTYPE_F32; P.nrows = nrows; P.D = D; P.G = G; P.Hq = Hq; P.rep = rep;
-  P.dg = kctx[0]->lay.d; P.obs = P.dg / 64; P.perm = perm; P.qp = qp;
+  P.dg = kctx[0]->lay.d; P.obs = P.dg / 16; P.perm = perm; P.qp = qp;
   for (int g = 0; g < G; ++g) { P.off[g] = off[g]; P.pit[g] = kctx[g]->PiT; P.stt[g] = kctx[g]->ST; }
-  const dim3 grid((nrows + kPrepRows - 1) / kPrepRows, G * 2 * P.obs);
-  decode_prep_kernel<<<grid, 256, 0, st>>>(P);
+  if (nrows > 256) {
+    P.obs = P.dg / 64;
+    const dim3 grid((nrows + kPrepRows - 1) / kPrepRows, G * 2 * P.obs);
+    decode_prep_wide_kernel<<<grid, 256, 0, st>>>(P);
+  } else {
+    const dim3 grid((nrows + kPrepRows - 1) / kPrepRows, G * 2 * P.obs);
+    decode_prep_kernel<<<grid, 256, 0, st>>>(P);
+  }
   count_launch();
   return check_launch("decode_prep_kernel");
 }
@@ -1122,7 +1212,10 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
   M.nsub = A.nsub;
   int pi_floats = 0;
   for (int g = 0; g < G; ++g) pi_floats += (M.off[g + 1] - M.off[g]) * (M.off[g + 1] - M.off[g]);
-  const int mdyn = pi_floats * (int)sizeof(float);
+  M.pi_floats = pi_floats;
+  const int64_t parts_bytes = (int64_t)kRep * W.part_ld * (int64_t)sizeof(float);
+  M.stage_parts = parts_bytes <= 128 * 1024 ? 1 : 0;
+  const int mdyn = pi_floats * (int)sizeof(float) + (M.stage_parts ? (int)parts_bytes : 0);
   cudaError_t em = cudaFuncSetAttribute(decode_merge_heads_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mdyn);
   if (em == cudaSuccess)
     em = cudaFuncSetAttribute(decode_merge_heads_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
