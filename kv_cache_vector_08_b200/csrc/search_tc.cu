@@ -15,14 +15,16 @@
 // so +-||r|| is exact; the centroids and the query carry fp16 rounding (2^-11 relative),
 // which moves a unit-vector score by ~1e-5.
 //
-// Roles (448 threads per CTA, one CTA per SM for a fixed query tile): warp 0 stages the
-// query atoms by TMA; warp 1 owns TMEM (two 256-column accumulators) and issues the
-// MMAs; warps 2-9 decode database atoms (thread = database row: code words -> fp16 by
-// byte-permute table lookups -> 128-byte-swizzled shared memory) and stage the chunk's
-// norms; warps 10-13 are the epilogue (thread = query: its 256 scores of the chunk from
-// TMEM, a running per-query top-k list in shared memory with the k-th score as threshold).
-// At the end every CTA writes its lists as candidates; the search merge kernel takes the
-// top-k of each query over the CTAs of its query tile.  Every wait is bounded; a timeout
+// Roles (576 threads per CTA, one CTA per SM for a fixed query tile): warp 0 stages the
+// query atoms by TMA (and, for 4-bit codes, the chunk's code words into a ring); warp 1
+// owns TMEM (two 256-column accumulators) and issues the MMAs; warps 2-9 decode database
+// atoms (thread = database row: code words -> fp16 by byte-permute table lookups ->
+// 128-byte-swizzled shared memory) and stage the chunk's norms; warps 10-17 are the
+// epilogue (thread = query x half of the chunk's columns when k <= 32, else query x all
+// of them on warps 10-13: scores from TMEM, a running top-k list in shared memory with
+// the k-th score as threshold).
+// At the end every list is written as candidates; the search merge kernel takes the top-k
+// of each query over the lists of its query tile.  Every wait is bounded; a timeout
 // records an error code in the context's error word and the CTA winds down.
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -48,7 +50,8 @@ constexpr int kSqStages = 2;
 constexpr int kSqCStages = 4;             // ring of code tiles (4-bit codes): 256 rows x 32 bytes each
 constexpr int kSqCStage = kSqN * 32;
 constexpr int kSqDecWarps = 8;
-constexpr int kSqEpiWarps = 4;
+constexpr int kSqEpiWarps = 8;            // two per TMEM lane quarter: each takes half of a chunk's columns
+constexpr int kSqHalfK = 32;               // the two halves keep separate lists when k <= this
 constexpr int kSqThreads = 64 + 32 * (kSqDecWarps + kSqEpiWarps);
 constexpr int kSqMaxK = 64;
 constexpr uint64_t kSqWaitNs = 2000000000ull;
@@ -63,8 +66,9 @@ struct SqArgs {
   int64_t N;                 // database vectors
   int nq, d, Kh, code_bytes, k;
   int cpq;                   // CTAs per query tile
+  int halves;                // epilogue lists per query and CTA (2 when k <= kSqHalfK, else 1)
   int64_t nchunks;
-  float* cand_s;             // [nq][cpq * k]
+  float* cand_s;             // [nq][cpq * halves * k]
   int64_t* cand_i;
   uint32_t ctab_lo[2], ctab_hi[2];   // 3-bit (neg, magnitude) code -> signed centroid fp16 bytes (P = 4)
   uint32_t ctab[32];                 // P-bit code -> signed centroid fp16 (other P)
@@ -106,7 +110,7 @@ __global__ void __launch_bounds__(kSqThreads, 1) search_tc_kernel(const __grid_c
   const int nloc = (int)((A.nchunks - cslot + A.cpq - 1) / A.cpq);
   const int KA = 2 * A.Kh / 64;                     // atoms per chunk (centroid + sign)
   constexpr int kDecThreads = 32 * kSqDecWarps;
-  constexpr int kEpiThreads = 32 * kSqEpiWarps;
+  const int kEpiThreads = 32 * (A.halves == 2 ? kSqEpiWarps : kSqEpiWarps / 2);   // active epilogue threads
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSqStages; ++s) {
@@ -351,60 +355,71 @@ __global__ void __launch_bounds__(kSqThreads, 1) search_tc_kernel(const __grid_c
     }
   } else {
     // ----------------------------------------------------------------------- epilogue
+    // warp e: TMEM lane quarter warp & 3 (query rows), column half e >> 2 of each chunk; with
+    // one half (k > kSqHalfK) the first four warps take all 256 columns and the rest idle
+    const int e = warp - 2 - kSqDecWarps;
     const int wq = warp & 3;
+    const int half = e >> 2;
+    const bool active = A.halves == 2 || half == 0;
+    const int col0 = A.halves == 2 ? half * (kSqN / 2) : 0;
+    const int ncol = A.halves == 2 ? kSqN / 2 : kSqN;
     const int qr = wq * 32 + lane;                  // query row of the tile (TMEM lane)
+    const int li = A.halves == 2 ? half * kSqM + qr : qr;   // this thread's list
+    const int ls = A.halves * kSqM;                 // list stride between entries
     const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
     const int k = A.k;
-    for (int j = 0; j < k; ++j) {
-      list_s[j * kSqM + qr] = -INFINITY;
-      list_i[j * kSqM + qr] = INT32_MAX;
-    }
-    float tau = -INFINITY;
-    for (int t = 0; t < nloc; ++t) {
-      const int b = t & 1;
-      const int64_t chunk = cslot + (int64_t)t * A.cpq;
-      if (!wait(acc_full + b, (uint32_t)((t >> 1) & 1)) || !wait(nrm_full + b, (uint32_t)((t >> 1) & 1))) {
-        fail(506);
-        break;
+    if (active) {
+      for (int j = 0; j < k; ++j) {
+        list_s[j * ls + li] = -INFINITY;
+        list_i[j * ls + li] = INT32_MAX;
       }
-      tc_fence_after();
-      for (int g = 0; g < kSqN / 32; ++g) {
-        uint32_t raw[32];
-        tmem_ld32(lane_base + (uint32_t)(b * kSqN + 32 * g), raw);
-        tmem_ld_wait();
-        if (g == kSqN / 32 - 1) {
-          tc_fence_before();
-          mbar_arrive(acc_empty + b);
+      float tau = -INFINITY;
+      for (int t = 0; t < nloc; ++t) {
+        const int b = t & 1;
+        const int64_t chunk = cslot + (int64_t)t * A.cpq;
+        if (!wait(acc_full + b, (uint32_t)((t >> 1) & 1)) || !wait(nrm_full + b, (uint32_t)((t >> 1) & 1))) {
+          fail(506);
+          break;
         }
+        tc_fence_after();
+        for (int g = 0; g < ncol / 32; ++g) {
+          uint32_t raw[32];
+          tmem_ld32(lane_base + (uint32_t)(b * kSqN + col0 + 32 * g), raw);
+          tmem_ld_wait();
+          if (g == ncol / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(acc_empty + b);
+          }
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = 32 * g + e;
-          const float sc = __uint_as_float(raw[e]) * s_norm[b * kSqN + c];
-          const int64_t id = chunk * kSqN + c;
-          if (sc > tau && id < A.N) {
-            // insert (ids rise within a CTA, so a later equal score stays behind)
-            int pos = k - 1;
-            while (pos > 0 && list_s[(pos - 1) * kSqM + qr] < sc) {
-              list_s[pos * kSqM + qr] = list_s[(pos - 1) * kSqM + qr];
-              list_i[pos * kSqM + qr] = list_i[(pos - 1) * kSqM + qr];
-              --pos;
+          for (int e2 = 0; e2 < 32; ++e2) {
+            const int c = col0 + 32 * g + e2;
+            const float sc = __uint_as_float(raw[e2]) * s_norm[b * kSqN + c];
+            const int64_t id = chunk * kSqN + c;
+            if (sc > tau && id < A.N) {
+              // insert (ids rise within a list, so a later equal score stays behind)
+              int pos = k - 1;
+              while (pos > 0 && list_s[(pos - 1) * ls + li] < sc) {
+                list_s[pos * ls + li] = list_s[(pos - 1) * ls + li];
+                list_i[pos * ls + li] = list_i[(pos - 1) * ls + li];
+                --pos;
+              }
+              list_s[pos * ls + li] = sc;
+              list_i[pos * ls + li] = (int32_t)id;
+              tau = list_s[(k - 1) * ls + li];
             }
-            list_s[pos * kSqM + qr] = sc;
-            list_i[pos * kSqM + qr] = (int32_t)id;
-            tau = list_s[(k - 1) * kSqM + qr];
           }
         }
+        mbar_arrive(nrm_empty + b);
       }
-      mbar_arrive(nrm_empty + b);
-    }
-    const int qg = qt * kSqM + qr;
-    if (qg < A.nq) {
-      float* cs = A.cand_s + (int64_t)qg * A.cpq * k + (int64_t)cslot * k;
-      int64_t* ci = A.cand_i + (int64_t)qg * A.cpq * k + (int64_t)cslot * k;
-      for (int j = 0; j < k; ++j) {
-        const int32_t id = list_i[j * kSqM + qr];
-        cs[j] = list_s[j * kSqM + qr];
-        ci[j] = id == INT32_MAX ? INT64_MAX : (int64_t)id;
+      const int qg = qt * kSqM + qr;
+      if (qg < A.nq) {
+        const int64_t per_q = (int64_t)A.cpq * A.halves * k;
+        const int64_t o = (int64_t)qg * per_q + ((int64_t)cslot * A.halves + (A.halves == 2 ? half : 0)) * k;
+        for (int j = 0; j < k; ++j) {
+          const int32_t id = list_i[j * ls + li];
+          A.cand_s[o + j] = list_s[j * ls + li];
+          A.cand_i[o + j] = id == INT32_MAX ? INT64_MAX : (int64_t)id;
+        }
       }
     }
   }
@@ -485,8 +500,9 @@ SqWs sq_ws(const tq_ctx* ctx, int64_t nq, int k, int sms) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   w.qop = 0;
   w.cs = up((size_t)w.nq_pad * 2 * w.Kh * sizeof(__half));
-  w.ci = w.cs + up((size_t)nq * w.cpq * k * sizeof(float));
-  w.total = w.ci + up((size_t)nq * w.cpq * k * sizeof(int64_t));
+  const int halves = k <= kSqHalfK ? 2 : 1;
+  w.ci = w.cs + up((size_t)nq * w.cpq * halves * k * sizeof(float));
+  w.total = w.ci + up((size_t)nq * w.cpq * halves * k * sizeof(int64_t));
   return w;
 }
 
@@ -559,6 +575,7 @@ int launch_search_tc(const tq_ctx* ctx, const float* q, int64_t nq, const tq_pac
   a.code_bytes = ctx->lay.code_bytes;
   a.k = k;
   a.cpq = W.cpq;
+  a.halves = k <= kSqHalfK ? 2 : 1;
   a.nchunks = (N + kSqN - 1) / kSqN;
   a.cand_s = cs;
   a.cand_i = ci;
@@ -593,7 +610,7 @@ int launch_search_tc(const tq_ctx* ctx, const float* q, int64_t nq, const tq_pac
     default: return fail(TQ_ERR_INTERNAL, "search: code layout");
   }
   if (r != TQ_OK) return r;
-  return launch_search_merge(cs, ci, nq, (int64_t)W.cpq * k, k, scores, ids, st);
+  return launch_search_merge(cs, ci, nq, (int64_t)W.cpq * a.halves * k, k, scores, ids, st);
 }
 
 }  // namespace tq
