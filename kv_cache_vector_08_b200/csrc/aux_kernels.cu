@@ -24,23 +24,60 @@ __device__ __forceinline__ bool better(float s1, int64_t i1, float s2, int64_t i
 }
 
 // ----------------------------------------------------------------------- query prepare
-// out[a] = (Pi q_a, S q_a); one thread per output coordinate.
+// out[a] = (Pi q_a, S q_a) in fp32.  CTA = 16 queries x 16 outputs (the outputs index the
+// concatenation [Pi q | S q]); the terms j run in chunks of 128: the chunk's 16 columns of
+// Pi^T / S^T and the 16 query rows are staged in shared memory with one round of loads,
+// thread (query, 4 outputs, quarter of the chunk) accumulates 4 dot products, and the
+// quarters (adjacent lanes) are summed by shuffles at the end.
+constexpr int kPqRows = 16, kPqCols = 16, kPqChunk = 128;
+
 template <typename T>
-__global__ void prepare_queries_kernel(const T* __restrict__ q, int64_t nq, int64_t ld, int d, int m,
-                                       const float* __restrict__ PiT, const float* __restrict__ ST,
-                                       float* __restrict__ out, int64_t out_ld) {
-  int64_t a = blockIdx.y;
-  int o = blockIdx.x * blockDim.x + threadIdx.x;
-  if (a >= nq || o >= d + m) return;
-  const T* qa = q + a * ld;
-  float acc = 0.f;
-  if (o < d) {
-    for (int j = 0; j < d; ++j) acc = fmaf(PiT[(size_t)j * d + o], load_f(qa + j), acc);
-  } else {
-    int r = o - d;
-    for (int j = 0; j < d; ++j) acc = fmaf(ST[(size_t)j * m + r], load_f(qa + j), acc);
+__global__ void __launch_bounds__(256) prepare_queries_kernel(const T* __restrict__ q, int64_t nq, int64_t ld, int d,
+                                                              int m, const float* __restrict__ PiT,
+                                                              const float* __restrict__ ST, float* __restrict__ out,
+                                                              int64_t out_ld) {
+  __shared__ float ms[kPqChunk][kPqCols + 1];
+  __shared__ float xs[kPqRows][kPqChunk + 1];
+  const int64_t r0 = (int64_t)blockIdx.x * kPqRows;
+  const int o0 = blockIdx.y * kPqCols;
+  const int t = threadIdx.x;
+  const int kq = t & 3, og = (t >> 2) & 3, r = t >> 4;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int k0 = 0; k0 < d; k0 += kPqChunk) {
+    const int kn = min(kPqChunk, d - k0);
+    for (int e = t; e < kPqChunk * kPqCols; e += 256) {
+      const int jj = e / kPqCols, oc = e % kPqCols, oo = o0 + oc;
+      float v = 0.f;
+      if (jj < kn) {
+        if (oo < d) v = __ldg(PiT + (size_t)(k0 + jj) * d + oo);
+        else if (oo < d + m) v = __ldg(ST + (size_t)(k0 + jj) * m + (oo - d));
+      }
+      ms[jj][oc] = v;
+    }
+    for (int e = t; e < kPqRows * kPqChunk; e += 256) {
+      const int rr = e / kPqChunk, jj = e % kPqChunk;
+      xs[rr][jj] = (r0 + rr < nq && jj < kn) ? load_f(q + (r0 + rr) * ld + k0 + jj) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int jj = kq; jj < kn; jj += 4) {
+      const float x = xs[r][jj];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = fmaf(ms[jj][4 * og + i], x, acc[i]);
+    }
+    __syncthreads();
   }
-  out[a * out_ld + o] = acc;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 1);
+    acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 2);
+  }
+  if (kq == 0 && r0 + r < nq)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int oo = o0 + 4 * og + i;
+      if (oo < d + m) out[(r0 + r) * out_ld + oo] = acc[i];
+    }
 }
 
 // One CTA per query: k rounds of arg-max over all candidates.
@@ -87,12 +124,12 @@ int launch_prepare_queries(const tq_ctx* ctx, const void* q, int q_dtype, int64_
                            int64_t out_ld, cudaStream_t st) {
   if (nq == 0) return TQ_OK;
   int d = ctx->lay.d, m = ctx->m;
-  dim3 grid(div_up(d + m, 128), (unsigned)nq);
+  dim3 grid((unsigned)div_up(nq, kPqRows), (unsigned)div_up(d + m, kPqCols));
   if (q_dtype == TQ_DTYPE_F32)
-    prepare_queries_kernel<float><<<grid, 128, 0, st>>>(static_cast<const float*>(q), nq, ld, d, m, ctx->PiT, ctx->ST,
+    prepare_queries_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(q), nq, ld, d, m, ctx->PiT, ctx->ST,
                                                         out, out_ld);
   else if (q_dtype == TQ_DTYPE_BF16)
-    prepare_queries_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(q), nq, ld, d, m,
+    prepare_queries_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), nq, ld, d, m,
                                                                 ctx->PiT, ctx->ST, out, out_ld);
   else
     return fail(TQ_ERR_INVALID_ARG, "query dtype must be TQ_DTYPE_F32 or TQ_DTYPE_BF16");

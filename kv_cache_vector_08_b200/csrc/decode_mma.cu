@@ -1007,8 +1007,8 @@ __global__ void __launch_bounds__(128) logits_mma_kernel(LogitArgs A) {
   const int64_t k0 = (int64_t)blockIdx.x * A.keys_per_cta;
   const int64_t k1 = min(A.n, k0 + A.keys_per_cta);
   const int qi = qb * kRep + l;
-  // the next tile's code words and norms are loaded before this tile is computed, so the
-  // global-memory latency overlaps the tensor-core work
+  // code words and norms of a warp's 16-key tiles are loaded three steps ahead of their
+  // use, so the global-memory latency overlaps the tensor-core work
   struct Tile {
     Words<GC::DG, GC::PK> wa, wb;
     float na, ra, nb, rb;
@@ -1025,11 +1025,7 @@ __global__ void __launch_bounds__(128) logits_mma_kernel(LogitArgs A) {
     T.nb = vb ? h2f(__ldg(A.norm + kb)) : 0.f;
     T.rb = vb ? h2f(__ldg(A.rnorm + kb)) : 0.f;
   };
-  Tile cur, nxt;
-  int64_t base = k0 + warp * 16;
-  if (base < k1) load(base, cur);
-  for (; base < k1; base += 64) {
-    if (base + 64 < k1) load(base + 64, nxt);
+  auto compute = [&](const Tile& cur, int64_t base) {
     const int64_t ka = base + g, kb = base + g + 8;
     const bool va = ka < k1, vb = kb < k1;
     float mse[4] = {0.f, 0.f, 0.f, 0.f}, sgn[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1057,16 +1053,32 @@ __global__ void __launch_bounds__(128) logits_mma_kernel(LogitArgs A) {
       if (va) A.out[(size_t)qi * A.n + ka] = la;
       if (vb) A.out[(size_t)qi * A.n + kb] = lb;
     }
-    cur = nxt;
+  };
+  // three 16-key tiles of this warp in flight: the tile three steps ahead is requested as
+  // soon as a tile's registers are free
+  Tile t0, t1, t2;
+  const int64_t b0 = k0 + warp * 16;
+  if (b0 < k1) load(b0, t0);
+  if (b0 + 64 < k1) load(b0 + 64, t1);
+  if (b0 + 128 < k1) load(b0 + 128, t2);
+  for (int64_t base = b0; base < k1; base += 192) {
+    compute(t0, base);
+    if (base + 192 < k1) load(base + 192, t0);
+    if (base + 64 >= k1) break;
+    compute(t1, base + 64);
+    if (base + 256 < k1) load(base + 256, t1);
+    if (base + 128 >= k1) break;
+    compute(t2, base + 128);
+    if (base + 320 < k1) load(base + 320, t2);
   }
 }
 
 template <class GC>
 int launch_logits_t(LogitArgs A, cudaStream_t st) {
   const int nqb = (A.nq + kRep - 1) / kRep;
-  // about 8 CTAs per SM in total (the query fragments are built once per CTA), whole
-  // 64-key steps per CTA
-  int64_t ctas = (int64_t)148 * 8 / nqb;
+  // about 4 CTAs per SM in total, one wave (the query fragments are built once per CTA),
+  // whole 64-key steps per CTA
+  int64_t ctas = (int64_t)148 * 4 / nqb;
   if (ctas < 1) ctas = 1;
   int64_t per = (A.n + ctas - 1) / ctas;
   per = ((per + 63) / 64) * 64;

@@ -260,13 +260,17 @@ def test_logits_on_oracle_codes(d, bits, n, nq):
     parity.assert_close(lg, oracle.estimate_inner_products(op, qn.astype(np.float64), o), "logits")
 
 
-def test_prepare_queries():
-    ctx = tq.Context(128, 4, 3, tq.MODE_PROD)
-    q = W.gaussian((7, 128), 1, 2).astype(np.float32)
+@pytest.mark.parametrize("d,nq", [(128, 7), (64, 1), (200, 33), (300, 16), (1536, 5)])
+def test_prepare_queries(d, nq):
+    """Pi q and S q of unit-variance queries: chunks of 128 terms, ragged query and output
+    blocks (d not a multiple of 16 or 128)."""
+    ctx = tq.Context(d, 4, 3, tq.MODE_PROD)
+    q = W.gaussian((nq, d), 1, 2).astype(np.float32)
     out = tq.prepare_queries(ctx, torch.tensor(q, device=DEV)).cpu().numpy()
-    qt, qs = oracle.prepare_query(oracle.make_params(128, 4, 3, 0), q.astype(np.float64))
-    assert np.abs(out[:, :128] - qt).max() < 1e-4
-    assert np.abs(out[:, 128:] - qs).max() < 1e-3
+    qt, qs = oracle.prepare_query(oracle.make_params(d, 4, 3, 0), q.astype(np.float64))
+    tol = 1e-4 * np.sqrt(d / 128.0)
+    assert np.abs(out[:, :d] - qt).max() < tol
+    assert np.abs(out[:, d:] - qs).max() < 10 * tol
 
 
 # ------------------------------------------------------------------------------ decode
