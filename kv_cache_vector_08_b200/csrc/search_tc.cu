@@ -390,10 +390,20 @@ __global__ void __launch_bounds__(kSqThreads, 1) search_tc_kernel(const __grid_c
             tc_fence_before();
             mbar_arrive(acc_empty + b);
           }
+          // the 32 scores first, then one test against the list's threshold: most groups
+          // of 32 hold no candidate once the list has filled
+          float sv[32];
+          float smax = -INFINITY;
+#pragma unroll
+          for (int e2 = 0; e2 < 32; ++e2) {
+            sv[e2] = __uint_as_float(raw[e2]) * s_norm[b * kSqN + col0 + 32 * g + e2];
+            smax = fmaxf(smax, sv[e2]);
+          }
+          if (!(smax > tau)) continue;
 #pragma unroll
           for (int e2 = 0; e2 < 32; ++e2) {
             const int c = col0 + 32 * g + e2;
-            const float sc = __uint_as_float(raw[e2]) * s_norm[b * kSqN + c];
+            const float sc = sv[e2];
             const int64_t id = chunk * kSqN + c;
             if (sc > tau && id < A.N) {
               // insert (ids rise within a list, so a later equal score stays behind)
