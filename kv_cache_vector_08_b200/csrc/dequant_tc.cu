@@ -258,14 +258,13 @@ __global__ void __launch_bounds__(kDqThreads, 1) dequant_tc_kernel(const __grid_
     for (int t = 0; t < nloc; ++t) {
       const int ab = t % NA;
       load_row(t + 1, nxt, nxt_n, nxt_v, nxt_r);       // one tile ahead: its loads fly during this tile
-      // codes -> fp16 (hi, lo) pairs of the centroids, two coordinates per 32-bit column
-      uint32_t hi[G0][16], lo[G0][16], sg[QJL ? G0 : 1][16];
-      if constexpr (P == 4) {
-        // 4-bit codes: slice u of a group is word u, coordinate j of the slice has its low
-        // three code bits in nibble j and its top bit at the msb of byte j (j < 4) or, after
-        // a shift by 4, of byte j - 4; one byte permute looks up four bytes
-#pragma unroll
-        for (int g = 0; g < G0; ++g) {
+      // codes -> fp16 (hi, lo) pairs of the centroids, two coordinates per 32-bit column, of
+      // this worker's group g (and, QJL, the fp16 +-||r|| pairs)
+      auto convert = [&](int g, uint32_t (&hi)[16], uint32_t (&lo)[16], uint32_t (&sg)[16]) {
+        if constexpr (P == 4) {
+          // 4-bit codes: slice u of a group is word u, coordinate j of the slice has its low
+          // three code bits in nibble j and its top bit at the msb of byte j (j < 4) or, after
+          // a shift by 4, of byte j - 4; one byte permute looks up four bytes
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const uint32_t w = cur[g * P + u];
@@ -278,14 +277,14 @@ __global__ void __launch_bounds__(kDqThreads, 1) dequant_tc_kernel(const __grid_
               const uint32_t hl = prmt(A.bt[0][0], A.bt[0][1], sl), hh8 = prmt(A.bt[1][0], A.bt[1][1], sl) ^ sgn;
               const uint32_t ll = prmt(A.bt[2][0], A.bt[2][1], sl), lh8 = prmt(A.bt[3][0], A.bt[3][1], sl) ^ sgn;
               const int i = 4 * u + 2 * hh;                // pair index of coordinates 8u + 4hh, +1
-              hi[g][i] = prmt(hl, hh8, 0x5140u);
-              hi[g][i + 1] = prmt(hl, hh8, 0x7362u);
-              lo[g][i] = prmt(ll, lh8, 0x5140u);
-              lo[g][i + 1] = prmt(ll, lh8, 0x7362u);
+              hi[i] = prmt(hl, hh8, 0x5140u);
+              hi[i + 1] = prmt(hl, hh8, 0x7362u);
+              lo[i] = prmt(ll, lh8, 0x5140u);
+              lo[i + 1] = prmt(ll, lh8, 0x7362u);
               if constexpr (QJL) {
                 const uint32_t nm = ~top;                  // fp16 sign set where the QJL bit is 0
-                sg[g][i] = (prmt(nm, 0u, 0x1404u) & 0x80008000u) | (cur_r | (cur_r << 16));
-                sg[g][i + 1] = (prmt(nm, 0u, 0x3424u) & 0x80008000u) | (cur_r | (cur_r << 16));
+                sg[i] = (prmt(nm, 0u, 0x1404u) & 0x80008000u) | (cur_r | (cur_r << 16));
+                sg[i + 1] = (prmt(nm, 0u, 0x3424u) & 0x80008000u) | (cur_r | (cur_r << 16));
               }
             }
           }
@@ -296,42 +295,60 @@ __global__ void __launch_bounds__(kDqThreads, 1) dequant_tc_kernel(const __grid_
             for (int e = 0; e < 32; ++e) {
               if (j0 + e >= A.d) {
                 const uint32_t keep = (e & 1) ? 0x0000FFFFu : 0xFFFF0000u;
-                hi[g][e / 2] &= keep;
-                lo[g][e / 2] &= keep;
-                if constexpr (QJL) sg[g][e / 2] &= keep;
+                hi[e / 2] &= keep;
+                lo[e / 2] &= keep;
+                if constexpr (QJL) sg[e / 2] &= keep;
               }
             }
           }
-        }
-      } else {
+        } else {
 #pragma unroll
-      for (int g = 0; g < G0; ++g) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int j = 32 * (g_lo + g) + e;
-          const uint32_t ca = group_code(cur + g * P, P, e), cb = group_code(cur + g * P, P, e + 1);
-          const uint32_t ta = (j < A.d) ? s_tbl[ca] : 0u;
-          const uint32_t tb = (j + 1 < A.d) ? s_tbl[cb] : 0u;
-          hi[g][e / 2] = __byte_perm(ta, tb, 0x5410);
-          lo[g][e / 2] = __byte_perm(ta, tb, 0x7632);
-          if constexpr (QJL) {
-            // +-||r|| (fp16; the sign bit set where the QJL sign bit is 0), zero past d
-            const uint32_t sa = (j < A.d) ? (cur_r | ((((ca >> (P - 1)) & 1u) ^ 1u) << 15)) : 0u;
-            const uint32_t sb = (j + 1 < A.d) ? (cur_r | ((((cb >> (P - 1)) & 1u) ^ 1u) << 15)) : 0u;
-            sg[g][e / 2] = sa | (sb << 16);
+          for (int e = 0; e < 32; e += 2) {
+            const int j = 32 * (g_lo + g) + e;
+            const uint32_t ca = group_code(cur + g * P, P, e), cb = group_code(cur + g * P, P, e + 1);
+            const uint32_t ta = (j < A.d) ? s_tbl[ca] : 0u;
+            const uint32_t tb = (j + 1 < A.d) ? s_tbl[cb] : 0u;
+            hi[e / 2] = __byte_perm(ta, tb, 0x5410);
+            lo[e / 2] = __byte_perm(ta, tb, 0x7632);
+            if constexpr (QJL) {
+              // +-||r|| (fp16; the sign bit set where the QJL sign bit is 0), zero past d
+              const uint32_t sa = (j < A.d) ? (cur_r | ((((ca >> (P - 1)) & 1u) ^ 1u) << 15)) : 0u;
+              const uint32_t sb = (j + 1 < A.d) ? (cur_r | ((((cb >> (P - 1)) & 1u) ^ 1u) << 15)) : 0u;
+              sg[e / 2] = sa | (sb << 16);
+            }
           }
         }
-      }
-      }
-      if (!wait(a_empty + ab, (uint32_t)(((t / NA) & 1) ^ 1))) { fail(304); ok = false; break; }
-      tc_fence_after();
+      };
       const uint32_t acol = lane_base + 256u + (uint32_t)(ab * 128);
+      if constexpr (!QJL) {
+        // all groups converted before the wait for the A buffer (the conversion overlaps the
+        // MMAs of the tile before)
+        uint32_t hi[G0][16], lo[G0][16], sg0[16];
 #pragma unroll
-      for (int g = 0; g < G0; ++g) {
-        if (g_lo + g < g_hi) {
-          tmem_st16(acol + (uint32_t)(16 * (g_lo + g)), hi[g]);
-          tmem_st16(acol + 64u + (uint32_t)(16 * (g_lo + g)), lo[g]);
-          if constexpr (QJL) tmem_st16(acol + 128u + (uint32_t)(16 * (g_lo + g)), sg[g]);
+        for (int g = 0; g < G0; ++g) convert(g, hi[g], lo[g], sg0);
+        if (!wait(a_empty + ab, (uint32_t)(((t / NA) & 1) ^ 1))) { fail(304); ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int g = 0; g < G0; ++g) {
+          if (g_lo + g < g_hi) {
+            tmem_st16(acol + (uint32_t)(16 * (g_lo + g)), hi[g]);
+            tmem_st16(acol + 64u + (uint32_t)(16 * (g_lo + g)), lo[g]);
+          }
+        }
+      } else {
+        // QJL: three operand halves per group would not fit in registers for every group at
+        // once, so each group is converted and stored in turn after the wait
+        if (!wait(a_empty + ab, (uint32_t)(((t / NA) & 1) ^ 1))) { fail(304); ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int g = 0; g < G0; ++g) {
+          if (g_lo + g < g_hi) {
+            uint32_t hi[16], lo[16], sg[16];
+            convert(g, hi, lo, sg);
+            tmem_st16(acol + (uint32_t)(16 * (g_lo + g)), hi);
+            tmem_st16(acol + 64u + (uint32_t)(16 * (g_lo + g)), lo);
+            tmem_st16(acol + 128u + (uint32_t)(16 * (g_lo + g)), sg);
+          }
         }
       }
       tmem_st_wait();
