@@ -226,7 +226,8 @@ int tq_prepare_queries(const tq_ctx* ctx, const float* q, int64_t nq, int64_t ld
  * 0..n-1 ([ADM] "computing attention logits" on 4-bit keys; [ZX] "两阶段内积量化"):
  *   logits[a*n + b] = norm_b * ( <Pi q_a, c[idx_b]> + sqrt(pi/2)/m * rnorm_b * <S q_a, 2 s_b - 1> )
  * (prod mode; MSE-mode contexts give the first term only).  q: device float32 [nq][d];
- * logits: device float32 [nq][n].  workspace: device, >= tq_attn_logits_workspace_size. */
+ * logits: device float32 [nq][n].  workspace: device, 16-byte aligned (else TQ_ERR_INVALID_ARG),
+ * >= tq_attn_logits_workspace_size. */
 size_t tq_attn_logits_workspace_size(const tq_ctx* ctx, int64_t nq);
 int tq_attn_logits(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* keys, int64_t n,
                    float* logits, void* workspace, size_t ws_bytes, tq_stream_t stream);

@@ -993,15 +993,19 @@ __global__ void __launch_bounds__(128) logits_mma_kernel(LogitArgs A) {
       const float h = __half2float(__float2half_rn(v));
       return lo ? v - h : h;
     };
+    // the thread's coordinates come four at a time (16-byte loads: d and 2d are multiples
+    // of 4, and each group of four starts at a multiple of 4)
 #pragma unroll
     for (int u = 0; u < GC::NS; ++u)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int c = GC::CQ * l + 8 * u + 4 * h;
-        bm[u][h][0] = pack_h2(part(src[c]), part(src[c + 1]));
-        bm[u][h][1] = pack_h2(part(src[c + 2]), part(src[c + 3]));
-        bs[u][h][0] = pack_h2(part(src[A.d + c]), part(src[A.d + c + 1]));
-        bs[u][h][1] = pack_h2(part(src[A.d + c + 2]), part(src[A.d + c + 3]));
+        const float4 vm = __ldg(reinterpret_cast<const float4*>(src + c));
+        const float4 vs = __ldg(reinterpret_cast<const float4*>(src + A.d + c));
+        bm[u][h][0] = pack_h2(part(vm.x), part(vm.y));
+        bm[u][h][1] = pack_h2(part(vm.z), part(vm.w));
+        bs[u][h][0] = pack_h2(part(vs.x), part(vs.y));
+        bs[u][h][1] = pack_h2(part(vs.z), part(vs.w));
       }
   }
   const int64_t k0 = (int64_t)blockIdx.x * A.keys_per_cta;
@@ -1259,6 +1263,8 @@ int launch_logits_mma(const tq_ctx* ctx, const float* q, int64_t nq, const tq_pa
   if (ctx->mode != TQ_MODE_PROD || (d != 64 && d != 128) || P < 2 || P > 4) return kNotHandled;
   if (nq > (int64_t)kRep * 65535) return kNotHandled;
   if ((reinterpret_cast<uintptr_t>(keys->codes) & 15) != 0) return kNotHandled;
+  if ((reinterpret_cast<uintptr_t>(ws) & 15) != 0)   // the prepared queries are read 16 bytes at a time
+    return fail(TQ_ERR_INVALID_ARG, "attn_logits: the workspace must be 16-byte aligned");
   float* qprep = static_cast<float*>(ws);
   int r = launch_prepare_queries(ctx, q, TQ_DTYPE_F32, nq, d, qprep, 2 * d, st);
   if (r != TQ_OK) return r;

@@ -20,7 +20,7 @@ import ctypes  # noqa: E402
 import kv_cache_vector_08_b200 as tq  # noqa: E402
 
 DEV = torch.device("cuda", 0)
-TQ_ERR_ALLOC, TQ_ERR_WORKSPACE = 4, 5
+TQ_ERR_INVALID_ARG, TQ_ERR_ALLOC, TQ_ERR_WORKSPACE = 1, 4, 5
 
 
 def _small_cache(d=128, n=512):
@@ -41,6 +41,13 @@ def test_undersized_workspaces_are_rejected():
     with pytest.raises(tq.TQError) as e:
         tq.attn_logits(ctx, q, pk, 512, workspace=small)
     assert e.value.status == TQ_ERR_WORKSPACE
+    # a workspace that is large enough but not 16-byte aligned is refused before any launch
+    big = torch.empty(need + 64, dtype=torch.uint8, device=DEV)
+    ps0 = pk.struct()
+    lg = torch.empty((4, 512), device=DEV)
+    st = L.tq_attn_logits(ctx.handle, ctypes.c_void_p(q.data_ptr()), 4, ctypes.byref(ps0), 512,
+                          ctypes.c_void_p(lg.data_ptr()), ctypes.c_void_p(big.data_ptr() + 4), need, None)
+    assert st == TQ_ERR_INVALID_ARG
     # search
     need = int(L.tq_search_workspace_size(ctx.handle, 4, 512, 10))
     out_s = torch.empty((4, 10), device=DEV)
