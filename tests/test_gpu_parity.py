@@ -356,6 +356,7 @@ def test_decode_end_to_end_matches_oracle_pipeline():
     (1536, 3000, 10, 4, 6), (3072, 700, 5, 4, 3), (96, 513, 33, 4, 6),     # wide / ragged chunk
     (128, 2000, 10, 4, 300), (128, 300, 1, 4, 129),                        # several query tiles
     (128, 2000, 10, 2, 6), (100, 1500, 7, 3, 6), (160, 1200, 10, 5, 6),    # 1-, 2-, 4-bit indices
+    (64, 900, 32, 4, 6),                                                   # largest k with two lists per query
 ])
 def test_search_topk_matches_oracle(d, N, k, bits, nq):
     db = W.unit_gaussian(N, d, 1, 10)
