@@ -328,6 +328,14 @@ def test_decode_matches_oracle(groups):
     parity.assert_close(out, ref, "decode %s" % (groups,))
 
 
+@pytest.mark.parametrize("groups", [((0, 128, 4, 4),), ((0, 64, 4, 4), (64, 64, 3, 3))])
+def test_decode_odd_max_len(groups):
+    """An odd cache length per (sequence, kv head): half of the caches start at an odd slot,
+    so their staged code and norm arrays land at odd offsets inside the stage buffers."""
+    out, ref, _ = _decode_case(2, 3, 12, 128, groups, [257, 130], 257, 21)
+    parity.assert_close(out, ref, "decode odd max_len %s" % (groups,))
+
+
 def test_decode_edge_lengths():
     """Empty sequence -> zeros; single token -> that token's dequantized value; ragged tails."""
     out, ref, (K, V, qn, kp, vp, offs) = _decode_case(4, 1, 4, 128, ((0, 128, 4, 4),), [0, 1, 129, 255], 256, 2)
