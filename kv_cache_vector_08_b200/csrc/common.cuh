@@ -104,6 +104,34 @@ namespace tq {
 void set_error(const std::string& msg);
 int fail(int code, const std::string& msg);
 int cuda_fail(cudaError_t e, const char* what);
+
+// Kernel attributes persist on a device: the dynamic shared-memory limit is raised only when
+// a launch needs more than any earlier launch of this kernel on the current device, and the
+// maximum carveout is requested once, instead of two driver calls before every launch.
+// (Like every attribute, they do not survive a cudaDeviceReset.)
+constexpr int kAttrDevices = 64;
+template <auto Kern>
+inline cudaError_t ensure_smem_attrs(int dyn_bytes, bool max_carveout) {
+  static int dyn_set[kAttrDevices];
+  static bool carve_set[kAttrDevices];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kAttrDevices) {
+    cudaGetLastError();
+    dev = -1;
+  }
+  if (dev < 0 || dyn_bytes > dyn_set[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_bytes);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0) dyn_set[dev] = dyn_bytes;
+  }
+  if (max_carveout && (dev < 0 || !carve_set[dev])) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(Kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0) carve_set[dev] = true;
+  }
+  return cudaSuccess;
+}
 void count_launch(uint64_t n = 1);
 
 // Limit of the pipeline waits of the dequantize, search and workspace-quantize kernels

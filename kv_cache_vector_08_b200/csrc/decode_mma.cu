@@ -1099,12 +1099,9 @@ int launch_mma_t(const MmaArgs& A, int nsplit, int BHkv, cudaStream_t st) {
   constexpr bool TWO = !std::is_same<G1, void>::value;
   using G1c = typename std::conditional<TWO, G1, G0>::type;
   const int dyn = std::max(kNStage * Stage<G0, G1c, TWO>::BYTES, kAccBytes);
-  cudaError_t ea = cudaFuncSetAttribute(decode_mma_kernel<G0, G1>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
-  if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncSetAttribute(decode_mma_kernel)");
   // one shared-memory carveout for the prep, decode and merge kernels, so they can share SMs
-  ea = cudaFuncSetAttribute(decode_mma_kernel<G0, G1>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                            cudaSharedmemCarveoutMaxShared);
-  if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncSetAttribute(decode_mma_kernel carveout)");
+  cudaError_t ea = ensure_smem_attrs<decode_mma_kernel<G0, G1>>(dyn, true);
+  if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncSetAttribute(decode_mma_kernel)");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nsplit, BHkv);
   cfg.blockDim = dim3((kWarps + 1) * 32);
@@ -1232,10 +1229,7 @@ int launch_decode_mma(const tq_ctx* const* kctx, const tq_ctx* const* vctx, cons
   const int64_t parts_bytes = (int64_t)kRep * W.part_ld * (int64_t)sizeof(float);
   M.stage_parts = parts_bytes <= 128 * 1024 ? 1 : 0;
   const int mdyn = pi_floats * (int)sizeof(float) + (M.stage_parts ? (int)parts_bytes : 0);
-  cudaError_t em = cudaFuncSetAttribute(decode_merge_heads_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mdyn);
-  if (em == cudaSuccess)
-    em = cudaFuncSetAttribute(decode_merge_heads_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                              cudaSharedmemCarveoutMaxShared);
+  cudaError_t em = ensure_smem_attrs<decode_merge_heads_kernel>(mdyn, true);
   if (em != cudaSuccess) return cuda_fail(em, "cudaFuncSetAttribute(decode_merge_heads_kernel)");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(B * Hkv * A.nsub);

@@ -380,7 +380,7 @@ int launch_dq_t(const CUtensorMap& tmb, const CUtensorMap& tms, int N, const DqA
   auto kern = dequant_tc_kernel<NG, P, QJL>;
   // one CTA per SM (it owns all 512 TMEM columns): ask for more than half the shared memory
   const int smem_bytes = SM::BYTES > 120 * 1024 ? SM::BYTES : 120 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  cudaError_t e = ensure_smem_attrs<dequant_tc_kernel<NG, P, QJL>>(smem_bytes, false);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(dequant_tc)");
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -463,7 +463,7 @@ int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& 
   constexpr int STAGE = 2 * kGenTile * 128 + 2 * kGenNb * 128;
   const int smem_bytes = kGenStages * STAGE + 256 + 1024;
   auto kern = quantize_gemm_kernel<P, KB, PROD, SIGN>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  cudaError_t e = ensure_smem_attrs<quantize_gemm_kernel<P, KB, PROD, SIGN>>(smem_bytes, false);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(quantize_gemm)");
   const int64_t units = (a.rows / kGenTile) * a.NB;
   const int grid = (int)std::min<int64_t>(units, sms);

@@ -698,7 +698,7 @@ int launch_tc_t(const tq_ctx* ctx, const void* x, int64_t n, int64_t ld, const t
   auto kern = quantize_tc_kernel<D, PROD, K>;
   // one CTA per SM: it owns all 512 TMEM columns (more than half the shared memory forces it)
   const int smem_bytes = SM::BYTES > 120 * 1024 ? SM::BYTES : 120 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  cudaError_t e = ensure_smem_attrs<quantize_tc_kernel<D, PROD, K>>(smem_bytes, false);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(quantize_tc)");
   const int64_t ntiles = (n + kTileM - 1) / kTileM;
   int sms = 148;

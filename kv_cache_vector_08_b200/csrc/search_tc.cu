@@ -530,7 +530,7 @@ int launch_sq_t(const CUtensorMap& tmq, const CUtensorMap& tmc, const SqArgs& a,
   const int smem = kSqStages * kSqStage + (P == 4 ? kSqCStages * kSqCStage : 0) + 2 * kSqMaxK * kSqM * 4 +
                    2 * kSqN * 4 + 32 * 4 + 256 + 1024;
   auto kern = search_tc_kernel<P>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = ensure_smem_attrs<search_tc_kernel<P>>(smem, false);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(search_tc)");
   kern<<<grid, kSqThreads, smem, st>>>(tmq, tmc, a);
   count_launch();
