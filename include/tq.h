@@ -29,6 +29,9 @@
  *     execution errors surface at the caller's next synchronisation.
  *   - A context is immutable after tq_init and may be used from several threads and
  *     streams at once.
+ *   - The library sets its kernels' shared-memory attributes on a device once and
+ *     remembers that it did: after a cudaDeviceReset of that device, load a fresh process
+ *     before calling the library on it again.
  *
  * Packed code layout (produced by tq_quantize_kv, read by every other call)
  *   A context with dimension d, MSE bits k (k = bits-1 in prod mode, k = bits in MSE
