@@ -897,7 +897,7 @@ def run_reference(args):
 
 
 # ------------------------------------------------------- small cases for profilers
-KERNEL_CASES = ("decode-serving-b16", "search-d1536-200k", "dequant-d128", "quantize-fp32-d1536", "logits-d128")
+KERNEL_CASES = ("decode-serving-b16", "search-d1536-200k", "search-d200-1m", "dequant-d128", "quantize-fp32-d1536", "logits-d128")
 
 
 def run_kernel_case(args):
@@ -932,8 +932,8 @@ def run_kernel_case(args):
         seq = torch.full((bench.B,), bench.T, dtype=torch.int32, device=dev)
         us = timed(lambda: bench.decode(seq))
         note = "%d token-heads" % (bench.B * bench.Hkv * bench.T)
-    elif case == "search-d1536-200k":
-        d, N, nq = 1536, 200000, 1000
+    elif case in ("search-d1536-200k", "search-d200-1m"):
+        d, N, nq = (1536, 200000, 1000) if case == "search-d1536-200k" else (200, 1000000, 1000)
         db = torch.nn.functional.normalize(torch.randn((N, d), generator=g, device=dev), dim=1)
         qs = torch.nn.functional.normalize(torch.randn((nq, d), generator=g, device=dev), dim=1)
         ctx = tq.Context(d, 4, 12, tq.MODE_PROD)
