@@ -277,20 +277,17 @@ __global__ void __launch_bounds__(kSqThreads, 1) search_tc_kernel(const __grid_c
         }
         if (!wait(empty + s, ph ^ 1)) { fail(505); ok = false; break; }
         uint8_t* dst = smem + s * kSqStage + kSqStageA + (row >> 3) * 1024 + rsw * 128;
-        // the atom's two code groups lie wholly inside d for a live row (every atom when 64
-        // divides d): that case skips the per-slice range checks
-        auto build = [&](auto full_tag) {
-          constexpr bool FULL = decltype(full_tag)::value;
+        // No range checks: coordinates >= d and rows past the database decode from zero
+        // words, the record's padding bytes or another row's codes, all to finite fp16
+        // values; those coordinates meet zero query entries (the query operand is zero past
+        // d) and those rows never enter a list (id >= N).
+        {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int g = 2 * ca + h;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {            // 8-coordinate slice u of group g: one 16-byte chunk
-              const int c0 = 32 * g + 8 * u;          // first coordinate of the slice
               uint32_t o[4];
-              if (!FULL && (!live || c0 >= A.d)) {
-                o[0] = o[1] = o[2] = o[3] = 0u;
-              } else if (!sign_atom) {
+              if (!sign_atom) {
                 if constexpr (P == 4) {
                   const uint32_t sel = w[h][u] & 0x77777777u;
 #pragma unroll
@@ -308,11 +305,6 @@ __global__ void __launch_bounds__(kSqThreads, 1) search_tc_kernel(const __grid_c
                     o[e / 2] = (va & 0xFFFFu) | (vb << 16);
                   }
                 }
-                if (!FULL && c0 + 8 > A.d) {                   // coordinates >= d are zero
-#pragma unroll
-                  for (int e = 0; e < 8; ++e)
-                    if (c0 + e >= A.d) o[e / 2] &= (e & 1) ? 0x0000FFFFu : 0xFFFF0000u;
-                }
               } else if constexpr (P == 4) {
                 // +-||r||: the fp16 sign bit set where the QJL sign bit is 0.  The sign bits of
                 // coordinates 0-3 are the byte msbs of the word, those of 4-7 after a shift by 4.
@@ -321,11 +313,6 @@ __global__ void __launch_bounds__(kSqThreads, 1) search_tc_kernel(const __grid_c
                   const uint32_t nm = ~(hh ? w[h][u] << 4 : w[h][u]);
                   o[2 * hh] = (prmt(nm, 0u, 0x1404u) & 0x80008000u) | rr;
                   o[2 * hh + 1] = (prmt(nm, 0u, 0x3424u) & 0x80008000u) | rr;
-                }
-                if (!FULL && c0 + 8 > A.d) {
-#pragma unroll
-                  for (int e = 0; e < 8; ++e)
-                    if (c0 + e >= A.d) o[e / 2] &= (e & 1) ? 0x0000FFFFu : 0xFFFF0000u;
                 }
               } else {
                 // +-||r||: the fp16 sign bit set where the QJL sign bit is 0
@@ -336,19 +323,12 @@ __global__ void __launch_bounds__(kSqThreads, 1) search_tc_kernel(const __grid_c
                       (w[h][code_bit_pos(P, 8 * u + e + 1, P - 1) >> 5] >> (code_bit_pos(P, 8 * u + e + 1, P - 1) & 31)) & 1u;
                   o[e / 2] = rr | ((sa ^ 1u) << 15) | ((sb ^ 1u) << 31);
                 }
-                if (!FULL && c0 + 8 > A.d) {
-#pragma unroll
-                  for (int e = 0; e < 8; ++e)
-                    if (c0 + e >= A.d) o[e / 2] &= (e & 1) ? 0x0000FFFFu : 0xFFFF0000u;
-                }
               }
               const int chunk16 = h * 4 + u;          // 16-byte chunk of the 128-byte row
               *reinterpret_cast<uint4*>(dst + ((chunk16 ^ rsw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
             }
           }
-        };
-        if (live && 64 * (ca + 1) <= A.d) build(std::true_type{});
-        else build(std::false_type{});
+        }
         fence_proxy_async_smem();
         mbar_arrive(full_b + s);
       }
