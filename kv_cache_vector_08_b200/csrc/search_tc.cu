@@ -475,6 +475,87 @@ __global__ void __launch_bounds__(256) search_query_kernel(const float* __restri
   }
 }
 
+// The same product for d a multiple of 8 (16-byte rows): CTA = 128 queries x 128 outputs of
+// one part, thread = 8 queries x 8 outputs (two 4 x 4 blocks 64 apart, so every shared-memory
+// read is one conflict-free 16-byte load), K in steps of 8 with the next step's global loads
+// in flight during the current step's 512 FMAs.  Every output sums its d terms in the same
+// order as the kernel above, so the two give identical operands.
+constexpr int kQgTile = 128;
+__global__ void __launch_bounds__(256) search_query_gemm_kernel(const float* __restrict__ q, int64_t nq, int d, int Kh,
+                                                                const float* __restrict__ PiT,
+                                                                const float* __restrict__ ST, float coef,
+                                                                __half* __restrict__ out) {
+  __shared__ __align__(16) float As[2][8][kQgTile + 4];   // [buffer][k][query]
+  __shared__ __align__(16) float Bs[2][8][kQgTile];       // [buffer][k][output]
+  const int64_t r0 = (int64_t)blockIdx.x * kQgTile;
+  const int o0 = blockIdx.y * kQgTile, part = blockIdx.z;
+  const float* M = part == 0 ? PiT : ST;
+  const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
+  // loader roles: A row t/2, k half t%2 (one 16-byte load); B k row t/32, outputs 4 (t%32)
+  const int ar = t >> 1, ak = 4 * (t & 1), bk = t >> 5, bo = 4 * (t & 31);
+  const bool a_ok = r0 + ar < nq, b_ok = o0 + bo < d;
+  const float* qa = q + (a_ok ? (r0 + ar) * d : 0) + ak;
+  const float* mb = M + (b_ok ? o0 + bo : 0) + (size_t)bk * d;
+  float4 ra = make_float4(0.f, 0.f, 0.f, 0.f), rb = ra;
+  auto fetch = [&](int k0) {
+    if (a_ok) ra = __ldg(reinterpret_cast<const float4*>(qa + k0));
+    if (b_ok) rb = __ldg(reinterpret_cast<const float4*>(mb + (size_t)k0 * d));
+  };
+  auto put = [&](int buf) {
+    As[buf][ak + 0][ar] = ra.x;
+    As[buf][ak + 1][ar] = ra.y;
+    As[buf][ak + 2][ar] = ra.z;
+    As[buf][ak + 3][ar] = ra.w;
+    *reinterpret_cast<float4*>(&Bs[buf][bk][bo]) = rb;
+  };
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  const int nk = d / 8;
+  fetch(0);
+  put(0);
+  __syncthreads();
+  for (int kt = 0; kt < nk; ++kt) {
+    const int cur = kt & 1;
+    if (kt + 1 < nk) fetch(8 * (kt + 1));
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[cur][kk][4 * ty]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[cur][kk][64 + 4 * ty]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[cur][kk][4 * tx]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[cur][kk][64 + 4 * tx]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    if (kt + 1 < nk) put(cur ^ 1);
+    __syncthreads();
+  }
+  const float sc = part == 0 ? 1.f : coef;
+  const int64_t K = 2 * (int64_t)Kh;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t row = r0 + (i < 4 ? 4 * ty + i : 64 + 4 * ty + i - 4);
+#pragma unroll
+    for (int jb = 0; jb < 2; ++jb) {
+      const int o = o0 + 64 * jb + 4 * tx;   // four outputs inside one 64-coordinate block
+      if (o < Kh) {
+        const __half2 lo = __floats2half2_rn(acc[i][4 * jb] * sc, acc[i][4 * jb + 1] * sc);
+        const __half2 hi = __floats2half2_rn(acc[i][4 * jb + 2] * sc, acc[i][4 * jb + 3] * sc);
+        uint2 v;
+        v.x = *reinterpret_cast<const uint32_t*>(&lo);
+        v.y = *reinterpret_cast<const uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(out + row * K + (int64_t)(o / 64) * 128 + part * 64 + (o % 64)) = v;
+      }
+    }
+  }
+}
+
 struct SqWs {
   size_t qop, cs, ci, total;
   int cpq, qtiles, Kh;
@@ -538,7 +619,14 @@ int launch_search_tc(const tq_ctx* ctx, const float* q, int64_t nq, const tq_pac
   int64_t* ci = reinterpret_cast<int64_t*>(base + W.ci);
   const int d = ctx->lay.d;
   // the query operand
-  {
+  if (d % 8 == 0 && (reinterpret_cast<uintptr_t>(q) & 15) == 0) {
+    const dim3 grid((unsigned)(W.nq_pad / kQgTile), (unsigned)((W.Kh + kQgTile - 1) / kQgTile), 2);
+    search_query_gemm_kernel<<<grid, 256, 0, st>>>(q, nq, d, W.Kh, ctx->PiT, ctx->ST, ctx->sqrt_pi_over_2_over_m,
+                                                   qop);
+    count_launch();
+    int r = check_launch("search_query_gemm_kernel");
+    if (r != TQ_OK) return r;
+  } else {
     const dim3 grid((unsigned)(W.nq_pad / 64), (unsigned)((W.Kh + 63) / 64), 2);
     search_query_kernel<<<grid, 256, 0, st>>>(q, nq, d, W.Kh, ctx->PiT, ctx->ST, ctx->sqrt_pi_over_2_over_m, qop);
     count_launch();
