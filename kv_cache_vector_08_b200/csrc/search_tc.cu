@@ -224,23 +224,31 @@ __global__ void __launch_bounds__(kSqThreads, 1) search_tc_kernel(const __grid_c
     const int NG = (A.d + 31) / 32;                 // code groups
     int64_t q = 0;
     bool ok = true;
+    // the row's norm and residual norm of chunk t + 1 load while chunk t is decoded
+    auto norms_of = [&](int tt, uint16_t& nv, uint16_t& rv) {
+      const int64_t idn = (cslot + (int64_t)tt * A.cpq) * kSqN + row;
+      nv = 0;
+      rv = 0;
+      if (tt < nloc && idn < A.N) {
+        nv = __ldg(A.norm + idn);
+        rv = __ldg(A.rnorm + idn);
+      }
+    };
+    uint16_t nxt_n, nxt_r;
+    norms_of(0, nxt_n, nxt_r);
     for (int t = 0; ok && t < nloc; ++t) {
       const int64_t chunk = cslot + (int64_t)t * A.cpq;
       const int64_t id = chunk * kSqN + row;
       const bool live = id < A.N;
       const uint8_t* rec = A.codes + (live ? id : 0) * (int64_t)A.code_bytes;
-      float rn = 0.f;
+      const uint16_t cur_n = nxt_n, cur_r = nxt_r;   // zero for a row past the database
+      norms_of(t + 1, nxt_n, nxt_r);
       // the chunk's norms for the epilogue
       const int nb = t & 1;
       if (!wait(nrm_empty + nb, (uint32_t)(((t >> 1) & 1) ^ 1))) { fail(504); ok = false; break; }
-      s_norm[nb * kSqN + row] = live ? __half2float(__ushort_as_half(A.norm[id])) : 0.f;
+      s_norm[nb * kSqN + row] = __half2float(__ushort_as_half(cur_n));
       mbar_arrive(nrm_full + nb);
-      uint32_t rbits = 0;
-      if (live) {
-        rn = __half2float(__ushort_as_half(A.rnorm[id]));
-        rbits = (uint32_t)A.rnorm[id] & 0x7FFFu;
-      }
-      (void)rn;
+      const uint32_t rbits = (uint32_t)cur_r & 0x7FFFu;
       const uint32_t rr = rbits | (rbits << 16);
       uint32_t w[2][P];                             // code words of the atom's two groups
       for (int a = 0; a < KA; ++a, ++q) {
