@@ -329,7 +329,9 @@ int tq_decode_attention_static(const tq_ctx* const* kctx, const tq_ctx* const* v
  * inner product ([TQN] "向量搜索中的应用"; [ADM] vector-search paragraph).  Ties keep the
  * lower id first.  q: device float32 [nq][d]; scores: device float32 [nq][k] (descending);
  * ids: device int64 [nq][k].  1 <= k <= 64, k <= N.
- * workspace: device, >= tq_search_workspace_size(ctx, nq, N, k). */
+ * workspace: device, >= tq_search_workspace_size(ctx, nq, N, k).
+ * Speed: with q 16-byte aligned and d a multiple of 8 the query projection runs as a
+ * register-blocked product; any other q gives the same results through a slower tiled one. */
 size_t tq_search_workspace_size(const tq_ctx* ctx, int64_t nq, int64_t N, int k);
 int tq_search_topk(const tq_ctx* ctx, const float* q, int64_t nq, const tq_packed* db, int64_t N,
                    int k, float* scores, int64_t* ids, void* workspace, size_t ws_bytes,
